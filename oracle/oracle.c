@@ -1,0 +1,377 @@
+/*
+ * ORACLE for the tensor-parallel reconciliation point -- TEST INFRASTRUCTURE.
+ *
+ * A plain, slow, obviously correct CPU implementation of what the GPU path
+ * computes. Only the test suite, the package smoke check and the benchmark's
+ * CPU-baseline leg load this library; the product path never does, and this
+ * file shares no code, header or table with the CUDA library.
+ *
+ * What it computes ("Interconnects e clusters", section 01 Conceito, and the
+ * all-reduce section of the NVL72 hosting post):
+ *   1. Partials. Each of N ranks owns the K/N-wide slice r of the projection
+ *      input; rank r's partial hidden vector is x_r . W_r (the weight matrix
+ *      is split between ranks, each rank computes a partial result over its
+ *      slice). Reading of an unstated step: the products are accumulated in
+ *      fp32, k ascending, starting from +0, each product rounded to fp32 and
+ *      then added (round-to-nearest-even, no fusion), and the sum is rounded
+ *      once to bf16 for the wire.
+ *   2. Ring all-reduce. The partials are summed before the residual stream
+ *      continues, by a ring all-reduce that puts 2(N-1)/N times the payload on
+ *      each rank's wire: a reduce-scatter in which each rank reduces one of N
+ *      slices, then a broadcast (all-gather) of the reduced slices. Simulated
+ *      literally with N rank-local buffers: at reduce-scatter step s rank r
+ *      sends chunk (r - s) mod N to rank (r + 1) mod N, which stores
+ *      bf16_rne(f32(received) + f32(own)). Reading: chunks are H/N-wide column
+ *      ranges of each token's hidden vector; chunk c is folded P_c, P_c+1, ...,
+ *      P_c-1, left to right.
+ *   3. Residual. out = bf16_rne(f32(residual) + f32(reduced)).
+ *
+ * Build: plain C11, -ffp-contract=off (no fused multiply-add), no fast-math,
+ * so every float operation is one IEEE round-to-nearest-even operation with
+ * subnormals kept.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_ERR_ARGS 1
+#define ORC_ERR_ALLOC 2
+#define ORC_ERR_RING 3
+
+/* ---------------------------------------------------------------- bf16 -- */
+
+/* bf16 bits -> float: the bf16 pattern is the top half of the float. */
+float orc_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* float -> bf16, round to nearest, ties to even, on the bit pattern: add
+ * 0x7FFF plus the bit that will become the last kept bit, keep the top half.
+ * A carry out of the fraction bumps the exponent, which is the correct result
+ * (up to overflow into infinity). NaN keeps its sign and becomes the quiet NaN
+ * 0x7FC0. Subnormals are not flushed. */
+uint16_t orc_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu) != 0u)
+        return (uint16_t)(((u >> 16) & 0x8000u) | 0x7FC0u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/* double -> bf16, correctly rounded (to nearest, ties to even) straight from
+ * the double, by scaling to the bf16 quantum of |v| and rounding to an
+ * integer: quantum 2^(e-8) for |v| in [2^(e-1), 2^e) (8 significant bits),
+ * never finer than the subnormal quantum 2^-133. Used to classify partials
+ * whose fp64 value lies near a bf16 rounding boundary. */
+uint16_t orc_bf16_rne_f64(double v)
+{
+    if (isnan(v))
+        return (uint16_t)((signbit(v) ? 0x8000u : 0u) | 0x7FC0u);
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (isinf(a))
+        return (uint16_t)(sign | 0x7F80u);
+    if (a == 0.0)
+        return sign;
+    int ex;
+    (void)frexp(a, &ex);               /* a = f * 2^ex, f in [0.5, 1) */
+    int q = ex - 8;
+    if (q < -133)
+        q = -133;
+    double r = nearbyint(ldexp(a, -q)); /* default rounding mode: ties to even */
+    double res = ldexp(r, q);
+    if (res >= 0x1p128)
+        return (uint16_t)(sign | 0x7F80u);
+    float rf = (float)res;             /* exact: res has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &rf, sizeof u);
+    return (uint16_t)(sign | (u >> 16));
+}
+
+/* ------------------------------------------------------------ partials -- */
+
+typedef struct {
+    int n_ranks;
+    int64_t tokens, k, n_rows, row_begin, row_end;
+    const uint16_t *x, *w_rows;
+    uint16_t *p;
+    double *p64, *pabs;
+} partial_job;
+
+static void partial_rows(const partial_job *j)
+{
+    const int64_t ks = j->k / j->n_ranks;
+    for (int r = 0; r < j->n_ranks; ++r)
+        for (int64_t m = 0; m < j->tokens; ++m)
+            for (int64_t i = j->row_begin; i < j->row_end; ++i) {
+                const uint16_t *xr = j->x + m * j->k + (int64_t)r * ks;
+                const uint16_t *wr = j->w_rows + i * j->k + (int64_t)r * ks;
+                float acc = 0.0f;
+                double d = 0.0, a = 0.0;
+                for (int64_t kk = 0; kk < ks; ++kk) {
+                    float prod = orc_f32(xr[kk]) * orc_f32(wr[kk]);
+                    acc = acc + prod;
+                    double dp = (double)orc_f32(xr[kk]) * (double)orc_f32(wr[kk]);
+                    d += dp;
+                    a += fabs(dp);
+                }
+                int64_t o = ((int64_t)r * j->tokens + m) * j->n_rows + i;
+                j->p[o] = orc_bf16_rne(acc);
+                if (j->p64)
+                    j->p64[o] = d;
+                if (j->pabs)
+                    j->pabs[o] = a;
+            }
+}
+
+static void *partial_thread(void *arg)
+{
+    partial_rows((const partial_job *)arg);
+    return NULL;
+}
+
+/* Partials of the selected output rows.
+ *   x       [tokens][k]     bf16 activations (the full projection input)
+ *   w_rows  [n_rows][k]     the selected rows h of the Linear weight W[H][K]
+ *   p       [n_ranks][tokens][n_rows]  bf16 partials (out)
+ *   p64     same shape, fp64 sum of the same products (out, may be NULL)
+ *   pabs    same shape, fp64 sum of |products| (out, may be NULL)
+ * Rows are split across n_threads threads; every element is computed by one
+ * thread in the same order, so the result does not depend on n_threads. */
+int orc_partials(int n_ranks, int64_t tokens, int64_t k, const uint16_t *x,
+                 int64_t n_rows, const uint16_t *w_rows, uint16_t *p, double *p64,
+                 double *pabs, int n_threads)
+{
+    if (n_ranks < 1 || tokens < 0 || k < 0 || n_rows < 0 || k % n_ranks != 0)
+        return ORC_ERR_ARGS;
+    if ((tokens && k && !x) || (n_rows && k && !w_rows) || (n_rows && tokens && !p))
+        return ORC_ERR_ARGS;
+    if (n_threads < 1)
+        n_threads = 1;
+    if (n_threads > n_rows)
+        n_threads = n_rows > 0 ? (int)n_rows : 1;
+    partial_job *jobs = calloc((size_t)n_threads, sizeof *jobs);
+    pthread_t *th = calloc((size_t)n_threads, sizeof *th);
+    if (!jobs || !th) {
+        free(jobs);
+        free(th);
+        return ORC_ERR_ALLOC;
+    }
+    for (int t = 0; t < n_threads; ++t) {
+        partial_job *j = &jobs[t];
+        j->n_ranks = n_ranks;
+        j->tokens = tokens;
+        j->k = k;
+        j->n_rows = n_rows;
+        j->row_begin = n_rows * t / n_threads;
+        j->row_end = n_rows * (t + 1) / n_threads;
+        j->x = x;
+        j->w_rows = w_rows;
+        j->p = p;
+        j->p64 = p64;
+        j->pabs = pabs;
+    }
+    int started = 0;
+    for (int t = 1; t < n_threads; ++t) {
+        if (pthread_create(&th[t], NULL, partial_thread, &jobs[t]) != 0)
+            break;
+        started = t;
+    }
+    partial_rows(&jobs[0]);
+    for (int t = 1; t <= started; ++t)
+        pthread_join(th[t], NULL);
+    for (int t = started + 1; t < n_threads; ++t) /* threads that failed to start */
+        partial_rows(&jobs[t]);
+    free(jobs);
+    free(th);
+    return ORC_OK;
+}
+
+/* ---------------------------------------------------------------- ring -- */
+
+/* Ring all-reduce of the partials, simulated message by message.
+ *   hidden    H, the full hidden size (chunks are H/N wide)
+ *   cols      [n_cols] the global column h of each stored column; the ring
+ *             runs on whatever subset of columns is given, each column in
+ *             the chunk h / (H/N) it belongs to
+ *   p         [n_ranks][tokens][n_cols] bf16 partials
+ *   reduced   [tokens][n_cols] bf16 all-reduced sum (out)
+ *   bytes_sent [n_ranks] bytes each rank put on its wire (out, may be NULL);
+ *             every message is a whole chunk of tokens * H/N bf16 values
+ * Returns ORC_ERR_RING if the ranks do not end with identical buffers. */
+int orc_ring(int n_ranks, int64_t tokens, int64_t hidden, int64_t n_cols,
+             const int64_t *cols, const uint16_t *p, uint16_t *reduced,
+             uint64_t *bytes_sent)
+{
+    if (n_ranks < 1 || tokens < 0 || hidden < 0 || n_cols < 0 || hidden % n_ranks != 0)
+        return ORC_ERR_ARGS;
+    const int N = n_ranks;
+    const int64_t hc = hidden / N;
+    const int64_t plane = tokens * n_cols;
+    for (int64_t i = 0; i < n_cols; ++i)
+        if (cols[i] < 0 || cols[i] >= hidden)
+            return ORC_ERR_ARGS;
+    if (bytes_sent)
+        for (int r = 0; r < N; ++r)
+            bytes_sent[r] = 0;
+    if (plane == 0)
+        return ORC_OK;
+
+    uint16_t *buf = malloc((size_t)N * (size_t)plane * sizeof *buf);  /* buf[r] */
+    uint16_t *msg = malloc((size_t)N * (size_t)plane * sizeof *msg);  /* in flight */
+    int *chunk_of = malloc((size_t)n_cols * sizeof *chunk_of);
+    if (!buf || !msg || !chunk_of) {
+        free(buf);
+        free(msg);
+        free(chunk_of);
+        return ORC_ERR_ALLOC;
+    }
+    memcpy(buf, p, (size_t)N * (size_t)plane * sizeof *buf);
+    for (int64_t i = 0; i < n_cols; ++i)
+        chunk_of[i] = (int)(cols[i] / hc);
+    const uint64_t chunk_bytes = (uint64_t)tokens * (uint64_t)hc * 2u;
+
+    /* Reduce-scatter: N-1 steps. All ranks send at once, then all receive. */
+    for (int s = 0; s < N - 1; ++s) {
+        for (int r = 0; r < N; ++r) {
+            int c = ((r - s) % N + N) % N;
+            for (int64_t m = 0; m < tokens; ++m)
+                for (int64_t i = 0; i < n_cols; ++i)
+                    if (chunk_of[i] == c)
+                        msg[(int64_t)r * plane + m * n_cols + i] =
+                            buf[(int64_t)r * plane + m * n_cols + i];
+            if (bytes_sent)
+                bytes_sent[r] += chunk_bytes;
+        }
+        for (int r = 0; r < N; ++r) {
+            int src = (r - 1 + N) % N;
+            int c = ((src - s) % N + N) % N;
+            for (int64_t m = 0; m < tokens; ++m)
+                for (int64_t i = 0; i < n_cols; ++i)
+                    if (chunk_of[i] == c) {
+                        int64_t o = m * n_cols + i;
+                        float recv = orc_f32(msg[(int64_t)src * plane + o]);
+                        float own = orc_f32(buf[(int64_t)r * plane + o]);
+                        buf[(int64_t)r * plane + o] = orc_bf16_rne(recv + own);
+                    }
+        }
+    }
+    /* All-gather: rank r now holds the reduced chunk (r + 1) mod N; N-1 steps
+     * pass the reduced chunks around the ring. */
+    for (int s = 0; s < N - 1; ++s) {
+        for (int r = 0; r < N; ++r) {
+            int c = ((r + 1 - s) % N + N) % N;
+            for (int64_t m = 0; m < tokens; ++m)
+                for (int64_t i = 0; i < n_cols; ++i)
+                    if (chunk_of[i] == c)
+                        msg[(int64_t)r * plane + m * n_cols + i] =
+                            buf[(int64_t)r * plane + m * n_cols + i];
+            if (bytes_sent)
+                bytes_sent[r] += chunk_bytes;
+        }
+        for (int r = 0; r < N; ++r) {
+            int src = (r - 1 + N) % N;
+            int c = ((src + 1 - s) % N + N) % N;
+            for (int64_t m = 0; m < tokens; ++m)
+                for (int64_t i = 0; i < n_cols; ++i)
+                    if (chunk_of[i] == c) {
+                        int64_t o = m * n_cols + i;
+                        buf[(int64_t)r * plane + o] = msg[(int64_t)src * plane + o];
+                    }
+        }
+    }
+    int rc = ORC_OK;
+    for (int r = 1; r < N; ++r)
+        if (memcmp(buf, buf + (int64_t)r * plane, (size_t)plane * sizeof *buf) != 0)
+            rc = ORC_ERR_RING;
+    memcpy(reduced, buf, (size_t)plane * sizeof *buf);
+    free(buf);
+    free(msg);
+    free(chunk_of);
+    return rc;
+}
+
+/* ------------------------------------------------------------ residual -- */
+
+void orc_residual(int64_t count, const uint16_t *residual, const uint16_t *reduced,
+                  uint16_t *out)
+{
+    for (int64_t i = 0; i < count; ++i)
+        out[i] = orc_bf16_rne(orc_f32(residual[i]) + orc_f32(reduced[i]));
+}
+
+/* ---------------------------------------------------------- whole point -- */
+
+/* One reconciliation point on the selected output columns.
+ *   x         [tokens][k]
+ *   w_rows    [n_cols][k]   rows cols[i] of the Linear weight W[H][K]
+ *   residual  [tokens][n_cols]  the residual at those columns
+ *   out       [tokens][n_cols]
+ *   partials  [n_ranks][tokens][n_cols] (out, may be NULL)
+ *   p64, pabs same shape (out, may be NULL)
+ *   bytes_sent [n_ranks] (out, may be NULL) */
+int orc_reconcile(int n_ranks, int64_t tokens, int64_t k, int64_t hidden, const uint16_t *x,
+                  int64_t n_cols, const int64_t *cols, const uint16_t *w_rows,
+                  const uint16_t *residual, uint16_t *out, uint16_t *partials, double *p64,
+                  double *pabs, uint64_t *bytes_sent, int n_threads)
+{
+    if (n_ranks < 1 || hidden % n_ranks != 0 || k % n_ranks != 0)
+        return ORC_ERR_ARGS;
+    const int64_t plane = tokens * n_cols;
+    uint16_t *p = partials;
+    uint16_t *red = malloc((size_t)(plane > 0 ? plane : 1) * sizeof *red);
+    if (!p)
+        p = malloc((size_t)(n_ranks * plane > 0 ? n_ranks * plane : 1) * sizeof *p);
+    if (!p || !red) {
+        if (!partials)
+            free(p);
+        free(red);
+        return ORC_ERR_ALLOC;
+    }
+    int rc = orc_partials(n_ranks, tokens, k, x, n_cols, w_rows, p, p64, pabs, n_threads);
+    if (rc == ORC_OK)
+        rc = orc_ring(n_ranks, tokens, hidden, n_cols, cols, p, red, bytes_sent);
+    if (rc == ORC_OK)
+        orc_residual(plane, residual, red, out);
+    if (!partials)
+        free(p);
+    free(red);
+    return rc;
+}
+
+/* ----------------------------------------------------------- byte model -- */
+
+/* Bytes one rank puts on its wire for a ring all-reduce of `points`
+ * reconciliations of tokens x hidden values of elem_bytes each:
+ * 2(N-1)/N times the payload (multiplied out before the one division). */
+uint64_t orc_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,
+                        int64_t points)
+{
+    if (n_ranks < 1 || tokens < 0 || hidden < 0 || elem_bytes < 0 || points < 0)
+        return 0;
+    uint64_t payload = (uint64_t)tokens * (uint64_t)hidden * (uint64_t)elem_bytes;
+    return 2u * (uint64_t)(n_ranks - 1) * payload * (uint64_t)points / (uint64_t)n_ranks;
+}
+
+/* ------------------------------------------------------- array helpers -- */
+
+void orc_bf16_rne_array(int64_t count, const float *in, uint16_t *out)
+{
+    for (int64_t i = 0; i < count; ++i)
+        out[i] = orc_bf16_rne(in[i]);
+}
+
+void orc_bf16_rne_f64_array(int64_t count, const double *in, uint16_t *out)
+{
+    for (int64_t i = 0; i < count; ++i)
+        out[i] = orc_bf16_rne_f64(in[i]);
+}

@@ -1,0 +1,97 @@
+"""Shared test helpers: bf16 bit views, exact rational rounding, golden files."""
+
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor -> numpy uint16 bit patterns (CPU copy)."""
+    assert t.dtype == torch.bfloat16
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def from_u16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+
+def bf16_value(b: int) -> Fraction:
+    """Exact rational value of a finite bf16 bit pattern."""
+    b = int(b) & 0xFFFF
+    sign = -1 if b & 0x8000 else 1
+    e = (b >> 7) & 0xFF
+    m = b & 0x7F
+    assert e != 0xFF, "not finite"
+    if e == 0:
+        return sign * Fraction(m, 1 << 7) * Fraction(1, 1 << 126)
+    return sign * (1 + Fraction(m, 1 << 7)) * Fraction(2) ** (e - 127)
+
+
+def round_bf16_exact(v: Fraction) -> int:
+    """Correct round-to-nearest-even of an exact rational to a bf16 pattern.
+
+    Written from the IEEE 754 definition: pick the representable value nearest
+    to v (8 significant bits, exponent -126..127, subnormal quantum 2^-133),
+    ties to the even significand, overflow to infinity when |v| reaches
+    (2 - 2^-8) * 2^127, the midpoint above the largest finite bf16.
+    """
+    sign = 0x8000 if v < 0 else 0
+    a = -v if v < 0 else v
+    if a == 0:
+        return sign
+    if a >= (2 - Fraction(1, 256)) * Fraction(2) ** 127:
+        return sign | 0x7F80
+    # exponent e with 2^e <= a < 2^(e+1)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    q = max(e - 7, -133)                     # quantum of the binade (or subnormal)
+    scaled = a / Fraction(2) ** q
+    n = math.floor(scaled)
+    rem = scaled - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    val = n * Fraction(2) ** q
+    if val >= Fraction(2) ** 128:
+        return sign | 0x7F80
+    # encode
+    if val < Fraction(2) ** -126:
+        mant = int(val / Fraction(2) ** -133)
+        return sign | mant
+    e2 = val.numerator.bit_length() - val.denominator.bit_length()
+    if Fraction(2) ** e2 > val:
+        e2 -= 1
+    mant = int((val / Fraction(2) ** e2 - 1) * 128)
+    return sign | ((e2 + 127) << 7) | mant
+
+
+def bf16_finite_patterns():
+    """All finite bf16 patterns as numpy uint16."""
+    a = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    return a[(a & 0x7F80) != 0x7F80]
+
+
+def round_bf16_float(v) -> int:
+    """Correct rounding of a finite float (float32 or float64) to bf16, with the
+    sign of zero kept (an exact rational has no signed zero)."""
+    v = float(v)
+    if v == 0.0:
+        return 0x8000 if math.copysign(1.0, v) < 0 else 0
+    return round_bf16_exact(Fraction(v))

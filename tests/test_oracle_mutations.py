@@ -1,0 +1,96 @@
+"""The pins catch plausible mistakes in the oracle.
+
+Each case compiles a copy of the oracle's C source with one planted mistake
+(on the CPU, in a temporary directory), loads it in place of the real library
+for the duration of the case, and checks that at least one of the named pins
+fails. The real oracle is restored afterwards.
+"""
+
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+
+import test_oracle_bf16 as tb
+import test_oracle_reconcile as trc
+import test_oracle_ring as trg
+
+SRC = open(obuild.SRC).read()
+
+
+def _integer_exact():
+    trc.test_integer_exact(4, 2, 256, 32)
+    trc.test_integer_exact(2, 3, 64, 16)
+
+MUTATIONS = {
+    # rounding: half-up instead of half-to-even
+    "round_half_up": ("u += 0x7FFFu + ((u >> 16) & 1u);", "u += 0x8000u;",
+                      [tb.test_bf16_rne_matches_exact_rounding_on_edges]),
+    # rounding: truncation
+    "round_truncate": ("u += 0x7FFFu + ((u >> 16) & 1u);", "u += 0u;",
+                       [tb.test_bf16_rne_matches_torch_conversion]),
+    # ring: chunks travel the other way round the ring
+    "ring_direction": ("int src = (r - 1 + N) % N;\n            int c = ((src - s) % N + N) % N;",
+                       "int src = (r + 1) % N;\n            int c = ((src - s) % N + N) % N;",
+                       [trg.test_ring_fold_order_golden]),
+    # ring: chunk c starts one rank late
+    "ring_start": ("int c = ((r - s) % N + N) % N;", "int c = ((r - s + 1) % N + N) % N;",
+                   [trg.test_ring_fold_order_golden]),
+    # partials: accumulate in double (not the fp32 reading)
+    "acc_double": ("float acc = 0.0f;", "double acc = 0.0;",
+                   [trc.test_partial_order_fp32_ascending]),
+    # partials: subtract instead of add
+    "acc_sign": ("acc = acc + prod;", "acc = acc - prod;",
+                 [_integer_exact]),
+    # partials: a rank reads the wrong slice of x
+    "x_slice": ("const uint16_t *xr = j->x + m * j->k + (int64_t)r * ks;",
+                "const uint16_t *xr = j->x + m * j->k;",
+                [_integer_exact]),
+    # residual dropped
+    "no_residual": ("out[i] = orc_bf16_rne(orc_f32(residual[i]) + orc_f32(reduced[i]));",
+                    "out[i] = reduced[i];",
+                    [_integer_exact]),
+    # byte model: N in place of N-1
+    "bytes_n": ("return 2u * (uint64_t)(n_ranks - 1) * payload",
+                "return 2u * (uint64_t)(n_ranks) * payload",
+                [trg.test_ring_bytes_pages_worked_example]),
+}
+
+
+def _build_mutant(name, old, new):
+    assert SRC.count(old) >= 1, f"mutation {name}: pattern not found"
+    d = tempfile.mkdtemp(prefix="orc_mut_")
+    src = os.path.join(d, "m.c")
+    lib = os.path.join(d, "libm.so")
+    with open(src, "w") as f:
+        f.write(SRC.replace(old, new))
+    subprocess.run(["gcc", *[c for c in obuild.CFLAGS if c != "-Werror"], src, "-o", lib, "-lm"],
+                   check=True)
+    return lib
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pin_catches_mutation(name, monkeypatch):
+    old, new, pins = MUTATIONS[name]
+    path = _build_mutant(name, old, new)
+    real = oracle.lib()
+    mutant = ctypes.CDLL(path)
+    for fn in ("orc_bf16_rne", "orc_bf16_rne_f64", "orc_f32", "orc_bf16_rne_array",
+               "orc_bf16_rne_f64_array", "orc_partials", "orc_ring", "orc_residual",
+               "orc_reconcile", "orc_ring_bytes"):
+        f = getattr(mutant, fn)
+        g = getattr(real, fn)
+        f.argtypes, f.restype = g.argtypes, g.restype
+    monkeypatch.setattr(oracle, "_lib", mutant)
+    caught = 0
+    for pin in pins:
+        try:
+            pin()
+        except (AssertionError, oracle.OracleError):
+            caught += 1
+    assert caught, f"no pin caught mutation {name}"
