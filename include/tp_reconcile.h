@@ -1,0 +1,166 @@
+/*
+ * tp_reconcile.h -- C ABI of the tensor-parallel reconciliation point on one
+ * B200 (sm_100a).
+ *
+ * The operation ("Interconnects e clusters", section 01 Conceito; NVL72 hosting
+ * post, All-reduce section): a row-parallel projection -- the attention
+ * out-projection or the FFN down-projection -- has its weight split across N
+ * tensor-parallel ranks along the input dimension K. Rank r owns the slice
+ * W_r = W[:, r*K/N : (r+1)*K/N] and computes the partial hidden vector
+ * P_r = x_r . W_r^T over its slice of the input x. The N partials are summed
+ * by a ring all-reduce -- a reduce-scatter in which each rank reduces one of
+ * N chunks of H/N hidden columns, then an all-gather of the reduced chunks --
+ * and the sum is added to the residual stream. Here all N ranks live in one
+ * GPU's memory: the ring is its summation order, carried out on the device.
+ *
+ * Arithmetic of the product (identical bit for bit to the oracle's reading of
+ * the pages):
+ *   P[r][m][h] = bf16_rne( sum_k x[m][r*Ks+k] * Wr[h][k] )   fp32 accumulate
+ *   chunk c = h / (H/N) is folded P_c, P_c+1, ..., P_c-1 (indices mod N), each
+ *   add being bf16_rne(f32(s) + f32(P)), then
+ *   out[m][h] = bf16_rne( f32(residual[m][h]) + f32(s) ).
+ * TP_VARIANT_EXACT accumulates each partial with fused multiply-adds in
+ * ascending k; TP_VARIANT_TENSOR accumulates on the tensor cores in fp32 in
+ * the hardware's order (see tp_plan_set_variant).
+ *
+ * Conventions for every function below:
+ *  - Element type: bf16 only (dtype argument TP_BF16). Tensors are dense and
+ *    row-major as stated per argument.
+ *  - Device pointers: every tensor argument is a CUDA device pointer on the
+ *    plan's device, 16-byte aligned; the caller allocates and owns it. The
+ *    library never allocates device memory and never synchronises the stream
+ *    on the compute path: calls are asynchronous on `stream` (a cudaStream_t
+ *    passed as void*; NULL means the legacy default stream).
+ *  - Errors: arguments are checked before anything is launched; a failed
+ *    check returns its status and launches nothing. A CUDA launch error maps
+ *    to TP_ERR_CUDA (tp_last_cuda_error gives the CUDA code).
+ *  - Threads: a plan is immutable after its set-up calls; concurrent calls
+ *    with one plan are safe as long as they use distinct output and
+ *    workspace buffers.
+ */
+#ifndef TP_RECONCILE_H
+#define TP_RECONCILE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tp_plan tp_plan; /* opaque, host side, owned by the caller */
+
+typedef enum {
+    TP_OK = 0,
+    TP_ERR_INVALID = 1,     /* bad shape, null pointer, aliasing, tokens > max */
+    TP_ERR_ALIGN = 2,       /* pointer not 16-byte aligned */
+    TP_ERR_UNSUPPORTED = 3, /* shape or variant this build has no kernel for */
+    TP_ERR_WORKSPACE = 4,   /* workspace missing or too small */
+    TP_ERR_CUDA = 5         /* CUDA runtime error (see tp_last_cuda_error) */
+} tp_status;
+
+enum { TP_BF16 = 0 };
+
+typedef enum {
+    TP_VARIANT_AUTO = 0,   /* EXACT for few tokens, TENSOR where built and faster */
+    TP_VARIANT_EXACT = 1,  /* CUDA cores, fp32 FMA chain per partial, k ascending */
+    TP_VARIANT_TENSOR = 2  /* tcgen05 tensor cores, fp32 accumulate in TMEM */
+} tp_variant;
+
+/* Creates a plan for one projection shape.
+ *   n_ranks     N, 1..8 tensor-parallel ranks
+ *   max_tokens  largest M any call will pass (>= 0)
+ *   k           projection input width K; K % N == 0 and (K/N) % 8 == 0
+ *   hidden      H; H % N == 0 and (H/N) % 8 == 0
+ *   dtype       TP_BF16
+ * Records the current CUDA device; every later call must run with that
+ * device current. On success *out owns a plan to release with
+ * tp_plan_destroy. Returns TP_ERR_INVALID on a bad shape or null out,
+ * TP_ERR_UNSUPPORTED for another dtype, TP_ERR_CUDA if no device is usable. */
+tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t k,
+                         int64_t hidden, int dtype);
+
+/* Chooses the partial kernel and whether the partials are staged.
+ *   variant  a tp_variant
+ *   staged   0: the partials stay on chip and one kernel does partials, ring
+ *            fold and residual add (no workspace); 1: the partial kernel
+ *            writes all N partials to the workspace and a separate ring
+ *            kernel (tp_ring_reduce's) folds them.
+ * Call before the plan is shared between threads. */
+tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
+
+/* Bytes of workspace tp_rowlinear_reconcile needs for `tokens` tokens with
+ * the plan's current setting: N*M*H*2 rounded up to 256 when staged, else 0.
+ * Returns 0 for a null plan. */
+size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
+
+/* S0, once per weight. Packs a torch Linear weight into the sharded layout.
+ *   w_hk      [H][K] bf16, the Linear weight (input)
+ *   w_packed  [N][H][K/N] bf16 (output): shard r is columns r*K/N ..
+ *             (r+1)*K/N-1 of w_hk, rank-major, K/N innermost, so each rank's
+ *             slice W_r is one contiguous block as on its own GPU
+ * ("Interconnects e clusters", 01 Conceito: each weight matrix is divided
+ * between the ranks.) The buffers must not overlap. */
+tp_status tp_pack_weights(const tp_plan* plan, const void* w_hk, void* w_packed, void* stream);
+
+/* S1-S4: one reconciliation point.
+ *   x          [M][K] bf16 activations (rank r reads columns r*K/N ..)
+ *   w_packed   [N][H][K/N] bf16 from tp_pack_weights
+ *   residual   [M][H] bf16
+ *   out        [M][H] bf16 (output); must not overlap any input or the workspace
+ *   tokens     M, 0 <= M <= max_tokens (M = 0 launches nothing)
+ *   workspace  tp_plan_workspace_bytes(plan, M) bytes of device memory, or
+ *              NULL when that is 0; contents on entry are ignored
+ * Partials per the header comment, summed in ring order, then the residual
+ * add ("Interconnects e clusters", 01 Conceito: the slices are summed before
+ * the residual stream continues). */
+tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void* w_packed,
+                                 const void* residual, void* out, int64_t tokens,
+                                 void* workspace, void* stream);
+
+/* S1 only: the N partials, no ring, no residual.
+ *   partials  [N][M][H] bf16 (output)
+ * Same x, w_packed and tokens rules as tp_rowlinear_reconcile. */
+tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* w_packed,
+                                void* partials, int64_t tokens, void* stream);
+
+/* S2-S4 only: ring reduce-scatter fold in ring order, the all-gather (one
+ * result buffer stands for every rank's copy) and the residual add.
+ *   partials  [N][M][H] bf16
+ *   residual  [M][H] bf16
+ *   out       [M][H] bf16 (output, must not overlap the inputs)
+ * (NVL72 hosting post, All-reduce section: each peer reduces one of N slices
+ * of the input, then broadcasts it to the rest.) */
+tp_status tp_ring_reduce(const tp_plan* plan, const void* partials, const void* residual,
+                         void* out, int64_t tokens, void* stream);
+
+/* S5: bytes each rank puts on its wire for `points` ring all-reduces of
+ * tokens x hidden elements of elem_bytes each: 2(N-1)/N times the payload
+ * ("Interconnects e clusters", 01 Conceito: 1.25 MiB per token at N=2 and
+ * about 1.875 MiB at N=4 for H=5120 bf16 and 128 reconciliations per token).
+ * Host only, exact (multiplies before the one division). Returns 0 for
+ * n_ranks < 1 or a negative argument. */
+uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,
+                       int64_t points);
+
+/* Releases a plan. NULL is allowed. */
+void tp_plan_destroy(tp_plan* plan);
+
+/* Static, NUL-terminated text for a status value. */
+const char* tp_status_string(tp_status status);
+
+/* The CUDA error code behind the calling thread's last TP_ERR_CUDA
+ * (0 if none). */
+int tp_last_cuda_error(void);
+
+/* Reads, and with reset != 0 clears, the device-side error word of the
+ * plan's device: bit 0 is set when a kernel's bounded wait on a pipeline
+ * barrier ran out (the kernel then stops early, so its output is invalid).
+ * Synchronises the device. */
+tp_status tp_device_error_flags(const tp_plan* plan, uint32_t* flags, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TP_RECONCILE_H */

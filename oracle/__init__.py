@@ -13,8 +13,8 @@ Functions and the passages they follow:
 * ``partials``  -- each rank's partial x_r . W_r over its K/N slice
   ("Interconnects e clusters", 01 Conceito: each weight matrix is split between
   ranks and each rank computes a partial result over its slice; bf16 on the
-  wire). fp32 accumulation, k ascending, one rounding to bf16 (reading of an
-  unstated step).
+  wire). fp32 accumulation by fused multiply-add, k ascending, one rounding
+  to bf16 (reading of an unstated step).
 * ``ring``      -- ring all-reduce simulated message by message: reduce-scatter
   of H/N chunks then all-gather ("Interconnects e clusters", 01 Conceito: a ring
   all-reduce puts 2(N-1)/N times the payload on each rank's wire; NVL72 hosting

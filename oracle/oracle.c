@@ -12,9 +12,11 @@
  *      input; rank r's partial hidden vector is x_r . W_r (the weight matrix
  *      is split between ranks, each rank computes a partial result over its
  *      slice). Reading of an unstated step: the products are accumulated in
- *      fp32, k ascending, starting from +0, each product rounded to fp32 and
- *      then added (round-to-nearest-even, no fusion), and the sum is rounded
- *      once to bf16 for the wire.
+ *      fp32, k ascending, starting from +0, each product added to the running
+ *      sum with one rounding (fused multiply-add, round-to-nearest-even; the
+ *      product of two bf16 values is exact in fp32 unless it underflows, so
+ *      this is also "round the product, then add" everywhere else), and the
+ *      sum is rounded once to bf16 for the wire.
  *   2. Ring all-reduce. The partials are summed before the residual stream
  *      continues, by a ring all-reduce that puts 2(N-1)/N times the payload on
  *      each rank's wire: a reduce-scatter in which each rank reduces one of N
@@ -26,9 +28,9 @@
  *      P_c-1, left to right.
  *   3. Residual. out = bf16_rne(f32(residual) + f32(reduced)).
  *
- * Build: plain C11, -ffp-contract=off (no fused multiply-add), no fast-math,
- * so every float operation is one IEEE round-to-nearest-even operation with
- * subnormals kept.
+ * Build: plain C11, -ffp-contract=off (no fused multiply-add other than the
+ * explicit fmaf), no fast-math, so every float operation is one IEEE
+ * round-to-nearest-even operation with subnormals kept.
  */
 #include <math.h>
 #include <pthread.h>
@@ -118,8 +120,7 @@ static void partial_rows(const partial_job *j)
                 float acc = 0.0f;
                 double d = 0.0, a = 0.0;
                 for (int64_t kk = 0; kk < ks; ++kk) {
-                    float prod = orc_f32(xr[kk]) * orc_f32(wr[kk]);
-                    acc = acc + prod;
+                    acc = fmaf(orc_f32(xr[kk]), orc_f32(wr[kk]), acc);
                     double dp = (double)orc_f32(xr[kk]) * (double)orc_f32(wr[kk]);
                     d += dp;
                     a += fabs(dp);

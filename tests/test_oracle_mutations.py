@@ -42,10 +42,17 @@ MUTATIONS = {
     "ring_start": ("int c = ((r - s) % N + N) % N;", "int c = ((r - s + 1) % N + N) % N;",
                    [trg.test_ring_fold_order_golden]),
     # partials: accumulate in double (not the fp32 reading)
-    "acc_double": ("float acc = 0.0f;", "double acc = 0.0;",
-                   [trc.test_partial_order_fp32_ascending]),
+    "acc_double": ([("float acc = 0.0f;", "double acc = 0.0;"),
+                    ("acc = fmaf(orc_f32(xr[kk]), orc_f32(wr[kk]), acc);",
+                     "acc = fma((double)orc_f32(xr[kk]), (double)orc_f32(wr[kk]), acc);")],
+                   None, [trc.test_partial_order_fp32_ascending]),
+    # partials: k descending
+    "k_descending": ("for (int64_t kk = 0; kk < ks; ++kk) {",
+                     "for (int64_t kk = ks - 1; kk >= 0; --kk) {",
+                     [trc.test_partial_order_fp32_ascending]),
     # partials: subtract instead of add
-    "acc_sign": ("acc = acc + prod;", "acc = acc - prod;",
+    "acc_sign": ("acc = fmaf(orc_f32(xr[kk]), orc_f32(wr[kk]), acc);",
+                 "acc = fmaf(-orc_f32(xr[kk]), orc_f32(wr[kk]), acc);",
                  [_integer_exact]),
     # partials: a rank reads the wrong slice of x
     "x_slice": ("const uint16_t *xr = j->x + m * j->k + (int64_t)r * ks;",
@@ -63,12 +70,16 @@ MUTATIONS = {
 
 
 def _build_mutant(name, old, new):
-    assert SRC.count(old) >= 1, f"mutation {name}: pattern not found"
+    edits = old if isinstance(old, list) else [(old, new)]
+    text = SRC
+    for o, n in edits:
+        assert text.count(o) >= 1, f"mutation {name}: pattern not found"
+        text = text.replace(o, n)
     d = tempfile.mkdtemp(prefix="orc_mut_")
     src = os.path.join(d, "m.c")
     lib = os.path.join(d, "libm.so")
     with open(src, "w") as f:
-        f.write(SRC.replace(old, new))
+        f.write(text)
     subprocess.run(["gcc", *[c for c in obuild.CFLAGS if c != "-Werror"], src, "-o", lib, "-lm"],
                    check=True)
     return lib
