@@ -1,0 +1,434 @@
+"""Benchmark of the reconciliation point on B200: one step = every point of a
+workload (all partials, ring folds and residual adds) over one batch.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                  [--variant auto|exact|tensor] [--staged] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0. With --gpus N > 1 it runs under
+torch.distributed.run, one process per GPU; every rank runs an independent
+replica of the step (the N tensor-parallel ranks of the method are emulated
+inside each GPU), so there is no data-path collective and the scaling is weak.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import KIND_RESIDUAL, KIND_W, KIND_X, get_config, point_tensor  # noqa: E402
+from workloads.configs import CONFIG_ORDER  # noqa: E402
+
+METRIC = "reconciliations/s & tokens/s on 1 B200; achieved HBM GB/s (TC util) vs peak"
+DEFAULT_CONFIG = "decode_n2"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------------ workload --
+
+class Workload:
+    """All points of one config resident on one GPU: packed weights, inputs, outputs.
+
+    x and the residual of all points live in two flat buffers (one host->device
+    copy each per end-to-end step); the outputs likewise (one copy back).
+    """
+
+    def __init__(self, cfg, device, variant="auto", staged=False):
+        import tensor_layer_reconciliation_b200 as tlr
+        self.cfg = cfg
+        self.device = device
+        m, h, n = cfg.tokens, cfg.hidden, cfg.n_ranks
+        self.plans = {}
+        for p in cfg.points:
+            if p.k not in self.plans:
+                self.plans[p.k] = tlr.Plan(n, m, p.k, h, variant=variant, staged=staged)
+        x_sizes = [m * p.k for p in cfg.points]
+        self.x_off = np.concatenate([[0], np.cumsum(x_sizes)]).astype(np.int64)
+        self.x_all = torch.empty(int(self.x_off[-1]), dtype=torch.bfloat16, device=device)
+        self.res_all = torch.empty(cfg.n_points * m * h, dtype=torch.bfloat16, device=device)
+        self.out_all = torch.empty(cfg.n_points * m * h, dtype=torch.bfloat16, device=device)
+        self.w_packed = []
+        ws_need = max(pl.workspace_bytes(m) for pl in self.plans.values())
+        self.workspace = (torch.empty(ws_need, dtype=torch.uint8, device=device)
+                          if ws_need else None)
+        for i, p in enumerate(cfg.points):
+            self.x(i).copy_(point_tensor(cfg, p, KIND_X, device))
+            self.res(i).copy_(point_tensor(cfg, p, KIND_RESIDUAL, device))
+            w = point_tensor(cfg, p, KIND_W, device)
+            self.w_packed.append(self.plans[p.k].pack_weights(w))
+            del w
+        torch.cuda.synchronize(device)
+
+    def x(self, i):
+        p = self.cfg.points[i]
+        return self.x_all[int(self.x_off[i]):int(self.x_off[i + 1])].view(self.cfg.tokens, p.k)
+
+    def res(self, i):
+        m, h = self.cfg.tokens, self.cfg.hidden
+        return self.res_all[i * m * h:(i + 1) * m * h].view(m, h)
+
+    def out(self, i):
+        m, h = self.cfg.tokens, self.cfg.hidden
+        return self.out_all[i * m * h:(i + 1) * m * h].view(m, h)
+
+    def step(self):
+        """One pass of the hot path over every point, on the current stream."""
+        for i, p in enumerate(self.cfg.points):
+            self.plans[p.k].reconcile(self.x(i), self.w_packed[i], self.res(i), out=self.out(i),
+                                      workspace=self.workspace)
+
+    def launches_per_step(self):
+        per = 2 if next(iter(self.plans.values())).staged else 1
+        return per * self.cfg.n_points
+
+    def capture(self):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            self.step()                      # warm the plans outside capture
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        torch.cuda.synchronize(self.device)
+        with torch.cuda.graph(g):
+            self.step()
+        return g
+
+
+# --------------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [s.strip() for s in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            if self.path:
+                try:
+                    os.unlink(self.path)
+                except OSError:
+                    pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------- oracle --
+
+def cpu_baseline(cfg, threads=None, target_s=12.0):
+    """The oracle as it stands on this host's cores, on a bounded sample.
+
+    Sample: the first point of each projection kind (all H columns, all M
+    tokens), repeated until about target_s seconds of oracle work; the step
+    time is extrapolated by the number of points of each kind.
+    """
+    import oracle
+    threads = threads or len(os.sched_getaffinity(0))
+    kinds = {}
+    for p in cfg.points:
+        kinds.setdefault(p.kind, []).append(p)
+    per_kind = {}
+    total_time, reps_done, desc = 0.0, 0, []
+    for kind, pts in kinds.items():
+        p = pts[0]
+        x = point_tensor(cfg, p, KIND_X).view(torch.int16).numpy().view(np.uint16)
+        w = point_tensor(cfg, p, KIND_W).view(torch.int16).numpy().view(np.uint16)
+        r = point_tensor(cfg, p, KIND_RESIDUAL).view(torch.int16).numpy().view(np.uint16)
+        rows = cfg.hidden
+        # bound one call to ~ target_s / number of kinds
+        t0 = time.perf_counter()
+        oracle.reconcile(cfg.n_ranks, cfg.hidden, x, np.ascontiguousarray(w[:64]),
+                         np.ascontiguousarray(r[:, :64]), cols=np.arange(64), threads=threads)
+        probe = (time.perf_counter() - t0) / 64
+        budget = target_s / len(kinds)
+        rows = int(max(64, min(cfg.hidden, budget / max(probe, 1e-9))))
+        cols = np.arange(rows)
+        t0 = time.perf_counter()
+        oracle.reconcile(cfg.n_ranks, cfg.hidden, x, np.ascontiguousarray(w[:rows]),
+                         np.ascontiguousarray(r[:, :rows]), cols=cols, threads=threads)
+        dt = time.perf_counter() - t0
+        per_point = dt * cfg.hidden / rows
+        per_kind[kind] = per_point
+        total_time += dt
+        reps_done += 1
+        desc.append(f"{kind} point {p.index} (K={p.k}): {rows} of {cfg.hidden} output columns")
+    step_s = sum(per_kind[p.kind] for p in cfg.points)
+    return {"step_s": step_s, "cores": threads, "sample": "; ".join(desc) +
+            f"; step time extrapolated over {cfg.n_points} points ({total_time:.1f} s measured)"}
+
+
+# --------------------------------------------------------------------- main --
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _max_over_ranks(v, world, device):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args, world, rank):
+    """The oracle (the reference arm of this build) timed on the host cores."""
+    if rank != 0:
+        return 0
+    cfg = get_config(args.config)
+    for _ in range(args.warmup):
+        cpu_baseline(cfg, target_s=1.0)
+    times = []
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(cfg, target_s=args.ref_seconds)
+        times.append(last["step_s"])
+    step_s = float(np.mean(times))
+    tok = cfg.tokens / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32-accumulate bf16", "data": "synthetic (seeded Philox)",
+        "reconciliations_per_s": cfg.n_points / step_s,
+        "config": {"workload": cfg.name, "n_ranks": cfg.n_ranks, "tokens": cfg.tokens,
+                   "hidden": cfg.hidden, "points": cfg.n_points},
+        "cpu_baseline": {"value": tok, "unit": "tokens/s", "cores": last["cores"],
+                         "kind": "oracle", "sample": last["sample"]},
+        "e2e": {"value": tok, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=CONFIG_ORDER)
+    ap.add_argument("--variant", default="auto", choices=["auto", "exact", "tensor"])
+    ap.add_argument("--staged", action="store_true")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=8.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world, rank, local = _dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    cfg = get_config(args.config)
+    wl = Workload(cfg, device, variant=args.variant, staged=args.staged)
+    peaks = _peaks()
+
+    graph = wl.capture()
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(device)
+
+    # ---- timed region: K graph replays, device-timed, max over ranks ------
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        _barrier(world)
+        torch.cuda.synchronize(device)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize(device)
+        _barrier(world)
+    step_ms = ev0.elapsed_time(ev1) / args.steps
+    step_ms = _max_over_ranks(step_ms, world, device)
+    clocks = clk.summary()
+
+    # ---- per-launch durations of the dominant kernel (events around each call)
+    per_launch = []
+    for _ in range(2):
+        evs = []
+        for i, p in enumerate(cfg.points):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            wl.plans[p.k].reconcile(wl.x(i), wl.w_packed[i], wl.res(i), out=wl.out(i),
+                                    workspace=wl.workspace)
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize(device)
+        per_launch.append([a.elapsed_time(b) for a, b in evs])
+    call_ms = np.mean(np.array(per_launch), axis=0)      # per point, ms
+
+    # ---- end to end through the public API with host buffers -------------
+    x_host = torch.empty(wl.x_all.shape, dtype=torch.bfloat16, pin_memory=True)
+    r_host = torch.empty(wl.res_all.shape, dtype=torch.bfloat16, pin_memory=True)
+    o_host = torch.empty(wl.out_all.shape, dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(wl.x_all.cpu())
+    r_host.copy_(wl.res_all.cpu())
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        wl.x_all.copy_(x_host, non_blocking=True)
+        wl.res_all.copy_(r_host, non_blocking=True)
+        graph.replay()
+        o_host.copy_(wl.out_all, non_blocking=True)
+    torch.cuda.synchronize(device)
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        wl.x_all.copy_(x_host, non_blocking=True)
+        wl.res_all.copy_(r_host, non_blocking=True)
+        graph.replay()
+        o_host.copy_(wl.out_all, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, device)
+    h2d = (wl.x_all.numel() + wl.res_all.numel()) * 2
+    d2h = wl.out_all.numel() * 2
+
+    # ---- numbers ---------------------------------------------------------
+    staged = args.staged
+    tokens_per_step = cfg.tokens * world
+    value = tokens_per_step / (step_ms * 1e-3)
+    recon = cfg.n_points * world / (step_ms * 1e-3)
+    alg_bytes = cfg.algorithmic_bytes(staged_partials=staged)
+    flops = cfg.flops()
+    tensor_bound = cfg.tokens >= 1024
+    kernel_ms = float(np.sum(call_ms))
+    if tensor_bound:
+        achieved = flops / (kernel_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None}
+    else:
+        achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None}
+    roof["peak_source"] = peaks["source"]
+    roof["kernel"] = "exact_partial_kernel (fused partials + ring fold + residual)" if not staged \
+        else "exact_partial_kernel + ring_reduce_kernel"
+    roof["launch_ms_mean"] = kernel_ms / cfg.n_points
+    roof["algorithmic_bytes_per_step"] = alg_bytes
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Philox4x32-10, Gaussian by 2^16-point inverse CDF)",
+        "reconciliations_per_s": recon,
+        "hbm_gbs_step": alg_bytes * world / (step_ms * 1e-3) / 1e9 / world,
+        "config": {"workload": cfg.name, "n_ranks": cfg.n_ranks, "tokens": cfg.tokens,
+                   "hidden": cfg.hidden, "points": cfg.n_points,
+                   "weights_gb_per_step": cfg.weight_bytes() / 1e9,
+                   "l2": "no flush: every step streams all points' distinct weights "
+                         f"({cfg.weight_bytes() / 1e9:.1f} GB), larger than the 126 MB L2",
+                   "variant": args.variant, "staged": staged,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "e2e": {"value": tokens_per_step / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": wl.launches_per_step() * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(cfg)
+        line["cpu_baseline"] = {"value": cfg.tokens / cb["step_s"], "unit": "tokens/s",
+                                "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"]}
+    del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

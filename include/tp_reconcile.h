@@ -44,6 +44,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define TP_API __attribute__((visibility("default")))
+#else
+#define TP_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -77,7 +83,7 @@ typedef enum {
  * device current. On success *out owns a plan to release with
  * tp_plan_destroy. Returns TP_ERR_INVALID on a bad shape or null out,
  * TP_ERR_UNSUPPORTED for another dtype, TP_ERR_CUDA if no device is usable. */
-tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t k,
+TP_API tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t k,
                          int64_t hidden, int dtype);
 
 /* Chooses the partial kernel and whether the partials are staged.
@@ -87,12 +93,12 @@ tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t
  *            writes all N partials to the workspace and a separate ring
  *            kernel (tp_ring_reduce's) folds them.
  * Call before the plan is shared between threads. */
-tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
+TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
 
 /* Bytes of workspace tp_rowlinear_reconcile needs for `tokens` tokens with
  * the plan's current setting: N*M*H*2 rounded up to 256 when staged, else 0.
  * Returns 0 for a null plan. */
-size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
+TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 
 /* S0, once per weight. Packs a torch Linear weight into the sharded layout.
  *   w_hk      [H][K] bf16, the Linear weight (input)
@@ -101,7 +107,7 @@ size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
  *             slice W_r is one contiguous block as on its own GPU
  * ("Interconnects e clusters", 01 Conceito: each weight matrix is divided
  * between the ranks.) The buffers must not overlap. */
-tp_status tp_pack_weights(const tp_plan* plan, const void* w_hk, void* w_packed, void* stream);
+TP_API tp_status tp_pack_weights(const tp_plan* plan, const void* w_hk, void* w_packed, void* stream);
 
 /* S1-S4: one reconciliation point.
  *   x          [M][K] bf16 activations (rank r reads columns r*K/N ..)
@@ -114,14 +120,14 @@ tp_status tp_pack_weights(const tp_plan* plan, const void* w_hk, void* w_packed,
  * Partials per the header comment, summed in ring order, then the residual
  * add ("Interconnects e clusters", 01 Conceito: the slices are summed before
  * the residual stream continues). */
-tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void* w_packed,
+TP_API tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void* w_packed,
                                  const void* residual, void* out, int64_t tokens,
                                  void* workspace, void* stream);
 
 /* S1 only: the N partials, no ring, no residual.
  *   partials  [N][M][H] bf16 (output)
  * Same x, w_packed and tokens rules as tp_rowlinear_reconcile. */
-tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* w_packed,
+TP_API tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* w_packed,
                                 void* partials, int64_t tokens, void* stream);
 
 /* S2-S4 only: ring reduce-scatter fold in ring order, the all-gather (one
@@ -131,7 +137,7 @@ tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* 
  *   out       [M][H] bf16 (output, must not overlap the inputs)
  * (NVL72 hosting post, All-reduce section: each peer reduces one of N slices
  * of the input, then broadcasts it to the rest.) */
-tp_status tp_ring_reduce(const tp_plan* plan, const void* partials, const void* residual,
+TP_API tp_status tp_ring_reduce(const tp_plan* plan, const void* partials, const void* residual,
                          void* out, int64_t tokens, void* stream);
 
 /* S5: bytes each rank puts on its wire for `points` ring all-reduces of
@@ -140,24 +146,24 @@ tp_status tp_ring_reduce(const tp_plan* plan, const void* partials, const void* 
  * about 1.875 MiB at N=4 for H=5120 bf16 and 128 reconciliations per token).
  * Host only, exact (multiplies before the one division). Returns 0 for
  * n_ranks < 1 or a negative argument. */
-uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,
+TP_API uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,
                        int64_t points);
 
 /* Releases a plan. NULL is allowed. */
-void tp_plan_destroy(tp_plan* plan);
+TP_API void tp_plan_destroy(tp_plan* plan);
 
 /* Static, NUL-terminated text for a status value. */
-const char* tp_status_string(tp_status status);
+TP_API const char* tp_status_string(tp_status status);
 
 /* The CUDA error code behind the calling thread's last TP_ERR_CUDA
  * (0 if none). */
-int tp_last_cuda_error(void);
+TP_API int tp_last_cuda_error(void);
 
 /* Reads, and with reset != 0 clears, the device-side error word of the
  * plan's device: bit 0 is set when a kernel's bounded wait on a pipeline
  * barrier ran out (the kernel then stops early, so its output is invalid).
  * Synchronises the device. */
-tp_status tp_device_error_flags(const tp_plan* plan, uint32_t* flags, int reset);
+TP_API tp_status tp_device_error_flags(const tp_plan* plan, uint32_t* flags, int reset);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,289 @@
+// Partial kernel on CUDA cores with the k-ascending fp32 FMA chain (S1),
+// optionally fused with the ring fold and the residual add (S2-S4).
+//
+// "Interconnects e clusters", 01 Conceito: each weight matrix is split
+// between ranks and each rank computes a partial result over its slice; the
+// slices are summed (all-reduce) before the residual stream continues.
+//
+// Work decomposition. A CTA owns BH output rows h0..h0+BH-1 for ALL N ranks
+// and MT tokens m0..m0+MT-1, so every partial an output element needs is
+// produced inside the CTA and the ring fold needs no second kernel.
+// Consumer thread t = r*BH + j runs the MT fp32 accumulation chains of
+// partial (rank r, row h0+j), one FMA per element in ascending k, so each
+// partial is exactly the k-ascending fp32 sum rounded once to bf16.
+//
+// Memory path. One producer thread streams 64-column k-blocks with 3-D TMA
+// bulk-tensor loads into a STAGES-deep shared-memory ring:
+//   W box {64 k, BH rows, N ranks} of w_packed [N][H][Ks], 128-byte swizzled
+//   x box {64 k, N ranks, MT tokens} of x viewed as [M][N][Ks]
+// Each stage has a "full" mbarrier (TMA transaction bytes) and an "empty"
+// mbarrier (one arrive per consumer warp). Weight loads for the first STAGES
+// blocks are issued before griddepcontrol.wait, so with programmatic
+// dependent launch they overlap the previous kernel's tail; activations,
+// the residual and the outputs are touched only after it.
+//
+// Shared-memory banks: a consumer reads 16-byte chunk c of its own 128-byte
+// row; with the 128-byte swizzle the physical chunk is c ^ (row & 7), so the
+// eight lanes of each quarter-warp hit eight different chunks.
+#pragma once
+
+#include "tp_common.cuh"
+
+namespace tpr {
+
+constexpr int kMaxStages = 16;
+constexpr int kKBlock = 64;  // bf16 columns per TMA box row (128 bytes)
+constexpr int kMaxExactChains = 512;                 // N * BH per CTA
+constexpr int kMaxExactThreads = kMaxExactChains + 32;  // + the producer warp
+
+struct ExactParams {
+    int n_ranks;     // N
+    int bh;          // output rows per CTA
+    int ks;          // K / N
+    int hidden;      // H
+    int hc;          // H / N
+    int tokens;      // M
+    int stages;      // pipeline depth, 2..kMaxStages
+    int fused;       // 1: fold + residual in-kernel; 0: write partials
+    uint32_t w_stage_bytes;  // stride of the W ring (multiple of 1024)
+    uint32_t x_stage_bytes;  // stride of the x ring (multiple of 128)
+    uint32_t w_box_bytes;    // 64 * bh * N * 2
+    uint32_t x_box_bytes;    // 64 * N * MT * 2
+    const uint16_t* residual;  // [M][H]
+    uint16_t* out;             // [M][H]           (fused)
+    uint16_t* partials;        // [N][M][H]        (not fused)
+};
+
+template <int MT>
+__global__ void __launch_bounds__(kMaxExactThreads, 1)
+    exact_partial_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                         const __grid_constant__ CUtensorMap tmap_x, const ExactParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // Align the dynamic shared-memory base to 1024 bytes (128-byte swizzle atom).
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int N = p.n_ranks, BH = p.bh, S = p.stages;
+    uint8_t* w_ring = smem;
+    uint8_t* x_ring = w_ring + static_cast<size_t>(S) * p.w_stage_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(x_ring + static_cast<size_t>(S) * p.x_stage_bytes);
+    uint64_t* empty = full + kMaxStages;
+    uint16_t* part = reinterpret_cast<uint16_t*>(empty + kMaxStages);  // [N][BH][MT]
+    __shared__ int abort_flag;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int consumer_warps = (blockDim.x >> 5) - 1;
+    const int n_consumers = consumer_warps * 32;
+    const int T = N * BH;  // chains-owning consumer threads
+    const int h0 = blockIdx.x * BH;
+    const int m0 = blockIdx.y * MT;
+    const int nkb = (p.ks + kKBlock - 1) / kKBlock;
+
+    if (tid == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], consumer_warps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+
+    if (warp == consumer_warps) {
+        // ------------------------------------------------------- producer --
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_w);
+            tma_prefetch_desc(&tmap_x);
+            const uint32_t tx = p.w_box_bytes + p.x_box_bytes;
+            const int pre = nkb < S ? nkb : S;
+            for (int kb = 0; kb < pre; ++kb) {
+                mbar_arrive_expect_tx(&full[kb], tx);
+                tma_load_3d(w_ring + static_cast<size_t>(kb) * p.w_stage_bytes, &tmap_w, &full[kb],
+                            kb * kKBlock, h0, 0);
+            }
+            pdl_wait();  // activations may be produced by the previous kernel
+            for (int kb = 0; kb < pre; ++kb)
+                tma_load_3d(x_ring + static_cast<size_t>(kb) * p.x_stage_bytes, &tmap_x, &full[kb],
+                            kb * kKBlock, 0, m0);
+            int issued = pre;
+            int s = 0;
+            uint32_t phase = 0;
+            for (int kb = pre; kb < nkb; ++kb) {
+                // stage kb % S, its (kb / S)-th reuse
+                s = kb % S;
+                phase = static_cast<uint32_t>(kb / S) & 1u;
+                if (!mbar_wait_bounded(&empty[s], phase ^ 1u)) {
+                    atomicExch(&abort_flag, 1);
+                    break;
+                }
+                if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
+                mbar_arrive_expect_tx(&full[s], tx);
+                tma_load_3d(w_ring + static_cast<size_t>(s) * p.w_stage_bytes, &tmap_w, &full[s],
+                            kb * kKBlock, h0, 0);
+                tma_load_3d(x_ring + static_cast<size_t>(s) * p.x_stage_bytes, &tmap_x, &full[s],
+                            kb * kKBlock, 0, m0);
+                issued = kb + 1;
+            }
+            // Never leave with bulk copies still landing in this CTA's memory:
+            // wait (bounded) for the last copies issued into every stage.
+            const int first = issued > S ? issued - S : 0;
+            for (int kb = first; kb < issued; ++kb)
+                if (!mbar_wait_bounded(&full[kb % S], static_cast<uint32_t>(kb / S) & 1u)) break;
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers --
+    const bool owner = tid < T;
+    const int r = owner ? tid / BH : 0;
+    const int row = tid;  // == r * BH + j: the thread's 128-byte row in a W box
+    float acc[MT];
+#pragma unroll
+    for (int i = 0; i < MT; ++i) acc[i] = 0.0f;
+
+    for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % S;
+        const uint32_t phase = static_cast<uint32_t>(kb / S) & 1u;
+        // Every lane waits (each needs the barrier's acquire); the warp then
+        // agrees, so a wait that ran out on one lane stops the whole warp.
+        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[s], phase));
+        if (!ok) {
+            atomicExch(&abort_flag, 1);
+            break;
+        }
+        if (owner) {
+            const uint8_t* wrow = w_ring + static_cast<size_t>(s) * p.w_stage_bytes + row * 128;
+            const uint8_t* xs = x_ring + static_cast<size_t>(s) * p.x_stage_bytes + r * 128;
+            const int rem = p.ks - kb * kKBlock;
+            const int nv = rem >= kKBlock ? 8 : rem >> 3;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                if (c < nv) {
+                    const uint4 wv = ld_shared_v4(wrow + ((c ^ (row & 7)) << 4));
+                    const float w0 = bf16_lo(wv.x), w1 = bf16_hi(wv.x);
+                    const float w2 = bf16_lo(wv.y), w3 = bf16_hi(wv.y);
+                    const float w4 = bf16_lo(wv.z), w5 = bf16_hi(wv.z);
+                    const float w6 = bf16_lo(wv.w), w7 = bf16_hi(wv.w);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const uint4 xv = ld_shared_v4(xs + mt * N * 128 + (c << 4));
+                        float a = acc[mt];
+                        a = __fmaf_rn(bf16_lo(xv.x), w0, a);
+                        a = __fmaf_rn(bf16_hi(xv.x), w1, a);
+                        a = __fmaf_rn(bf16_lo(xv.y), w2, a);
+                        a = __fmaf_rn(bf16_hi(xv.y), w3, a);
+                        a = __fmaf_rn(bf16_lo(xv.z), w4, a);
+                        a = __fmaf_rn(bf16_hi(xv.z), w5, a);
+                        a = __fmaf_rn(bf16_lo(xv.w), w6, a);
+                        a = __fmaf_rn(bf16_hi(xv.w), w7, a);
+                        acc[mt] = a;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+
+    // Every consumer thread reaches this barrier (no early return above).
+    asm volatile("bar.sync 1, %0;" ::"r"(n_consumers) : "memory");
+    if (*reinterpret_cast<volatile int*>(&abort_flag)) return;
+    pdl_wait();  // the residual and the outputs belong to the stream's order
+
+    const int j = tid - r * BH;
+    if (!p.fused) {
+        if (owner && h0 + j < p.hidden) {
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+                if (m0 + mt < p.tokens)
+                    p.partials[(static_cast<size_t>(r) * p.tokens + m0 + mt) * p.hidden + h0 + j] =
+                        f32_to_bf16_rne(acc[mt]);
+        }
+        return;
+    }
+
+    if (owner) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) part[(r * BH + j) * MT + mt] = f32_to_bf16_rne(acc[mt]);
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(n_consumers) : "memory");
+    // Ring fold: chunk c = h / (H/N) starts at rank c and adds ranks c+1, ...,
+    // c-1 (mod N) from the left; then the residual.
+    for (int o = tid; o < BH * MT; o += n_consumers) {
+        const int mt = o / BH, jj = o - mt * BH;
+        const int h = h0 + jj, m = m0 + mt;
+        if (h >= p.hidden || m >= p.tokens) continue;
+        const int c = h / p.hc;
+        uint16_t acc16 = part[(c * BH + jj) * MT + mt];
+        for (int i = 1; i < N; ++i) {
+            int rr = c + i;
+            if (rr >= N) rr -= N;
+            acc16 = bf16_add(acc16, part[(rr * BH + jj) * MT + mt]);
+        }
+        const size_t o_idx = static_cast<size_t>(m) * p.hidden + h;
+        p.out[o_idx] = bf16_add(p.residual[o_idx], acc16);
+    }
+}
+
+// ------------------------------------------------------------------ S2-S4 --
+// Ring reduce-scatter fold over partials staged in memory, the all-gather
+// (one result buffer stands for every rank's copy) and the residual add.
+// Thread per 8 consecutive columns (16-byte vectors; H/N % 8 == 0 keeps a
+// vector inside one chunk), grid-stride.
+__global__ void __launch_bounds__(256)
+    ring_reduce_kernel(const uint16_t* __restrict__ partials, const uint16_t* __restrict__ residual,
+                       uint16_t* __restrict__ out, int n_ranks, int64_t tokens, int hidden, int hc) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int64_t hv = hidden >> 3;
+    const int64_t total = tokens * hv;
+    const size_t plane = static_cast<size_t>(tokens) * hidden;
+    for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < total;
+         v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t m = v / hv;
+        const int h = static_cast<int>(v - m * hv) << 3;
+        const int c = h / hc;
+        const size_t off = static_cast<size_t>(m) * hidden + h;
+        uint4 a = ld_global_nc_v4(partials + static_cast<size_t>(c) * plane + off);
+        uint16_t s[8];
+        s[0] = a.x & 0xFFFF; s[1] = a.x >> 16; s[2] = a.y & 0xFFFF; s[3] = a.y >> 16;
+        s[4] = a.z & 0xFFFF; s[5] = a.z >> 16; s[6] = a.w & 0xFFFF; s[7] = a.w >> 16;
+        for (int i = 1; i < n_ranks; ++i) {
+            int rr = c + i;
+            if (rr >= n_ranks) rr -= n_ranks;
+            const uint4 b = ld_global_nc_v4(partials + static_cast<size_t>(rr) * plane + off);
+            s[0] = bf16_add(s[0], b.x & 0xFFFF); s[1] = bf16_add(s[1], b.x >> 16);
+            s[2] = bf16_add(s[2], b.y & 0xFFFF); s[3] = bf16_add(s[3], b.y >> 16);
+            s[4] = bf16_add(s[4], b.z & 0xFFFF); s[5] = bf16_add(s[5], b.z >> 16);
+            s[6] = bf16_add(s[6], b.w & 0xFFFF); s[7] = bf16_add(s[7], b.w >> 16);
+        }
+        const uint4 rv = ld_global_nc_v4(residual + off);
+        uint4 o;
+        o.x = bf16_add(rv.x & 0xFFFF, s[0]) | (static_cast<uint32_t>(bf16_add(rv.x >> 16, s[1])) << 16);
+        o.y = bf16_add(rv.y & 0xFFFF, s[2]) | (static_cast<uint32_t>(bf16_add(rv.y >> 16, s[3])) << 16);
+        o.z = bf16_add(rv.z & 0xFFFF, s[4]) | (static_cast<uint32_t>(bf16_add(rv.z >> 16, s[5])) << 16);
+        o.w = bf16_add(rv.w & 0xFFFF, s[6]) | (static_cast<uint32_t>(bf16_add(rv.w >> 16, s[7])) << 16);
+        st_global_v4(out + off, o);
+    }
+}
+
+// --------------------------------------------------------------------- S0 --
+// Linear weight [H][K] -> [N][H][K/N]: shard r is columns r*Ks .. r*Ks+Ks-1.
+__global__ void __launch_bounds__(256)
+    pack_weights_kernel(const uint16_t* __restrict__ w, uint16_t* __restrict__ wp, int hidden,
+                        int64_t k, int64_t ks) {
+    const int64_t kv = k >> 3;
+    const int64_t total = static_cast<int64_t>(hidden) * kv;
+    for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < total;
+         v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t h = v / kv;
+        const int64_t col = (v - h * kv) << 3;
+        const int64_t r = col / ks;
+        const int64_t kk = col - r * ks;
+        const uint4 val = ld_global_nc_v4(w + h * k + col);
+        st_global_v4(wp + (r * hidden + h) * ks + kk, val);
+    }
+}
+
+}  // namespace tpr

@@ -1,0 +1,414 @@
+// Host side of the C ABI declared in include/tp_reconcile.h: plan set-up,
+// argument checks, TMA descriptors and kernel launches. No device memory is
+// allocated here and nothing synchronises the caller's stream except
+// tp_device_error_flags, which says so.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "tp_kernels_exact.cuh"
+#include "tp_reconcile.h"
+
+struct tp_plan {
+    int n_ranks;
+    int64_t max_tokens, k, hidden, ks, hc;
+    int device;
+    int sm_count;
+    int smem_optin;
+    int variant;
+    int staged;
+};
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+tp_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = static_cast<int>(e);
+    return TP_ERR_CUDA;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        g_encode_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        else if (g_encode_err == cudaSuccess)
+            g_encode_err = cudaErrorSymbolNotFound;
+    });
+    return g_encode;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+    if (!a || !b || an == 0 || bn == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + bn && b0 < a0 + an;
+}
+
+tp_status check_device(const tp_plan* p) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return dev == p->device ? TP_OK : TP_ERR_INVALID;
+}
+
+// --------------------------------------------------------- exact variant --
+
+struct ExactConfig {
+    int mt, bh, grid_x, grid_y, stages, threads;
+    size_t smem;
+    uint32_t w_stage, x_stage;
+};
+
+constexpr size_t kSmemBudgetShared = 110 * 1024;   // two CTAs per SM
+constexpr size_t kSmemBudgetAlone = 200 * 1024;
+
+ExactConfig exact_config(const tp_plan* p, int64_t tokens) {
+    ExactConfig c{};
+    c.mt = tokens <= 1 ? 1 : tokens <= 2 ? 2 : tokens <= 4 ? 4 : 8;
+    const int n = p->n_ranks;
+    const int64_t mtiles = (tokens + c.mt - 1) / c.mt;
+    int64_t htiles = std::max<int64_t>(1, p->sm_count / std::max<int64_t>(1, mtiles));
+    int64_t bh = (p->hidden + htiles - 1) / htiles;
+    const int64_t bh_cap = std::min<int64_t>(256, tpr::kMaxExactChains / n);
+    bh = std::max<int64_t>(1, std::min<int64_t>(bh, std::min<int64_t>(bh_cap, p->hidden)));
+    c.bh = static_cast<int>(bh);
+    c.grid_x = static_cast<int>((p->hidden + bh - 1) / bh);
+    c.grid_y = static_cast<int>(mtiles);
+    const int chains = n * c.bh;
+    c.threads = ((chains + 31) / 32 + 1) * 32;
+    c.w_stage = static_cast<uint32_t>(((static_cast<size_t>(chains) * 128 + 1023) / 1024) * 1024);
+    c.x_stage = static_cast<uint32_t>(static_cast<size_t>(n) * c.mt * 128);
+    const size_t fixed = 2 * tpr::kMaxStages * sizeof(uint64_t) +
+                         static_cast<size_t>(chains) * c.mt * sizeof(uint16_t) + 1024;
+    const size_t stage = c.w_stage + c.x_stage;
+    size_t budget = stage <= 16 * 1024 ? kSmemBudgetShared : kSmemBudgetAlone;
+    budget = std::min<size_t>(budget, static_cast<size_t>(p->smem_optin));
+    int stages = budget > fixed ? static_cast<int>((budget - fixed) / stage) : 0;
+    c.stages = std::min(stages, tpr::kMaxStages);
+    c.smem = fixed + static_cast<size_t>(c.stages) * stage;
+    return c;
+}
+
+tp_status encode_maps(const tp_plan* p, const ExactConfig& c, const void* x, const void* w,
+                      int64_t tokens, CUtensorMap* mw, CUtensorMap* mx) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc) return cuda_fail(g_encode_err);
+    const cuuint32_t estr[3] = {1, 1, 1};
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->ks),
+                                    static_cast<cuuint64_t>(p->hidden),
+                                    static_cast<cuuint64_t>(p->n_ranks)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks) * 2,
+                                       static_cast<cuuint64_t>(p->hidden * p->ks) * 2};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(tpr::kKBlock),
+                                   static_cast<cuuint32_t>(c.bh),
+                                   static_cast<cuuint32_t>(p->n_ranks)};
+        CUresult r = enc(mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    }
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->ks),
+                                    static_cast<cuuint64_t>(p->n_ranks),
+                                    static_cast<cuuint64_t>(tokens)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks) * 2,
+                                       static_cast<cuuint64_t>(p->k) * 2};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(tpr::kKBlock),
+                                   static_cast<cuuint32_t>(p->n_ranks),
+                                   static_cast<cuuint32_t>(c.mt)};
+        CUresult r = enc(mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    }
+    return TP_OK;
+}
+
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+tp_status launch_exact(const tp_plan* p, const void* x, const void* w, const void* residual,
+                       void* out, void* partials, int64_t tokens, bool fused,
+                       cudaStream_t stream) {
+    const ExactConfig c = exact_config(p, tokens);
+    if (c.stages < 2) return TP_ERR_UNSUPPORTED;
+    CUtensorMap mw, mx;
+    tp_status st = encode_maps(p, c, x, w, tokens, &mw, &mx);
+    if (st != TP_OK) return st;
+    tpr::ExactParams prm{};
+    prm.n_ranks = p->n_ranks;
+    prm.bh = c.bh;
+    prm.ks = static_cast<int>(p->ks);
+    prm.hidden = static_cast<int>(p->hidden);
+    prm.hc = static_cast<int>(p->hc);
+    prm.tokens = static_cast<int>(tokens);
+    prm.stages = c.stages;
+    prm.fused = fused ? 1 : 0;
+    prm.w_stage_bytes = c.w_stage;
+    prm.x_stage_bytes = c.x_stage;
+    prm.w_box_bytes = static_cast<uint32_t>(tpr::kKBlock * c.bh * p->n_ranks * 2);
+    prm.x_box_bytes = static_cast<uint32_t>(tpr::kKBlock * p->n_ranks * c.mt * 2);
+    prm.residual = static_cast<const uint16_t*>(residual);
+    prm.out = static_cast<uint16_t*>(out);
+    prm.partials = static_cast<uint16_t*>(partials);
+    const dim3 grid(c.grid_x, c.grid_y), block(c.threads);
+    cudaError_t e;
+    switch (c.mt) {
+        case 1: e = launch_pdl(tpr::exact_partial_kernel<1>, grid, block, c.smem, stream, mw, mx, prm); break;
+        case 2: e = launch_pdl(tpr::exact_partial_kernel<2>, grid, block, c.smem, stream, mw, mx, prm); break;
+        case 4: e = launch_pdl(tpr::exact_partial_kernel<4>, grid, block, c.smem, stream, mw, mx, prm); break;
+        default: e = launch_pdl(tpr::exact_partial_kernel<8>, grid, block, c.smem, stream, mw, mx, prm); break;
+    }
+    return e == cudaSuccess ? TP_OK : cuda_fail(e);
+}
+
+tp_status launch_ring(const tp_plan* p, const void* partials, const void* residual, void* out,
+                      int64_t tokens, cudaStream_t stream) {
+    const int64_t total = tokens * (p->hidden / 8);
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(p->sm_count) * 8);
+    cudaError_t e = launch_pdl(tpr::ring_reduce_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                               stream, static_cast<const uint16_t*>(partials),
+                               static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out),
+                               p->n_ranks, tokens, static_cast<int>(p->hidden),
+                               static_cast<int>(p->hc));
+    return e == cudaSuccess ? TP_OK : cuda_fail(e);
+}
+
+// Lets every exact kernel use the device's opt-in shared memory less its own
+// static shared memory; returns the smallest such dynamic allowance.
+cudaError_t set_kernel_attrs(int smem_optin, int* dyn_max) {
+    const void* kernels[4] = {reinterpret_cast<const void*>(tpr::exact_partial_kernel<1>),
+                              reinterpret_cast<const void*>(tpr::exact_partial_kernel<2>),
+                              reinterpret_cast<const void*>(tpr::exact_partial_kernel<4>),
+                              reinterpret_cast<const void*>(tpr::exact_partial_kernel<8>)};
+    int lowest = smem_optin;
+    for (const void* k : kernels) {
+        cudaFuncAttributes fa{};
+        cudaError_t e = cudaFuncGetAttributes(&fa, k);
+        if (e != cudaSuccess) return e;
+        const int dyn = smem_optin - static_cast<int>(fa.sharedSizeBytes);
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+        if (e != cudaSuccess) return e;
+        lowest = std::min(lowest, dyn);
+    }
+    *dyn_max = lowest;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t k, int64_t hidden,
+                         int dtype) {
+    if (!out) return TP_ERR_INVALID;
+    *out = nullptr;
+    if (dtype != TP_BF16) return TP_ERR_UNSUPPORTED;
+    if (n_ranks < 1 || n_ranks > 8 || max_tokens < 0 || k <= 0 || hidden <= 0) return TP_ERR_INVALID;
+    if (k % n_ranks != 0 || hidden % n_ranks != 0) return TP_ERR_INVALID;
+    if ((k / n_ranks) % 8 != 0 || (hidden / n_ranks) % 8 != 0) return TP_ERR_INVALID;
+    if (hidden > INT32_MAX || k > INT32_MAX || max_tokens > INT32_MAX) return TP_ERR_UNSUPPORTED;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int sms = 0, optin = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return cuda_fail(e);
+    int dyn_max = 0;
+    if ((e = set_kernel_attrs(optin, &dyn_max)) != cudaSuccess) return cuda_fail(e);
+    tp_plan* p = new (std::nothrow) tp_plan{};
+    if (!p) return TP_ERR_INVALID;
+    p->n_ranks = n_ranks;
+    p->max_tokens = max_tokens;
+    p->k = k;
+    p->hidden = hidden;
+    p->ks = k / n_ranks;
+    p->hc = hidden / n_ranks;
+    p->device = dev;
+    p->sm_count = sms;
+    p->smem_optin = dyn_max;
+    p->variant = TP_VARIANT_AUTO;
+    p->staged = 0;
+    *out = p;
+    return TP_OK;
+}
+
+tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged) {
+    if (!plan) return TP_ERR_INVALID;
+    if (variant != TP_VARIANT_AUTO && variant != TP_VARIANT_EXACT && variant != TP_VARIANT_TENSOR)
+        return TP_ERR_INVALID;
+    if (staged != 0 && staged != 1) return TP_ERR_INVALID;
+    plan->variant = variant;
+    plan->staged = staged;
+    return TP_OK;
+}
+
+size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens) {
+    if (!plan || tokens <= 0 || !plan->staged) return 0;
+    const size_t b = static_cast<size_t>(plan->n_ranks) * static_cast<size_t>(tokens) *
+                     static_cast<size_t>(plan->hidden) * 2;
+    return (b + 255) / 256 * 256;
+}
+
+tp_status tp_pack_weights(const tp_plan* plan, const void* w_hk, void* w_packed, void* stream) {
+    if (!plan || !w_hk || !w_packed) return TP_ERR_INVALID;
+    if (!aligned16(w_hk) || !aligned16(w_packed)) return TP_ERR_ALIGN;
+    const size_t bytes = static_cast<size_t>(plan->hidden) * plan->k * 2;
+    if (overlaps(w_hk, bytes, w_packed, bytes)) return TP_ERR_INVALID;
+    tp_status st = check_device(plan);
+    if (st != TP_OK) return st;
+    const int64_t total = plan->hidden * (plan->k / 8);
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(plan->sm_count) * 16);
+    tpr::pack_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(w_hk), static_cast<uint16_t*>(w_packed),
+        static_cast<int>(plan->hidden), plan->k, plan->ks);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TP_OK : cuda_fail(e);
+}
+
+static tp_status check_point_args(const tp_plan* plan, const void* x, const void* w, int64_t tokens) {
+    if (!plan) return TP_ERR_INVALID;
+    if (tokens < 0 || tokens > plan->max_tokens) return TP_ERR_INVALID;
+    if (tokens > 0 && (!x || !w)) return TP_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(w)) return TP_ERR_ALIGN;
+    return TP_OK;
+}
+
+static int effective_variant(const tp_plan* plan, int64_t tokens) {
+    (void)tokens;
+    if (plan->variant == TP_VARIANT_AUTO) return TP_VARIANT_EXACT;
+    return plan->variant;
+}
+
+tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void* w_packed,
+                                 const void* residual, void* out, int64_t tokens, void* workspace,
+                                 void* stream) {
+    tp_status st = check_point_args(plan, x, w_packed, tokens);
+    if (st != TP_OK) return st;
+    if (tokens == 0) return TP_OK;
+    if (!residual || !out) return TP_ERR_INVALID;
+    if (!aligned16(residual) || !aligned16(out) || !aligned16(workspace)) return TP_ERR_ALIGN;
+    const size_t mh = static_cast<size_t>(tokens) * plan->hidden * 2;
+    const size_t xb = static_cast<size_t>(tokens) * plan->k * 2;
+    const size_t wb = static_cast<size_t>(plan->hidden) * plan->k * 2;
+    const size_t ws = tp_plan_workspace_bytes(plan, tokens);
+    if (overlaps(out, mh, x, xb) || overlaps(out, mh, w_packed, wb) ||
+        overlaps(out, mh, residual, mh) || overlaps(out, mh, workspace, ws))
+        return TP_ERR_INVALID;
+    if (plan->staged && !workspace) return TP_ERR_WORKSPACE;
+    if ((st = check_device(plan)) != TP_OK) return st;
+    const int variant = effective_variant(plan, tokens);
+    if (variant != TP_VARIANT_EXACT) return TP_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!plan->staged)
+        return launch_exact(plan, x, w_packed, residual, out, nullptr, tokens, true, s);
+    st = launch_exact(plan, x, w_packed, nullptr, nullptr, workspace, tokens, false, s);
+    if (st != TP_OK) return st;
+    return launch_ring(plan, workspace, residual, out, tokens, s);
+}
+
+tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* w_packed,
+                                void* partials, int64_t tokens, void* stream) {
+    tp_status st = check_point_args(plan, x, w_packed, tokens);
+    if (st != TP_OK) return st;
+    if (tokens == 0) return TP_OK;
+    if (!partials) return TP_ERR_INVALID;
+    if (!aligned16(partials)) return TP_ERR_ALIGN;
+    const size_t pb = static_cast<size_t>(plan->n_ranks) * tokens * plan->hidden * 2;
+    if (overlaps(partials, pb, x, static_cast<size_t>(tokens) * plan->k * 2) ||
+        overlaps(partials, pb, w_packed, static_cast<size_t>(plan->hidden) * plan->k * 2))
+        return TP_ERR_INVALID;
+    if ((st = check_device(plan)) != TP_OK) return st;
+    const int variant = effective_variant(plan, tokens);
+    if (variant != TP_VARIANT_EXACT) return TP_ERR_UNSUPPORTED;
+    return launch_exact(plan, x, w_packed, nullptr, nullptr, partials, tokens, false,
+                        static_cast<cudaStream_t>(stream));
+}
+
+tp_status tp_ring_reduce(const tp_plan* plan, const void* partials, const void* residual, void* out,
+                         int64_t tokens, void* stream) {
+    if (!plan) return TP_ERR_INVALID;
+    if (tokens < 0 || tokens > plan->max_tokens) return TP_ERR_INVALID;
+    if (tokens == 0) return TP_OK;
+    if (!partials || !residual || !out) return TP_ERR_INVALID;
+    if (!aligned16(partials) || !aligned16(residual) || !aligned16(out)) return TP_ERR_ALIGN;
+    const size_t mh = static_cast<size_t>(tokens) * plan->hidden * 2;
+    if (overlaps(out, mh, partials, mh * plan->n_ranks) || overlaps(out, mh, residual, mh))
+        return TP_ERR_INVALID;
+    tp_status st = check_device(plan);
+    if (st != TP_OK) return st;
+    return launch_ring(plan, partials, residual, out, tokens, static_cast<cudaStream_t>(stream));
+}
+
+uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes, int64_t points) {
+    if (n_ranks < 1 || tokens < 0 || hidden < 0 || elem_bytes < 0 || points < 0) return 0;
+    const uint64_t payload = static_cast<uint64_t>(tokens) * static_cast<uint64_t>(hidden) *
+                             static_cast<uint64_t>(elem_bytes) * static_cast<uint64_t>(points);
+    return 2ull * static_cast<uint64_t>(n_ranks - 1) * payload / static_cast<uint64_t>(n_ranks);
+}
+
+void tp_plan_destroy(tp_plan* plan) { delete plan; }
+
+const char* tp_status_string(tp_status status) {
+    switch (status) {
+        case TP_OK: return "ok";
+        case TP_ERR_INVALID: return "invalid argument";
+        case TP_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case TP_ERR_UNSUPPORTED: return "unsupported shape, dtype or variant";
+        case TP_ERR_WORKSPACE: return "workspace missing or too small";
+        case TP_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+int tp_last_cuda_error(void) { return t_last_cuda_error; }
+
+tp_status tp_device_error_flags(const tp_plan* plan, uint32_t* flags, int reset) {
+    if (!plan || !flags) return TP_ERR_INVALID;
+    tp_status st = check_device(plan);
+    if (st != TP_OK) return st;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e);
+    uint32_t v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, tpr::g_device_error, sizeof v)) != cudaSuccess) return cuda_fail(e);
+    if (reset) {
+        const uint32_t zero = 0;
+        if ((e = cudaMemcpyToSymbol(tpr::g_device_error, &zero, sizeof zero)) != cudaSuccess)
+            return cuda_fail(e);
+    }
+    *flags = v;
+    return TP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,151 @@
+"""Torch-facing wrapper of the C ABI: a ``Plan`` owns one tp_plan handle.
+
+PyTorch supplies device memory and the current stream; every tensor goes to
+the library as a data pointer after its device, dtype, shape and layout are
+checked here. Nothing is computed in Python.
+"""
+
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import TPError
+
+_VARIANTS = {"auto": _lib.TP_VARIANT_AUTO, "exact": _lib.TP_VARIANT_EXACT,
+             "tensor": _lib.TP_VARIANT_TENSOR}
+
+
+def _check(t: torch.Tensor, name: str, shape) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+class Plan:
+    """One projection shape: N ranks, up to max_tokens tokens, K inputs, H outputs."""
+
+    def __init__(self, n_ranks: int, max_tokens: int, k: int, hidden: int,
+                 variant: str = "auto", staged: bool = False):
+        st, h = _lib.tp_plan_create(n_ranks, max_tokens, k, hidden, _lib.TP_BF16)
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_plan_create")
+        self._h = h
+        self.n_ranks, self.max_tokens, self.k, self.hidden = n_ranks, max_tokens, k, hidden
+        self.ks, self.hc = k // n_ranks, hidden // n_ranks
+        self.device = torch.cuda.current_device()
+        self.set_variant(variant, staged)
+
+    def set_variant(self, variant: str = "auto", staged: bool = False) -> None:
+        st = _lib.tp_plan_set_variant(self._h, _VARIANTS[variant], int(bool(staged)))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_plan_set_variant")
+        self.variant, self.staged = variant, bool(staged)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _lib.tp_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self, tokens: int) -> int:
+        return _lib.tp_plan_workspace_bytes(self._h, tokens)
+
+    def pack_weights(self, w_hk: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+        """Linear weight [H, K] -> packed shards [N, H, K/N]."""
+        if out is None:
+            out = torch.empty(self.n_ranks, self.hidden, self.ks, dtype=torch.bfloat16,
+                              device=w_hk.device)
+        a = _check(w_hk, "w_hk", (self.hidden, self.k))
+        b = _check(out, "w_packed", (self.n_ranks, self.hidden, self.ks))
+        st = _lib.tp_pack_weights(self._h, a, b, _stream(stream))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_pack_weights")
+        return out
+
+    def reconcile(self, x: torch.Tensor, w_packed: torch.Tensor, residual: torch.Tensor,
+                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+        """out [M, H] = residual + ring-ordered sum over ranks of x_r . W_r^T."""
+        m = x.shape[0]
+        if out is None:
+            out = torch.empty(m, self.hidden, dtype=torch.bfloat16, device=x.device)
+        px = _check(x, "x", (m, self.k))
+        pw = _check(w_packed, "w_packed", (self.n_ranks, self.hidden, self.ks))
+        pr = _check(residual, "residual", (m, self.hidden))
+        po = _check(out, "out", (m, self.hidden))
+        need = self.workspace_bytes(m)
+        pws = 0
+        if need:
+            if workspace is None:
+                workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+            if workspace.numel() * workspace.element_size() < need or workspace.device.type != "cuda":
+                raise ValueError("workspace too small")
+            pws = workspace.data_ptr()
+        st = _lib.tp_rowlinear_reconcile(self._h, px, pw, pr, po, m, pws, _stream(stream))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_rowlinear_reconcile")
+        return out
+
+    def partials(self, x: torch.Tensor, w_packed: torch.Tensor,
+                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """The N partials [N, M, H] (S1 only)."""
+        m = x.shape[0]
+        if out is None:
+            out = torch.empty(self.n_ranks, m, self.hidden, dtype=torch.bfloat16, device=x.device)
+        px = _check(x, "x", (m, self.k))
+        pw = _check(w_packed, "w_packed", (self.n_ranks, self.hidden, self.ks))
+        po = _check(out, "partials", (self.n_ranks, m, self.hidden))
+        st = _lib.tp_rowlinear_partials(self._h, px, pw, po, m, _stream(stream))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_rowlinear_partials")
+        return out
+
+    def ring_reduce(self, partials: torch.Tensor, residual: torch.Tensor,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """S2-S4 on given partials [N, M, H]."""
+        m = partials.shape[1]
+        if out is None:
+            out = torch.empty(m, self.hidden, dtype=torch.bfloat16, device=partials.device)
+        pp = _check(partials, "partials", (self.n_ranks, m, self.hidden))
+        pr = _check(residual, "residual", (m, self.hidden))
+        po = _check(out, "out", (m, self.hidden))
+        st = _lib.tp_ring_reduce(self._h, pp, pr, po, m, _stream(stream))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_ring_reduce")
+        return out
+
+    def device_error_flags(self, reset: bool = False) -> int:
+        st, flags = _lib.tp_device_error_flags(self._h, int(reset))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_device_error_flags")
+        return flags
+
+
+def ring_bytes(n_ranks: int, tokens: int, hidden: int, elem_bytes: int = 2, points: int = 1) -> int:
+    return _lib.tp_ring_bytes(n_ranks, tokens, hidden, elem_bytes, points)
