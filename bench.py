@@ -184,8 +184,9 @@ class ClockSampler:
 def cpu_baseline(cfg, threads=None, target_s=12.0):
     """The oracle as it stands on this host's cores, on a bounded sample.
 
-    Sample: the first point of each projection kind (all H columns, all M
-    tokens), repeated until about target_s seconds of oracle work; the step
+    Sample: the first point of each projection kind (all M tokens; all H
+    output columns, or a leading block of them for the large workloads), run
+    repeatedly for about target_s seconds of oracle work in total; the step
     time is extrapolated by the number of points of each kind.
     """
     import oracle
@@ -193,34 +194,34 @@ def cpu_baseline(cfg, threads=None, target_s=12.0):
     kinds = {}
     for p in cfg.points:
         kinds.setdefault(p.kind, []).append(p)
-    per_kind = {}
-    total_time, reps_done, desc = 0.0, 0, []
+    per_kind, desc, measured = {}, [], 0.0
+    budget = target_s / len(kinds)
     for kind, pts in kinds.items():
         p = pts[0]
         x = point_tensor(cfg, p, KIND_X).view(torch.int16).numpy().view(np.uint16)
         w = point_tensor(cfg, p, KIND_W).view(torch.int16).numpy().view(np.uint16)
         r = point_tensor(cfg, p, KIND_RESIDUAL).view(torch.int16).numpy().view(np.uint16)
-        rows = cfg.hidden
-        # bound one call to ~ target_s / number of kinds
+        # columns per call: all of them unless one call would exceed the budget
         t0 = time.perf_counter()
-        oracle.reconcile(cfg.n_ranks, cfg.hidden, x, np.ascontiguousarray(w[:64]),
-                         np.ascontiguousarray(r[:, :64]), cols=np.arange(64), threads=threads)
-        probe = (time.perf_counter() - t0) / 64
-        budget = target_s / len(kinds)
-        rows = int(max(64, min(cfg.hidden, budget / max(probe, 1e-9))))
-        cols = np.arange(rows)
-        t0 = time.perf_counter()
-        oracle.reconcile(cfg.n_ranks, cfg.hidden, x, np.ascontiguousarray(w[:rows]),
-                         np.ascontiguousarray(r[:, :rows]), cols=cols, threads=threads)
-        dt = time.perf_counter() - t0
-        per_point = dt * cfg.hidden / rows
-        per_kind[kind] = per_point
-        total_time += dt
-        reps_done += 1
-        desc.append(f"{kind} point {p.index} (K={p.k}): {rows} of {cfg.hidden} output columns")
+        oracle.reconcile(cfg.n_ranks, cfg.hidden, x, np.ascontiguousarray(w[:16]),
+                         np.ascontiguousarray(r[:, :16]), cols=np.arange(16), threads=threads)
+        per_col = (time.perf_counter() - t0) / 16
+        cols = int(max(16, min(cfg.hidden, budget / max(per_col, 1e-9))))
+        wc, rc, cc = (np.ascontiguousarray(w[:cols]), np.ascontiguousarray(r[:, :cols]),
+                      np.arange(cols))
+        reps, spent = 0, 0.0
+        while spent < budget or reps == 0:
+            t0 = time.perf_counter()
+            oracle.reconcile(cfg.n_ranks, cfg.hidden, x, wc, rc, cols=cc, threads=threads)
+            spent += time.perf_counter() - t0
+            reps += 1
+        per_kind[kind] = spent / reps * cfg.hidden / cols
+        measured += spent
+        desc.append(f"{kind} point {p.index} (K={p.k}): {cols} of {cfg.hidden} output columns "
+                    f"x {reps} runs")
     step_s = sum(per_kind[p.kind] for p in cfg.points)
     return {"step_s": step_s, "cores": threads, "sample": "; ".join(desc) +
-            f"; step time extrapolated over {cfg.n_points} points ({total_time:.1f} s measured)"}
+            f"; step time extrapolated over {cfg.n_points} points ({measured:.1f} s measured)"}
 
 
 # --------------------------------------------------------------------- main --

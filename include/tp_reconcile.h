@@ -100,6 +100,10 @@ TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
  * Returns 0 for a null plan. */
 TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 
+/* Bytes of the packed weight buffer tp_pack_weights writes: N*H*(K/N)*2,
+ * the size of the Linear weight. Returns 0 for a null plan. */
+TP_API size_t tp_plan_packed_bytes(const tp_plan* plan);
+
 /* S0, once per weight. Packs a torch Linear weight into the sharded layout.
  *   w_hk      [H][K] bf16, the Linear weight (input)
  *   w_packed  [N][H][K/N] bf16 (output): shard r is columns r*K/N ..

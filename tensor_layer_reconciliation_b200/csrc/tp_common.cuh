@@ -72,14 +72,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
         : "memory");
 }
 
+// Suspend-time hint for try_wait: a waiting thread sleeps until the phase
+// completes or this many nanoseconds pass, instead of polling the barrier
+// (polling threads compete with the bulk copies for the shared-memory path).
+constexpr uint32_t kSuspendHintNs = 1000000u;  // 1 ms
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -89,9 +94,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t spins = 0;
     while (!mbar_try_wait(bar, parity)) {
-        if ((++spins & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
             atomicOr(&g_device_error, kErrWaitTimeout);
             return false;
         }
@@ -124,6 +128,59 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // Lets the next grid in the stream start its prologue early.
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Two steps of an fp32 accumulation chain on a pair of bf16 values each:
+// acc = fma(x.lo, w.lo, acc); acc = fma(x.hi, w.hi, acc). The mixed-precision
+// FMA multiplies the bf16 operands exactly and rounds once to fp32, the same
+// as fmaf on their fp32 widenings; the low half (the earlier k) goes first.
+__device__ __forceinline__ float fma2_bf16(uint32_t x, uint32_t w, float acc) {
+    asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+        "mov.b32 {xl, xh}, %1;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, xl, wl, %0;\n\t"
+        "fma.rn.f32.bf16 %0, xh, wh, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(x), "r"(w));
+    return acc;
+}
+
+// Four chain steps sharing one x pair: two rows (a, b) of the same rank,
+// each advanced by x.lo then x.hi (k ascending within each chain); the two
+// chains interleave so each FMA's latency hides behind the other chain's.
+__device__ __forceinline__ void fma4_bf16(uint32_t x, uint32_t wa, uint32_t wb, float& a,
+                                          float& b) {
+    asm("{\n\t.reg .b16 xl, xh, al, ah, bl, bh;\n\t"
+        "mov.b32 {xl, xh}, %2;\n\t"
+        "mov.b32 {al, ah}, %3;\n\t"
+        "mov.b32 {bl, bh}, %4;\n\t"
+        "fma.rn.f32.bf16 %0, xl, al, %0;\n\t"
+        "fma.rn.f32.bf16 %1, xl, bl, %1;\n\t"
+        "fma.rn.f32.bf16 %0, xh, ah, %0;\n\t"
+        "fma.rn.f32.bf16 %1, xh, bh, %1;\n\t}"
+        : "+f"(a), "+f"(b)
+        : "r"(x), "r"(wa), "r"(wb));
+}
+
+// 1-D bulk copy global -> this CTA's shared memory (no multicast); both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 5-D tiled bulk tensor load into this CTA's shared memory (no multicast).
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+        "r"(c3), "r"(c4)
+        : "memory");
 }
 
 // ------------------------------------------------------------ vector loads --

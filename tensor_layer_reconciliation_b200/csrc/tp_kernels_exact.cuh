@@ -153,33 +153,35 @@ __global__ void __launch_bounds__(kMaxExactThreads, 1)
             break;
         }
         if (owner) {
-            const uint8_t* wrow = w_ring + static_cast<size_t>(s) * p.w_stage_bytes + row * 128;
-            const uint8_t* xs = x_ring + static_cast<size_t>(s) * p.x_stage_bytes + r * 128;
+            // Plain shared-memory loads (ordered after the barrier wait by its
+            // memory clobber) so the compiler can issue the block's loads
+            // ahead of the FMA chain.
+            const uint4* wrow = reinterpret_cast<const uint4*>(
+                w_ring + static_cast<size_t>(s) * p.w_stage_bytes + row * 128);
+            const uint4* xs = reinterpret_cast<const uint4*>(
+                x_ring + static_cast<size_t>(s) * p.x_stage_bytes + r * 128);
+            const int sw = row & 7;
             const int rem = p.ks - kb * kKBlock;
-            const int nv = rem >= kKBlock ? 8 : rem >> 3;
+            const int nv = rem >= kKBlock ? 8 : rem >> 3;  // K/N % 8 == 0: whole 16-byte vectors
+            uint4 wv[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                if (c < nv) {
-                    const uint4 wv = ld_shared_v4(wrow + ((c ^ (row & 7)) << 4));
-                    const float w0 = bf16_lo(wv.x), w1 = bf16_hi(wv.x);
-                    const float w2 = bf16_lo(wv.y), w3 = bf16_hi(wv.y);
-                    const float w4 = bf16_lo(wv.z), w5 = bf16_hi(wv.z);
-                    const float w6 = bf16_lo(wv.w), w7 = bf16_hi(wv.w);
+            for (int c = 0; c < 8; ++c)
+                if (c < nv) wv[c] = wrow[c ^ sw];
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        const uint4 xv = ld_shared_v4(xs + mt * N * 128 + (c << 4));
-                        float a = acc[mt];
-                        a = __fmaf_rn(bf16_lo(xv.x), w0, a);
-                        a = __fmaf_rn(bf16_hi(xv.x), w1, a);
-                        a = __fmaf_rn(bf16_lo(xv.y), w2, a);
-                        a = __fmaf_rn(bf16_hi(xv.y), w3, a);
-                        a = __fmaf_rn(bf16_lo(xv.z), w4, a);
-                        a = __fmaf_rn(bf16_hi(xv.z), w5, a);
-                        a = __fmaf_rn(bf16_lo(xv.w), w6, a);
-                        a = __fmaf_rn(bf16_hi(xv.w), w7, a);
-                        acc[mt] = a;
+            for (int mt = 0; mt < MT; ++mt) {
+                const uint4* xm = xs + mt * N * 8;
+                float a = acc[mt];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (c < nv) {
+                        const uint4 xv = xm[c];
+                        a = fma2_bf16(xv.x, wv[c].x, a);
+                        a = fma2_bf16(xv.y, wv[c].y, a);
+                        a = fma2_bf16(xv.z, wv[c].z, a);
+                        a = fma2_bf16(xv.w, wv[c].w, a);
                     }
                 }
+                acc[mt] = a;
             }
         }
         __syncwarp();

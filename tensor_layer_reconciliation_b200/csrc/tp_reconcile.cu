@@ -281,6 +281,10 @@ size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens) {
     return (b + 255) / 256 * 256;
 }
 
+size_t tp_plan_packed_bytes(const tp_plan* plan) {
+    return plan ? static_cast<size_t>(plan->hidden) * static_cast<size_t>(plan->k) * 2 : 0;
+}
+
 tp_status tp_pack_weights(const tp_plan* plan, const void* w_hk, void* w_packed, void* stream) {
     if (!plan || !w_hk || !w_packed) return TP_ERR_INVALID;
     if (!aligned16(w_hk) || !aligned16(w_packed)) return TP_ERR_ALIGN;

@@ -75,14 +75,18 @@ class Plan:
     def workspace_bytes(self, tokens: int) -> int:
         return _lib.tp_plan_workspace_bytes(self._h, tokens)
 
+    @property
+    def packed_numel(self) -> int:
+        """bf16 elements of the packed weight buffer (tiled shards, see tp_reconcile.h)."""
+        return _lib.tp_plan_packed_bytes(self._h) // 2
+
     def pack_weights(self, w_hk: torch.Tensor, out: Optional[torch.Tensor] = None,
                      stream=None) -> torch.Tensor:
-        """Linear weight [H, K] -> packed shards [N, H, K/N]."""
+        """Linear weight [H, K] -> packed tiled shards (flat bf16 tensor)."""
         if out is None:
-            out = torch.empty(self.n_ranks, self.hidden, self.ks, dtype=torch.bfloat16,
-                              device=w_hk.device)
+            out = torch.empty(self.packed_numel, dtype=torch.bfloat16, device=w_hk.device)
         a = _check(w_hk, "w_hk", (self.hidden, self.k))
-        b = _check(out, "w_packed", (self.n_ranks, self.hidden, self.ks))
+        b = _check(out, "w_packed", (self.packed_numel,))
         st = _lib.tp_pack_weights(self._h, a, b, _stream(stream))
         if st != _lib.TP_OK:
             raise TPError(st, "tp_pack_weights")
@@ -96,7 +100,7 @@ class Plan:
         if out is None:
             out = torch.empty(m, self.hidden, dtype=torch.bfloat16, device=x.device)
         px = _check(x, "x", (m, self.k))
-        pw = _check(w_packed, "w_packed", (self.n_ranks, self.hidden, self.ks))
+        pw = _check(w_packed, "w_packed", (self.packed_numel,))
         pr = _check(residual, "residual", (m, self.hidden))
         po = _check(out, "out", (m, self.hidden))
         need = self.workspace_bytes(m)
@@ -119,7 +123,7 @@ class Plan:
         if out is None:
             out = torch.empty(self.n_ranks, m, self.hidden, dtype=torch.bfloat16, device=x.device)
         px = _check(x, "x", (m, self.k))
-        pw = _check(w_packed, "w_packed", (self.n_ranks, self.hidden, self.ks))
+        pw = _check(w_packed, "w_packed", (self.packed_numel,))
         po = _check(out, "partials", (self.n_ranks, m, self.hidden))
         st = _lib.tp_rowlinear_partials(self._h, px, pw, po, m, _stream(stream))
         if st != _lib.TP_OK:

@@ -61,7 +61,7 @@ def test_zero_tokens_launches_nothing(dev):
     plan = tlr.Plan(2, 4, 256, 64)
     x = torch.empty(0, 256, dtype=torch.bfloat16, device=dev)
     r = torch.empty(0, 64, dtype=torch.bfloat16, device=dev)
-    wp = torch.zeros(2, 64, 128, dtype=torch.bfloat16, device=dev)
+    wp = torch.zeros(plan.packed_numel, dtype=torch.bfloat16, device=dev)
     out = plan.reconcile(x, wp, r)
     assert out.shape == (0, 64)
 
