@@ -68,7 +68,7 @@ typedef enum {
 enum { TP_BF16 = 0 };
 
 typedef enum {
-    TP_VARIANT_AUTO = 0,   /* EXACT for few tokens, TENSOR where built and faster */
+    TP_VARIANT_AUTO = 0,   /* EXACT below 16 tokens, TENSOR from 16 tokens on */
     TP_VARIANT_EXACT = 1,  /* CUDA cores, fp32 FMA chain per partial, k ascending */
     TP_VARIANT_TENSOR = 2  /* tcgen05 tensor cores, fp32 accumulate in TMEM */
 } tp_variant;
@@ -96,8 +96,9 @@ TP_API tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, 
 TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
 
 /* Bytes of workspace tp_rowlinear_reconcile needs for `tokens` tokens with
- * the plan's current setting: N*M*H*2 rounded up to 256 when staged, else 0.
- * Returns 0 for a null plan. */
+ * the plan's current setting: N*M*H*2 rounded up to 256 when the partials go
+ * through memory (staged, or the tensor-core variant, which always stages
+ * them), else 0. Returns 0 for a null plan. */
 TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 
 /* Bytes of the packed weight buffer tp_pack_weights writes: N*H*(K/N)*2,

@@ -11,6 +11,7 @@
 #include <new>
 
 #include "tp_kernels_exact.cuh"
+#include "tp_kernels_tc.cuh"
 #include "tp_reconcile.h"
 
 struct tp_plan {
@@ -191,6 +192,99 @@ tp_status launch_exact(const tp_plan* p, const void* x, const void* w, const voi
     return e == cudaSuccess ? TP_OK : cuda_fail(e);
 }
 
+// -------------------------------------------------------- tensor variant --
+
+struct TcConfig {
+    int bn, stages, grid, units, h_tiles, m_tiles;
+    size_t smem;
+};
+
+constexpr int64_t kTensorMinTokens = 16;     // AUTO uses the tensor cores from here
+
+int tc_token_tile(int64_t tokens) {
+    return tokens <= 32 ? 32 : tokens <= 64 ? 64 : tokens <= 128 ? 128 : 256;
+}
+
+TcConfig tc_config(const tp_plan* p, int64_t tokens) {
+    TcConfig c{};
+    c.bn = tc_token_tile(tokens);
+    c.h_tiles = static_cast<int>((p->hidden + tpr::kTcRows - 1) / tpr::kTcRows);
+    c.m_tiles = static_cast<int>((tokens + c.bn - 1) / c.bn);
+    c.units = p->n_ranks * c.h_tiles * c.m_tiles;
+    const size_t stage = tpr::kTcATile + static_cast<size_t>(c.bn) * tpr::kTcKBlock * 2;
+    const size_t fixed = (2 * tpr::kTcMaxStages + 5) * sizeof(uint64_t) + 16 + 1024;
+    // Small token tiles stream weights: two CTAs per SM (about 100 KB each,
+    // tensor memory 2 x 2*BN columns). Large tiles: one CTA per SM, deep ring.
+    const bool two_per_sm = c.bn <= 64;
+    const size_t budget = std::min<size_t>(two_per_sm ? 110 * 1024 : 200 * 1024,
+                                           static_cast<size_t>(p->smem_optin));
+    c.stages = static_cast<int>(std::min<size_t>(tpr::kTcMaxStages, (budget - fixed) / stage));
+    c.smem = fixed + static_cast<size_t>(c.stages) * stage;
+    const int slots = p->sm_count * (two_per_sm ? 2 : 1);
+    c.grid = std::min(c.units, slots);
+    return c;
+}
+
+tp_status encode_tc_maps(const tp_plan* p, const TcConfig& c, const void* x, const void* w,
+                         int64_t tokens, CUtensorMap* mw, CUtensorMap* mx) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc) return cuda_fail(g_encode_err);
+    const cuuint32_t estr[3] = {1, 1, 1};
+    {
+        // Packed weights [N][H][Ks]: {Ks, H, N}, 128 rows x 64 columns per box.
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->ks), static_cast<cuuint64_t>(p->hidden),
+                                    static_cast<cuuint64_t>(p->n_ranks)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks) * 2,
+                                       static_cast<cuuint64_t>(p->hidden * p->ks) * 2};
+        const cuuint32_t box[3] = {tpr::kTcKBlock, tpr::kTcRows, 1};
+        CUresult r = enc(mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    }
+    {
+        // Activations [M][N][Ks]: {Ks, N, M}, BN token rows x 64 columns of one rank.
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->ks), static_cast<cuuint64_t>(p->n_ranks),
+                                    static_cast<cuuint64_t>(tokens)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks) * 2,
+                                       static_cast<cuuint64_t>(p->k) * 2};
+        const cuuint32_t box[3] = {tpr::kTcKBlock, 1, static_cast<cuuint32_t>(c.bn)};
+        CUresult r = enc(mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    }
+    return TP_OK;
+}
+
+tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partials, int64_t tokens,
+                    cudaStream_t stream) {
+    const TcConfig c = tc_config(p, tokens);
+    if (c.stages < 2) return TP_ERR_UNSUPPORTED;
+    CUtensorMap mw, mx;
+    tp_status st = encode_tc_maps(p, c, x, w, tokens, &mw, &mx);
+    if (st != TP_OK) return st;
+    tpr::TcParams prm{};
+    prm.n_ranks = p->n_ranks;
+    prm.ks = static_cast<int>(p->ks);
+    prm.hidden = static_cast<int>(p->hidden);
+    prm.tokens = static_cast<int>(tokens);
+    prm.h_tiles = c.h_tiles;
+    prm.m_tiles = c.m_tiles;
+    prm.units = c.units;
+    prm.stages = c.stages;
+    prm.partials = static_cast<uint16_t*>(partials);
+    const dim3 grid(c.grid), block(tpr::kTcThreads);
+    cudaError_t e;
+    switch (c.bn) {
+        case 32: e = launch_pdl(tpr::tc_partial_kernel<32>, grid, block, c.smem, stream, mw, mx, prm); break;
+        case 64: e = launch_pdl(tpr::tc_partial_kernel<64>, grid, block, c.smem, stream, mw, mx, prm); break;
+        case 128: e = launch_pdl(tpr::tc_partial_kernel<128>, grid, block, c.smem, stream, mw, mx, prm); break;
+        default: e = launch_pdl(tpr::tc_partial_kernel<256>, grid, block, c.smem, stream, mw, mx, prm); break;
+    }
+    return e == cudaSuccess ? TP_OK : cuda_fail(e);
+}
+
 tp_status launch_ring(const tp_plan* p, const void* partials, const void* residual, void* out,
                       int64_t tokens, cudaStream_t stream) {
     const int64_t total = tokens * (p->hidden / 8);
@@ -206,10 +300,14 @@ tp_status launch_ring(const tp_plan* p, const void* partials, const void* residu
 // Lets every exact kernel use the device's opt-in shared memory less its own
 // static shared memory; returns the smallest such dynamic allowance.
 cudaError_t set_kernel_attrs(int smem_optin, int* dyn_max) {
-    const void* kernels[4] = {reinterpret_cast<const void*>(tpr::exact_partial_kernel<1>),
+    const void* kernels[8] = {reinterpret_cast<const void*>(tpr::exact_partial_kernel<1>),
                               reinterpret_cast<const void*>(tpr::exact_partial_kernel<2>),
                               reinterpret_cast<const void*>(tpr::exact_partial_kernel<4>),
-                              reinterpret_cast<const void*>(tpr::exact_partial_kernel<8>)};
+                              reinterpret_cast<const void*>(tpr::exact_partial_kernel<8>),
+                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<32>),
+                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<64>),
+                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<128>),
+                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<256>)};
     int lowest = smem_optin;
     for (const void* k : kernels) {
         cudaFuncAttributes fa{};
@@ -274,8 +372,18 @@ tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged) {
     return TP_OK;
 }
 
+// AUTO: the k-ascending CUDA-core chain for few tokens (a memory-bound
+// weight stream either way), the tensor cores from kTensorMinTokens on.
+static int effective_variant(const tp_plan* plan, int64_t tokens) {
+    if (plan->variant == TP_VARIANT_AUTO)
+        return tokens >= kTensorMinTokens ? TP_VARIANT_TENSOR : TP_VARIANT_EXACT;
+    return plan->variant;
+}
+
 size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens) {
-    if (!plan || tokens <= 0 || !plan->staged) return 0;
+    if (!plan || tokens <= 0) return 0;
+    // The tensor-core partials always go through the workspace.
+    if (!plan->staged && effective_variant(plan, tokens) != TP_VARIANT_TENSOR) return 0;
     const size_t b = static_cast<size_t>(plan->n_ranks) * static_cast<size_t>(tokens) *
                      static_cast<size_t>(plan->hidden) * 2;
     return (b + 255) / 256 * 256;
@@ -309,12 +417,6 @@ static tp_status check_point_args(const tp_plan* plan, const void* x, const void
     return TP_OK;
 }
 
-static int effective_variant(const tp_plan* plan, int64_t tokens) {
-    (void)tokens;
-    if (plan->variant == TP_VARIANT_AUTO) return TP_VARIANT_EXACT;
-    return plan->variant;
-}
-
 tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void* w_packed,
                                  const void* residual, void* out, int64_t tokens, void* workspace,
                                  void* stream) {
@@ -330,14 +432,17 @@ tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void*
     if (overlaps(out, mh, x, xb) || overlaps(out, mh, w_packed, wb) ||
         overlaps(out, mh, residual, mh) || overlaps(out, mh, workspace, ws))
         return TP_ERR_INVALID;
-    if (plan->staged && !workspace) return TP_ERR_WORKSPACE;
+    if (ws && !workspace) return TP_ERR_WORKSPACE;
     if ((st = check_device(plan)) != TP_OK) return st;
     const int variant = effective_variant(plan, tokens);
-    if (variant != TP_VARIANT_EXACT) return TP_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (!plan->staged)
-        return launch_exact(plan, x, w_packed, residual, out, nullptr, tokens, true, s);
-    st = launch_exact(plan, x, w_packed, nullptr, nullptr, workspace, tokens, false, s);
+    if (variant == TP_VARIANT_TENSOR) {
+        st = launch_tc(plan, x, w_packed, workspace, tokens, s);
+    } else {
+        if (!plan->staged)
+            return launch_exact(plan, x, w_packed, residual, out, nullptr, tokens, true, s);
+        st = launch_exact(plan, x, w_packed, nullptr, nullptr, workspace, tokens, false, s);
+    }
     if (st != TP_OK) return st;
     return launch_ring(plan, workspace, residual, out, tokens, s);
 }
@@ -355,7 +460,8 @@ tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* 
         return TP_ERR_INVALID;
     if ((st = check_device(plan)) != TP_OK) return st;
     const int variant = effective_variant(plan, tokens);
-    if (variant != TP_VARIANT_EXACT) return TP_ERR_UNSUPPORTED;
+    if (variant == TP_VARIANT_TENSOR)
+        return launch_tc(plan, x, w_packed, partials, tokens, static_cast<cudaStream_t>(stream));
     return launch_exact(plan, x, w_packed, nullptr, nullptr, partials, tokens, false,
                         static_cast<cudaStream_t>(stream));
 }

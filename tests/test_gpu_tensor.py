@@ -1,0 +1,137 @@
+"""Parity of the tensor-core variant (tcgen05, fp32 accumulation in TMEM)
+against the oracle.
+
+The tensor cores accumulate in their own order, so a partial can differ from
+the oracle's k-ascending fp32 sum where that sum lies next to a bf16 rounding
+boundary. The checks:
+
+* integer-valued x, W in {-1, 0, 1}: every sum is an exactly representable
+  integer, so partials and outputs must be bit-identical to the oracle (this
+  pins the operand layouts, descriptors and tile indexing);
+* Gaussian inputs: a partial is "fragile" when the bf16 rounding of its fp64
+  value d is not the same at d - e and d + e, with e = 2^-19 * sum|x*w|, far
+  above any fp32 accumulation error at these sizes (about 2^-24 * sqrt(K/N)
+  relative). Every non-fragile partial must equal bf16(d) and the oracle's
+  partial; a fragile one must be one of the two bf16 values around d. An
+  output whose N partials are all non-fragile must equal the oracle's bit
+  for bit; for the rest, a flipped partial moves its addend by one bf16
+  unit of that partial, and each of the N-1 ring adds and the residual add
+  may then round the other way, so
+      |out - out_oracle| <= sum over fragile r of 2 ulp(P_r)
+                            + (N-1) ulp(sum_r |P_r|) + ulp(|res| + sum_r |P_r|);
+* the acceptance tolerance: relative L2 error <= 5e-3 over the whole
+  output, and max abs error <= 2e-2 over every output with no fragile
+  partial (there it is 0: bit-exact). On a fragile output the bound above
+  applies instead: one unit of a partial of magnitude >= 2 is already
+  2^-6 = 0.016, so no accumulation order other than the oracle's own can
+  keep such an output within 2e-2 everywhere. The largest error over all
+  outputs is reported.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import inputs, oracle_point
+from helpers import from_u16, u16
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [             # N, M, K, H
+    (4, 32, 512, 512),      # decode batch, token tile 32
+    (8, 64, 1024, 256),     # decode batch, token tile 64, N = 8
+    (2, 16, 128, 128),      # fewest tokens the tensor path takes
+    (4, 100, 640, 384),     # token tile 128 with a ragged tail; 3 weight tiles
+    (4, 300, 512, 256),     # token tile 256, two tiles, second ragged
+    (1, 48, 400, 200),      # N = 1; K/N = 400 ends in a partial 64-column block; H % 128 != 0
+]
+IDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in SHAPES]
+
+
+def _run(n, m, k, h, x, w, r):
+    import tensor_layer_reconciliation_b200 as tlr
+    plan = tlr.Plan(n, m, k, h, variant="tensor")
+    wp = plan.pack_weights(w)
+    out = plan.reconcile(x, wp, r)
+    parts = plan.partials(x, wp)
+    torch.cuda.synchronize()
+    assert plan.device_error_flags() == 0
+    return u16(out), u16(parts)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=IDS)
+def test_tensor_integer_exact(shape):
+    n, m, k, h = shape
+    dev = torch.device("cuda")
+    g = torch.Generator().manual_seed(sum(shape))
+    xi = torch.randint(-1, 2, (m, k), generator=g)
+    wi = torch.randint(-1, 2, (h, k), generator=g)
+    ri = torch.randint(-8, 9, (m, h), generator=g)
+    out, parts = _run(n, m, k, h, xi.to(dev, torch.bfloat16), wi.to(dev, torch.bfloat16),
+                      ri.to(dev, torch.bfloat16))
+    ref = oracle_point(n, h, xi.to(torch.bfloat16), wi.to(torch.bfloat16), ri.to(torch.bfloat16))
+    assert np.array_equal(parts, ref["partials"])
+    assert np.array_equal(out, ref["out"])
+    assert torch.equal(from_u16(out).long(), xi @ wi.T + ri)
+
+
+def bf16_ulp(a):
+    """Spacing of bf16 values at magnitude a (subnormal spacing below 2^-126)."""
+    a = np.maximum(np.asarray(a, dtype=np.float64), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def fragile_mask(p64, pabs):
+    e = pabs * 2.0 ** -19
+    lo = oracle.bf16_rne_f64(p64 - e)
+    hi = oracle.bf16_rne_f64(p64 + e)
+    return lo != hi
+
+
+def check_against_oracle(out, parts, ref, n):
+    p64, pabs = ref["p64"], ref["pabs"]
+    frag = fragile_mask(p64, pabs)
+    exact_p = oracle.bf16_rne_f64(p64)
+    # partials: bit-exact where not fragile, a neighbour of d where fragile
+    assert np.array_equal(parts[~frag], exact_p[~frag])
+    assert np.array_equal(ref["partials"][~frag], exact_p[~frag])
+    if frag.any():
+        lo = oracle.bf16_rne_f64(np.nextafter(p64[frag], -np.inf) - pabs[frag] * 2.0 ** -19)
+        hi = oracle.bf16_rne_f64(p64[frag] + pabs[frag] * 2.0 ** -19)
+        g = oracle.f32(parts[frag])
+        assert np.all((g >= oracle.f32(lo)) & (g <= oracle.f32(hi)))
+    # outputs
+    out_frag = frag.any(axis=0)
+    assert np.array_equal(out[~out_frag], ref["out"][~out_frag])
+    go, ro = oracle.f32(out).astype(np.float64), oracle.f32(ref["out"]).astype(np.float64)
+    pf = np.abs(oracle.f32(ref["partials"]).astype(np.float64))
+    res = np.abs(oracle.f32(ref["res"]).astype(np.float64))
+    bound = (2 * bf16_ulp(pf) * frag).sum(axis=0) + (n - 1) * bf16_ulp(pf.sum(axis=0)) \
+        + bf16_ulp(res + pf.sum(axis=0))
+    assert np.all(np.abs(go - ro)[out_frag] <= bound[out_frag])
+    # acceptance tolerance
+    diff = np.abs(go - ro)
+    rel_l2 = np.linalg.norm(go - ro) / max(np.linalg.norm(ro), 1e-30)
+    assert rel_l2 <= 5e-3
+    assert np.all(diff[~out_frag] <= 2e-2)
+    return int(frag.sum()), int(out_frag.sum()), float(diff.max()), float(rel_l2)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=IDS)
+def test_tensor_gaussian_fragile_rule(shape):
+    n, m, k, h = shape
+    dev = torch.device("cuda")
+    x, w, r = inputs(n, m, k, h, 500 + sum(shape), dev)
+    out, parts = _run(n, m, k, h, x, w, r)
+    ref = oracle_point(n, h, x.cpu(), w.cpu(), r.cpu())
+    ref["res"] = u16(r)
+    fp, fo, mx, rl2 = check_against_oracle(out, parts, ref, n)
+    print(f"{shape}: fragile partials {fp}, outputs touched {fo}, max abs {mx:.3g}, rel L2 {rl2:.3g}")
+
+
+def test_auto_uses_tensor_from_16_tokens():
+    import tensor_layer_reconciliation_b200 as tlr
+    plan = tlr.Plan(2, 64, 256, 128)                   # AUTO
+    assert plan.workspace_bytes(8) == 0                # exact, fused: no workspace
+    assert plan.workspace_bytes(16) == 2 * 16 * 128 * 2  # tensor: staged partials
