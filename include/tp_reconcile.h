@@ -129,6 +129,31 @@ TP_API tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, cons
                                  const void* residual, void* out, int64_t tokens,
                                  void* workspace, void* stream);
 
+/* One reconciliation point exactly like tp_rowlinear_reconcile (same
+ * arguments, same kernels, same result), for callers that cannot allocate
+ * device memory: code that runs while a CUDA graph is being captured
+ * (allocation is not an operation a capture can record), latency-critical
+ * decode loops (cudaMalloc may synchronize the device), and hosts whose
+ * device memory is budgeted up front by an embedding framework. Instead of a
+ * caller-supplied workspace, the partials that this call stages (the
+ * tensor-core variant, or a staged plan) go to a fixed scratch array inside
+ * the library: 16 MiB, a file-scope device array that every GPU loading the
+ * library holds until the process exits. Its device address is looked up
+ * once per device when a plan is created on it, so this call does no set-up
+ * of its own and allocates nothing.
+ *  - Returns TP_ERR_WORKSPACE, launching nothing, when the call needs more
+ *    scratch than that: tp_plan_workspace_bytes(plan, tokens) > 16 MiB
+ *    (N*M*H*2 bytes; e.g. N=8, M=64, H=4096 needs 4 MiB).
+ *  - Every call, from every plan and thread on a device, shares the one
+ *    array, which keeps the last call's partials; each call writes every
+ *    partial it reads, so nothing needs clearing. Calls whose kernels overlap
+ *    on the GPU (different streams without ordering between them) race on
+ *    the array and give wrong results: order them on one stream.
+ * The pages describe no counterpart of this entry point. */
+TP_API tp_status tp_rowlinear_reconcile_noalloc(const tp_plan* plan, const void* x,
+                                                const void* w_packed, const void* residual,
+                                                void* out, int64_t tokens, void* stream);
+
 /* S1 only: the N partials, no ring, no residual.
  *   partials  [N][M][H] bf16 (output)
  * Same x, w_packed and tokens rules as tp_rowlinear_reconcile. */

@@ -21,7 +21,8 @@ TP_VARIANT_AUTO, TP_VARIANT_EXACT, TP_VARIANT_TENSOR = 0, 1, 2
 EXPORTED = (
     "tp_plan_create", "tp_plan_set_variant", "tp_plan_workspace_bytes", "tp_plan_packed_bytes",
     "tp_pack_weights",
-    "tp_rowlinear_reconcile", "tp_rowlinear_partials", "tp_ring_reduce", "tp_ring_bytes",
+    "tp_rowlinear_reconcile", "tp_rowlinear_reconcile_noalloc", "tp_rowlinear_partials",
+    "tp_ring_reduce", "tp_ring_bytes",
     "tp_plan_destroy", "tp_status_string", "tp_last_cuda_error", "tp_device_error_flags",
 )
 
@@ -54,6 +55,8 @@ def _load() -> ctypes.CDLL:
     L.tp_pack_weights.restype = ctypes.c_int
     L.tp_rowlinear_reconcile.argtypes = [vp, vp, vp, vp, vp, i64, vp, vp]
     L.tp_rowlinear_reconcile.restype = ctypes.c_int
+    L.tp_rowlinear_reconcile_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, vp]
+    L.tp_rowlinear_reconcile_noalloc.restype = ctypes.c_int
     L.tp_rowlinear_partials.argtypes = [vp, vp, vp, vp, i64, vp]
     L.tp_rowlinear_partials.restype = ctypes.c_int
     L.tp_ring_reduce.argtypes = [vp, vp, vp, vp, i64, vp]
@@ -106,6 +109,12 @@ def tp_pack_weights(plan, w_hk: int, w_packed: int, stream: int) -> int:
 def tp_rowlinear_reconcile(plan, x: int, w_packed: int, residual: int, out: int, tokens: int,
                            workspace: int, stream: int) -> int:
     return LIB.tp_rowlinear_reconcile(plan, x, w_packed, residual, out, tokens, workspace, stream)
+
+
+def tp_rowlinear_reconcile_noalloc(plan, x: int, w_packed: int, residual: int, out: int,
+                                   tokens: int, stream: int) -> int:
+    """tp_rowlinear_reconcile with the library's fixed scratch instead of a workspace."""
+    return LIB.tp_rowlinear_reconcile_noalloc(plan, x, w_packed, residual, out, tokens, stream)
 
 
 def tp_rowlinear_partials(plan, x: int, w_packed: int, partials: int, tokens: int,

@@ -14,6 +14,12 @@
 #include "tp_kernels_tc.cuh"
 #include "tp_reconcile.h"
 
+// Fixed scratch for tp_rowlinear_reconcile_noalloc: the staged partials
+// (N * M * H bf16) of callers that cannot allocate device memory. Every GPU
+// that loads this library holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
 struct tp_plan {
     int n_ranks;
     int64_t max_tokens, k, hidden, ks, hc;
@@ -22,11 +28,32 @@ struct tp_plan {
     int smem_optin;
     int variant;
     int staged;
+    void* noalloc_scratch;  // device address of g_noalloc_scratch on this plan's device
 };
 
 namespace {
 
 thread_local int t_last_cuda_error = 0;
+
+// Device address of the no-alloc scratch array, looked up once per device
+// (cudaGetSymbolAddress with that device current). In host code the array's
+// name is only a host-side stand-in, never a device address.
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+cudaError_t noalloc_scratch_for(int dev, void** out) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = ptr;
+    }
+    *out = g_scratch_addr[dev];
+    return cudaSuccess;
+}
 
 tp_status cuda_fail(cudaError_t e) {
     t_last_cuda_error = static_cast<int>(e);
@@ -345,6 +372,8 @@ tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t
         return cuda_fail(e);
     int dyn_max = 0;
     if ((e = set_kernel_attrs(optin, &dyn_max)) != cudaSuccess) return cuda_fail(e);
+    void* scratch = nullptr;
+    if ((e = noalloc_scratch_for(dev, &scratch)) != cudaSuccess) return cuda_fail(e);
     tp_plan* p = new (std::nothrow) tp_plan{};
     if (!p) return TP_ERR_INVALID;
     p->n_ranks = n_ranks;
@@ -358,6 +387,7 @@ tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t
     p->smem_optin = dyn_max;
     p->variant = TP_VARIANT_AUTO;
     p->staged = 0;
+    p->noalloc_scratch = scratch;
     *out = p;
     return TP_OK;
 }
@@ -445,6 +475,16 @@ tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void*
     }
     if (st != TP_OK) return st;
     return launch_ring(plan, workspace, residual, out, tokens, s);
+}
+
+tp_status tp_rowlinear_reconcile_noalloc(const tp_plan* plan, const void* x, const void* w_packed,
+                                         const void* residual, void* out, int64_t tokens,
+                                         void* stream) {
+    if (!plan) return TP_ERR_INVALID;
+    if (tokens < 0 || tokens > plan->max_tokens) return TP_ERR_INVALID;
+    if (tp_plan_workspace_bytes(plan, tokens) > kNoAllocScratchBytes) return TP_ERR_WORKSPACE;
+    return tp_rowlinear_reconcile(plan, x, w_packed, residual, out, tokens,
+                                  plan->noalloc_scratch, stream);
 }
 
 tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* w_packed,
