@@ -14,6 +14,7 @@ inside each GPU), so there is no data-path collective and the scaling is weak.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import os
@@ -48,6 +49,32 @@ def _peaks():
                 "source": "fallback"}
 
 
+# DRAM bytes (read + write) per reconciliation call, averaged over the points
+# of a workload, from ncu captures of the kernels as they are built from the
+# sources whose digest is recorded; a digest that no longer matches the
+# sources means the kernels changed since, and the traffic is reported null.
+PROFILED_TRAFFIC = {
+    # (workload, path): (bytes per call, kernel-source digest, profile summary)
+}
+
+
+def _kernel_source_digest():
+    import hashlib
+    d = hashlib.sha256()
+    src = os.path.join(ROOT, "tensor_layer_reconciliation_b200", "csrc")
+    for name in sorted(os.listdir(src)):
+        with open(os.path.join(src, name), "rb") as f:
+            d.update(name.encode() + b"\0" + f.read())
+    return d.hexdigest()[:16]
+
+
+def _profiled_traffic(workload, path):
+    rec = PROFILED_TRAFFIC.get((workload, path))
+    if rec is None or rec[1] != _kernel_source_digest():
+        return None
+    return rec[0]
+
+
 # ------------------------------------------------------------------ workload --
 
 class Workload:
@@ -73,8 +100,8 @@ class Workload:
         self.out_all = torch.empty(cfg.n_points * m * h, dtype=torch.bfloat16, device=device)
         self.w_packed = []
         ws_need = max(pl.workspace_bytes(m) for pl in self.plans.values())
-        self.workspace = (torch.empty(ws_need, dtype=torch.uint8, device=device)
-                          if ws_need else None)
+        self.workspace = (torch.zeros(ws_need, dtype=torch.uint8, device=device)
+                          if ws_need else None)   # counter head zero on first use
         for i, p in enumerate(cfg.points):
             self.x(i).copy_(point_tensor(cfg, p, KIND_X, device))
             self.res(i).copy_(point_tensor(cfg, p, KIND_RESIDUAL, device))
@@ -101,9 +128,23 @@ class Workload:
             self.plans[p.k].reconcile(self.x(i), self.w_packed[i], self.res(i), out=self.out(i),
                                       workspace=self.workspace)
 
+    def run_eager(self):
+        """One step as plain calls of the public API, one per point."""
+        for i, p in enumerate(self.cfg.points):
+            self.plans[p.k].reconcile(self.x(i), self.w_packed[i], self.res(i), out=self.out(i),
+                                      workspace=self.workspace)
+
+    def path_name(self):
+        """Which kernels one call runs: 'tensor' (tensor-core partials, staged),
+        'exact-staged' or 'exact-fused'."""
+        pl = next(iter(self.plans.values()))
+        if pl.effective_variant(self.cfg.tokens) == "tensor":
+            return "tensor"
+        return "exact-staged" if pl.staged else "exact-fused"
+
     def launches_per_step(self):
-        per = 2 if next(iter(self.plans.values())).staged else 1
-        return per * self.cfg.n_points
+        staged = any(pl.workspace_bytes(self.cfg.tokens) for pl in self.plans.values())
+        return (2 if staged else 1) * self.cfg.n_points
 
     def capture(self):
         g = torch.cuda.CUDAGraph()
@@ -242,6 +283,12 @@ def _max_over_ranks(v, world, device):
     return float(t.item())
 
 
+def _job_rate(units_per_rank, ms_per_step_max, world):
+    """Whole-job rate: every rank's units of one step over the slowest rank's
+    step time (weak scaling, one replica per rank)."""
+    return units_per_rank * world / (ms_per_step_max * 1e-3)
+
+
 def _barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -290,6 +337,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=8.0)
+    ap.add_argument("--points", type=int, default=0,
+                    help="run only the first P points of the workload (small profiling cases)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -308,6 +357,9 @@ def main(argv=None):
                                 device_id=device)
 
     cfg = get_config(args.config)
+    if args.points:
+        cfg = dataclasses.replace(cfg, layers=1, layer_points=cfg.layer_points)
+        cfg.points[:] = cfg.points[:args.points]
     wl = Workload(cfg, device, variant=args.variant, staged=args.staged)
     peaks = _peaks()
 
@@ -332,7 +384,11 @@ def main(argv=None):
     step_ms = _max_over_ranks(step_ms, world, device)
     clocks = clk.summary()
 
-    # ---- per-launch durations of the dominant kernel (events around each call)
+    # ---- per-call durations outside a graph (for reference only) ---------
+    # Each call is the hot path of one point: the partial kernel (fused with the
+    # fold on the exact path) and, on staged paths, the ring fold kernel. Eager
+    # launches add host gaps between calls; the roofline uses the graph time.
+    staged_path = any(pl.workspace_bytes(cfg.tokens) for pl in wl.plans.values())
     per_launch = []
     for _ in range(2):
         evs = []
@@ -345,29 +401,32 @@ def main(argv=None):
             evs.append((a, b))
         torch.cuda.synchronize(device)
         per_launch.append([a.elapsed_time(b) for a, b in evs])
-    call_ms = np.mean(np.array(per_launch), axis=0)      # per point, ms
+    call_ms_eager = np.mean(np.array(per_launch), axis=0)      # per point, ms
 
     # ---- end to end through the public API with host buffers -------------
+    # Every step: x and residual of all points host->device (pinned), one
+    # reconcile call per point through the C ABI (no graph), outputs back.
     x_host = torch.empty(wl.x_all.shape, dtype=torch.bfloat16, pin_memory=True)
     r_host = torch.empty(wl.res_all.shape, dtype=torch.bfloat16, pin_memory=True)
     o_host = torch.empty(wl.out_all.shape, dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(wl.x_all.cpu())
     r_host.copy_(wl.res_all.cpu())
     e2e_steps = max(3, min(args.steps, 10))
-    for _ in range(2):
+
+    def e2e_step():
         wl.x_all.copy_(x_host, non_blocking=True)
         wl.res_all.copy_(r_host, non_blocking=True)
-        graph.replay()
+        wl.run_eager()
         o_host.copy_(wl.out_all, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
     torch.cuda.synchronize(device)
     _barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        wl.x_all.copy_(x_host, non_blocking=True)
-        wl.res_all.copy_(r_host, non_blocking=True)
-        graph.replay()
-        o_host.copy_(wl.out_all, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, device)
@@ -375,27 +434,35 @@ def main(argv=None):
     d2h = wl.out_all.numel() * 2
 
     # ---- numbers ---------------------------------------------------------
-    staged = args.staged
-    tokens_per_step = cfg.tokens * world
-    value = tokens_per_step / (step_ms * 1e-3)
-    recon = cfg.n_points * world / (step_ms * 1e-3)
-    alg_bytes = cfg.algorithmic_bytes(staged_partials=staged)
+    value = _job_rate(cfg.tokens, step_ms, world)
+    recon = _job_rate(cfg.n_points, step_ms, world)
+    step_bytes = cfg.algorithmic_bytes(staged_partials=staged_path)
     flops = cfg.flops()
     tensor_bound = cfg.tokens >= 1024
-    kernel_ms = float(np.sum(call_ms))
+    # The hot path of one point is one reconciliation call: the partial kernel
+    # and, on staged paths, the ring fold kernel, chained by programmatic
+    # dependent launch inside the graph. Its average duration is the graph's
+    # device time over the timed region divided by the points per step.
+    call_ms = step_ms / cfg.n_points
+    kern_bytes = step_bytes   # weights, activations, residual, output (+ staged partials)
+    kern_name = ("reconciliation call: tc_partial_kernel then ring fold kernel" if staged_path
+                 else "reconciliation call: exact_partial_kernel (partials + ring fold + residual)")
     if tensor_bound:
-        achieved = flops / (kernel_ms * 1e-3) / 1e12
+        achieved = flops / (step_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None}
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
     else:
-        achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
+        achieved = kern_bytes / (step_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None}
-    roof["peak_source"] = peaks["source"]
-    roof["kernel"] = "exact_partial_kernel (fused partials + ring fold + residual)" if not staged \
-        else "exact_partial_kernel + ring_reduce_kernel"
-    roof["launch_ms_mean"] = kernel_ms / cfg.n_points
-    roof["algorithmic_bytes_per_step"] = alg_bytes
+                "frac": achieved / peaks["hbm_gbs"]}
+    roof["traffic"] = _profiled_traffic(cfg.name, wl.path_name())
+    roof["traffic_unit"] = "bytes per call (DRAM read + write, ncu), averaged over the points"
+    roof["peak_source"] = peaks["source"] + " (burst: the step is timed alone)"
+    roof["kernel"] = kern_name
+    roof["call_ms_mean"] = call_ms
+    roof["call_ms_mean_eager"] = float(np.mean(call_ms_eager))
+    roof["algorithmic_bytes_per_call"] = kern_bytes / cfg.n_points
+    roof["algorithmic_flops_per_call"] = flops / cfg.n_points
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -403,17 +470,19 @@ def main(argv=None):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Philox4x32-10, Gaussian by 2^16-point inverse CDF)",
         "reconciliations_per_s": recon,
-        "hbm_gbs_step": alg_bytes * world / (step_ms * 1e-3) / 1e9 / world,
+        "hbm_gbs_step": step_bytes / (step_ms * 1e-3) / 1e9,
+        "tflops_step": flops / (step_ms * 1e-3) / 1e12,
         "config": {"workload": cfg.name, "n_ranks": cfg.n_ranks, "tokens": cfg.tokens,
                    "hidden": cfg.hidden, "points": cfg.n_points,
                    "weights_gb_per_step": cfg.weight_bytes() / 1e9,
                    "l2": "no flush: every step streams all points' distinct weights "
                          f"({cfg.weight_bytes() / 1e9:.1f} GB), larger than the 126 MB L2",
-                   "variant": args.variant, "staged": staged,
+                   "variant": args.variant, "staged_partials": staged_path,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof,
-        "e2e": {"value": tokens_per_step / (e2e_ms * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "e2e": {"value": _job_rate(cfg.tokens, e2e_ms, world), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "mode": "pinned host copies + one C-ABI reconcile call per point, no graph"},
         "gpu_launches": wl.launches_per_step() * args.steps,
         "clocks": clocks,
     }

@@ -68,7 +68,7 @@ typedef enum {
 enum { TP_BF16 = 0 };
 
 typedef enum {
-    TP_VARIANT_AUTO = 0,   /* EXACT below 16 tokens, TENSOR from 16 tokens on */
+    TP_VARIANT_AUTO = 0,   /* TENSOR (the fastest on B200 at every token count) */
     TP_VARIANT_EXACT = 1,  /* CUDA cores, fp32 FMA chain per partial, k ascending */
     TP_VARIANT_TENSOR = 2  /* tcgen05 tensor cores, fp32 accumulate in TMEM */
 } tp_variant;
@@ -86,20 +86,28 @@ typedef enum {
 TP_API tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t k,
                          int64_t hidden, int dtype);
 
-/* Chooses the partial kernel and whether the partials are staged.
+/* Chooses the partial kernel and, for EXACT, whether the partials are staged.
  *   variant  a tp_variant
- *   staged   0: the partials stay on chip and one kernel does partials, ring
- *            fold and residual add (no workspace); 1: the partial kernel
- *            writes all N partials to the workspace and a separate ring
- *            kernel (tp_ring_reduce's) folds them.
+ *   staged   EXACT: 0 keeps the partials on chip, one kernel doing partials,
+ *            ring fold and residual add (no workspace); 1 writes all N
+ *            partials to the workspace and a separate ring kernel
+ *            (tp_ring_reduce's) folds them. TENSOR always stages its
+ *            partials and folds them in a separate ring kernel.
  * Call before the plan is shared between threads. */
 TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
 
 /* Bytes of workspace tp_rowlinear_reconcile needs for `tokens` tokens with
- * the plan's current setting: N*M*H*2 rounded up to 256 when the partials go
- * through memory (staged, or the tensor-core variant, which always stages
- * them), else 0. Returns 0 for a null plan. */
+ * the plan's current setting; 0 when the partials stay on chip (EXACT, not
+ * staged). The tensor-core variant always sends its partials through the
+ * workspace: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of K parts)
+ * when it splits K across CTAs to fill the SMs; rounded up to 256. Returns 0
+ * for a null plan. */
 TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
+
+/* The partial kernel a call with `tokens` tokens runs under the plan's
+ * current setting: TP_VARIANT_EXACT or TP_VARIANT_TENSOR (AUTO resolved).
+ * Returns -1 for a null plan or tokens < 1. A query only; launches nothing. */
+TP_API int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens);
 
 /* Bytes of the packed weight buffer tp_pack_weights writes: N*H*(K/N)*2,
  * the size of the Linear weight. Returns 0 for a null plan. */

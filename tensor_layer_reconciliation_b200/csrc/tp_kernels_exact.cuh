@@ -270,6 +270,60 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// S2-S4 over k-split partials: rank r's partial is first assembled as
+// bf16_rne(part_0 + part_1 + ... ) -- the fp32 sums of its K parts added in
+// split order -- then folded in ring order as above.
+__global__ void __launch_bounds__(256)
+    ring_reduce_splits_kernel(const float* __restrict__ parts, int splits,
+                              const uint16_t* __restrict__ residual, uint16_t* __restrict__ out,
+                              int n_ranks, int64_t tokens, int hidden, int hc) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int64_t hv = hidden >> 3;
+    const int64_t total = tokens * hv;
+    const size_t plane = static_cast<size_t>(tokens) * hidden;
+    for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < total;
+         v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t m = v / hv;
+        const int h = static_cast<int>(v - m * hv) << 3;
+        const int c = h / hc;
+        const size_t off = static_cast<size_t>(m) * hidden + h;
+        uint16_t s[8];
+        for (int i = 0; i < n_ranks; ++i) {
+            int rr = c + i;
+            if (rr >= n_ranks) rr -= n_ranks;
+            float a[8];
+            {
+                const float4* src = reinterpret_cast<const float4*>(parts + static_cast<size_t>(rr) * plane + off);
+                const float4 lo = src[0], hi = src[1];
+                a[0] = lo.x; a[1] = lo.y; a[2] = lo.z; a[3] = lo.w;
+                a[4] = hi.x; a[5] = hi.y; a[6] = hi.z; a[7] = hi.w;
+            }
+            for (int sp = 1; sp < splits; ++sp) {
+                const float4* src = reinterpret_cast<const float4*>(
+                    parts + (static_cast<size_t>(sp) * n_ranks + rr) * plane + off);
+                const float4 lo = src[0], hi = src[1];
+                a[0] = __fadd_rn(a[0], lo.x); a[1] = __fadd_rn(a[1], lo.y);
+                a[2] = __fadd_rn(a[2], lo.z); a[3] = __fadd_rn(a[3], lo.w);
+                a[4] = __fadd_rn(a[4], hi.x); a[5] = __fadd_rn(a[5], hi.y);
+                a[6] = __fadd_rn(a[6], hi.z); a[7] = __fadd_rn(a[7], hi.w);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint16_t pr = f32_to_bf16_rne(a[e]);
+                s[e] = i == 0 ? pr : bf16_add(s[e], pr);
+            }
+        }
+        const uint4 rv = ld_global_nc_v4(residual + off);
+        uint4 o;
+        o.x = bf16_add(rv.x & 0xFFFF, s[0]) | (static_cast<uint32_t>(bf16_add(rv.x >> 16, s[1])) << 16);
+        o.y = bf16_add(rv.y & 0xFFFF, s[2]) | (static_cast<uint32_t>(bf16_add(rv.y >> 16, s[3])) << 16);
+        o.z = bf16_add(rv.z & 0xFFFF, s[4]) | (static_cast<uint32_t>(bf16_add(rv.z >> 16, s[5])) << 16);
+        o.w = bf16_add(rv.w & 0xFFFF, s[6]) | (static_cast<uint32_t>(bf16_add(rv.w >> 16, s[7])) << 16);
+        st_global_v4(out + off, o);
+    }
+}
+
 // --------------------------------------------------------------------- S0 --
 // Linear weight [H][K] -> [N][H][K/N]: shard r is columns r*Ks .. r*Ks+Ks-1.
 __global__ void __launch_bounds__(256)

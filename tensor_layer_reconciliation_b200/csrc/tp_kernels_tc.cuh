@@ -4,7 +4,7 @@
 // result over its slice of the weight matrix; prefill runs every position
 // of the prompt at once, which makes the partial a dense contraction.
 //
-// Work unit = (rank r, 128 rows of H, BN tokens): the tile
+// Work unit = (rank r, 128 rows of H, BN tokens, k-split s): the tile
 //     P[r][m0 .. m0+BN)[h0 .. h0+128) = x_r[m0 ..][:] . W_r[h0 ..][:]^T
 // computed as D = A * B^T on tcgen05 with A = the 128 x 64 weight block
 // (rows of W_r, K-major) and B = the BN x 64 activation block (rows of x_r,
@@ -25,6 +25,15 @@
 //   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, one
 //              round-to-nearest-even to bf16 per partial, stores to the
 //              partial buffer [N][M][H] (32 consecutive h per warp store).
+// When there are fewer units than SMs (few ranks, small H) the K range of
+// each unit is split in SPLITS contiguous parts handled by different CTAs;
+// each part's fp32 sum is stored unrounded in [SPLITS][N][M][H] and the
+// ring kernel adds the parts in split order before the one rounding to bf16.
+// Units run token tile fastest, so CTAs working at the same time share each
+// weight tile through L2 (prefill reads every weight tile for 16 token tiles).
+// The ring fold stays a kernel of its own: folding inside the CTA that
+// completes a tile (measured) serialises N * SPLITS * 128 * BN reads behind
+// that CTA's next accumulator and is slower for every token count above one.
 // Accumulation order inside the tensor core is the hardware's; the partial
 // is the fp32 sum rounded once to bf16, like the oracle's, but only equal to
 // it where the two fp32 sums round to the same bf16 value.
@@ -47,9 +56,11 @@ struct TcParams {
     int tokens;    // M
     int h_tiles;   // ceil(H / 128)
     int m_tiles;   // ceil(M / BN)
-    int units;     // N * h_tiles * m_tiles
+    int splits;    // k-splits per (rank, h tile, m tile)
+    int units;     // N * h_tiles * m_tiles * splits
     int stages;    // 2 .. kTcMaxStages
-    uint16_t* partials;  // [N][M][H]
+    uint16_t* partials;     // [N][M][H] bf16 (splits == 1)
+    float* partials_f32;    // [splits][N][M][H] fp32 sums of each k part (splits > 1)
 };
 
 template <int BN>
@@ -80,16 +91,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int my_units = p.units > static_cast<int>(blockIdx.x)
                              ? (p.units - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                              : 0;
-    const int iters = my_units * nkb;
-    // unit index -> (rank, h tile, m tile); ranks innermost
-    auto unit_of = [&](int lu, int& r, int& ht, int& mt) {
+    // unit index -> (rank, h tile, m tile, split); token tile fastest
+    auto unit_of = [&](int lu, int& r, int& ht, int& mt, int& sp) {
         const int u = static_cast<int>(blockIdx.x) + lu * static_cast<int>(gridDim.x);
-        r = u % p.n_ranks;
-        const int rest = u / p.n_ranks;
-        ht = rest % p.h_tiles;
-        mt = rest / p.h_tiles;
+        mt = u % p.m_tiles;
+        int t = u / p.m_tiles;
+        sp = t % p.splits;
+        t /= p.splits;
+        ht = t % p.h_tiles;
+        r = t / p.h_tiles;
     };
-
+    // k-blocks [kb_lo, kb_hi) of split sp
+    auto split_range = [&](int sp, int& kb_lo, int& kb_hi) {
+        kb_lo = sp * nkb / p.splits;
+        kb_hi = (sp + 1) * nkb / p.splits;
+    };
     if (threadIdx.x == 0) {
         abort_flag = 0;
         for (int s = 0; s < S; ++s) {
@@ -119,38 +135,53 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_prefetch_desc(&tmap_w);
             tma_prefetch_desc(&tmap_x);
             const uint32_t tx = kTcATile + kBTile;
-            auto load_a = [&](int i, int s) {
-                int r, ht, mt;
-                unit_of(i / nkb, r, ht, mt);
-                tma_load_3d(a_ring + static_cast<size_t>(s) * kTcATile, &tmap_w, &full[s],
-                            (i % nkb) * kTcKBlock, ht * kTcRows, r);
+            // Walk (unit, k-block) in issue order.
+            int lu = 0, kb = 0, kb_hi = 0, r = 0, ht = 0, mt = 0, sp = 0;
+            auto enter_unit = [&]() {
+                if (lu < my_units) {
+                    unit_of(lu, r, ht, mt, sp);
+                    split_range(sp, kb, kb_hi);
+                }
             };
-            auto load_b = [&](int i, int s) {
-                int r, ht, mt;
-                unit_of(i / nkb, r, ht, mt);
-                tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, &full[s],
-                            (i % nkb) * kTcKBlock, r, mt * BN);
+            auto advance = [&]() {
+                if (++kb == kb_hi) {
+                    ++lu;
+                    enter_unit();
+                }
             };
-            const int pre = iters < S ? iters : S;
-            for (int i = 0; i < pre; ++i) {
-                mbar_arrive_expect_tx(&full[i], tx);
-                load_a(i, i);
+            enter_unit();
+            int pre_r[kTcMaxStages], pre_mt[kTcMaxStages], pre_kb[kTcMaxStages];
+            int pre = 0;
+            while (pre < S && lu < my_units) {
+                mbar_arrive_expect_tx(&full[pre], tx);
+                tma_load_3d(a_ring + static_cast<size_t>(pre) * kTcATile, &tmap_w, &full[pre],
+                            kb * kTcKBlock, ht * kTcRows, r);
+                pre_r[pre] = r;
+                pre_mt[pre] = mt;
+                pre_kb[pre] = kb;
+                ++pre;
+                advance();
             }
             pdl_wait();  // activations may be produced by the previous kernel
-            for (int i = 0; i < pre; ++i) load_b(i, i);
+            for (int i = 0; i < pre; ++i)
+                tma_load_3d(b_ring + static_cast<size_t>(i) * kBTile, &tmap_x, &full[i],
+                            pre_kb[i] * kTcKBlock, pre_r[i], pre_mt[i] * BN);
             int issued = pre;
             int s = pre % S;
             uint32_t phase = pre >= S ? 1u : 0u;   // parity of slot s's next fill
-            for (int i = pre; i < iters; ++i) {
+            while (lu < my_units) {
                 if (!mbar_wait_bounded(&empty[s], phase ^ 1u)) {
                     atomicExch(&abort_flag, 1);
                     break;
                 }
                 if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
                 mbar_arrive_expect_tx(&full[s], tx);
-                load_a(i, s);
-                load_b(i, s);
-                issued = i + 1;
+                tma_load_3d(a_ring + static_cast<size_t>(s) * kTcATile, &tmap_w, &full[s],
+                            kb * kTcKBlock, ht * kTcRows, r);
+                tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, &full[s],
+                            kb * kTcKBlock, r, mt * BN);
+                ++issued;
+                advance();
                 if (++s == S) {
                     s = 0;
                     phase ^= 1u;
@@ -174,8 +205,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t d = tmem_base + static_cast<uint32_t>(b * BN);
+                int r, ht, mt, sp, kb_lo, kb_hi;
+                unit_of(lu, r, ht, mt, sp);
+                split_range(sp, kb_lo, kb_hi);
                 bool ok = true;
-                for (int kb = 0; kb < nkb; ++kb, ++i) {
+                for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
                     const int s = i % S;
                     if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / S) & 1u)) {
                         ok = false;
@@ -186,7 +220,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const uint64_t bd = smem_desc_k128(b_ring + static_cast<size_t>(s) * kBTile);
 #pragma unroll
                     for (int kk = 0; kk < kTcKBlock / 16; ++kk)
-                        umma_bf16(d, ad + 2ull * kk, bd + 2ull * kk, kIdesc, (kb | kk) != 0);
+                        umma_bf16(d, ad + 2ull * kk, bd + 2ull * kk, kIdesc,
+                                  (kb != kb_lo) || (kk != 0));
                     umma_commit(&empty[s]);  // frees the stage when these MMAs finish
                 }
                 if (!ok) {
@@ -205,16 +240,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int lu = 0; lu < my_units; ++lu) {
             const int b = lu & 1;
             const uint32_t aph = static_cast<uint32_t>(lu >> 1) & 1u;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&acc_full[b], aph))) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&acc_full[b], aph)))
                 atomicExch(&abort_flag, 1);
-                break;
-            }
+            // The four epilogue warps leave together.
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
             tc_fence_after_sync();
-            int r, ht, mt;
-            unit_of(lu, r, ht, mt);
+            int r, ht, mt, sp;
+            unit_of(lu, r, ht, mt, sp);
             const int h = ht * kTcRows + q * 32 + lane;
             const int m0 = mt * BN;
-            uint16_t* dst = p.partials + static_cast<size_t>(r) * p.tokens * p.hidden + h;
+            const size_t plane = static_cast<size_t>(p.tokens) * p.hidden;
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
@@ -222,12 +258,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                    static_cast<uint32_t>(b * BN + c0),
                                v);
                 if (h < p.hidden) {
+                    if (p.splits == 1) {
+                        uint16_t* dst = p.partials + static_cast<size_t>(r) * plane + h;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int m = m0 + c0 + i;
-                        if (m < p.tokens)
-                            dst[static_cast<size_t>(m) * p.hidden] =
-                                f32_to_bf16_rne(__uint_as_float(v[i]));
+                        for (int i = 0; i < 32; ++i) {
+                            const int m = m0 + c0 + i;
+                            if (m < p.tokens)
+                                dst[static_cast<size_t>(m) * p.hidden] =
+                                    f32_to_bf16_rne(__uint_as_float(v[i]));
+                        }
+                    } else {
+                        float* dst = p.partials_f32 +
+                                     (static_cast<size_t>(sp) * p.n_ranks + r) * plane + h;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int m = m0 + c0 + i;
+                            if (m < p.tokens) dst[static_cast<size_t>(m) * p.hidden] = __uint_as_float(v[i]);
+                        }
                     }
                 }
             }

@@ -222,22 +222,22 @@ tp_status launch_exact(const tp_plan* p, const void* x, const void* w, const voi
 // -------------------------------------------------------- tensor variant --
 
 struct TcConfig {
-    int bn, stages, grid, units, h_tiles, m_tiles;
+    int bn, stages, grid, units, h_tiles, m_tiles, splits;
     size_t smem;
 };
 
-constexpr int64_t kTensorMinTokens = 16;     // AUTO uses the tensor cores from here
+constexpr int64_t kTensorMinTokens = 1;      // AUTO uses the tensor cores from here
 
 int tc_token_tile(int64_t tokens) {
     return tokens <= 32 ? 32 : tokens <= 64 ? 64 : tokens <= 128 ? 128 : 256;
 }
 
-TcConfig tc_config(const tp_plan* p, int64_t tokens) {
+TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split) {
     TcConfig c{};
     c.bn = tc_token_tile(tokens);
     c.h_tiles = static_cast<int>((p->hidden + tpr::kTcRows - 1) / tpr::kTcRows);
     c.m_tiles = static_cast<int>((tokens + c.bn - 1) / c.bn);
-    c.units = p->n_ranks * c.h_tiles * c.m_tiles;
+    const int base_units = p->n_ranks * c.h_tiles * c.m_tiles;
     const size_t stage = tpr::kTcATile + static_cast<size_t>(c.bn) * tpr::kTcKBlock * 2;
     const size_t fixed = (2 * tpr::kTcMaxStages + 5) * sizeof(uint64_t) + 16 + 1024;
     // Small token tiles stream weights: two CTAs per SM (about 100 KB each,
@@ -248,6 +248,12 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens) {
     c.stages = static_cast<int>(std::min<size_t>(tpr::kTcMaxStages, (budget - fixed) / stage));
     c.smem = fixed + static_cast<size_t>(c.stages) * stage;
     const int slots = p->sm_count * (two_per_sm ? 2 : 1);
+    // Fewer units than SMs: split K so every SM streams weights.
+    const int nkb = static_cast<int>((p->ks + tpr::kTcKBlock - 1) / tpr::kTcKBlock);
+    c.splits = 1;
+    if (allow_split && base_units < p->sm_count)
+        c.splits = std::max(1, std::min({slots / base_units, nkb, 8}));
+    c.units = base_units * c.splits;
     c.grid = std::min(c.units, slots);
     return c;
 }
@@ -284,9 +290,11 @@ tp_status encode_tc_maps(const tp_plan* p, const TcConfig& c, const void* x, con
     return TP_OK;
 }
 
+// The tensor-core partials: bf16 [N][M][H] when the units are not split, or
+// fp32 k-part sums [splits][N][M][H] (allow_split) for the ring kernel to add.
 tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partials, int64_t tokens,
-                    cudaStream_t stream) {
-    const TcConfig c = tc_config(p, tokens);
+                    bool allow_split, cudaStream_t stream) {
+    const TcConfig c = tc_config(p, tokens, allow_split);
     if (c.stages < 2) return TP_ERR_UNSUPPORTED;
     CUtensorMap mw, mx;
     tp_status st = encode_tc_maps(p, c, x, w, tokens, &mw, &mx);
@@ -298,9 +306,11 @@ tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partia
     prm.tokens = static_cast<int>(tokens);
     prm.h_tiles = c.h_tiles;
     prm.m_tiles = c.m_tiles;
+    prm.splits = c.splits;
     prm.units = c.units;
     prm.stages = c.stages;
     prm.partials = static_cast<uint16_t*>(partials);
+    prm.partials_f32 = static_cast<float*>(partials);
     const dim3 grid(c.grid), block(tpr::kTcThreads);
     cudaError_t e;
     switch (c.bn) {
@@ -309,6 +319,17 @@ tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partia
         case 128: e = launch_pdl(tpr::tc_partial_kernel<128>, grid, block, c.smem, stream, mw, mx, prm); break;
         default: e = launch_pdl(tpr::tc_partial_kernel<256>, grid, block, c.smem, stream, mw, mx, prm); break;
     }
+    return e == cudaSuccess ? TP_OK : cuda_fail(e);
+}
+
+tp_status launch_ring_splits(const tp_plan* p, const void* parts, int splits, const void* residual,
+                             void* out, int64_t tokens, cudaStream_t stream) {
+    const int64_t total = tokens * (p->hidden / 8);
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(p->sm_count) * 8);
+    cudaError_t e = launch_pdl(tpr::ring_reduce_splits_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256),
+                               0, stream, static_cast<const float*>(parts), splits,
+                               static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out),
+                               p->n_ranks, tokens, static_cast<int>(p->hidden), static_cast<int>(p->hc));
     return e == cudaSuccess ? TP_OK : cuda_fail(e);
 }
 
@@ -402,20 +423,30 @@ tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged) {
     return TP_OK;
 }
 
-// AUTO: the k-ascending CUDA-core chain for few tokens (a memory-bound
-// weight stream either way), the tensor cores from kTensorMinTokens on.
+// AUTO: the tensor cores (fastest at every token count measured on B200,
+// including single-token decode, where a 32-token tile is padded but the
+// point is bound by the weight stream). EXACT stays selectable: its partials
+// are the k-ascending fp32 sums bit for bit.
 static int effective_variant(const tp_plan* plan, int64_t tokens) {
     if (plan->variant == TP_VARIANT_AUTO)
         return tokens >= kTensorMinTokens ? TP_VARIANT_TENSOR : TP_VARIANT_EXACT;
     return plan->variant;
 }
 
+int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens) {
+    if (!plan || tokens < 1) return -1;
+    return effective_variant(plan, tokens);
+}
+
 size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens) {
     if (!plan || tokens <= 0) return 0;
-    // The tensor-core partials always go through the workspace.
-    if (!plan->staged && effective_variant(plan, tokens) != TP_VARIANT_TENSOR) return 0;
+    // The tensor-core partials always go through the workspace, as fp32 k-part
+    // sums when the units are split.
+    const bool tensor = effective_variant(plan, tokens) == TP_VARIANT_TENSOR;
+    if (!plan->staged && !tensor) return 0;
+    const int splits = tensor ? tc_config(plan, tokens, true).splits : 1;
     const size_t b = static_cast<size_t>(plan->n_ranks) * static_cast<size_t>(tokens) *
-                     static_cast<size_t>(plan->hidden) * 2;
+                     static_cast<size_t>(plan->hidden) * (splits > 1 ? 4u * splits : 2u);
     return (b + 255) / 256 * 256;
 }
 
@@ -467,7 +498,10 @@ tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void*
     const int variant = effective_variant(plan, tokens);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (variant == TP_VARIANT_TENSOR) {
-        st = launch_tc(plan, x, w_packed, workspace, tokens, s);
+        st = launch_tc(plan, x, w_packed, workspace, tokens, true, s);
+        const int splits = tc_config(plan, tokens, true).splits;
+        if (st == TP_OK && splits > 1)
+            return launch_ring_splits(plan, workspace, splits, residual, out, tokens, s);
     } else {
         if (!plan->staged)
             return launch_exact(plan, x, w_packed, residual, out, nullptr, tokens, true, s);
@@ -501,7 +535,7 @@ tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* 
     if ((st = check_device(plan)) != TP_OK) return st;
     const int variant = effective_variant(plan, tokens);
     if (variant == TP_VARIANT_TENSOR)
-        return launch_tc(plan, x, w_packed, partials, tokens, static_cast<cudaStream_t>(stream));
+        return launch_tc(plan, x, w_packed, partials, tokens, false, static_cast<cudaStream_t>(stream));
     return launch_exact(plan, x, w_packed, nullptr, nullptr, partials, tokens, false,
                         static_cast<cudaStream_t>(stream));
 }

@@ -75,6 +75,13 @@ class Plan:
     def workspace_bytes(self, tokens: int) -> int:
         return _lib.tp_plan_workspace_bytes(self._h, tokens)
 
+    def effective_variant(self, tokens: int) -> str:
+        """'exact' or 'tensor': the partial kernel a call with this many tokens runs."""
+        v = _lib.tp_plan_kernel_variant(self._h, tokens)
+        if v < 0:
+            raise ValueError("tokens must be >= 1")
+        return "tensor" if v == _lib.TP_VARIANT_TENSOR else "exact"
+
     @property
     def packed_numel(self) -> int:
         """bf16 elements of the packed weight buffer (tiled shards, see tp_reconcile.h)."""

@@ -105,7 +105,7 @@ def test_guard_zones_untouched(dev):
     import tensor_layer_reconciliation_b200 as tlr
     n, m, k, h = 2, 3, 400, 1200
     x, w, r = inputs(n, m, k, h, 6, dev)
-    plan = tlr.Plan(n, m, k, h, staged=True)
+    plan = tlr.Plan(n, m, k, h, variant="exact", staged=True)
     wp = plan.pack_weights(w)
     g = 4096
     sentinel = torch.tensor(0x7BCD, dtype=torch.int16)

@@ -41,7 +41,9 @@ pytestmark = pytest.mark.gpu
 SHAPES = [             # N, M, K, H
     (4, 32, 512, 512),      # decode batch, token tile 32
     (8, 64, 1024, 256),     # decode batch, token tile 64, N = 8
-    (2, 16, 128, 128),      # fewest tokens the tensor path takes
+    (2, 16, 128, 128),      # 16 tokens in a 32-token tile
+    (2, 1, 8192, 512),      # one token: K split 8 ways across CTAs (fp32 parts)
+    (4, 3, 2048, 640),      # three tokens, K split, H % 128 != 0
     (4, 100, 640, 384),     # token tile 128 with a ragged tail; 3 weight tiles
     (4, 300, 512, 256),     # token tile 256, two tiles, second ragged
     (1, 48, 400, 200),      # N = 1; K/N = 400 ends in a partial 64-column block; H % 128 != 0
@@ -130,8 +132,13 @@ def test_tensor_gaussian_fragile_rule(shape):
     print(f"{shape}: fragile partials {fp}, outputs touched {fo}, max abs {mx:.3g}, rel L2 {rl2:.3g}")
 
 
-def test_auto_uses_tensor_from_16_tokens():
+def test_auto_uses_tensor_cores():
     import tensor_layer_reconciliation_b200 as tlr
     plan = tlr.Plan(2, 64, 256, 128)                   # AUTO
-    assert plan.workspace_bytes(8) == 0                # exact, fused: no workspace
-    assert plan.workspace_bytes(16) == 2 * 16 * 128 * 2  # tensor: staged partials
+    assert plan.effective_variant(1) == "tensor"
+    assert plan.effective_variant(64) == "tensor"
+    assert plan.workspace_bytes(1) > 0                 # tensor: staged partials
+    plan.set_variant("exact")
+    assert plan.effective_variant(1) == "exact"
+    assert plan.workspace_bytes(1) == 0                # exact, fused: no workspace
+    assert tlr.tp_plan_kernel_variant(plan.handle, 0) == -1
