@@ -229,10 +229,15 @@ __global__ void __launch_bounds__(kMaxExactThreads, 1)
 }
 
 // ------------------------------------------------------------------ S2-S4 --
+constexpr int kMaxRanks = 8;     // tp_plan_create accepts 1 .. 8 ranks
+constexpr int kMaxSplits = 8;    // k-splits of the tensor-core partials
+
 // Ring reduce-scatter fold over partials staged in memory, the all-gather
 // (one result buffer stands for every rank's copy) and the residual add.
 // Thread per 8 consecutive columns (16-byte vectors; H/N % 8 == 0 keeps a
-// vector inside one chunk), grid-stride.
+// vector inside one chunk), grid-stride. The N partial vectors of a thread
+// are all loaded before the first add (the rank loop is unrolled to the
+// largest N), so their memory latencies overlap instead of adding up.
 __global__ void __launch_bounds__(256)
     ring_reduce_kernel(const uint16_t* __restrict__ partials, const uint16_t* __restrict__ residual,
                        uint16_t* __restrict__ out, int n_ranks, int64_t tokens, int hidden, int hc) {
@@ -247,20 +252,29 @@ __global__ void __launch_bounds__(256)
         const int h = static_cast<int>(v - m * hv) << 3;
         const int c = h / hc;
         const size_t off = static_cast<size_t>(m) * hidden + h;
-        uint4 a = ld_global_nc_v4(partials + static_cast<size_t>(c) * plane + off);
-        uint16_t s[8];
-        s[0] = a.x & 0xFFFF; s[1] = a.x >> 16; s[2] = a.y & 0xFFFF; s[3] = a.y >> 16;
-        s[4] = a.z & 0xFFFF; s[5] = a.z >> 16; s[6] = a.w & 0xFFFF; s[7] = a.w >> 16;
-        for (int i = 1; i < n_ranks; ++i) {
-            int rr = c + i;
-            if (rr >= n_ranks) rr -= n_ranks;
-            const uint4 b = ld_global_nc_v4(partials + static_cast<size_t>(rr) * plane + off);
-            s[0] = bf16_add(s[0], b.x & 0xFFFF); s[1] = bf16_add(s[1], b.x >> 16);
-            s[2] = bf16_add(s[2], b.y & 0xFFFF); s[3] = bf16_add(s[3], b.y >> 16);
-            s[4] = bf16_add(s[4], b.z & 0xFFFF); s[5] = bf16_add(s[5], b.z >> 16);
-            s[6] = bf16_add(s[6], b.w & 0xFFFF); s[7] = bf16_add(s[7], b.w >> 16);
+        uint4 pv[kMaxRanks];
+#pragma unroll
+        for (int i = 0; i < kMaxRanks; ++i) {
+            if (i < n_ranks) {
+                int rr = c + i;   // ring order: the chunk's owner first
+                if (rr >= n_ranks) rr -= n_ranks;
+                pv[i] = ld_global_nc_v4(partials + static_cast<size_t>(rr) * plane + off);
+            }
         }
         const uint4 rv = ld_global_nc_v4(residual + off);
+        uint16_t s[8];
+        s[0] = pv[0].x & 0xFFFF; s[1] = pv[0].x >> 16; s[2] = pv[0].y & 0xFFFF; s[3] = pv[0].y >> 16;
+        s[4] = pv[0].z & 0xFFFF; s[5] = pv[0].z >> 16; s[6] = pv[0].w & 0xFFFF; s[7] = pv[0].w >> 16;
+#pragma unroll
+        for (int i = 1; i < kMaxRanks; ++i) {
+            if (i < n_ranks) {
+                const uint4 b = pv[i];
+                s[0] = bf16_add(s[0], b.x & 0xFFFF); s[1] = bf16_add(s[1], b.x >> 16);
+                s[2] = bf16_add(s[2], b.y & 0xFFFF); s[3] = bf16_add(s[3], b.y >> 16);
+                s[4] = bf16_add(s[4], b.z & 0xFFFF); s[5] = bf16_add(s[5], b.z >> 16);
+                s[6] = bf16_add(s[6], b.w & 0xFFFF); s[7] = bf16_add(s[7], b.w >> 16);
+            }
+        }
         uint4 o;
         o.x = bf16_add(rv.x & 0xFFFF, s[0]) | (static_cast<uint32_t>(bf16_add(rv.x >> 16, s[1])) << 16);
         o.y = bf16_add(rv.y & 0xFFFF, s[2]) | (static_cast<uint32_t>(bf16_add(rv.y >> 16, s[3])) << 16);
@@ -272,55 +286,48 @@ __global__ void __launch_bounds__(256)
 
 // S2-S4 over k-split partials: rank r's partial is first assembled as
 // bf16_rne(part_0 + part_1 + ... ) -- the fp32 sums of its K parts added in
-// split order -- then folded in ring order as above.
+// split order -- then folded in ring order as above. Few tokens take this
+// path (it exists to fill the SMs when there are few units), so a thread
+// takes one output element and loads all N * SPLITS parts before adding.
+// Grid: x over H in blocks of 256 columns, y over tokens (grid-stride).
 __global__ void __launch_bounds__(256)
     ring_reduce_splits_kernel(const float* __restrict__ parts, int splits,
                               const uint16_t* __restrict__ residual, uint16_t* __restrict__ out,
                               int n_ranks, int64_t tokens, int hidden, int hc) {
     pdl_launch_dependents();
     pdl_wait();
-    const int64_t hv = hidden >> 3;
-    const int64_t total = tokens * hv;
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= hidden) return;
+    const int c = h / hc;
     const size_t plane = static_cast<size_t>(tokens) * hidden;
-    for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < total;
-         v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t m = v / hv;
-        const int h = static_cast<int>(v - m * hv) << 3;
-        const int c = h / hc;
+    for (int64_t m = blockIdx.y; m < tokens; m += gridDim.y) {
         const size_t off = static_cast<size_t>(m) * hidden + h;
-        uint16_t s[8];
-        for (int i = 0; i < n_ranks; ++i) {
-            int rr = c + i;
-            if (rr >= n_ranks) rr -= n_ranks;
-            float a[8];
-            {
-                const float4* src = reinterpret_cast<const float4*>(parts + static_cast<size_t>(rr) * plane + off);
-                const float4 lo = src[0], hi = src[1];
-                a[0] = lo.x; a[1] = lo.y; a[2] = lo.z; a[3] = lo.w;
-                a[4] = hi.x; a[5] = hi.y; a[6] = hi.z; a[7] = hi.w;
-            }
-            for (int sp = 1; sp < splits; ++sp) {
-                const float4* src = reinterpret_cast<const float4*>(
-                    parts + (static_cast<size_t>(sp) * n_ranks + rr) * plane + off);
-                const float4 lo = src[0], hi = src[1];
-                a[0] = __fadd_rn(a[0], lo.x); a[1] = __fadd_rn(a[1], lo.y);
-                a[2] = __fadd_rn(a[2], lo.z); a[3] = __fadd_rn(a[3], lo.w);
-                a[4] = __fadd_rn(a[4], hi.x); a[5] = __fadd_rn(a[5], hi.y);
-                a[6] = __fadd_rn(a[6], hi.z); a[7] = __fadd_rn(a[7], hi.w);
-            }
+        float a[kMaxRanks][kMaxSplits];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const uint16_t pr = f32_to_bf16_rne(a[e]);
-                s[e] = i == 0 ? pr : bf16_add(s[e], pr);
+        for (int i = 0; i < kMaxRanks; ++i) {
+            if (i < n_ranks) {
+                int rr = c + i;
+                if (rr >= n_ranks) rr -= n_ranks;
+#pragma unroll
+                for (int sp = 0; sp < kMaxSplits; ++sp)
+                    if (sp < splits)
+                        a[i][sp] = parts[(static_cast<size_t>(sp) * n_ranks + rr) * plane + off];
             }
         }
-        const uint4 rv = ld_global_nc_v4(residual + off);
-        uint4 o;
-        o.x = bf16_add(rv.x & 0xFFFF, s[0]) | (static_cast<uint32_t>(bf16_add(rv.x >> 16, s[1])) << 16);
-        o.y = bf16_add(rv.y & 0xFFFF, s[2]) | (static_cast<uint32_t>(bf16_add(rv.y >> 16, s[3])) << 16);
-        o.z = bf16_add(rv.z & 0xFFFF, s[4]) | (static_cast<uint32_t>(bf16_add(rv.z >> 16, s[5])) << 16);
-        o.w = bf16_add(rv.w & 0xFFFF, s[6]) | (static_cast<uint32_t>(bf16_add(rv.w >> 16, s[7])) << 16);
-        st_global_v4(out + off, o);
+        const uint16_t rv = residual[off];
+        uint16_t s = 0;
+#pragma unroll
+        for (int i = 0; i < kMaxRanks; ++i) {
+            if (i < n_ranks) {
+                float f = a[i][0];
+#pragma unroll
+                for (int sp = 1; sp < kMaxSplits; ++sp)
+                    if (sp < splits) f = __fadd_rn(f, a[i][sp]);
+                const uint16_t pr = f32_to_bf16_rne(f);
+                s = i == 0 ? pr : bf16_add(s, pr);
+            }
+        }
+        out[off] = bf16_add(rv, s);
     }
 }
 

@@ -252,7 +252,7 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split) {
     const int nkb = static_cast<int>((p->ks + tpr::kTcKBlock - 1) / tpr::kTcKBlock);
     c.splits = 1;
     if (allow_split && base_units < p->sm_count)
-        c.splits = std::max(1, std::min({slots / base_units, nkb, 8}));
+        c.splits = std::max(1, std::min({slots / base_units, nkb, tpr::kMaxSplits}));
     c.units = base_units * c.splits;
     c.grid = std::min(c.units, slots);
     return c;
@@ -324,10 +324,10 @@ tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partia
 
 tp_status launch_ring_splits(const tp_plan* p, const void* parts, int splits, const void* residual,
                              void* out, int64_t tokens, cudaStream_t stream) {
-    const int64_t total = tokens * (p->hidden / 8);
-    const int64_t blocks = std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(p->sm_count) * 8);
-    cudaError_t e = launch_pdl(tpr::ring_reduce_splits_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256),
-                               0, stream, static_cast<const float*>(parts), splits,
+    const dim3 grid(static_cast<unsigned>((p->hidden + 255) / 256),
+                    static_cast<unsigned>(std::min<int64_t>(tokens, 65535)));
+    cudaError_t e = launch_pdl(tpr::ring_reduce_splits_kernel, grid, dim3(256), 0, stream,
+                               static_cast<const float*>(parts), splits,
                                static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out),
                                p->n_ranks, tokens, static_cast<int>(p->hidden), static_cast<int>(p->hc));
     return e == cudaSuccess ? TP_OK : cuda_fail(e);
