@@ -143,8 +143,7 @@ class Workload:
         return "exact-staged" if pl.staged else "exact-fused"
 
     def launches_per_step(self):
-        staged = any(pl.workspace_bytes(self.cfg.tokens) for pl in self.plans.values())
-        return (2 if staged else 1) * self.cfg.n_points
+        return sum(self.plans[p.k].launches(self.cfg.tokens) for p in self.cfg.points)
 
     def capture(self):
         g = torch.cuda.CUDAGraph()

@@ -100,14 +100,22 @@ TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
  * the plan's current setting; 0 when the partials stay on chip (EXACT, not
  * staged). The tensor-core variant always sends its partials through the
  * workspace: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of K parts)
- * when it splits K across CTAs to fill the SMs; rounded up to 256. Returns 0
- * for a null plan. */
+ * when it splits K across CTAs to fill the SMs. Layout: a counter block of
+ * one 32-bit counter per 128-row H tile (256-byte rounded; the in-kernel fold
+ * of one or two tokens counts stored parts there), then the partials.
+ * Rounded up to 256 in all. Returns 0 for a null plan. */
 TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 
 /* The partial kernel a call with `tokens` tokens runs under the plan's
  * current setting: TP_VARIANT_EXACT or TP_VARIANT_TENSOR (AUTO resolved).
  * Returns -1 for a null plan or tokens < 1. A query only; launches nothing. */
 TP_API int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens);
+
+/* Kernels one tp_rowlinear_reconcile call with `tokens` tokens launches under
+ * the plan's current setting: 1 (EXACT not staged; TENSOR with 1 or 2 tokens,
+ * which folds inside its partial kernel) or 2 (a partial kernel, then a ring
+ * fold kernel); 0 for tokens = 0; -1 for a null plan or tokens < 0. */
+TP_API int tp_plan_launches(const tp_plan* plan, int64_t tokens);
 
 /* Bytes of the packed weight buffer tp_pack_weights writes: N*H*(K/N)*2,
  * the size of the Linear weight. Returns 0 for a null plan. */
@@ -129,7 +137,13 @@ TP_API tp_status tp_pack_weights(const tp_plan* plan, const void* w_hk, void* w_
  *   out        [M][H] bf16 (output); must not overlap any input or the workspace
  *   tokens     M, 0 <= M <= max_tokens (M = 0 launches nothing)
  *   workspace  tp_plan_workspace_bytes(plan, M) bytes of device memory, or
- *              NULL when that is 0; contents on entry are ignored
+ *              NULL when that is 0. Zero it before its first use: its fold
+ *              counters (see tp_plan_workspace_bytes) must start at zero, and
+ *              every call that sets no device error flag leaves them zero
+ *              again, so one zeroed workspace serves any number of calls (of
+ *              any plans with the same H, in stream order). After a call that
+ *              set a device error flag, zero it again. The rest of its
+ *              contents on entry are ignored.
  * Partials per the header comment, summed in ring order, then the residual
  * add ("Interconnects e clusters", 01 Conceito: the slices are summed before
  * the residual stream continues). */
@@ -150,11 +164,15 @@ TP_API tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, cons
  * once per device when a plan is created on it, so this call does no set-up
  * of its own and allocates nothing.
  *  - Returns TP_ERR_WORKSPACE, launching nothing, when the call needs more
- *    scratch than that: tp_plan_workspace_bytes(plan, tokens) > 16 MiB
- *    (N*M*H*2 bytes; e.g. N=8, M=64, H=4096 needs 4 MiB).
+ *    scratch than that: staged partials above 16 MiB - 4 KiB (N*M*H*2
+ *    bytes, or splits*N*M*H*4; e.g. N=8, M=64, H=4096 needs 4 MiB), or
+ *    H > 131072 (the first 4 KiB hold the fold counters of every plan).
  *  - Every call, from every plan and thread on a device, shares the one
  *    array, which keeps the last call's partials; each call writes every
- *    partial it reads, so nothing needs clearing. Calls whose kernels overlap
+ *    partial it reads. The fold counters at its start are zero when the
+ *    library is loaded and every call that sets no device error flag leaves
+ *    them zero; after one that does, this entry point may give wrong results
+ *    until the process restarts. Calls whose kernels overlap
  *    on the GPU (different streams without ordering between them) race on
  *    the array and give wrong results: order them on one stream.
  * The pages describe no counterpart of this entry point. */

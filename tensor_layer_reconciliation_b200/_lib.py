@@ -19,7 +19,7 @@ TP_BF16 = 0
 TP_VARIANT_AUTO, TP_VARIANT_EXACT, TP_VARIANT_TENSOR = 0, 1, 2
 
 EXPORTED = (
-    "tp_plan_create", "tp_plan_set_variant", "tp_plan_workspace_bytes", "tp_plan_kernel_variant",
+    "tp_plan_create", "tp_plan_set_variant", "tp_plan_workspace_bytes", "tp_plan_kernel_variant", "tp_plan_launches",
     "tp_plan_packed_bytes",
     "tp_pack_weights",
     "tp_rowlinear_reconcile", "tp_rowlinear_reconcile_noalloc", "tp_rowlinear_partials",
@@ -52,6 +52,8 @@ def _load() -> ctypes.CDLL:
     L.tp_plan_workspace_bytes.restype = sz
     L.tp_plan_kernel_variant.argtypes = [vp, i64]
     L.tp_plan_kernel_variant.restype = ctypes.c_int
+    L.tp_plan_launches.argtypes = [vp, i64]
+    L.tp_plan_launches.restype = ctypes.c_int
     L.tp_plan_packed_bytes.argtypes = [vp]
     L.tp_plan_packed_bytes.restype = sz
     L.tp_pack_weights.argtypes = [vp, vp, vp, vp]
@@ -103,6 +105,10 @@ def tp_plan_workspace_bytes(plan, tokens: int) -> int:
 
 def tp_plan_kernel_variant(plan, tokens: int) -> int:
     return LIB.tp_plan_kernel_variant(plan, tokens)
+
+
+def tp_plan_launches(plan, tokens: int) -> int:
+    return LIB.tp_plan_launches(plan, tokens)
 
 
 def tp_plan_packed_bytes(plan) -> int:

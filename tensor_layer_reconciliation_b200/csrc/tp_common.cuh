@@ -103,6 +103,115 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     return true;
 }
 
+// Named barrier `id` over `nthreads` threads that also ORs a flag across
+// them: every participant gets the same answer, so a decision taken on it
+// (leaving a loop whose next iteration meets the barrier again) is uniform.
+__device__ __forceinline__ bool bar_sync_any(int id, int nthreads, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, p;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+// ---------------------------------------------------------- ring fold --
+constexpr int kMaxRanks = 8;     // tp_plan_create accepts 1 .. 8 ranks
+constexpr int kMaxSplits = 8;    // k-splits of the tensor-core partials
+
+// S2-S3 for one output element (token m, column h at offset `off` of an
+// [M][H] plane) from partials staged in memory: starting at the owner c of
+// the element's chunk, the ranks' partials are added in ring order, each add
+// rounded to bf16. Every load is issued before the first add (loops unrolled
+// to the largest counts), so one memory latency covers them all. kL2 loads
+// through L2 only, for data written earlier by the same kernel.
+template <bool kL2>
+__device__ __forceinline__ uint16_t ring_fold_bf16(const uint16_t* partials, int n_ranks, size_t plane,
+                                                   size_t off, int c) {
+    uint16_t v[kMaxRanks];
+#pragma unroll
+    for (int i = 0; i < kMaxRanks; ++i) {
+        if (i < n_ranks) {
+            int rr = c + i;
+            if (rr >= n_ranks) rr -= n_ranks;
+            const uint16_t* a = partials + static_cast<size_t>(rr) * plane + off;
+            v[i] = kL2 ? __ldcg(a) : *a;
+        }
+    }
+    uint16_t s = v[0];
+#pragma unroll
+    for (int i = 1; i < kMaxRanks; ++i)
+        if (i < n_ranks) s = bf16_add(s, v[i]);
+    return s;
+}
+
+// As ring_fold_bf16 over k-split fp32 parts [SPLITS][N][M][H]: rank r's
+// partial is bf16_rne(part_0 + part_1 + ...), the parts added in split
+// (k-ascending) order in fp32, before the ring-order bf16 adds.
+template <bool kL2>
+__device__ __forceinline__ uint16_t ring_fold_f32_parts(const float* parts, int splits, int n_ranks,
+                                                        size_t plane, size_t off, int c) {
+    float a[kMaxRanks][kMaxSplits];
+#pragma unroll
+    for (int i = 0; i < kMaxRanks; ++i) {
+        if (i < n_ranks) {
+            int rr = c + i;
+            if (rr >= n_ranks) rr -= n_ranks;
+#pragma unroll
+            for (int sp = 0; sp < kMaxSplits; ++sp)
+                if (sp < splits) {
+                    const float* q = parts + (static_cast<size_t>(sp) * n_ranks + rr) * plane + off;
+                    a[i][sp] = kL2 ? __ldcg(q) : *q;
+                }
+        }
+    }
+    uint16_t s = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxRanks; ++i) {
+        if (i < n_ranks) {
+            float f = a[i][0];
+#pragma unroll
+            for (int sp = 1; sp < kMaxSplits; ++sp)
+                if (sp < splits) f = __fadd_rn(f, a[i][sp]);
+            const uint16_t pr = f32_to_bf16_rne(f);
+            s = i == 0 ? pr : bf16_add(s, pr);
+        }
+    }
+    return s;
+}
+
+// ring_fold_f32_parts for callers short of registers (the tensor-core
+// kernel's in-kernel fold): ranks one after another, the parts of a rank
+// loaded together. Same sums in the same order, so the same result.
+template <bool kL2>
+__device__ __forceinline__ uint16_t ring_fold_f32_parts_by_rank(const float* parts, int splits,
+                                                                int n_ranks, size_t plane, size_t off,
+                                                                int c) {
+    uint16_t s = 0;
+#pragma unroll 1
+    for (int i = 0; i < n_ranks; ++i) {
+        int rr = c + i;
+        if (rr >= n_ranks) rr -= n_ranks;
+        const float* q = parts + static_cast<size_t>(rr) * plane + off;
+        const size_t step = static_cast<size_t>(n_ranks) * plane;
+        float a[kMaxSplits];
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplits; ++sp)
+            if (sp < splits) a[sp] = kL2 ? __ldcg(q + sp * step) : q[sp * step];
+        float f = a[0];
+#pragma unroll
+        for (int sp = 1; sp < kMaxSplits; ++sp)
+            if (sp < splits) f = __fadd_rn(f, a[sp]);
+        const uint16_t pr = f32_to_bf16_rne(f);
+        s = i == 0 ? pr : bf16_add(s, pr);
+    }
+    return s;
+}
+
 // --------------------------------------------------------------------- TMA --
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

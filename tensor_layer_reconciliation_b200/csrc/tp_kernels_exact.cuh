@@ -229,9 +229,6 @@ __global__ void __launch_bounds__(kMaxExactThreads, 1)
 }
 
 // ------------------------------------------------------------------ S2-S4 --
-constexpr int kMaxRanks = 8;     // tp_plan_create accepts 1 .. 8 ranks
-constexpr int kMaxSplits = 8;    // k-splits of the tensor-core partials
-
 // Ring reduce-scatter fold over partials staged in memory, the all-gather
 // (one result buffer stands for every rank's copy) and the residual add.
 // Thread per 8 consecutive columns (16-byte vectors; H/N % 8 == 0 keeps a
@@ -302,31 +299,8 @@ __global__ void __launch_bounds__(256)
     const size_t plane = static_cast<size_t>(tokens) * hidden;
     for (int64_t m = blockIdx.y; m < tokens; m += gridDim.y) {
         const size_t off = static_cast<size_t>(m) * hidden + h;
-        float a[kMaxRanks][kMaxSplits];
-#pragma unroll
-        for (int i = 0; i < kMaxRanks; ++i) {
-            if (i < n_ranks) {
-                int rr = c + i;
-                if (rr >= n_ranks) rr -= n_ranks;
-#pragma unroll
-                for (int sp = 0; sp < kMaxSplits; ++sp)
-                    if (sp < splits)
-                        a[i][sp] = parts[(static_cast<size_t>(sp) * n_ranks + rr) * plane + off];
-            }
-        }
+        const uint16_t s = ring_fold_f32_parts<false>(parts, splits, n_ranks, plane, off, c);
         const uint16_t rv = residual[off];
-        uint16_t s = 0;
-#pragma unroll
-        for (int i = 0; i < kMaxRanks; ++i) {
-            if (i < n_ranks) {
-                float f = a[i][0];
-#pragma unroll
-                for (int sp = 1; sp < kMaxSplits; ++sp)
-                    if (sp < splits) f = __fadd_rn(f, a[i][sp]);
-                const uint16_t pr = f32_to_bf16_rne(f);
-                s = i == 0 ? pr : bf16_add(s, pr);
-            }
-        }
         out[off] = bf16_add(rv, s);
     }
 }

@@ -31,9 +31,14 @@
 // ring kernel adds the parts in split order before the one rounding to bf16.
 // Units run token tile fastest, so CTAs working at the same time share each
 // weight tile through L2 (prefill reads every weight tile for 16 token tiles).
-// The ring fold stays a kernel of its own: folding inside the CTA that
-// completes a tile (measured) serialises N * SPLITS * 128 * BN reads behind
-// that CTA's next accumulator and is slower for every token count above one.
+// Folding (S2-S4): for one or two tokens the CTA that stores the last of
+// the N * SPLITS parts of an (H tile, token tile) -- found with a per-tile
+// counter in the workspace -- folds that tile itself, each epilogue thread
+// one row h, so a call is one kernel and the next call's kernel waits on one
+// grid instead of two. For more tokens the fold stays a kernel of its own:
+// there the CTA that completes a tile would read N * SPLITS * 128 * BN
+// values behind its next accumulator (measured slower from 32 tokens up),
+// while a separate kernel spreads that work over the whole GPU.
 // Accumulation order inside the tensor core is the hardware's; the partial
 // is the fp32 sum rounded once to bf16, like the oracle's, but only equal to
 // it where the two fp32 sums round to the same bf16 value.
@@ -61,6 +66,12 @@ struct TcParams {
     int stages;    // 2 .. kTcMaxStages
     uint16_t* partials;     // [N][M][H] bf16 (splits == 1)
     float* partials_f32;    // [splits][N][M][H] fp32 sums of each k part (splits > 1)
+    // In-kernel fold (S2-S4), few tokens only; fold == 0 leaves it to the ring kernel.
+    int fold;
+    int hc;                       // H / N, the chunk each rank owns in the ring
+    unsigned int* counters;       // [h_tiles][m_tiles] parts stored so far; zero between calls
+    const uint16_t* residual;     // [M][H]
+    uint16_t* out;                // [M][H]
 };
 
 template <int BN>
@@ -85,6 +96,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* mma_done = acc_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     __shared__ int abort_flag;
+    __shared__ int fold_mine;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nkb = (p.ks + kTcKBlock - 1) / kTcKBlock;
@@ -237,14 +249,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else {
         // ---------------------------------------------------------- epilogue --
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        pdl_wait();  // the fold reads the residual and writes the output in stream order
         for (int lu = 0; lu < my_units; ++lu) {
             const int b = lu & 1;
             const uint32_t aph = static_cast<uint32_t>(lu >> 1) & 1u;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&acc_full[b], aph)))
-                atomicExch(&abort_flag, 1);
-            // The four epilogue warps leave together.
-            asm volatile("bar.sync 2, 128;" ::: "memory");
-            if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
+            bool bad = !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&acc_full[b], aph));
+            if (bad) atomicExch(&abort_flag, 1);
+            bad = bad || *reinterpret_cast<volatile int*>(&abort_flag) != 0;
+            // The four epilogue warps leave together: one answer for all of them.
+            if (bar_sync_any(2, 128, bad)) break;
             tc_fence_after_sync();
             int r, ht, mt, sp;
             unit_of(lu, r, ht, mt, sp);
@@ -281,6 +294,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[b]);
+            if (p.fold) {
+                // The CTA that stores the last of the N * SPLITS parts of this
+                // (H tile, token tile) folds the tile: ring order, residual add.
+                __threadfence();  // this thread's parts are visible before the count
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                unsigned int* cnt = p.counters + ht * p.m_tiles + mt;
+                if (warp == 2 && lane == 0)
+                    fold_mine = atomicAdd(cnt, 1u) == static_cast<unsigned int>(p.n_ranks * p.splits - 1);
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                if (fold_mine) {
+                    __threadfence();  // the other CTAs' parts, counted above, are read after it
+                    if (h < p.hidden) {
+                        const int c = h / p.hc;
+                        const int m_end = min(m0 + BN, p.tokens);
+                        for (int m = m0; m < m_end; ++m) {
+                            const size_t off = static_cast<size_t>(m) * p.hidden + h;
+                            const uint16_t sum =
+                                p.splits == 1
+                                    ? ring_fold_bf16<true>(p.partials, p.n_ranks, plane, off, c)
+                                    : ring_fold_f32_parts_by_rank<true>(p.partials_f32, p.splits,
+                                                                        p.n_ranks, plane, off, c);
+                            p.out[off] = bf16_add(p.residual[off], sum);
+                        }
+                    }
+                    if (warp == 2 && lane == 0) atomicExch(cnt, 0u);  // zero for the next call
+                }
+            }
         }
     }
 

@@ -14,10 +14,13 @@
 #include "tp_kernels_tc.cuh"
 #include "tp_reconcile.h"
 
-// Fixed scratch for tp_rowlinear_reconcile_noalloc: the staged partials
-// (N * M * H bf16) of callers that cannot allocate device memory. Every GPU
-// that loads this library holds it until the process exits.
+// Fixed scratch for tp_rowlinear_reconcile_noalloc: fold counters and the
+// staged partials of callers that cannot allocate device memory. Every GPU
+// that loads this library holds it until the process exits. Its first
+// kNoAllocCounterBytes hold the counters of every plan (zero-initialised,
+// left zero by each call), the rest the partials.
 constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB
+constexpr size_t kNoAllocCounterBytes = 4096;       // 1024 H tiles: H <= 131072
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 struct tp_plan {
@@ -292,10 +295,20 @@ tp_status encode_tc_maps(const tp_plan* p, const TcConfig& c, const void* x, con
 
 // The tensor-core partials: bf16 [N][M][H] when the units are not split, or
 // fp32 k-part sums [splits][N][M][H] (allow_split) for the ring kernel to add.
+size_t tc_partial_bytes(const tp_plan* p, const TcConfig& c, int64_t tokens) {
+    return static_cast<size_t>(p->n_ranks) * static_cast<size_t>(tokens) *
+           static_cast<size_t>(p->hidden) * (c.splits > 1 ? 4u * c.splits : 2u);
+}
+
+// fold: the kernel also runs S2-S4 (residual, out) for few tokens, counting
+// stored parts per H tile in `counters` (zero on entry, zero on return);
+// else a ring kernel must follow.
 tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partials, int64_t tokens,
-                    bool allow_split, cudaStream_t stream) {
+                    bool allow_split, bool fold, unsigned int* counters, const void* residual,
+                    void* out, cudaStream_t stream) {
     const TcConfig c = tc_config(p, tokens, allow_split);
     if (c.stages < 2) return TP_ERR_UNSUPPORTED;
+    if (fold && c.m_tiles != 1) return TP_ERR_UNSUPPORTED;
     CUtensorMap mw, mx;
     tp_status st = encode_tc_maps(p, c, x, w, tokens, &mw, &mx);
     if (st != TP_OK) return st;
@@ -311,6 +324,11 @@ tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partia
     prm.stages = c.stages;
     prm.partials = static_cast<uint16_t*>(partials);
     prm.partials_f32 = static_cast<float*>(partials);
+    prm.fold = fold ? 1 : 0;
+    prm.hc = static_cast<int>(p->hc);
+    prm.counters = fold ? counters : nullptr;
+    prm.residual = static_cast<const uint16_t*>(residual);
+    prm.out = static_cast<uint16_t*>(out);
     const dim3 grid(c.grid), block(tpr::kTcThreads);
     cudaError_t e;
     switch (c.bn) {
@@ -438,16 +456,41 @@ int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens) {
     return effective_variant(plan, tokens);
 }
 
+// The tensor path folds inside its partial kernel up to this many tokens.
+constexpr int64_t kFoldMaxTokens = 2;
+
+static bool tc_folds(int64_t tokens) { return tokens <= kFoldMaxTokens; }
+
+// Fold counter block at the start of every workspace: one uint32 per
+// 128-row H tile, 256-byte rounded, reserved on every staged path so that
+// calls of other variants or token counts sharing the workspace leave the
+// counters alone.
+static size_t counter_block_bytes(const tp_plan* plan) {
+    const size_t tiles = static_cast<size_t>((plan->hidden + tpr::kTcRows - 1) / tpr::kTcRows);
+    return (tiles * 4 + 255) / 256 * 256;
+}
+
+// Bytes of staged partials a call writes (0: none, the exact fused kernel).
+static size_t partial_bytes(const tp_plan* plan, int64_t tokens) {
+    if (effective_variant(plan, tokens) == TP_VARIANT_TENSOR)
+        return tc_partial_bytes(plan, tc_config(plan, tokens, true), tokens);
+    if (!plan->staged) return 0;
+    return static_cast<size_t>(plan->n_ranks) * static_cast<size_t>(tokens) *
+           static_cast<size_t>(plan->hidden) * 2;
+}
+
 size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens) {
     if (!plan || tokens <= 0) return 0;
-    // The tensor-core partials always go through the workspace, as fp32 k-part
-    // sums when the units are split.
-    const bool tensor = effective_variant(plan, tokens) == TP_VARIANT_TENSOR;
-    if (!plan->staged && !tensor) return 0;
-    const int splits = tensor ? tc_config(plan, tokens, true).splits : 1;
-    const size_t b = static_cast<size_t>(plan->n_ranks) * static_cast<size_t>(tokens) *
-                     static_cast<size_t>(plan->hidden) * (splits > 1 ? 4u * splits : 2u);
-    return (b + 255) / 256 * 256;
+    const size_t pb = partial_bytes(plan, tokens);
+    if (pb == 0) return 0;
+    return (counter_block_bytes(plan) + pb + 255) / 256 * 256;
+}
+
+int tp_plan_launches(const tp_plan* plan, int64_t tokens) {
+    if (!plan || tokens < 0) return -1;
+    if (tokens == 0) return 0;
+    if (effective_variant(plan, tokens) == TP_VARIANT_TENSOR) return tc_folds(tokens) ? 1 : 2;
+    return plan->staged ? 2 : 1;
 }
 
 size_t tp_plan_packed_bytes(const tp_plan* plan) {
@@ -478,37 +521,56 @@ static tp_status check_point_args(const tp_plan* plan, const void* x, const void
     return TP_OK;
 }
 
-tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void* w_packed,
-                                 const void* residual, void* out, int64_t tokens, void* workspace,
-                                 void* stream) {
+// Argument checks shared by both reconcile entry points (all but the workspace).
+static tp_status check_reconcile_args(const tp_plan* plan, const void* x, const void* w_packed,
+                                      const void* residual, const void* out, int64_t tokens) {
     tp_status st = check_point_args(plan, x, w_packed, tokens);
-    if (st != TP_OK) return st;
-    if (tokens == 0) return TP_OK;
+    if (st != TP_OK || tokens == 0) return st;
     if (!residual || !out) return TP_ERR_INVALID;
-    if (!aligned16(residual) || !aligned16(out) || !aligned16(workspace)) return TP_ERR_ALIGN;
+    if (!aligned16(residual) || !aligned16(out)) return TP_ERR_ALIGN;
     const size_t mh = static_cast<size_t>(tokens) * plan->hidden * 2;
     const size_t xb = static_cast<size_t>(tokens) * plan->k * 2;
     const size_t wb = static_cast<size_t>(plan->hidden) * plan->k * 2;
-    const size_t ws = tp_plan_workspace_bytes(plan, tokens);
-    if (overlaps(out, mh, x, xb) || overlaps(out, mh, w_packed, wb) ||
-        overlaps(out, mh, residual, mh) || overlaps(out, mh, workspace, ws))
+    if (overlaps(out, mh, x, xb) || overlaps(out, mh, w_packed, wb) || overlaps(out, mh, residual, mh))
         return TP_ERR_INVALID;
-    if (ws && !workspace) return TP_ERR_WORKSPACE;
-    if ((st = check_device(plan)) != TP_OK) return st;
-    const int variant = effective_variant(plan, tokens);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (variant == TP_VARIANT_TENSOR) {
-        st = launch_tc(plan, x, w_packed, workspace, tokens, true, s);
+    return TP_OK;
+}
+
+// S1-S4 with the fold counters and the staged partials given apart.
+static tp_status reconcile_launch(const tp_plan* plan, const void* x, const void* w_packed,
+                                  const void* residual, void* out, int64_t tokens,
+                                  unsigned int* counters, void* partials, cudaStream_t s) {
+    tp_status st = check_device(plan);
+    if (st != TP_OK) return st;
+    if (effective_variant(plan, tokens) == TP_VARIANT_TENSOR) {
+        const bool fold = tc_folds(tokens);
+        st = launch_tc(plan, x, w_packed, partials, tokens, true, fold, counters, residual, out, s);
+        if (st != TP_OK || fold) return st;
         const int splits = tc_config(plan, tokens, true).splits;
-        if (st == TP_OK && splits > 1)
-            return launch_ring_splits(plan, workspace, splits, residual, out, tokens, s);
+        if (splits > 1) return launch_ring_splits(plan, partials, splits, residual, out, tokens, s);
     } else {
         if (!plan->staged)
             return launch_exact(plan, x, w_packed, residual, out, nullptr, tokens, true, s);
-        st = launch_exact(plan, x, w_packed, nullptr, nullptr, workspace, tokens, false, s);
+        st = launch_exact(plan, x, w_packed, nullptr, nullptr, partials, tokens, false, s);
+        if (st != TP_OK) return st;
     }
-    if (st != TP_OK) return st;
-    return launch_ring(plan, workspace, residual, out, tokens, s);
+    return launch_ring(plan, partials, residual, out, tokens, s);
+}
+
+tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, const void* w_packed,
+                                 const void* residual, void* out, int64_t tokens, void* workspace,
+                                 void* stream) {
+    tp_status st = check_reconcile_args(plan, x, w_packed, residual, out, tokens);
+    if (st != TP_OK || tokens == 0) return st;
+    if (!aligned16(workspace)) return TP_ERR_ALIGN;
+    const size_t ws = tp_plan_workspace_bytes(plan, tokens);
+    if (overlaps(out, static_cast<size_t>(tokens) * plan->hidden * 2, workspace, ws)) return TP_ERR_INVALID;
+    if (ws && !workspace) return TP_ERR_WORKSPACE;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    return reconcile_launch(plan, x, w_packed, residual, out, tokens,
+                            reinterpret_cast<unsigned int*>(base),
+                            ws ? base + counter_block_bytes(plan) : nullptr,
+                            static_cast<cudaStream_t>(stream));
 }
 
 tp_status tp_rowlinear_reconcile_noalloc(const tp_plan* plan, const void* x, const void* w_packed,
@@ -516,9 +578,16 @@ tp_status tp_rowlinear_reconcile_noalloc(const tp_plan* plan, const void* x, con
                                          void* stream) {
     if (!plan) return TP_ERR_INVALID;
     if (tokens < 0 || tokens > plan->max_tokens) return TP_ERR_INVALID;
-    if (tp_plan_workspace_bytes(plan, tokens) > kNoAllocScratchBytes) return TP_ERR_WORKSPACE;
-    return tp_rowlinear_reconcile(plan, x, w_packed, residual, out, tokens,
-                                  plan->noalloc_scratch, stream);
+    // Refused before anything is touched when the scratch cannot hold it.
+    if (counter_block_bytes(plan) > kNoAllocCounterBytes ||
+        partial_bytes(plan, tokens) > kNoAllocScratchBytes - kNoAllocCounterBytes)
+        return TP_ERR_WORKSPACE;
+    tp_status st = check_reconcile_args(plan, x, w_packed, residual, out, tokens);
+    if (st != TP_OK || tokens == 0) return st;
+    uint8_t* base = static_cast<uint8_t*>(plan->noalloc_scratch);
+    return reconcile_launch(plan, x, w_packed, residual, out, tokens,
+                            reinterpret_cast<unsigned int*>(base), base + kNoAllocCounterBytes,
+                            static_cast<cudaStream_t>(stream));
 }
 
 tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* w_packed,
@@ -535,7 +604,8 @@ tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* 
     if ((st = check_device(plan)) != TP_OK) return st;
     const int variant = effective_variant(plan, tokens);
     if (variant == TP_VARIANT_TENSOR)
-        return launch_tc(plan, x, w_packed, partials, tokens, false, static_cast<cudaStream_t>(stream));
+        return launch_tc(plan, x, w_packed, partials, tokens, false, false, nullptr, nullptr,
+                         nullptr, static_cast<cudaStream_t>(stream));
     return launch_exact(plan, x, w_packed, nullptr, nullptr, partials, tokens, false,
                         static_cast<cudaStream_t>(stream));
 }

@@ -82,6 +82,10 @@ class Plan:
             raise ValueError("tokens must be >= 1")
         return "tensor" if v == _lib.TP_VARIANT_TENSOR else "exact"
 
+    def launches(self, tokens: int) -> int:
+        """Kernels one reconcile call with this many tokens launches."""
+        return _lib.tp_plan_launches(self._h, tokens)
+
     @property
     def packed_numel(self) -> int:
         """bf16 elements of the packed weight buffer (tiled shards, see tp_reconcile.h)."""
@@ -113,8 +117,8 @@ class Plan:
         need = self.workspace_bytes(m)
         pws = 0
         if need:
-            if workspace is None:
-                workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+            if workspace is None:   # fold counters start at zero
+                workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
             if workspace.numel() * workspace.element_size() < need or workspace.device.type != "cuda":
                 raise ValueError("workspace too small")
             pws = workspace.data_ptr()

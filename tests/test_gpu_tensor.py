@@ -42,7 +42,9 @@ SHAPES = [             # N, M, K, H
     (4, 32, 512, 512),      # decode batch, token tile 32
     (8, 64, 1024, 256),     # decode batch, token tile 64, N = 8
     (2, 16, 128, 128),      # 16 tokens in a 32-token tile
-    (2, 1, 8192, 512),      # one token: K split 8 ways across CTAs (fp32 parts)
+    (2, 1, 8192, 512),      # one token: K split 8 ways across CTAs, folded in the kernel
+    (8, 1, 2048, 1024),     # one token, N = 8: K split 4 ways, folded in the kernel
+    (2, 2, 4096, 384),      # two tokens (the most folded in the kernel), H % 128 != 0
     (4, 3, 2048, 640),      # three tokens, K split, H % 128 != 0
     (4, 100, 640, 384),     # token tile 128 with a ragged tail; 3 weight tiles
     (4, 300, 512, 256),     # token tile 256, two tiles, second ragged
@@ -142,3 +144,29 @@ def test_auto_uses_tensor_cores():
     assert plan.effective_variant(1) == "exact"
     assert plan.workspace_bytes(1) == 0                # exact, fused: no workspace
     assert tlr.tp_plan_kernel_variant(plan.handle, 0) == -1
+
+
+def test_fold_counters_return_to_zero():
+    """One zeroed workspace serves many calls: the in-kernel fold (one or two
+    tokens) counts stored parts per tile in the workspace's first bytes and
+    the folding CTA sets each count back to zero."""
+    import tensor_layer_reconciliation_b200 as tlr
+    dev = torch.device("cuda")
+    n, k, h = 4, 4096, 640
+    plan = tlr.Plan(n, 2, k, h)                        # AUTO
+    for m in (1, 2):
+        assert plan.launches(m) == 1                   # partials and fold in one kernel
+        need = plan.workspace_bytes(m)
+        ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+        h_tiles = (h + 127) // 128
+        counter_bytes = (h_tiles * 4 + 255) // 256 * 256
+        for seed in (31, 32, 33):
+            x, w, r = inputs(n, m, k, h, seed + 10 * m, dev)
+            wp = plan.pack_weights(w)
+            out = plan.reconcile(x, wp, r, workspace=ws)
+            fresh = plan.reconcile(x, wp, r)           # its own zeroed workspace
+            torch.cuda.synchronize()
+            assert plan.device_error_flags() == 0
+            assert torch.equal(out.view(torch.int16), fresh.view(torch.int16))
+            assert int(torch.count_nonzero(ws[:counter_bytes])) == 0
+    assert plan.launches(3) == 2                       # from three tokens: a ring kernel follows

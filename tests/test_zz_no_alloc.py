@@ -49,6 +49,28 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert torch.equal(out.view(torch.int16), out_ref.view(torch.int16)), f"call {call}"
 
 
+def test_noalloc_single_token_fold_twice():
+    """One token: the tensor-core kernel folds in place, using counters at
+    the start of the scratch array that each call must leave at zero."""
+    import tensor_layer_reconciliation_b200 as tlr
+    dev = torch.device("cuda")
+    n, m, k, h = 2, 1, 4096, 1024
+    plan = tlr.Plan(n, m, k, h)            # AUTO
+    assert plan.launches(m) == 1 and plan.workspace_bytes(m) > 0
+    stream = torch.cuda.current_stream().cuda_stream
+    for call, seed in enumerate((21, 22)):
+        x, w, r = inputs(n, m, k, h, seed, dev)
+        wp = plan.pack_weights(w)
+        ref = plan.reconcile(x, wp, r)
+        out = torch.full((m, h), float("nan"), dtype=torch.bfloat16, device=dev)
+        st = tlr.tp_rowlinear_reconcile_noalloc(plan.handle, _ptr(x), _ptr(wp), _ptr(r), _ptr(out),
+                                                m, stream)
+        assert st == tlr.TP_OK
+        torch.cuda.synchronize()
+        assert plan.device_error_flags() == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), f"call {call}"
+
+
 def test_noalloc_fused_path_needs_no_scratch():
     import tensor_layer_reconciliation_b200 as tlr
     dev = torch.device("cuda")
