@@ -297,6 +297,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (p.fold) {
                 // The CTA that stores the last of the N * SPLITS parts of this
                 // (H tile, token tile) folds the tile: ring order, residual add.
+                // Residual of this thread's row, loaded while the count goes round.
+                uint16_t res[2] = {0, 0};
+                if (h < p.hidden)
+                    for (int m = m0, i = 0; m < p.tokens && i < 2; ++m, ++i)
+                        res[i] = p.residual[static_cast<size_t>(m) * p.hidden + h];
                 __threadfence();  // this thread's parts are visible before the count
                 asm volatile("bar.sync 2, 128;" ::: "memory");
                 unsigned int* cnt = p.counters + ht * p.m_tiles + mt;
@@ -307,15 +312,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     __threadfence();  // the other CTAs' parts, counted above, are read after it
                     if (h < p.hidden) {
                         const int c = h / p.hc;
-                        const int m_end = min(m0 + BN, p.tokens);
-                        for (int m = m0; m < m_end; ++m) {
+                        // at most two tokens here (m_tiles == 1, tokens <= 2)
+                        for (int m = m0, i = 0; m < p.tokens && i < 2; ++m, ++i) {
                             const size_t off = static_cast<size_t>(m) * p.hidden + h;
                             const uint16_t sum =
                                 p.splits == 1
                                     ? ring_fold_bf16<true>(p.partials, p.n_ranks, plane, off, c)
+                                : p.n_ranks * p.splits <= 16
+                                    ? ring_fold_f32_parts16<true>(p.partials_f32, p.splits,
+                                                                  p.n_ranks, plane, off, c)
                                     : ring_fold_f32_parts_by_rank<true>(p.partials_f32, p.splits,
                                                                         p.n_ranks, plane, off, c);
-                            p.out[off] = bf16_add(p.residual[off], sum);
+                            p.out[off] = bf16_add(res[i], sum);
                         }
                     }
                     if (warp == 2 && lane == 0) atomicExch(cnt, 0u);  // zero for the next call

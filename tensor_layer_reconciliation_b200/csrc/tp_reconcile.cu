@@ -308,7 +308,7 @@ tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partia
                     void* out, cudaStream_t stream) {
     const TcConfig c = tc_config(p, tokens, allow_split);
     if (c.stages < 2) return TP_ERR_UNSUPPORTED;
-    if (fold && c.m_tiles != 1) return TP_ERR_UNSUPPORTED;
+    if (fold && (c.m_tiles != 1 || tokens > 2)) return TP_ERR_UNSUPPORTED;  // the kernel folds <= 2 rows
     CUtensorMap mw, mx;
     tp_status st = encode_tc_maps(p, c, x, w, tokens, &mw, &mx);
     if (st != TP_OK) return st;
