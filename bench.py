@@ -55,6 +55,13 @@ def _peaks():
 # sources means the kernels changed since, and the traffic is reported null.
 PROFILED_TRAFFIC = {
     # (workload, path): (bytes per call, kernel-source digest, profile summary)
+    ("decode_n2", "tensor"): (119145344, "3268512489d4754e", "profiles/tc_partial_decode_n2.md"),
+    ("decode_n4_m32", "tensor"): (120157696, "3268512489d4754e",
+                                  "profiles/tc_partial_ring_decode_n4_m32.md"),
+    ("decode_n8_m64", "tensor"): (83345920, "3268512489d4754e",
+                                  "profiles/tc_partial_ring_decode_n8_m64.md"),
+    ("prefill_n4", "tensor"): (807557888, "3268512489d4754e", "profiles/tc_partial_ring_prefill_n4.md"),
+    ("decode_n2", "exact-fused"): (117277824, "3268512489d4754e", "profiles/exact_partial_decode_n2.md"),
 }
 
 
@@ -456,6 +463,8 @@ def main(argv=None):
                 "frac": achieved / peaks["hbm_gbs"]}
     roof["traffic"] = _profiled_traffic(cfg.name, wl.path_name())
     roof["traffic_unit"] = "bytes per call (DRAM read + write, ncu), averaged over the points"
+    rec = PROFILED_TRAFFIC.get((cfg.name, wl.path_name()))
+    roof["traffic_source"] = rec[2] if roof["traffic"] is not None else None
     roof["peak_source"] = peaks["source"] + " (burst: the step is timed alone)"
     roof["kernel"] = kern_name
     roof["call_ms_mean"] = call_ms
