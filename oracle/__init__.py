@@ -86,6 +86,9 @@ def lib():
         L.orc_ring_bytes.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                      ctypes.c_int64]
         L.orc_ring_bytes.restype = ctypes.c_uint64
+        L.orc_allreduce_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                          ctypes.c_int, ctypes.c_int64]
+        L.orc_allreduce_bytes.restype = ctypes.c_uint64
         _lib = L
     return _lib
 
@@ -224,6 +227,16 @@ def reconcile(n_ranks: int, hidden: int, x: np.ndarray, w_rows: np.ndarray,
 
 def ring_bytes(n_ranks: int, tokens: int, hidden: int, elem_bytes: int, points: int) -> int:
     return int(lib().orc_ring_bytes(n_ranks, tokens, hidden, elem_bytes, points))
+
+
+ALLREDUCE_SCHEMES = {"ring": 0, "naive": 1, "sharp": 2}
+
+
+def allreduce_bytes(scheme: str, n_ranks: int, tokens: int, hidden: int, elem_bytes: int,
+                    points: int) -> int:
+    """Per-rank NVLink bytes of one all-reduce scheme (see orc_allreduce_bytes)."""
+    return int(lib().orc_allreduce_bytes(ALLREDUCE_SCHEMES[scheme], n_ranks, tokens, hidden,
+                                         elem_bytes, points))
 
 
 def cores() -> int:

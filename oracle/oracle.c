@@ -363,6 +363,55 @@ uint64_t orc_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_by
     return 2u * (uint64_t)(n_ranks - 1) * payload * (uint64_t)points / (uint64_t)n_ranks;
 }
 
+/*
+ * Bytes one rank's NVLink port carries for the all-reduce of `payload` bytes
+ * per rank, under three schemes of the all-reduce section of the NVL72
+ * hosting post, counted message by message over slices of B/N bytes (B =
+ * tokens * hidden * elem_bytes * points):
+ *   0 ring (reduce the slices, then broadcast): rank r receives slice r from
+ *     each of its N-1 peers and sends its reduced slice r to each of them;
+ *     2(N-1) slice messages (the same count as the first page's
+ *     reduce-scatter plus all-gather).
+ *   1 naive: rank r loads every peer's whole buffer: N-1 buffers of N slices.
+ *   2 switch reduction (SHARP): slice r is summed inside the switch, which
+ *     reads it from the N-1 peers and hands rank r one reduced slice; counted
+ *     for slice r: N-1 peer reads plus 1 slice from the switch.
+ * One rank communicates nothing. Exact: slice messages are counted, then
+ * multiplied by B before the one division by N.
+ */
+uint64_t orc_allreduce_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,
+                             int64_t points)
+{
+    if (n_ranks < 1 || tokens < 0 || hidden < 0 || elem_bytes < 0 || points < 0)
+        return 0;
+    if (n_ranks == 1)
+        return 0;
+    uint64_t slices = 0;  /* slice messages counted at rank 0 */
+    const int r = 0;
+    if (scheme == 0) {
+        for (int peer = 0; peer < n_ranks; ++peer)
+            if (peer != r)
+                slices += 1;  /* peer's slice r arrives for the reduction */
+        for (int peer = 0; peer < n_ranks; ++peer)
+            if (peer != r)
+                slices += 1;  /* reduced slice r goes out to the peer */
+    } else if (scheme == 1) {
+        for (int peer = 0; peer < n_ranks; ++peer)
+            if (peer != r)
+                for (int c = 0; c < n_ranks; ++c)
+                    slices += 1;  /* every slice of the peer's buffer */
+    } else if (scheme == 2) {
+        for (int peer = 0; peer < n_ranks; ++peer)
+            if (peer != r)
+                slices += 1;  /* the switch reads the peer's slice r */
+        slices += 1;          /* the reduced slice r from the switch */
+    } else {
+        return 0;
+    }
+    const uint64_t b = (uint64_t)tokens * (uint64_t)hidden * (uint64_t)elem_bytes * (uint64_t)points;
+    return slices * b / (uint64_t)n_ranks;
+}
+
 /* ------------------------------------------------------- array helpers -- */
 
 void orc_bf16_rne_array(int64_t count, const float *in, uint16_t *out)

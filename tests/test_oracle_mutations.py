@@ -19,6 +19,7 @@ from oracle import build as obuild
 import test_oracle_bf16 as tb
 import test_oracle_reconcile as trc
 import test_oracle_ring as trg
+import test_oracle_allreduce as tar
 
 SRC = open(obuild.SRC).read()
 
@@ -66,6 +67,14 @@ MUTATIONS = {
     "bytes_n": ("return 2u * (uint64_t)(n_ranks - 1) * payload",
                 "return 2u * (uint64_t)(n_ranks) * payload",
                 [trg.test_ring_bytes_pages_worked_example]),
+    # all-reduce schemes: the switch hands back every slice, not one
+    "sharp_all_slices": ("        slices += 1;          /* the reduced slice r from the switch */",
+                         "        slices += (uint64_t)n_ranks;",
+                         [tar.test_allreduce_bytes_golden]),
+    # all-reduce schemes: the naive reader also counts its own buffer
+    "naive_self": ("                for (int c = 0; c < n_ranks; ++c)\n                    slices += 1;  /* every slice of the peer's buffer */",
+                   "                for (int c = 0; c < n_ranks; ++c)\n                    slices += 1;  /* every slice of the peer's buffer */\n        slices += (uint64_t)n_ranks;",
+                   [tar.test_allreduce_bytes_golden]),
 }
 
 
@@ -93,7 +102,7 @@ def test_pin_catches_mutation(name, monkeypatch):
     mutant = ctypes.CDLL(path)
     for fn in ("orc_bf16_rne", "orc_bf16_rne_f64", "orc_f32", "orc_bf16_rne_array",
                "orc_bf16_rne_f64_array", "orc_partials", "orc_ring", "orc_residual",
-               "orc_reconcile", "orc_ring_bytes"):
+               "orc_reconcile", "orc_ring_bytes", "orc_allreduce_bytes"):
         f = getattr(mutant, fn)
         g = getattr(real, fn)
         f.argtypes, f.restype = g.argtypes, g.restype
