@@ -205,6 +205,29 @@ TP_API tp_status tp_ring_reduce(const tp_plan* plan, const void* partials, const
 TP_API uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,
                        int64_t points);
 
+/* All-reduce schemes of tp_allreduce_bytes. */
+typedef enum {
+    TP_ALLREDUCE_RING = 0,   /* reduce the slices, then broadcast them */
+    TP_ALLREDUCE_NAIVE = 1,  /* every rank loads every peer's whole buffer */
+    TP_ALLREDUCE_SWITCH = 2  /* the switch sums each slice (SHARP, multimem) */
+} tp_allreduce_scheme;
+
+/* Bytes one rank's NVLink port carries for the all-reduce of B = tokens *
+ * hidden * elem_bytes * points bytes per rank, under the schemes of the NVL72
+ * hosting post's All-reduce section:
+ *   RING    2(N-1)/N * B   (= tp_ring_bytes; N ranks move 2(N-1)B in all)
+ *   NAIVE   (N-1) * B      (N(N-1)B read in all)
+ *   SWITCH  B              (the peers' N-1 copies of the rank's slice are
+ *                           read by the switch, which returns one reduced
+ *                           slice: N/(2(N-1)) of the ring's transfers)
+ * Reading: the switch scheme counts, like the page, the transfers of the
+ * reduction of one rank's slice on both sides of the switch. Host only,
+ * exact (multiplies before the one division). Returns 0 for one rank, an
+ * unknown scheme, n_ranks < 1 or a negative argument. The pages' kernels for
+ * these schemes run across GPUs; this is their byte model only. */
+TP_API uint64_t tp_allreduce_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hidden,
+                                   int elem_bytes, int64_t points);
+
 /* Releases a plan. NULL is allowed. */
 TP_API void tp_plan_destroy(tp_plan* plan);
 

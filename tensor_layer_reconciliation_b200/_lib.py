@@ -23,7 +23,7 @@ EXPORTED = (
     "tp_plan_packed_bytes",
     "tp_pack_weights",
     "tp_rowlinear_reconcile", "tp_rowlinear_reconcile_noalloc", "tp_rowlinear_partials",
-    "tp_ring_reduce", "tp_ring_bytes",
+    "tp_ring_reduce", "tp_ring_bytes", "tp_allreduce_bytes",
     "tp_plan_destroy", "tp_status_string", "tp_last_cuda_error", "tp_device_error_flags",
 )
 
@@ -68,6 +68,8 @@ def _load() -> ctypes.CDLL:
     L.tp_ring_reduce.restype = ctypes.c_int
     L.tp_ring_bytes.argtypes = [ctypes.c_int, i64, i64, ctypes.c_int, i64]
     L.tp_ring_bytes.restype = ctypes.c_uint64
+    L.tp_allreduce_bytes.argtypes = [ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int, i64]
+    L.tp_allreduce_bytes.restype = ctypes.c_uint64
     L.tp_plan_destroy.argtypes = [vp]
     L.tp_plan_destroy.restype = None
     L.tp_status_string.argtypes = [ctypes.c_int]
@@ -137,6 +139,14 @@ def tp_rowlinear_partials(plan, x: int, w_packed: int, partials: int, tokens: in
 
 def tp_ring_reduce(plan, partials: int, residual: int, out: int, tokens: int, stream: int) -> int:
     return LIB.tp_ring_reduce(plan, partials, residual, out, tokens, stream)
+
+
+TP_ALLREDUCE_RING, TP_ALLREDUCE_NAIVE, TP_ALLREDUCE_SWITCH = 0, 1, 2
+
+
+def tp_allreduce_bytes(scheme: int, n_ranks: int, tokens: int, hidden: int, elem_bytes: int,
+                       points: int) -> int:
+    return int(LIB.tp_allreduce_bytes(scheme, n_ranks, tokens, hidden, elem_bytes, points))
 
 
 def tp_ring_bytes(n_ranks: int, tokens: int, hidden: int, elem_bytes: int, points: int) -> int:

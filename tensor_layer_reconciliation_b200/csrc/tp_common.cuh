@@ -35,6 +35,15 @@ __device__ __forceinline__ uint16_t bf16_add(uint16_t a, uint16_t b) {
     return f32_to_bf16_rne(__fadd_rn(bf16_bits_to_f32(a), bf16_bits_to_f32(b)));
 }
 
+// Two ring adds at once on packed bf16 pairs: add.rn.bf16x2 rounds the exact
+// sum once to bf16, which equals bf16_add's fp32 add then rounding (fp32 holds
+// more than 2 * 8 + 2 bits, so the double rounding is innocuous).
+__device__ __forceinline__ uint32_t bf16x2_add(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -632,6 +632,20 @@ uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_byt
     return 2ull * static_cast<uint64_t>(n_ranks - 1) * payload / static_cast<uint64_t>(n_ranks);
 }
 
+uint64_t tp_allreduce_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,
+                            int64_t points) {
+    if (n_ranks < 2 || tokens < 0 || hidden < 0 || elem_bytes < 0 || points < 0) return 0;
+    const uint64_t n = static_cast<uint64_t>(n_ranks);
+    const uint64_t b = static_cast<uint64_t>(tokens) * static_cast<uint64_t>(hidden) *
+                       static_cast<uint64_t>(elem_bytes) * static_cast<uint64_t>(points);
+    switch (scheme) {
+        case TP_ALLREDUCE_RING: return 2ull * (n - 1) * b / n;
+        case TP_ALLREDUCE_NAIVE: return (n - 1) * b;
+        case TP_ALLREDUCE_SWITCH: return b;
+        default: return 0;
+    }
+}
+
 void tp_plan_destroy(tp_plan* plan) { delete plan; }
 
 const char* tp_status_string(tp_status status) {

@@ -94,3 +94,21 @@ def test_product_does_not_import_oracle():
             text = open(f).read()
             assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
             assert "liboracle" not in text and "oracle.c" not in text, f
+
+
+@pytest.mark.parametrize("scheme", ["ring", "naive", "sharp"])
+def test_allreduce_bytes_matches_oracle(scheme):
+    """The library's all-reduce byte model (host code) against the oracle's
+    message count, over rank counts, shapes and bad arguments."""
+    import oracle
+    import tensor_layer_reconciliation_b200 as tlr
+    code = {"ring": tlr.TP_ALLREDUCE_RING, "naive": tlr.TP_ALLREDUCE_NAIVE,
+            "sharp": tlr.TP_ALLREDUCE_SWITCH}[scheme]
+    for n in range(0, 10):
+        for m, h, e, pts in [(1, 5120, 2, 128), (32, 5120, 2, 128), (3, 840, 4, 7), (0, 5, 2, 1),
+                             (64, 4096, 2, 96), (5, 7, 1, 3), (2, -1, 2, 1)]:
+            assert tlr.tp_allreduce_bytes(code, n, m, h, e, pts) == \
+                oracle.allreduce_bytes(scheme, n, m, h, e, pts), (n, m, h, e, pts)
+    assert tlr.tp_allreduce_bytes(code, 4, 1, 5120, 2, 128) == \
+        oracle.allreduce_bytes(scheme, 4, 1, 5120, 2, 128)
+    assert tlr.tp_allreduce_bytes(9, 4, 1, 5120, 2, 128) == 0
