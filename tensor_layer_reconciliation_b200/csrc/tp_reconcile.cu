@@ -12,6 +12,7 @@
 
 #include "tp_kernels_exact.cuh"
 #include "tp_kernels_tc.cuh"
+#include "tp_kernels_tc2.cuh"
 #include "tp_reconcile.h"
 
 // Fixed scratch for tp_rowlinear_reconcile_noalloc: fold counters and the
@@ -261,7 +262,9 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split) {
     return c;
 }
 
-tp_status encode_tc_maps(const tp_plan* p, const TcConfig& c, const void* x, const void* w,
+// x_box_tokens: token rows of one activation box (the 1-SM kernel's BN, or
+// the half tile a CTA of a pair stages).
+tp_status encode_tc_maps(const tp_plan* p, int x_box_tokens, const void* x, const void* w,
                          int64_t tokens, CUtensorMap* mw, CUtensorMap* mx) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
     if (!enc) return cuda_fail(g_encode_err);
@@ -284,7 +287,7 @@ tp_status encode_tc_maps(const tp_plan* p, const TcConfig& c, const void* x, con
                                     static_cast<cuuint64_t>(tokens)};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks) * 2,
                                        static_cast<cuuint64_t>(p->k) * 2};
-        const cuuint32_t box[3] = {tpr::kTcKBlock, 1, static_cast<cuuint32_t>(c.bn)};
+        const cuuint32_t box[3] = {tpr::kTcKBlock, 1, static_cast<cuuint32_t>(x_box_tokens)};
         CUresult r = enc(mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides,
                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -300,6 +303,37 @@ size_t tc_partial_bytes(const tp_plan* p, const TcConfig& c, int64_t tokens) {
            static_cast<size_t>(p->hidden) * (c.splits > 1 ? 4u * c.splits : 2u);
 }
 
+// The partials [N][M][H] of a prefill-sized call on CTA pairs: units of
+// (rank, 256 rows of H, 256 tokens), two CTAs per unit, one per SM.
+tp_status launch_tc2(const tp_plan* p, const void* x, const void* w, void* partials, int64_t tokens,
+                     cudaStream_t stream) {
+    const int h_pairs = static_cast<int>((p->hidden + 2 * tpr::kTcRows - 1) / (2 * tpr::kTcRows));
+    const int m_tiles = static_cast<int>((tokens + tpr::kTc2Tokens - 1) / tpr::kTc2Tokens);
+    const int units = p->n_ranks * h_pairs * m_tiles;
+    const size_t fixed = (2 * tpr::kTc2MaxStages + 5) * sizeof(uint64_t) + 16 + 1024;
+    const size_t budget = std::min<size_t>(200 * 1024, static_cast<size_t>(p->smem_optin));
+    const int stages = static_cast<int>(std::min<size_t>(tpr::kTc2MaxStages, (budget - fixed) / tpr::kTc2Stage));
+    if (stages < 2) return TP_ERR_UNSUPPORTED;
+    const size_t smem = fixed + static_cast<size_t>(stages) * tpr::kTc2Stage;
+    const int pairs = std::min(units, p->sm_count / 2);
+    CUtensorMap mw, mx;
+    tp_status st = encode_tc_maps(p, tpr::kTc2HalfTokens, x, w, tokens, &mw, &mx);
+    if (st != TP_OK) return st;
+    tpr::Tc2Params prm{};
+    prm.n_ranks = p->n_ranks;
+    prm.ks = static_cast<int>(p->ks);
+    prm.hidden = static_cast<int>(p->hidden);
+    prm.tokens = static_cast<int>(tokens);
+    prm.h_pairs = h_pairs;
+    prm.m_tiles = m_tiles;
+    prm.units = units;
+    prm.stages = stages;
+    prm.partials = static_cast<uint16_t*>(partials);
+    cudaError_t e = launch_pdl(tpr::tc2_partial_kernel, dim3(static_cast<unsigned>(2 * pairs)),
+                               dim3(tpr::kTcThreads), smem, stream, mw, mx, prm);
+    return e == cudaSuccess ? TP_OK : cuda_fail(e);
+}
+
 // fold: the kernel also runs S2-S4 (residual, out) for few tokens, counting
 // stored parts per H tile in `counters` (zero on entry, zero on return);
 // else a ring kernel must follow.
@@ -309,8 +343,11 @@ tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partia
     const TcConfig c = tc_config(p, tokens, allow_split);
     if (c.stages < 2) return TP_ERR_UNSUPPORTED;
     if (fold && (c.m_tiles != 1 || tokens > 2)) return TP_ERR_UNSUPPORTED;  // the kernel folds <= 2 rows
+    // Prefill-sized tiles without a k-split run on CTA pairs (2-SM MMA).
+    if (c.bn == tpr::kTc2Tokens && c.splits == 1 && !fold && p->sm_count >= 2)
+        return launch_tc2(p, x, w, partials, tokens, stream);
     CUtensorMap mw, mx;
-    tp_status st = encode_tc_maps(p, c, x, w, tokens, &mw, &mx);
+    tp_status st = encode_tc_maps(p, c.bn, x, w, tokens, &mw, &mx);
     if (st != TP_OK) return st;
     tpr::TcParams prm{};
     prm.n_ranks = p->n_ranks;
@@ -366,14 +403,15 @@ tp_status launch_ring(const tp_plan* p, const void* partials, const void* residu
 // Lets every exact kernel use the device's opt-in shared memory less its own
 // static shared memory; returns the smallest such dynamic allowance.
 cudaError_t set_kernel_attrs(int smem_optin, int* dyn_max) {
-    const void* kernels[8] = {reinterpret_cast<const void*>(tpr::exact_partial_kernel<1>),
+    const void* kernels[9] = {reinterpret_cast<const void*>(tpr::exact_partial_kernel<1>),
                               reinterpret_cast<const void*>(tpr::exact_partial_kernel<2>),
                               reinterpret_cast<const void*>(tpr::exact_partial_kernel<4>),
                               reinterpret_cast<const void*>(tpr::exact_partial_kernel<8>),
                               reinterpret_cast<const void*>(tpr::tc_partial_kernel<32>),
                               reinterpret_cast<const void*>(tpr::tc_partial_kernel<64>),
                               reinterpret_cast<const void*>(tpr::tc_partial_kernel<128>),
-                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<256>)};
+                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<256>),
+                              reinterpret_cast<const void*>(tpr::tc2_partial_kernel)};
     int lowest = smem_optin;
     for (const void* k : kernels) {
         cudaFuncAttributes fa{};

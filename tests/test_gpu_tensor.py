@@ -49,6 +49,9 @@ SHAPES = [             # N, M, K, H
     (4, 100, 640, 384),     # token tile 128 with a ragged tail; 3 weight tiles
     (4, 300, 512, 256),     # token tile 256, two tiles, second ragged
     (1, 48, 400, 200),      # N = 1; K/N = 400 ends in a partial 64-column block; H % 128 != 0
+    (8, 512, 1024, 4096),   # prefill-sized: CTA pairs (2-SM MMA), 16 H-tile pairs, 2 token tiles
+    (8, 300, 1024, 4224),   # CTA pairs, odd H-tile count (last pair half out of range), ragged tokens
+    (1, 260, 512, 768),     # CTA pairs for the partials, N = 1, ragged second token tile
 ]
 IDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in SHAPES]
 
