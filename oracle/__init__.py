@@ -47,6 +47,7 @@ _F64P = ctypes.POINTER(ctypes.c_double)
 _F32P = ctypes.POINTER(ctypes.c_float)
 _I64P = ctypes.POINTER(ctypes.c_int64)
 _U64P = ctypes.POINTER(ctypes.c_uint64)
+_U8P = ctypes.POINTER(ctypes.c_uint8)
 
 ORC_OK, ORC_ERR_ARGS, ORC_ERR_ALLOC, ORC_ERR_RING = 0, 1, 2, 3
 
@@ -89,6 +90,15 @@ def lib():
         L.orc_allreduce_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
                                           ctypes.c_int, ctypes.c_int64]
         L.orc_allreduce_bytes.restype = ctypes.c_uint64
+        L.orc_e4m3_rne.argtypes = [ctypes.c_double]
+        L.orc_e4m3_rne.restype = ctypes.c_uint8
+        L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_value.restype = ctypes.c_double
+        L.orc_mx_quantize.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, _U16P, _U8P, _U8P]
+        L.orc_mx_quantize.restype = ctypes.c_int
+        L.orc_mx_dequant_bf16.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, _U8P, _U8P,
+                                          _U16P]
+        L.orc_mx_dequant_bf16.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -227,6 +237,42 @@ def reconcile(n_ranks: int, hidden: int, x: np.ndarray, w_rows: np.ndarray,
 
 def ring_bytes(n_ranks: int, tokens: int, hidden: int, elem_bytes: int, points: int) -> int:
     return int(lib().orc_ring_bytes(n_ranks, tokens, hidden, elem_bytes, points))
+
+
+def e4m3_rne(v: float) -> int:
+    """E4M3 code of the exact value v, nearest even, saturating at 448."""
+    return int(lib().orc_e4m3_rne(float(v)))
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().orc_e4m3_value(int(code)))
+
+
+def mx_quantize(n_ranks: int, w_hk: np.ndarray):
+    """Linear weight [H, K] bf16 -> (q [N, H, K/N] uint8 E4M3 codes,
+    scales [N, H, K/N/32] uint8 E8M0 bytes)."""
+    w = _u16(w_hk)
+    h, k = w.shape
+    ks = k // n_ranks
+    q = np.empty((n_ranks, h, ks), dtype=np.uint8)
+    sc = np.empty((n_ranks, h, ks // 32), dtype=np.uint8)
+    rc = lib().orc_mx_quantize(n_ranks, h, k, _ptr(w, _U16P), _ptr(q, _U8P), _ptr(sc, _U8P))
+    if rc != ORC_OK:
+        raise OracleError(f"orc_mx_quantize failed with {rc}")
+    return q, sc
+
+
+def mx_dequant_bf16(n_ranks: int, q: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """MXFP8 shards -> the dequantised Linear weight [H, K] as bf16 bit patterns."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    n, h, ks = q.shape
+    w = np.empty((h, n * ks), dtype=np.uint16)
+    rc = lib().orc_mx_dequant_bf16(n_ranks, h, n * ks, _ptr(q, _U8P), _ptr(scales, _U8P),
+                                   _ptr(w, _U16P))
+    if rc != ORC_OK:
+        raise OracleError(f"orc_mx_dequant_bf16 failed with {rc}")
+    return w
 
 
 ALLREDUCE_SCHEMES = {"ring": 0, "naive": 1, "sharp": 2}

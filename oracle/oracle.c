@@ -27,6 +27,10 @@
  *      ranges of each token's hidden vector; chunk c is folded P_c, P_c+1, ...,
  *      P_c-1, left to right.
  *   3. Residual. out = bf16_rne(f32(residual) + f32(reduced)).
+ *   4. MXFP8 weight shards (the "next" weight format): quantisation of the
+ *      Linear weight to E4M3 codes with one E8M0 scale per 32 weights of a
+ *      rank's slice, and back; a reconciliation over such shards is the
+ *      point above over the dequantised weights (exact in bf16).
  *
  * Build: plain C11, -ffp-contract=off (no fused multiply-add other than the
  * explicit fmaf), no fast-math, so every float operation is one IEEE
@@ -410,6 +414,130 @@ uint64_t orc_allreduce_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hi
     }
     const uint64_t b = (uint64_t)tokens * (uint64_t)hidden * (uint64_t)elem_bytes * (uint64_t)points;
     return slices * b / (uint64_t)n_ranks;
+}
+
+/* -------------------------------------------------- MXFP8 weight shards -- */
+/*
+ * Micro-scaled FP8 weights (the NVL72 hosting post quantises the MoE GEMM's
+ * weights to MXFP8; the format itself is the OCP Microscaling (MX) v1.0
+ * specification's MXFP8 E4M3): every block of 32 consecutive weights along
+ * K, inside one rank's slice, shares one E8M0 scale X = 2^s (byte s + 127),
+ * and each weight is stored as the FP8 E4M3 value nearest to w / X.
+ *   s = floor(log2(max |w| of the block)) - 8   (8 = E4M3's largest exponent),
+ *       clamped to [-127, 127]; an all-zero block takes s = -127;
+ *   w / X rounded to nearest, ties to even, on the E4M3 grid (3 fraction
+ *       bits; normals 2^-6 .. 448, subnormals in steps of 2^-9), saturating
+ *       at +-448 (the block maximum can exceed 448 before rounding).
+ * Reading: the specification leaves the rounding and overflow of the
+ * element conversion to the implementation; round-to-nearest-even with
+ * saturation is used, as for the bf16 rounding of the rest of the path.
+ */
+
+/* E4M3 code of the exact value v (|v| < 2^10), rounded to nearest even,
+ * saturating at 448. */
+uint8_t orc_e4m3_rne(double v)
+{
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs(v);
+    if (a >= 448.0)
+        return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {                 /* subnormal: multiples of 2^-9 */
+        const double q = a * 512.0;           /* exact: a has few significant bits */
+        double m = floor(q);
+        const double rem = q - m;
+        if (rem > 0.5 || (rem == 0.5 && fmod(m, 2.0) == 1.0))
+            m += 1.0;
+        return sign | (uint8_t)m;             /* m == 8 is the smallest normal, 0x08 */
+    }
+    int e;
+    (void)frexp(a, &e);
+    e -= 1;                                   /* a = f * 2^e, f in [1, 2) */
+    const double q = (ldexp(a, -e) - 1.0) * 8.0;
+    double m = floor(q);
+    const double rem = q - m;
+    if (rem > 0.5 || (rem == 0.5 && fmod(m, 2.0) == 1.0))
+        m += 1.0;
+    if (m == 8.0) {
+        m = 0.0;
+        e += 1;
+    }
+    return sign | (uint8_t)(((e + 7) << 3) | (int)m);
+}
+
+/* Value of an E4M3 code (never NaN here: the encoder does not produce 0x7F). */
+double orc_e4m3_value(uint8_t c)
+{
+    const int ex = (c >> 3) & 0xF, m = c & 7;
+    const double mag = ex == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, ex - 7);
+    return (c & 0x80) ? -mag : mag;
+}
+
+/* Shared exponent of a block from its largest magnitude. */
+static int mx_shared_exp(double amax)
+{
+    if (amax == 0.0)
+        return -127;
+    int e;
+    (void)frexp(amax, &e);
+    int s = (e - 1) - 8;
+    if (s < -127)
+        s = -127;
+    if (s > 127)
+        s = 127;
+    return s;
+}
+
+/* Linear weight [hidden][k] (bf16) -> per-rank MXFP8 shards:
+ *   q      [n_ranks][hidden][k/n_ranks] E4M3 codes
+ *   scales [n_ranks][hidden][k/n_ranks/32] E8M0 bytes (s + 127)
+ * k/n_ranks must be a multiple of 32 (blocks never straddle two ranks). */
+int orc_mx_quantize(int n_ranks, int64_t hidden, int64_t k, const uint16_t *w_hk, uint8_t *q,
+                    uint8_t *scales)
+{
+    if (n_ranks < 1 || hidden < 0 || k < 0 || k % n_ranks != 0 || (k / n_ranks) % 32 != 0)
+        return ORC_ERR_ARGS;
+    const int64_t ks = k / n_ranks, nb = ks / 32;
+    for (int r = 0; r < n_ranks; ++r)
+        for (int64_t h = 0; h < hidden; ++h)
+            for (int64_t b = 0; b < nb; ++b) {
+                const uint16_t *w = w_hk + h * k + (int64_t)r * ks + 32 * b;
+                double amax = 0.0;
+                for (int i = 0; i < 32; ++i) {
+                    const double a = fabs((double)orc_f32(w[i]));
+                    if (a > amax)
+                        amax = a;
+                }
+                const int s = mx_shared_exp(amax);
+                const int64_t row = (int64_t)r * hidden + h;
+                scales[row * nb + b] = (uint8_t)(s + 127);
+                for (int i = 0; i < 32; ++i)
+                    q[row * ks + 32 * b + i] = orc_e4m3_rne(ldexp((double)orc_f32(w[i]), -s));
+            }
+    return ORC_OK;
+}
+
+/* Dequantised shards back in the Linear layout [hidden][k] as bf16: every
+ * value E4M3 * 2^s has at most 4 significant bits, so it is exact in bf16
+ * unless it leaves bf16's range (returns ORC_ERR_ARGS then, which only
+ * blocks whose largest weight is below 2^-116 can cause). */
+int orc_mx_dequant_bf16(int n_ranks, int64_t hidden, int64_t k, const uint8_t *q,
+                        const uint8_t *scales, uint16_t *w_hk)
+{
+    if (n_ranks < 1 || hidden < 0 || k < 0 || k % n_ranks != 0 || (k / n_ranks) % 32 != 0)
+        return ORC_ERR_ARGS;
+    const int64_t ks = k / n_ranks, nb = ks / 32;
+    for (int r = 0; r < n_ranks; ++r)
+        for (int64_t h = 0; h < hidden; ++h)
+            for (int64_t j = 0; j < ks; ++j) {
+                const int64_t row = (int64_t)r * hidden + h;
+                const int s = (int)scales[row * nb + j / 32] - 127;
+                const double v = ldexp(orc_e4m3_value(q[row * ks + j]), s);
+                const uint16_t b = orc_bf16_rne_f64(v);
+                if ((double)orc_f32(b) != v)
+                    return ORC_ERR_ARGS;
+                w_hk[h * k + (int64_t)r * ks + j] = b;
+            }
+    return ORC_OK;
 }
 
 /* ------------------------------------------------------- array helpers -- */

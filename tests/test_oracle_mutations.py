@@ -20,6 +20,7 @@ import test_oracle_bf16 as tb
 import test_oracle_reconcile as trc
 import test_oracle_ring as trg
 import test_oracle_allreduce as tar
+import test_oracle_mx as tmx
 
 SRC = open(obuild.SRC).read()
 
@@ -75,6 +76,16 @@ MUTATIONS = {
     "naive_self": ("                for (int c = 0; c < n_ranks; ++c)\n                    slices += 1;  /* every slice of the peer's buffer */",
                    "                for (int c = 0; c < n_ranks; ++c)\n                    slices += 1;  /* every slice of the peer's buffer */\n        slices += (uint64_t)n_ranks;",
                    [tar.test_allreduce_bytes_golden]),
+    # MXFP8: element rounding half away from zero instead of to even
+    "e4m3_half_up": ("if (rem > 0.5 || (rem == 0.5 && fmod(m, 2.0) == 1.0))",
+                     "if (rem >= 0.5)",
+                     [tmx.test_e4m3_midpoints_go_to_even_and_saturation]),
+    # MXFP8: shared exponent from E4M3's bias instead of its largest exponent
+    "mx_exp_off_by_one": ("int s = (e - 1) - 8;", "int s = (e - 1) - 7;",
+                          [tmx.test_scale_rule_and_block_max]),
+    # MXFP8: no saturation at 448
+    "e4m3_no_saturation": ("    if (a >= 448.0)\n        return sign | 0x7E;\n", "",
+                           [tmx.test_e4m3_midpoints_go_to_even_and_saturation]),
 }
 
 
@@ -102,7 +113,8 @@ def test_pin_catches_mutation(name, monkeypatch):
     mutant = ctypes.CDLL(path)
     for fn in ("orc_bf16_rne", "orc_bf16_rne_f64", "orc_f32", "orc_bf16_rne_array",
                "orc_bf16_rne_f64_array", "orc_partials", "orc_ring", "orc_residual",
-               "orc_reconcile", "orc_ring_bytes", "orc_allreduce_bytes"):
+               "orc_reconcile", "orc_ring_bytes", "orc_allreduce_bytes", "orc_e4m3_rne",
+               "orc_e4m3_value", "orc_mx_quantize", "orc_mx_dequant_bf16"):
         f = getattr(mutant, fn)
         g = getattr(real, fn)
         f.argtypes, f.restype = g.argtypes, g.restype
