@@ -91,10 +91,11 @@ class Workload:
     copy each per end-to-end step); the outputs likewise (one copy back).
     """
 
-    def __init__(self, cfg, device, variant="auto", staged=False):
+    def __init__(self, cfg, device, variant="auto", staged=False, weights="bf16"):
         import tensor_layer_reconciliation_b200 as tlr
         self.cfg = cfg
         self.device = device
+        self.weights = weights
         m, h, n = cfg.tokens, cfg.hidden, cfg.n_ranks
         self.plans = {}
         for p in cfg.points:
@@ -113,7 +114,10 @@ class Workload:
             self.x(i).copy_(point_tensor(cfg, p, KIND_X, device))
             self.res(i).copy_(point_tensor(cfg, p, KIND_RESIDUAL, device))
             w = point_tensor(cfg, p, KIND_W, device)
-            self.w_packed.append(self.plans[p.k].pack_weights(w))
+            if weights == "mxfp8":        # (E4M3 codes, E8M0 scales) per point
+                self.w_packed.append(self.plans[p.k].pack_weights_mxfp8(w))
+            else:
+                self.w_packed.append(self.plans[p.k].pack_weights(w))
             del w
         torch.cuda.synchronize(device)
 
@@ -129,21 +133,40 @@ class Workload:
         m, h = self.cfg.tokens, self.cfg.hidden
         return self.out_all[i * m * h:(i + 1) * m * h].view(m, h)
 
+    def call(self, i, stream=None):
+        """The reconciliation of point i through the public API."""
+        plan = self.plans[self.cfg.points[i].k]
+        if self.weights == "mxfp8":
+            q, sc = self.w_packed[i]
+            plan.reconcile_mxfp8(self.x(i), q, sc, self.res(i), out=self.out(i), stream=stream)
+        else:
+            plan.reconcile(self.x(i), self.w_packed[i], self.res(i), out=self.out(i),
+                           workspace=self.workspace, stream=stream)
+
     def step(self):
         """One pass of the hot path over every point, on the current stream."""
-        for i, p in enumerate(self.cfg.points):
-            self.plans[p.k].reconcile(self.x(i), self.w_packed[i], self.res(i), out=self.out(i),
-                                      workspace=self.workspace)
+        for i in range(self.cfg.n_points):
+            self.call(i)
+
+    def weight_bytes_read(self):
+        """Bytes of packed weights one step reads."""
+        if self.weights == "mxfp8":
+            return sum(q.numel() + sc.numel() for q, sc in self.w_packed)
+        return self.cfg.weight_bytes()
 
     def path_name(self):
         """Which kernels one call runs: 'tensor' (tensor-core partials, staged),
-        'exact-staged' or 'exact-fused'."""
+        'exact-staged', 'exact-fused' or 'mxfp8' (MXFP8 shards, one fused kernel)."""
+        if self.weights == "mxfp8":
+            return "mxfp8"
         pl = next(iter(self.plans.values()))
         if pl.effective_variant(self.cfg.tokens) == "tensor":
             return "tensor"
         return "exact-staged" if pl.staged else "exact-fused"
 
     def launches_per_step(self):
+        if self.weights == "mxfp8":
+            return self.cfg.n_points
         return sum(self.plans[p.k].launches(self.cfg.tokens) for p in self.cfg.points)
 
     def capture(self):
@@ -315,9 +338,7 @@ class HostPipeline:
                 compute.wait_event(self.ev_out[c])
             with torch.cuda.stream(compute):
                 for i in range(a, b):
-                    p = wl.cfg.points[i]
-                    wl.plans[p.k].reconcile(wl.x(i), wl.w_packed[i], wl.res(i), out=wl.out(i),
-                                            workspace=wl.workspace, stream=compute)
+                    wl.call(i, stream=compute)
             self.ev_done[c].record(compute)
             self.s_out.wait_event(self.ev_done[c])
             with torch.cuda.stream(self.s_out):
@@ -398,6 +419,8 @@ def main(argv=None):
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=CONFIG_ORDER)
     ap.add_argument("--variant", default="auto", choices=["auto", "exact", "tensor"])
     ap.add_argument("--staged", action="store_true")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp8"],
+                    help="mxfp8: MXFP8 weight shards (decode, at most 4 tokens)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=8.0)
@@ -424,7 +447,9 @@ def main(argv=None):
     if args.points:
         cfg = dataclasses.replace(cfg, layers=1, layer_points=cfg.layer_points)
         cfg.points[:] = cfg.points[:args.points]
-    wl = Workload(cfg, device, variant=args.variant, staged=args.staged)
+    if args.weights == "mxfp8" and cfg.tokens > 4:
+        ap.error("--weights mxfp8 takes decode workloads of at most 4 tokens")
+    wl = Workload(cfg, device, variant=args.variant, staged=args.staged, weights=args.weights)
     peaks = _peaks()
 
     graph = wl.capture()
@@ -458,15 +483,15 @@ def main(argv=None):
     # Each call is the hot path of one point: the partial kernel (fused with the
     # fold on the exact path) and, on staged paths, the ring fold kernel. Eager
     # launches add host gaps between calls; the roofline uses the graph time.
-    staged_path = any(pl.workspace_bytes(cfg.tokens) for pl in wl.plans.values())
+    staged_path = (args.weights == "bf16" and
+                   any(pl.workspace_bytes(cfg.tokens) for pl in wl.plans.values()))
     per_launch = []
     for _ in range(2):
         evs = []
         for i, p in enumerate(cfg.points):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            wl.plans[p.k].reconcile(wl.x(i), wl.w_packed[i], wl.res(i), out=wl.out(i),
-                                    workspace=wl.workspace)
+            wl.call(i)
             b.record(stream)
             evs.append((a, b))
         torch.cuda.synchronize(device)
@@ -503,6 +528,9 @@ def main(argv=None):
     value = _job_rate(cfg.tokens, step_ms, world)
     recon = _job_rate(cfg.n_points, step_ms, world)
     step_bytes = cfg.algorithmic_bytes(staged_partials=staged_path)
+    if args.weights == "mxfp8":   # codes + scales in place of bf16 weights; nothing staged
+        step_bytes = (cfg.algorithmic_bytes(staged_partials=False) - cfg.weight_bytes()
+                      + wl.weight_bytes_read())
     flops = cfg.flops()
     tensor_bound = cfg.tokens >= 1024
     # The hot path of one point is one reconciliation call: the partial kernel
@@ -511,8 +539,17 @@ def main(argv=None):
     # device time over the timed region divided by the points per step.
     call_ms = step_ms / cfg.n_points
     kern_bytes = step_bytes   # weights, activations, residual, output (+ staged partials)
-    kern_name = ("reconciliation call: tc_partial_kernel then ring fold kernel" if staged_path
-                 else "reconciliation call: exact_partial_kernel (partials + ring fold + residual)")
+    path = wl.path_name()
+    one_kernel = wl.launches_per_step() == cfg.n_points
+    kern_name = {
+        "mxfp8": "reconciliation call: mx_reconcile_kernel (MXFP8 partials, ring fold, residual)",
+        "exact-fused": "reconciliation call: exact_partial_kernel (partials, ring fold, residual)",
+        "exact-staged": "reconciliation call: exact_partial_kernel then ring_reduce_kernel",
+        "tensor": ("reconciliation call: tc_partial_kernel (partials, in-kernel ring fold, residual)"
+                   if one_kernel else
+                   "reconciliation call: tc_partial_kernel (tc2_partial_kernel on CTA pairs "
+                   "from 129 tokens) then a ring fold kernel"),
+    }[path]
     if tensor_bound:
         achieved = flops / (step_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
@@ -543,7 +580,8 @@ def main(argv=None):
         "tflops_step": flops / (step_ms * 1e-3) / 1e12,
         "config": {"workload": cfg.name, "n_ranks": cfg.n_ranks, "tokens": cfg.tokens,
                    "hidden": cfg.hidden, "points": cfg.n_points,
-                   "weights_gb_per_step": cfg.weight_bytes() / 1e9,
+                   "weights_gb_per_step": wl.weight_bytes_read() / 1e9,
+                   "weights": args.weights,
                    "l2": "no flush: every step streams all points' distinct weights "
                          f"({cfg.weight_bytes() / 1e9:.1f} GB), larger than the 126 MB L2",
                    "variant": args.variant, "staged_partials": staged_path,

@@ -205,6 +205,41 @@ TP_API tp_status tp_ring_reduce(const tp_plan* plan, const void* partials, const
 TP_API uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,
                        int64_t points);
 
+/* ---------------------------------------------------------------------
+ * MXFP8 weight shards. The NVL72 hosting post stores the MoE GEMM's weights
+ * as MXFP8; the layout here is the OCP Microscaling v1.0 MXFP8 (E4M3)
+ * format applied to each rank's slice: every 32 consecutive weights along
+ * K share one E8M0 scale X = 2^s (byte s + 127), s = floor(log2 max|w|) - 8
+ * clamped to [-127, 127] (-127 for an all-zero run), and each weight is the
+ * E4M3 code nearest to w / X, ties to even, saturating at +-448. The
+ * reconciliation over such shards is S1-S4 over the dequantised weights
+ * E4M3 * X, which are exact in bf16 for any run whose largest weight is at
+ * least 2^-116.
+ * ------------------------------------------------------------------- */
+
+/* Sizes of the two shard buffers: q_bytes = H*K (one E4M3 code per weight,
+ * [N][H][K/N]), scale_bytes = H*K/32 ([N][H][K/N/32]). TP_ERR_UNSUPPORTED
+ * when K/N is not a multiple of 32; TP_ERR_INVALID for null arguments. */
+TP_API tp_status tp_plan_mxfp8_bytes(const tp_plan* plan, size_t* q_bytes, size_t* scale_bytes);
+
+/* S0 for MXFP8: Linear weight [H][K] bf16 -> w_q [N][H][K/N] codes and
+ * w_scales [N][H][K/N/32] scales (device buffers of tp_plan_mxfp8_bytes'
+ * sizes; w_hk and w_q 16-byte aligned; no overlap). Asynchronous on
+ * `stream`; the result is identical, bit for bit, to the format's
+ * definition above. */
+TP_API tp_status tp_pack_weights_mxfp8(const tp_plan* plan, const void* w_hk, void* w_q,
+                                       void* w_scales, void* stream);
+
+/* S1-S4 for decode over MXFP8 shards, one kernel, no workspace:
+ *   x, residual, out as in tp_rowlinear_reconcile; w_q, w_scales from
+ *   tp_pack_weights_mxfp8; tokens 0 .. 4 (more: TP_ERR_UNSUPPORTED, the
+ *   fused kernel streams the shards once for all tokens of a decode step).
+ * Partials are fp32 sums rounded once to bf16, in an order of its own
+ * (lanes of a warp split K), then folded in ring order with the residual. */
+TP_API tp_status tp_rowlinear_reconcile_mxfp8(const tp_plan* plan, const void* x, const void* w_q,
+                                              const void* w_scales, const void* residual,
+                                              void* out, int64_t tokens, void* stream);
+
 /* All-reduce schemes of tp_allreduce_bytes. */
 typedef enum {
     TP_ALLREDUCE_RING = 0,   /* reduce the slices, then broadcast them */

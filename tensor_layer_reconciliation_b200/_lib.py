@@ -24,6 +24,7 @@ EXPORTED = (
     "tp_pack_weights",
     "tp_rowlinear_reconcile", "tp_rowlinear_reconcile_noalloc", "tp_rowlinear_partials",
     "tp_ring_reduce", "tp_ring_bytes", "tp_allreduce_bytes",
+    "tp_plan_mxfp8_bytes", "tp_pack_weights_mxfp8", "tp_rowlinear_reconcile_mxfp8",
     "tp_plan_destroy", "tp_status_string", "tp_last_cuda_error", "tp_device_error_flags",
 )
 
@@ -68,6 +69,12 @@ def _load() -> ctypes.CDLL:
     L.tp_ring_reduce.restype = ctypes.c_int
     L.tp_ring_bytes.argtypes = [ctypes.c_int, i64, i64, ctypes.c_int, i64]
     L.tp_ring_bytes.restype = ctypes.c_uint64
+    L.tp_plan_mxfp8_bytes.argtypes = [vp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.tp_plan_mxfp8_bytes.restype = ctypes.c_int
+    L.tp_pack_weights_mxfp8.argtypes = [vp, vp, vp, vp, vp]
+    L.tp_pack_weights_mxfp8.restype = ctypes.c_int
+    L.tp_rowlinear_reconcile_mxfp8.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp]
+    L.tp_rowlinear_reconcile_mxfp8.restype = ctypes.c_int
     L.tp_allreduce_bytes.argtypes = [ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int, i64]
     L.tp_allreduce_bytes.restype = ctypes.c_uint64
     L.tp_plan_destroy.argtypes = [vp]
@@ -139,6 +146,21 @@ def tp_rowlinear_partials(plan, x: int, w_packed: int, partials: int, tokens: in
 
 def tp_ring_reduce(plan, partials: int, residual: int, out: int, tokens: int, stream: int) -> int:
     return LIB.tp_ring_reduce(plan, partials, residual, out, tokens, stream)
+
+
+def tp_plan_mxfp8_bytes(plan):
+    q, sc = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    st = LIB.tp_plan_mxfp8_bytes(plan, ctypes.byref(q), ctypes.byref(sc))
+    return st, q.value, sc.value
+
+
+def tp_pack_weights_mxfp8(plan, w_hk: int, w_q: int, w_scales: int, stream: int) -> int:
+    return LIB.tp_pack_weights_mxfp8(plan, w_hk, w_q, w_scales, stream)
+
+
+def tp_rowlinear_reconcile_mxfp8(plan, x: int, w_q: int, w_scales: int, residual: int, out: int,
+                                 tokens: int, stream: int) -> int:
+    return LIB.tp_rowlinear_reconcile_mxfp8(plan, x, w_q, w_scales, residual, out, tokens, stream)
 
 
 TP_ALLREDUCE_RING, TP_ALLREDUCE_NAIVE, TP_ALLREDUCE_SWITCH = 0, 1, 2

@@ -13,6 +13,7 @@
 #include "tp_kernels_exact.cuh"
 #include "tp_kernels_tc.cuh"
 #include "tp_kernels_tc2.cuh"
+#include "tp_kernels_mx.cuh"
 #include "tp_reconcile.h"
 
 // Fixed scratch for tp_rowlinear_reconcile_noalloc: fold counters and the
@@ -668,6 +669,80 @@ uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_byt
     const uint64_t payload = static_cast<uint64_t>(tokens) * static_cast<uint64_t>(hidden) *
                              static_cast<uint64_t>(elem_bytes) * static_cast<uint64_t>(points);
     return 2ull * static_cast<uint64_t>(n_ranks - 1) * payload / static_cast<uint64_t>(n_ranks);
+}
+
+// ---------------------------------------------------- MXFP8 weight shards --
+
+tp_status tp_plan_mxfp8_bytes(const tp_plan* plan, size_t* q_bytes, size_t* scale_bytes) {
+    if (!plan || !q_bytes || !scale_bytes) return TP_ERR_INVALID;
+    if (plan->ks % tpr::kMxBlock != 0) return TP_ERR_UNSUPPORTED;
+    *q_bytes = static_cast<size_t>(plan->hidden) * static_cast<size_t>(plan->k);
+    *scale_bytes = *q_bytes / tpr::kMxBlock;
+    return TP_OK;
+}
+
+tp_status tp_pack_weights_mxfp8(const tp_plan* plan, const void* w_hk, void* w_q, void* w_scales,
+                                void* stream) {
+    if (!plan || !w_hk || !w_q || !w_scales) return TP_ERR_INVALID;
+    if (plan->ks % tpr::kMxBlock != 0) return TP_ERR_UNSUPPORTED;
+    if (!aligned16(w_hk) || !aligned16(w_q)) return TP_ERR_ALIGN;
+    const size_t wb = static_cast<size_t>(plan->hidden) * plan->k * 2;
+    const size_t qb = wb / 2, sb = qb / tpr::kMxBlock;
+    if (overlaps(w_hk, wb, w_q, qb) || overlaps(w_hk, wb, w_scales, sb) || overlaps(w_q, qb, w_scales, sb))
+        return TP_ERR_INVALID;
+    tp_status st = check_device(plan);
+    if (st != TP_OK) return st;
+    const int64_t blocks_total = static_cast<int64_t>(plan->n_ranks) * plan->hidden * (plan->ks / tpr::kMxBlock);
+    const int64_t grid = std::min<int64_t>((blocks_total + 255) / 256, static_cast<int64_t>(plan->sm_count) * 16);
+    tpr::pack_weights_mx_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(w_hk), static_cast<uint8_t*>(w_q), static_cast<uint8_t*>(w_scales),
+        plan->n_ranks, static_cast<int>(plan->hidden), plan->k, plan->ks);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TP_OK : cuda_fail(e);
+}
+
+tp_status tp_rowlinear_reconcile_mxfp8(const tp_plan* plan, const void* x, const void* w_q,
+                                       const void* w_scales, const void* residual, void* out,
+                                       int64_t tokens, void* stream) {
+    if (!plan) return TP_ERR_INVALID;
+    if (tokens < 0 || tokens > plan->max_tokens) return TP_ERR_INVALID;
+    if (tokens == 0) return TP_OK;
+    if (tokens > tpr::kMxMaxTokens || plan->ks % tpr::kMxBlock != 0) return TP_ERR_UNSUPPORTED;
+    if (!x || !w_q || !w_scales || !residual || !out) return TP_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(w_q) || !aligned16(residual) || !aligned16(out)) return TP_ERR_ALIGN;
+    const size_t mh = static_cast<size_t>(tokens) * plan->hidden * 2;
+    const size_t xb = static_cast<size_t>(tokens) * plan->k * 2;
+    const size_t qb = static_cast<size_t>(plan->hidden) * plan->k, sb = qb / tpr::kMxBlock;
+    if (overlaps(out, mh, x, xb) || overlaps(out, mh, w_q, qb) || overlaps(out, mh, w_scales, sb) ||
+        overlaps(out, mh, residual, mh))
+        return TP_ERR_INVALID;
+    tp_status st = check_device(plan);
+    if (st != TP_OK) return st;
+    tpr::MxParams prm{};
+    prm.n_ranks = plan->n_ranks;
+    prm.hidden = static_cast<int>(plan->hidden);
+    prm.hc = static_cast<int>(plan->hc);
+    prm.tokens = static_cast<int>(tokens);
+    prm.k = plan->k;
+    prm.ks = plan->ks;
+    prm.x = static_cast<const uint16_t*>(x);
+    prm.q = static_cast<const uint8_t*>(w_q);
+    prm.scales = static_cast<const uint8_t*>(w_scales);
+    prm.residual = static_cast<const uint16_t*>(residual);
+    prm.out = static_cast<uint16_t*>(out);
+    const int64_t rows_per_cta = tpr::kMxWarps;
+    const int64_t grid = std::min<int64_t>((plan->hidden + rows_per_cta - 1) / rows_per_cta,
+                                           static_cast<int64_t>(plan->sm_count) * 32);
+    const dim3 g(static_cast<unsigned>(grid)), b(tpr::kMxWarps * 32);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    switch (tokens) {
+        case 1: e = launch_pdl(tpr::mx_reconcile_kernel<1>, g, b, 0, s, prm); break;
+        case 2: e = launch_pdl(tpr::mx_reconcile_kernel<2>, g, b, 0, s, prm); break;
+        case 3: e = launch_pdl(tpr::mx_reconcile_kernel<3>, g, b, 0, s, prm); break;
+        default: e = launch_pdl(tpr::mx_reconcile_kernel<4>, g, b, 0, s, prm); break;
+    }
+    return e == cudaSuccess ? TP_OK : cuda_fail(e);
 }
 
 uint64_t tp_allreduce_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,

@@ -127,6 +127,46 @@ class Plan:
             raise TPError(st, "tp_rowlinear_reconcile")
         return out
 
+    # ---------------------------------------------------- MXFP8 shards --
+
+    def mxfp8_bytes(self):
+        """(code bytes, scale bytes) of this plan's MXFP8 shards."""
+        st, q, sc = _lib.tp_plan_mxfp8_bytes(self._h)
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_plan_mxfp8_bytes")
+        return q, sc
+
+    def pack_weights_mxfp8(self, w_hk: torch.Tensor, stream=None):
+        """Linear weight [H, K] -> (E4M3 codes, E8M0 scales) as flat uint8 tensors."""
+        qb, sb = self.mxfp8_bytes()
+        q = torch.empty(qb, dtype=torch.uint8, device=w_hk.device)
+        sc = torch.empty(sb, dtype=torch.uint8, device=w_hk.device)
+        a = _check(w_hk, "w_hk", (self.hidden, self.k))
+        st = _lib.tp_pack_weights_mxfp8(self._h, a, q.data_ptr(), sc.data_ptr(), _stream(stream))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_pack_weights_mxfp8")
+        return q, sc
+
+    def reconcile_mxfp8(self, x: torch.Tensor, w_q: torch.Tensor, w_scales: torch.Tensor,
+                        residual: torch.Tensor, out: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+        """out [M, H] = residual + ring-ordered sum of x_r . dequant(W_r)^T (M <= 4)."""
+        m = x.shape[0]
+        if out is None:
+            out = torch.empty(m, self.hidden, dtype=torch.bfloat16, device=x.device)
+        qb, sb = self.mxfp8_bytes()
+        for t, name, n in ((w_q, "w_q", qb), (w_scales, "w_scales", sb)):
+            if t.dtype != torch.uint8 or t.numel() != n or t.device.type != "cuda" or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CUDA uint8 tensor of {n} bytes")
+        px = _check(x, "x", (m, self.k))
+        pr = _check(residual, "residual", (m, self.hidden))
+        po = _check(out, "out", (m, self.hidden))
+        st = _lib.tp_rowlinear_reconcile_mxfp8(self._h, px, w_q.data_ptr(), w_scales.data_ptr(), pr, po,
+                                               m, _stream(stream))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_rowlinear_reconcile_mxfp8")
+        return out
+
     def partials(self, x: torch.Tensor, w_packed: torch.Tensor,
                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         """The N partials [N, M, H] (S1 only)."""

@@ -96,14 +96,16 @@ def fragile_mask(p64, pabs):
     return lo != hi
 
 
-def check_against_oracle(out, parts, ref, n):
+def check_against_oracle(out, parts, ref, n, outputs_only=False):
     p64, pabs = ref["p64"], ref["pabs"]
     frag = fragile_mask(p64, pabs)
     exact_p = oracle.bf16_rne_f64(p64)
     # partials: bit-exact where not fragile, a neighbour of d where fragile
-    assert np.array_equal(parts[~frag], exact_p[~frag])
+    # (outputs_only: the kernel keeps its partials on chip; only the oracle's are checked)
     assert np.array_equal(ref["partials"][~frag], exact_p[~frag])
-    if frag.any():
+    if not outputs_only:
+        assert np.array_equal(parts[~frag], exact_p[~frag])
+    if frag.any() and not outputs_only:
         lo = oracle.bf16_rne_f64(np.nextafter(p64[frag], -np.inf) - pabs[frag] * 2.0 ** -19)
         hi = oracle.bf16_rne_f64(p64[frag] + pabs[frag] * 2.0 ** -19)
         g = oracle.f32(parts[frag])
