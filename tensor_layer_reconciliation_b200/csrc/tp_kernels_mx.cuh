@@ -17,7 +17,7 @@ namespace tpr {
 
 constexpr int kMxBlock = 32;        // weights per shared scale
 constexpr int kMxMaxTokens = 4;     // decode token counts the fused kernel takes (MT = tokens)
-constexpr int kMxWarps = 8;         // rows in flight per CTA (one per warp)
+constexpr int kMxWarps = 4;         // output rows in flight per CTA (one per warp)
 
 // Two f32 values -> two E4M3 codes, nearest even, saturating at +-448; the
 // code of `lo` in bits 0-7 of the result.
@@ -111,15 +111,21 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------- S1-S4 --
-// One warp per output row h, all N ranks: lane i takes 16 consecutive
-// weights of every 512 (so a warp load is 512 contiguous bytes), multiplies
-// them by the bf16 activations in fp32 and scales the 16-term sum by the
-// block's 2^s; the warp's sums meet by shuffles. The N partials of the row
-// then fold in ring order from the chunk's owner and meet the residual, so
-// nothing is staged. Weight loads of the first iteration are issued before
-// griddepcontrol.wait. The summation order differs from the oracle's
-// k-ascending chain: a partial can round to the other bf16 neighbour where
-// its exact value lies next to a rounding boundary.
+// One warp per output row h (grid-stride), all N ranks in turn. Lane i
+// takes the 32 consecutive codes of one scale block out of every 1024 (two
+// 16-byte loads: a warp load is 1024 contiguous bytes), two such chunks in
+// flight at a time. The codes become exact f32 values (E4M3 -> f16x2 ->
+// f32), the bf16 activations f32 pairs, and the 32 products of a chunk are
+// summed with packed f32x2 fused multiply-adds (two interleaved chains), the
+// chunk's sum scaled by 2^s into the lane's accumulator; lanes meet by
+// shuffles. The N partials of the row then fold in ring order from the
+// chunk's owner and meet the residual: nothing is staged. Codes of the first
+// chunks are loaded before griddepcontrol.wait. The summation order differs
+// from the oracle's k-ascending chain, so a partial can round to the other
+// bf16 neighbour where its exact value lies next to a rounding boundary.
+constexpr int kMxLaneChunk = kMxBlock;                 // codes per lane per step
+constexpr int kMxWarpStep = 32 * kMxLaneChunk;         // 1024 codes per warp step
+
 struct MxParams {
     int n_ranks;
     int hidden;
@@ -134,12 +140,52 @@ struct MxParams {
     uint16_t* out;             // [M][H]
 };
 
+// d (f32x2) += a (f32x2) * b (f32x2), each lane of the pair rounded once.
+__device__ __forceinline__ void fma_f32x2(uint64_t& d, uint64_t a, uint64_t b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+
+// Sum of the 32 products of one chunk: codes in q0, q1 (32 bytes), the
+// activations' 32 bf16 at xp (64 bytes, 16-byte aligned).
+__device__ __forceinline__ float mx_chunk_dot(const uint4& q0, const uint4& q1, const uint16_t* xp) {
+    const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const uint4* x4 = reinterpret_cast<const uint4*>(xp);
+    uint64_t s0 = 0, s1 = 0;   // two chains of f32x2 sums
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint4 xv = __ldg(x4 + j);              // 8 activations: codes 8j .. 8j+7
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t c = qw[2 * j + i];            // 4 codes
+            const uint32_t a = f16x2_from_e4m3x2(static_cast<uint16_t>(c & 0xFFFF));
+            const uint32_t b = f16x2_from_e4m3x2(static_cast<uint16_t>(c >> 16));
+            const uint64_t w01 = pack_f32x2(f16_lo_to_f32(a), f16_hi_to_f32(a));
+            const uint64_t w23 = pack_f32x2(f16_lo_to_f32(b), f16_hi_to_f32(b));
+            const uint32_t x01 = xw[2 * i], x23 = xw[2 * i + 1];
+            fma_f32x2(s0, pack_f32x2(bf16_lo(x01), bf16_hi(x01)), w01);
+            fma_f32x2(s1, pack_f32x2(bf16_lo(x23), bf16_hi(x23)), w23);
+        }
+    }
+    const float a0 = __uint_as_float(static_cast<uint32_t>(s0));
+    const float a1 = __uint_as_float(static_cast<uint32_t>(s0 >> 32));
+    const float b0 = __uint_as_float(static_cast<uint32_t>(s1));
+    const float b1 = __uint_as_float(static_cast<uint32_t>(s1 >> 32));
+    return (a0 + a1) + (b0 + b1);
+}
+
+// One token: at most 56 registers, so 9 CTAs (36 warps) fit on an SM and a
+// 5120-row call runs in one wave on 148 SMs.
 template <int MT>
-__global__ void __launch_bounds__(kMxWarps * 32)
+__global__ void __launch_bounds__(kMxWarps * 32, MT == 1 ? 9 : 4)
     mx_reconcile_kernel(const MxParams p) {
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t nb = p.ks / kMxBlock;
+    const int ks = static_cast<int>(p.ks);
+    const int nb = ks / kMxBlock;
     bool waited = false;
     for (int h = blockIdx.x * kMxWarps + warp; h < p.hidden; h += gridDim.x * kMxWarps) {
         float part[kMaxRanks][MT];
@@ -149,60 +195,36 @@ __global__ void __launch_bounds__(kMxWarps * 32)
             for (int m = 0; m < MT; ++m) part[r][m] = 0.0f;
 #pragma unroll 1
         for (int r = 0; r < p.n_ranks; ++r) {
-            const uint8_t* qrow = p.q + (static_cast<int64_t>(r) * p.hidden + h) * p.ks;
-            const uint8_t* srow = p.scales + (static_cast<int64_t>(r) * p.hidden + h) * nb;
-            const uint16_t* xr = p.x + static_cast<int64_t>(r) * p.ks;
+            const int64_t row = static_cast<int64_t>(r) * p.hidden + h;
+            const uint8_t* qrow = p.q + row * ks;
+            const uint8_t* srow = p.scales + row * nb;
+            const uint16_t* xr = p.x + static_cast<int64_t>(r) * ks;
             float acc[MT];
 #pragma unroll
             for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
-            // Groups of 4 x 512 weights: a lane's four 16-byte loads are in
-            // flight together.
-            for (int64_t g = static_cast<int64_t>(lane) * 16; g < p.ks; g += 4 * 512) {
-                uint4 qv[4];
-                uint32_t sb[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int64_t k0 = g + u * 512;
-                    qv[u] = k0 < p.ks ? ld_global_nc_v4(qrow + k0) : make_uint4(0, 0, 0, 0);
-                    sb[u] = k0 < p.ks ? srow[k0 / kMxBlock] : 0u;
+            for (int k0 = lane * kMxLaneChunk; k0 < ks; k0 += 2 * kMxWarpStep) {
+                const int k1 = k0 + kMxWarpStep;
+                const bool has1 = k1 < ks;
+                const uint4* qa = reinterpret_cast<const uint4*>(qrow + k0);
+                const uint4 qa0 = ld_global_nc_v4(qa), qa1 = ld_global_nc_v4(qa + 1);
+                const uint32_t sa = srow[k0 / kMxBlock];
+                uint4 qb0 = make_uint4(0, 0, 0, 0), qb1 = qb0;
+                uint32_t sbb = 0;
+                if (has1) {
+                    const uint4* qb = reinterpret_cast<const uint4*>(qrow + k1);
+                    qb0 = ld_global_nc_v4(qb);
+                    qb1 = ld_global_nc_v4(qb + 1);
+                    sbb = srow[k1 / kMxBlock];
                 }
                 if (!waited) {
                     pdl_wait();   // activations and residual follow the stream's order
                     waited = true;
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int64_t k0 = g + u * 512;
-                    if (k0 < p.ks) {
-                        const float sc = e8m0_to_f32(sb[u]);
-                        float w[16];
-                        const uint32_t qw[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint32_t a = f16x2_from_e4m3x2(static_cast<uint16_t>(qw[i] & 0xFFFF));
-                            const uint32_t b = f16x2_from_e4m3x2(static_cast<uint16_t>(qw[i] >> 16));
-                            w[4 * i] = f16_lo_to_f32(a);
-                            w[4 * i + 1] = f16_hi_to_f32(a);
-                            w[4 * i + 2] = f16_lo_to_f32(b);
-                            w[4 * i + 3] = f16_hi_to_f32(b);
-                        }
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) {
-                            // every warp of the CTA reads the same activations: keep them in L1
-                            const uint4* xp =
-                                reinterpret_cast<const uint4*>(xr + static_cast<int64_t>(m) * p.k + k0);
-                            const uint4 x0 = __ldg(xp);
-                            const uint4 x1 = __ldg(xp + 1);
-                            const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                            float s16 = 0.0f;
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                s16 = fmaf(bf16_lo(xw[i]), w[2 * i], s16);
-                                s16 = fmaf(bf16_hi(xw[i]), w[2 * i + 1], s16);
-                            }
-                            acc[m] = fmaf(s16, sc, acc[m]);
-                        }
-                    }
+                for (int m = 0; m < MT; ++m) {
+                    const uint16_t* xm = xr + static_cast<int64_t>(m) * p.k;
+                    acc[m] = fmaf(mx_chunk_dot(qa0, qa1, xm + k0), e8m0_to_f32(sa), acc[m]);
+                    if (has1) acc[m] = fmaf(mx_chunk_dot(qb0, qb1, xm + k1), e8m0_to_f32(sbb), acc[m]);
                 }
             }
 #pragma unroll
@@ -222,27 +244,32 @@ __global__ void __launch_bounds__(kMxWarps * 32)
             waited = true;
         }
         // S2-S4: lane m folds token m's partials in ring order, adds the residual.
-        const int c = h / p.hc;
+        if (lane < MT) {
+            const int c = h / p.hc;
+            float pm[kMaxRanks];
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            if (lane == m) {
-                uint16_t s = 0;
+            for (int rr = 0; rr < kMaxRanks; ++rr) {
+                pm[rr] = part[rr][0];
 #pragma unroll
-                for (int i = 0; i < kMaxRanks; ++i) {
-                    if (i < p.n_ranks) {
-                        int rr = c + i;
-                        if (rr >= p.n_ranks) rr -= p.n_ranks;
-                        float pv = 0.0f;
-#pragma unroll
-                        for (int j = 0; j < kMaxRanks; ++j)
-                            if (j == rr) pv = part[j][m];
-                        const uint16_t pb = f32_to_bf16_rne(pv);
-                        s = i == 0 ? pb : bf16_add(s, pb);
-                    }
-                }
-                const size_t o = static_cast<size_t>(m) * p.hidden + h;
-                p.out[o] = bf16_add(p.residual[o], s);
+                for (int m = 1; m < MT; ++m)
+                    if (lane == m) pm[rr] = part[rr][m];
             }
+            uint16_t s = 0;
+#pragma unroll
+            for (int i = 0; i < kMaxRanks; ++i) {
+                if (i < p.n_ranks) {
+                    int rr = c + i;
+                    if (rr >= p.n_ranks) rr -= p.n_ranks;
+                    float pv = pm[0];
+#pragma unroll
+                    for (int j = 1; j < kMaxRanks; ++j)
+                        if (j == rr) pv = pm[j];
+                    const uint16_t pb = f32_to_bf16_rne(pv);
+                    s = i == 0 ? pb : bf16_add(s, pb);
+                }
+            }
+            const size_t o = static_cast<size_t>(lane) * p.hidden + h;
+            p.out[o] = bf16_add(p.residual[o], s);
         }
     }
     if (!waited) pdl_wait();

@@ -730,8 +730,8 @@ tp_status tp_rowlinear_reconcile_mxfp8(const tp_plan* plan, const void* x, const
     prm.scales = static_cast<const uint8_t*>(w_scales);
     prm.residual = static_cast<const uint16_t*>(residual);
     prm.out = static_cast<uint16_t*>(out);
-    const int64_t rows_per_cta = tpr::kMxWarps;
-    const int64_t grid = std::min<int64_t>((plan->hidden + rows_per_cta - 1) / rows_per_cta,
+    // one warp per output row (grid-stride beyond 32 CTAs per SM)
+    const int64_t grid = std::min<int64_t>((plan->hidden + tpr::kMxWarps - 1) / tpr::kMxWarps,
                                            static_cast<int64_t>(plan->sm_count) * 32);
     const dim3 g(static_cast<unsigned>(grid)), b(tpr::kMxWarps * 32);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
