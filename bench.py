@@ -55,13 +55,14 @@ def _peaks():
 # sources means the kernels changed since, and the traffic is reported null.
 PROFILED_TRAFFIC = {
     # (workload, path): (bytes per call, kernel-source digest, profile summary)
-    ("decode_n2", "tensor"): (119145344, "3268512489d4754e", "profiles/tc_partial_decode_n2.md"),
-    ("decode_n4_m32", "tensor"): (120157696, "3268512489d4754e",
+    ("decode_n2", "tensor"): (118179712, "5b328d70d0c875e6", "profiles/tc_partial_decode_n2.md"),
+    ("decode_n4_m32", "tensor"): (119969664, "5b328d70d0c875e6",
                                   "profiles/tc_partial_ring_decode_n4_m32.md"),
-    ("decode_n8_m64", "tensor"): (83345920, "3268512489d4754e",
+    ("decode_n8_m64", "tensor"): (83670016, "5b328d70d0c875e6",
                                   "profiles/tc_partial_ring_decode_n8_m64.md"),
-    ("prefill_n4", "tensor"): (807557888, "3268512489d4754e", "profiles/tc_partial_ring_prefill_n4.md"),
-    ("decode_n2", "exact-fused"): (117277824, "3268512489d4754e", "profiles/exact_partial_decode_n2.md"),
+    ("prefill_n4", "tensor"): (832162304, "5b328d70d0c875e6", "profiles/tc2_partial_ring_prefill_n4.md"),
+    ("decode_n2", "exact-fused"): (117850112, "5b328d70d0c875e6", "profiles/exact_partial_decode_n2.md"),
+    ("decode_n2", "mxfp8"): (61455872, "5b328d70d0c875e6", "profiles/mx_reconcile_decode_n2.md"),
 }
 
 
