@@ -382,7 +382,7 @@ def _barrier(world):
 
 
 def run_reference(args, world, rank):
-    """The oracle (the reference arm of this build) timed on the host cores."""
+    """The reference arm: the oracle timed on the host cores."""
     if rank != 0:
         return 0
     cfg = get_config(args.config)

@@ -60,7 +60,7 @@ typedef enum {
     TP_OK = 0,
     TP_ERR_INVALID = 1,     /* bad shape, null pointer, aliasing, tokens > max */
     TP_ERR_ALIGN = 2,       /* pointer not 16-byte aligned */
-    TP_ERR_UNSUPPORTED = 3, /* shape or variant this build has no kernel for */
+    TP_ERR_UNSUPPORTED = 3, /* shape or variant the library has no kernel for */
     TP_ERR_WORKSPACE = 4,   /* workspace missing or too small */
     TP_ERR_CUDA = 5         /* CUDA runtime error (see tp_last_cuda_error) */
 } tp_status;
