@@ -1,4 +1,6 @@
-// Partial kernel on the tensor cores (S1) for batched decode and prefill.
+// Partial kernel on the tensor cores (S1) for decode, and for any call with a
+// k-split; prompts of more than 128 tokens without a split run on CTA pairs
+// (tp_kernels_tc2.cuh).
 //
 // "Interconnects e clusters", 01 Conceito: each rank computes a partial
 // result over its slice of the weight matrix; prefill runs every position
@@ -30,7 +32,7 @@
 // each part's fp32 sum is stored unrounded in [SPLITS][N][M][H] and the
 // ring kernel adds the parts in split order before the one rounding to bf16.
 // Units run token tile fastest, so CTAs working at the same time share each
-// weight tile through L2 (prefill reads every weight tile for 16 token tiles).
+// weight tile through L2 (a tile of weights serves every token tile of a call).
 // Folding (S2-S4): for one or two tokens the CTA that stores the last of
 // the N * SPLITS parts of an (H tile, token tile) -- found with a per-tile
 // counter in the workspace -- folds that tile itself, each epilogue thread
