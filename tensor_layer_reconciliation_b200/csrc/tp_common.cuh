@@ -263,7 +263,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 3-D tiled bulk tensor load into this CTA's shared memory (no multicast).
+// 3-D tiled bulk tensor load into this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2) {
     asm volatile(
@@ -316,7 +316,7 @@ __device__ __forceinline__ void fma4_bf16(uint32_t x, uint32_t wa, uint32_t wb, 
         : "r"(x), "r"(wa), "r"(wb));
 }
 
-// 1-D bulk copy global -> this CTA's shared memory (no multicast); both
+// 1-D bulk copy global -> this CTA's shared memory only; both
 // addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile(
@@ -326,7 +326,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
         : "memory");
 }
 
-// 5-D tiled bulk tensor load into this CTA's shared memory (no multicast).
+// 5-D tiled bulk tensor load into this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2, int c3, int c4) {
     asm volatile(

@@ -185,7 +185,7 @@ __device__ __forceinline__ void umma_commit_pair_mc(const uint64_t* bar, uint16_
 }
 
 // 3-D tiled load into this CTA's shared memory whose completed bytes count on
-// the leader CTA's barrier (`leader_bar` from pair_leader_addr). No multicast.
+// the leader CTA's barrier (`leader_bar` from pair_leader_addr); each CTA loads its own half.
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t leader_bar,
                                                  int c0, int c1, int c2) {
     asm volatile(
