@@ -91,19 +91,23 @@ TP_API tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, 
  *   staged   EXACT: 0 keeps the partials on chip, one kernel doing partials,
  *            ring fold and residual add (no workspace); 1 writes all N
  *            partials to the workspace and a separate ring kernel
- *            (tp_ring_reduce's) folds them. TENSOR always stages its
- *            partials and folds them in a separate ring kernel.
+ *            (tp_ring_reduce's) folds them. TENSOR (and AUTO) ignore it:
+ *            they always write their partials to the workspace; with one
+ *            or two tokens the partial kernel itself folds them (the CTA
+ *            that stores the last part of a tile folds that tile), from
+ *            three tokens up a ring kernel follows.
  * Call before the plan is shared between threads. */
 TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
 
 /* Bytes of workspace tp_rowlinear_reconcile needs for `tokens` tokens with
  * the plan's current setting; 0 when the partials stay on chip (EXACT, not
- * staged). The tensor-core variant always sends its partials through the
- * workspace: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of K parts)
- * when it splits K across CTAs to fill the SMs. Layout: a counter block of
- * one 32-bit counter per 128-row H tile (256-byte rounded; the in-kernel fold
- * of one or two tokens counts stored parts there), then the partials.
- * Rounded up to 256 in all. Returns 0 for a null plan. */
+ * staged). The tensor-core variant always writes its partials to the
+ * workspace, whether its own kernel folds them (one or two tokens) or a
+ * ring kernel does: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of K
+ * parts) when it splits K across CTAs to fill the SMs. Layout: a counter
+ * block of one 32-bit counter per 128-row H tile (256-byte rounded; the
+ * in-kernel fold counts stored parts there), then the partials. Rounded up
+ * to 256 in all. Returns 0 for a null plan or tokens <= 0. */
 TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 
 /* The partial kernel a call with `tokens` tokens runs under the plan's
@@ -172,7 +176,7 @@ TP_API tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, cons
  *    partial it reads. The fold counters at its start are zero when the
  *    library is loaded and every call that sets no device error flag leaves
  *    them zero; after one that does, this entry point may give wrong results
- *    until the process restarts. Calls whose kernels overlap
+ *    until tp_device_error_flags with reset != 0 clears them. Calls whose kernels overlap
  *    on the GPU (different streams without ordering between them) race on
  *    the array and give wrong results: order them on one stream.
  * The pages describe no counterpart of this entry point. */
@@ -263,6 +267,22 @@ typedef enum {
 TP_API uint64_t tp_allreduce_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hidden,
                                    int elem_bytes, int64_t points);
 
+/* Bytes one rank's NVLink port carries for the combine step of an MoE layer
+ * (NVL72 hosting post, MoE dispatch/combine section): the combine first
+ * accumulates, on each rank, the weighted contributions of the experts the
+ * rank hosts for every token, then all-reduces the accumulated
+ * [tokens][hidden] buffer of elem_bytes elements across the N ranks under
+ * `scheme` (a tp_allreduce_scheme).
+ *   local_accumulate 1  the post's combine: one all-reduce, tp_allreduce_bytes
+ *                       of the buffer (points = 1), whatever top_k is;
+ *                    0  for comparison: each of a token's top_k expert slots
+ *                       all-reduced on its own, top_k times that.
+ * Host only, exact. Returns 0 for top_k < 1, local_accumulate not 0 or 1,
+ * and wherever tp_allreduce_bytes returns 0. A byte model only: the expert
+ * GEMMs and the routing are not part of this library. */
+TP_API uint64_t tp_moe_combine_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hidden,
+                                     int elem_bytes, int64_t top_k, int local_accumulate);
+
 /* Releases a plan. NULL is allowed. */
 TP_API void tp_plan_destroy(tp_plan* plan);
 
@@ -275,8 +295,13 @@ TP_API int tp_last_cuda_error(void);
 
 /* Reads, and with reset != 0 clears, the device-side error word of the
  * plan's device: bit 0 is set when a kernel's bounded wait on a pipeline
- * barrier ran out (the kernel then stops early, so its output is invalid).
- * Synchronises the device. */
+ * barrier ran out (the kernel then stops early, so its output is invalid;
+ * copies or tensor-core operations it had in flight may not have finished
+ * when it returned, so the context should be discarded, e.g. by
+ * cudaDeviceReset, before results are trusted again). With reset != 0 and a
+ * nonzero word it also zeroes the fold counters of the library's own
+ * scratch array (tp_rowlinear_reconcile_noalloc); a caller's workspace must
+ * be zeroed by the caller. Synchronises the device. */
 TP_API tp_status tp_device_error_flags(const tp_plan* plan, uint32_t* flags, int reset);
 
 #ifdef __cplusplus

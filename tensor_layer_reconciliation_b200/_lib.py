@@ -23,7 +23,7 @@ EXPORTED = (
     "tp_plan_packed_bytes",
     "tp_pack_weights",
     "tp_rowlinear_reconcile", "tp_rowlinear_reconcile_noalloc", "tp_rowlinear_partials",
-    "tp_ring_reduce", "tp_ring_bytes", "tp_allreduce_bytes",
+    "tp_ring_reduce", "tp_ring_bytes", "tp_allreduce_bytes", "tp_moe_combine_bytes",
     "tp_plan_mxfp8_bytes", "tp_pack_weights_mxfp8", "tp_rowlinear_reconcile_mxfp8",
     "tp_plan_destroy", "tp_status_string", "tp_last_cuda_error", "tp_device_error_flags",
 )
@@ -77,6 +77,9 @@ def _load() -> ctypes.CDLL:
     L.tp_rowlinear_reconcile_mxfp8.restype = ctypes.c_int
     L.tp_allreduce_bytes.argtypes = [ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int, i64]
     L.tp_allreduce_bytes.restype = ctypes.c_uint64
+    L.tp_moe_combine_bytes.argtypes = [ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int, i64,
+                                       ctypes.c_int]
+    L.tp_moe_combine_bytes.restype = ctypes.c_uint64
     L.tp_plan_destroy.argtypes = [vp]
     L.tp_plan_destroy.restype = None
     L.tp_status_string.argtypes = [ctypes.c_int]
@@ -169,6 +172,12 @@ TP_ALLREDUCE_RING, TP_ALLREDUCE_NAIVE, TP_ALLREDUCE_SWITCH = 0, 1, 2
 def tp_allreduce_bytes(scheme: int, n_ranks: int, tokens: int, hidden: int, elem_bytes: int,
                        points: int) -> int:
     return int(LIB.tp_allreduce_bytes(scheme, n_ranks, tokens, hidden, elem_bytes, points))
+
+
+def tp_moe_combine_bytes(scheme: int, n_ranks: int, tokens: int, hidden: int, elem_bytes: int,
+                         top_k: int, local_accumulate: int = 1) -> int:
+    return int(LIB.tp_moe_combine_bytes(scheme, n_ranks, tokens, hidden, elem_bytes, top_k,
+                                        local_accumulate))
 
 
 def tp_ring_bytes(n_ranks: int, tokens: int, hidden: int, elem_bytes: int, points: int) -> int:

@@ -299,54 +299,7 @@ __device__ __forceinline__ float fma2_bf16(uint32_t x, uint32_t w, float acc) {
     return acc;
 }
 
-// Four chain steps sharing one x pair: two rows (a, b) of the same rank,
-// each advanced by x.lo then x.hi (k ascending within each chain); the two
-// chains interleave so each FMA's latency hides behind the other chain's.
-__device__ __forceinline__ void fma4_bf16(uint32_t x, uint32_t wa, uint32_t wb, float& a,
-                                          float& b) {
-    asm("{\n\t.reg .b16 xl, xh, al, ah, bl, bh;\n\t"
-        "mov.b32 {xl, xh}, %2;\n\t"
-        "mov.b32 {al, ah}, %3;\n\t"
-        "mov.b32 {bl, bh}, %4;\n\t"
-        "fma.rn.f32.bf16 %0, xl, al, %0;\n\t"
-        "fma.rn.f32.bf16 %1, xl, bl, %1;\n\t"
-        "fma.rn.f32.bf16 %0, xh, ah, %0;\n\t"
-        "fma.rn.f32.bf16 %1, xh, bh, %1;\n\t}"
-        : "+f"(a), "+f"(b)
-        : "r"(x), "r"(wa), "r"(wb));
-}
-
-// 1-D bulk copy global -> this CTA's shared memory only; both
-// addresses 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// 5-D tiled bulk tensor load into this CTA's shared memory only.
-__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int c0, int c1, int c2, int c3, int c4) {
-    asm volatile(
-        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
-        "r"(c3), "r"(c4)
-        : "memory");
-}
-
 // ------------------------------------------------------------ vector loads --
-
-__device__ __forceinline__ uint4 ld_shared_v4(const void* p) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(smem_u32(p))
-                 : "memory");
-    return v;
-}
 
 __device__ __forceinline__ uint4 ld_global_nc_v4(const void* p) {
     uint4 v;

@@ -125,8 +125,9 @@ __global__ void __launch_bounds__(kMaxExactThreads, 1)
                             kb * kKBlock, 0, m0);
                 issued = kb + 1;
             }
-            // Never leave with bulk copies still landing in this CTA's memory:
-            // wait (bounded) for the last copies issued into every stage.
+            // Wait (bounded) for the last copies issued into every stage. A wait
+            // that runs out has set the device error word; the launch's results
+            // are then invalid and the context should be discarded.
             const int first = issued > S ? issued - S : 0;
             for (int kb = first; kb < issued; ++kb)
                 if (!mbar_wait_bounded(&full[kb % S], static_cast<uint32_t>(kb / S) & 1u)) break;

@@ -201,7 +201,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     phase ^= 1u;
                 }
             }
-            // Never leave with bulk copies still landing in this CTA's memory.
+            // Wait (bounded) for the copies still landing in this CTA's memory.
+            // A wait that runs out has set the device error word; the launch's
+            // results are then invalid and the context should be discarded.
             const int first = issued > S ? issued - S : 0;
             for (int i = first; i < issued; ++i)
                 if (!mbar_wait_bounded(&full[i % S], static_cast<uint32_t>(i / S) & 1u)) break;
@@ -245,8 +247,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 umma_commit(&acc_full[b]);
             }
             // Every MMA issued has finished before the tensor memory is freed.
+            // A first wait that runs out (error word set) gets one more bound.
             umma_commit(mma_done);
-            (void)mbar_wait_bounded(mma_done, 0);
+            if (!mbar_wait_bounded(mma_done, 0)) (void)mbar_wait_bounded(mma_done, 0);
         }
     } else {
         // ---------------------------------------------------------- epilogue --

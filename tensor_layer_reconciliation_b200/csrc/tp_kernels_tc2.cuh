@@ -222,7 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             // Every MMA issued has finished before the tensor memory is freed.
             if (issued_any) {
                 umma_commit_pair_mc(mma_done, 0x1);
-                (void)mbar_wait_bounded(mma_done, 0);
+                if (!mbar_wait_bounded(mma_done, 0)) (void)mbar_wait_bounded(mma_done, 0);
             }
         }
     } else {

@@ -40,23 +40,16 @@ namespace {
 
 thread_local int t_last_cuda_error = 0;
 
-// Device address of the no-alloc scratch array, looked up once per device
-// (cudaGetSymbolAddress with that device current). In host code the array's
-// name is only a host-side stand-in, never a device address.
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-cudaError_t noalloc_scratch_for(int dev, void** out) {
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
-        void* ptr = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = ptr;
-    }
-    *out = g_scratch_addr[dev];
+// Device address of the no-alloc scratch array on the current device. In host
+// code the array's name is only a host-side stand-in, never a device address:
+// cudaGetSymbolAddress, with the device current, gives the address kernels
+// use. It is looked up again at every plan creation (a cheap query), so a
+// plan made after cudaDeviceReset gets the array of the new context.
+cudaError_t noalloc_scratch_current(void** out) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    *out = ptr;
     return cudaSuccess;
 }
 
@@ -256,7 +249,7 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split) {
     // Fewer units than SMs: split K so every SM streams weights.
     const int nkb = static_cast<int>((p->ks + tpr::kTcKBlock - 1) / tpr::kTcKBlock);
     c.splits = 1;
-    if (allow_split && base_units < p->sm_count)
+    if (allow_split && base_units > 0 && base_units < p->sm_count)
         c.splits = std::max(1, std::min({slots / base_units, nkb, tpr::kMaxSplits}));
     c.units = base_units * c.splits;
     c.grid = std::min(c.units, slots);
@@ -451,7 +444,7 @@ tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t
     int dyn_max = 0;
     if ((e = set_kernel_attrs(optin, &dyn_max)) != cudaSuccess) return cuda_fail(e);
     void* scratch = nullptr;
-    if ((e = noalloc_scratch_for(dev, &scratch)) != cudaSuccess) return cuda_fail(e);
+    if ((e = noalloc_scratch_current(&scratch)) != cudaSuccess) return cuda_fail(e);
     tp_plan* p = new (std::nothrow) tp_plan{};
     if (!p) return TP_ERR_INVALID;
     p->n_ranks = n_ranks;
@@ -617,12 +610,13 @@ tp_status tp_rowlinear_reconcile_noalloc(const tp_plan* plan, const void* x, con
                                          void* stream) {
     if (!plan) return TP_ERR_INVALID;
     if (tokens < 0 || tokens > plan->max_tokens) return TP_ERR_INVALID;
+    if (tokens == 0) return TP_OK;   // nothing to launch, nothing staged
     // Refused before anything is touched when the scratch cannot hold it.
     if (counter_block_bytes(plan) > kNoAllocCounterBytes ||
         partial_bytes(plan, tokens) > kNoAllocScratchBytes - kNoAllocCounterBytes)
         return TP_ERR_WORKSPACE;
     tp_status st = check_reconcile_args(plan, x, w_packed, residual, out, tokens);
-    if (st != TP_OK || tokens == 0) return st;
+    if (st != TP_OK) return st;
     uint8_t* base = static_cast<uint8_t*>(plan->noalloc_scratch);
     return reconcile_launch(plan, x, w_packed, residual, out, tokens,
                             reinterpret_cast<unsigned int*>(base), base + kNoAllocCounterBytes,
@@ -759,6 +753,13 @@ uint64_t tp_allreduce_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hid
     }
 }
 
+uint64_t tp_moe_combine_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hidden, int elem_bytes,
+                              int64_t top_k, int local_accumulate) {
+    if (top_k < 1 || (local_accumulate != 0 && local_accumulate != 1)) return 0;
+    const uint64_t one = tp_allreduce_bytes(scheme, n_ranks, tokens, hidden, elem_bytes, 1);
+    return local_accumulate ? one : static_cast<uint64_t>(top_k) * one;
+}
+
 void tp_plan_destroy(tp_plan* plan) { delete plan; }
 
 const char* tp_status_string(tp_status status) {
@@ -786,6 +787,10 @@ tp_status tp_device_error_flags(const tp_plan* plan, uint32_t* flags, int reset)
     if (reset) {
         const uint32_t zero = 0;
         if ((e = cudaMemcpyToSymbol(tpr::g_device_error, &zero, sizeof zero)) != cudaSuccess)
+            return cuda_fail(e);
+        // A call that ran out of a wait may have left fold counters of the
+        // no-alloc scratch above zero; clear them (device idle: synchronised above).
+        if (v != 0 && (e = cudaMemset(plan->noalloc_scratch, 0, kNoAllocCounterBytes)) != cudaSuccess)
             return cuda_fail(e);
     }
     *flags = v;
