@@ -23,6 +23,10 @@ Functions and the passages they follow:
 * ``residual``  -- the residual add after reconciliation (01 Conceito: the
   slices are summed before the residual stream continues).
 * ``ring_bytes`` -- 2(N-1)/N x payload per rank (01 Conceito, worked example).
+* ``allreduce_bytes`` -- per-rank bytes of the ring, naive and switch-reduction
+  all-reduce schemes (NVL72 hosting post, All-reduce section).
+* ``moe_combine_bytes`` -- per-rank bytes of an MoE combine: local weighted
+  accumulation, then one all-reduce (NVL72 hosting post, MoE dispatch/combine).
 
 Pins that tie each function to the pages or to mathematics (not to itself)
 live in ``tests/test_oracle_*.py``. Parity unpinned: the exact fp32 rounding of
@@ -90,6 +94,10 @@ def lib():
         L.orc_allreduce_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
                                           ctypes.c_int, ctypes.c_int64]
         L.orc_allreduce_bytes.restype = ctypes.c_uint64
+        L.orc_moe_combine_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                            ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
+                                            ctypes.c_int]
+        L.orc_moe_combine_bytes.restype = ctypes.c_uint64
         L.orc_e4m3_rne.argtypes = [ctypes.c_double]
         L.orc_e4m3_rne.restype = ctypes.c_uint8
         L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
@@ -283,6 +291,16 @@ def allreduce_bytes(scheme: str, n_ranks: int, tokens: int, hidden: int, elem_by
     """Per-rank NVLink bytes of one all-reduce scheme (see orc_allreduce_bytes)."""
     return int(lib().orc_allreduce_bytes(ALLREDUCE_SCHEMES[scheme], n_ranks, tokens, hidden,
                                          elem_bytes, points))
+
+
+def moe_combine_bytes(scheme: str, n_ranks: int, tokens: int, hidden: int, elem_bytes: int,
+                      top_k: int, local_accumulate: bool = True) -> int:
+    """Per-rank NVLink bytes of an MoE combine: the weighted contributions of
+    each rank's experts accumulated locally, then one all-reduce of the
+    [tokens][hidden] buffer (NVL72 hosting post, MoE dispatch/combine);
+    local_accumulate=False all-reduces each of the top_k expert slots apart."""
+    return int(lib().orc_moe_combine_bytes(ALLREDUCE_SCHEMES[scheme], n_ranks, tokens, hidden,
+                                           elem_bytes, top_k, int(bool(local_accumulate))))
 
 
 def cores() -> int:

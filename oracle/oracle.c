@@ -416,6 +416,32 @@ uint64_t orc_allreduce_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hi
     return slices * b / (uint64_t)n_ranks;
 }
 
+/*
+ * Bytes one rank's NVLink port carries for the combine step of an MoE layer
+ * (NVL72 hosting post, MoE dispatch/combine section): the combine kernel
+ * first accumulates, on each rank, the weighted contributions of the experts
+ * that rank hosts for every token, then all-reduces the accumulated
+ * [tokens][hidden] buffer across the ranks. Counted buffer by buffer:
+ *   local_accumulate = 1  every rank all-reduces one [tokens][hidden]
+ *                         buffer, whatever top_k and the routing are;
+ *   local_accumulate = 0  (for comparison) each of the top_k expert slots of
+ *                         a token is all-reduced as its own [tokens][hidden]
+ *                         buffer, the weighted sum taken afterwards.
+ * Each buffer costs orc_allreduce_bytes under `scheme` (points = 1).
+ * Returns 0 for top_k < 1 or the arguments orc_allreduce_bytes rejects.
+ */
+uint64_t orc_moe_combine_bytes(int scheme, int n_ranks, int64_t tokens, int64_t hidden,
+                               int elem_bytes, int64_t top_k, int local_accumulate)
+{
+    if (top_k < 1 || (local_accumulate != 0 && local_accumulate != 1))
+        return 0;
+    const int64_t buffers = local_accumulate ? 1 : top_k;
+    uint64_t total = 0;
+    for (int64_t b = 0; b < buffers; ++b)
+        total += orc_allreduce_bytes(scheme, n_ranks, tokens, hidden, elem_bytes, 1);
+    return total;
+}
+
 /* -------------------------------------------------- MXFP8 weight shards -- */
 /*
  * Micro-scaled FP8 weights (the NVL72 hosting post quantises the MoE GEMM's

@@ -95,3 +95,25 @@ def round_bf16_float(v) -> int:
     if v == 0.0:
         return 0x8000 if math.copysign(1.0, v) < 0 else 0
     return round_bf16_exact(Fraction(v))
+
+
+def round_f32_exact(v: Fraction) -> Fraction:
+    """Correct round-to-nearest-even of an exact rational to an IEEE binary32
+    value (returned as an exact rational), from the format's definition: 24
+    significant bits, exponent down to -126, subnormal quantum 2^-149;
+    |v| at or above the largest finite value's upper midpoint is refused."""
+    if v == 0:
+        return Fraction(0)
+    a = -v if v < 0 else v
+    assert a < (2 - Fraction(1, 1 << 24)) * Fraction(2) ** 127, "overflow"
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    q = max(e - 23, -149)
+    scaled = a / Fraction(2) ** q
+    n = math.floor(scaled)
+    rem = scaled - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    r = n * Fraction(2) ** q
+    return -r if v < 0 else r

@@ -115,3 +115,19 @@ def test_allreduce_bytes_matches_oracle(scheme):
     assert tlr.tp_allreduce_bytes(code, 4, 1, 5120, 2, 128) == \
         oracle.allreduce_bytes(scheme, 4, 1, 5120, 2, 128)
     assert tlr.tp_allreduce_bytes(9, 4, 1, 5120, 2, 128) == 0
+
+
+@pytest.mark.parametrize("scheme", ["ring", "naive", "sharp"])
+def test_moe_combine_bytes_matches_oracle(scheme):
+    """The library's MoE-combine byte model (host code) against the oracle's
+    buffer-by-buffer count, with and without the local accumulation."""
+    import tensor_layer_reconciliation_b200 as tlr
+    code = {"ring": tlr.TP_ALLREDUCE_RING, "naive": tlr.TP_ALLREDUCE_NAIVE,
+            "sharp": tlr.TP_ALLREDUCE_SWITCH}[scheme]
+    for n in range(0, 10):
+        for m, h, e, k in [(1, 5120, 2, 8), (64, 4096, 2, 8), (3, 840, 4, 1), (0, 5, 2, 2),
+                           (5, 7, 1, 3), (2, -1, 2, 2), (4, 16, 2, 0)]:
+            for local in (0, 1):
+                assert tlr.tp_moe_combine_bytes(code, n, m, h, e, k, local) == \
+                    oracle.moe_combine_bytes(scheme, n, m, h, e, k, bool(local)), (n, m, h, e, k, local)
+    assert tlr.tp_moe_combine_bytes(code, 4, 1, 16, 2, 2, 2) == 0

@@ -6,7 +6,10 @@ switch reduction), against what the pages fix:
   N(N-1)B in total; reducing slices and broadcasting them moves (N-1)B/N per
   peer each way, 2(N-1)B in total; the switch reduction moves the fraction
   N/(2(N-1)) of the ring's transfers (a 33% saving at four peers);
-* one rank communicates nothing.
+* one rank communicates nothing;
+* the MoE combine (same post, dispatch/combine section) accumulates each
+  rank's expert contributions locally and then all-reduces one buffer, so its
+  cost is one all-reduce whatever top_k is (golden file, invariants).
 """
 
 from fractions import Fraction
@@ -45,3 +48,24 @@ def test_allreduce_single_rank_and_bad_args():
         assert oracle.allreduce_bytes(s, 0, 4, 5120, 2, 128) == 0
         assert oracle.allreduce_bytes(s, 4, -1, 5120, 2, 128) == 0
     assert int(oracle.lib().orc_allreduce_bytes(7, 4, 1, 5120, 2, 128)) == 0
+
+
+def test_moe_combine_bytes_golden():
+    rows = golden_rows("moe_combine_bytes.txt")
+    assert len(rows) == 4
+    for scheme, n, m, h, e, k, local, want in rows:
+        got = oracle.moe_combine_bytes(scheme, int(n), int(m), int(h), int(e), int(k), local == "1")
+        assert got == int(want), (scheme, n, m, h, e, k, local)
+
+
+@pytest.mark.parametrize("scheme", ["ring", "naive", "sharp"])
+def test_moe_combine_invariants(scheme):
+    for n in range(1, 9):
+        one = oracle.allreduce_bytes(scheme, n, 7, 840, 2, 1)
+        for top_k in (1, 2, 8):
+            # local accumulation: one all-reduce of the [tokens][hidden] buffer
+            assert oracle.moe_combine_bytes(scheme, n, 7, 840, 2, top_k, True) == one
+            # slots reduced apart: top_k all-reduces
+            assert oracle.moe_combine_bytes(scheme, n, 7, 840, 2, top_k, False) == top_k * one
+    assert oracle.moe_combine_bytes(scheme, 4, 7, 840, 2, 0, True) == 0
+    assert int(oracle.lib().orc_moe_combine_bytes(0, 4, 7, 840, 2, 2, 2)) == 0

@@ -48,6 +48,10 @@ MUTATIONS = {
                     ("acc = fmaf(orc_f32(xr[kk]), orc_f32(wr[kk]), acc);",
                      "acc = fma((double)orc_f32(xr[kk]), (double)orc_f32(wr[kk]), acc);")],
                    None, [trc.test_partial_order_fp32_ascending]),
+    # partials: the product rounded to fp32 before it is added
+    "round_then_add": ("acc = fmaf(orc_f32(xr[kk]), orc_f32(wr[kk]), acc);",
+                       "acc = acc + orc_f32(xr[kk]) * orc_f32(wr[kk]);",
+                       [trc.test_partial_adds_each_product_with_one_rounding]),
     # partials: k descending
     "k_descending": ("for (int64_t kk = 0; kk < ks; ++kk) {",
                      "for (int64_t kk = ks - 1; kk >= 0; --kk) {",
@@ -76,6 +80,10 @@ MUTATIONS = {
     "naive_self": ("                for (int c = 0; c < n_ranks; ++c)\n                    slices += 1;  /* every slice of the peer's buffer */",
                    "                for (int c = 0; c < n_ranks; ++c)\n                    slices += 1;  /* every slice of the peer's buffer */\n        slices += (uint64_t)n_ranks;",
                    [tar.test_allreduce_bytes_golden]),
+    # MoE combine: the local accumulation is skipped (every slot all-reduced)
+    "combine_no_local_acc": ("const int64_t buffers = local_accumulate ? 1 : top_k;",
+                             "const int64_t buffers = top_k;",
+                             [tar.test_moe_combine_bytes_golden]),
     # MXFP8: element rounding half away from zero instead of to even
     "e4m3_half_up": ("if (rem > 0.5 || (rem == 0.5 && fmod(m, 2.0) == 1.0))",
                      "if (rem >= 0.5)",
@@ -113,7 +121,8 @@ def test_pin_catches_mutation(name, monkeypatch):
     mutant = ctypes.CDLL(path)
     for fn in ("orc_bf16_rne", "orc_bf16_rne_f64", "orc_f32", "orc_bf16_rne_array",
                "orc_bf16_rne_f64_array", "orc_partials", "orc_ring", "orc_residual",
-               "orc_reconcile", "orc_ring_bytes", "orc_allreduce_bytes", "orc_e4m3_rne",
+               "orc_reconcile", "orc_ring_bytes", "orc_allreduce_bytes", "orc_moe_combine_bytes",
+               "orc_e4m3_rne",
                "orc_e4m3_value", "orc_mx_quantize", "orc_mx_dequant_bf16"):
         f = getattr(mutant, fn)
         g = getattr(real, fn)

@@ -4,6 +4,9 @@
   rounding is exact, so the output must equal the int64 product x.W + res;
 * a crafted order-sensitive dot product: fp32 accumulation with k ascending
   gives 0 where the exact sum is 1 (the accumulator reading);
+* a crafted dot product with a subnormal product: each product is added to
+  the running fp32 sum with one rounding (fused multiply-add), which gives a
+  different bf16 partial than rounding the product first and then adding;
 * each partial lies within the textbook error bound of recursive fp32
   summation (Higham, "Accuracy and Stability of Numerical Algorithms", 4.2:
   |error| <= gamma_(n-1) * sum |x_k w_k|) of the exact rational dot product,
@@ -21,7 +24,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import bf16_value, round_bf16_exact, u16
+from helpers import bf16_value, round_bf16_exact, round_f32_exact, u16
 from workloads import KIND_RESIDUAL, KIND_W, KIND_X, get_config, point_tensor
 
 U = 2.0 ** -8          # bf16 unit roundoff
@@ -57,6 +60,37 @@ def test_partial_order_fp32_ascending():
     p, p64, _ = oracle.partials(1, x, w)
     assert oracle.f32(p)[0, 0, 0] == 0.0
     assert p64[0, 0, 0] == 1.0
+
+
+# Four products, k ascending (hand-derived): p0 = (1 + 2^-7) 2^-124 = b, a bf16
+# value with an odd last bit; p1 = 2^-132, half a bf16 unit of b, so the sum
+# is the bf16 midpoint m = b + 2^-132; p2 = -2^-147, one fp32 unit in this
+# binade, so the sum is m - 2^-147; p3 = 1.75 * 2^-149, a product below the
+# fp32 normal range. Fused: m - 2^-147 + 0.4375 units rounds back to
+# m - 2^-147, below the midpoint, and the partial is b (0x0181). Product
+# rounded first: 1.75 * 2^-149 becomes 2^-148 (subnormal quantum 2^-149),
+# the sum m - 2^-148 is an fp32 tie that goes to the even m, and m is a bf16
+# tie that goes to the even b + 2^-131 (0x0182).
+FMA_PIN_X = [0x3F81, 0x1E80, 0xB880, 0x37E0]     # 1+2^-7, 2^-66, -2^-14, 1.75*2^-16
+FMA_PIN_W = [0x0180, 0x1E80, 0x0001, 0x0001]     # 2^-124, 2^-66, 2^-133, 2^-133
+
+
+def _chain(xs, ws, fused):
+    acc = Fraction(0)
+    for xb, wb in zip(xs, ws):
+        prod = bf16_value(xb) * bf16_value(wb)
+        acc = round_f32_exact(acc + (prod if fused else round_f32_exact(prod)))
+    return round_bf16_exact(acc)
+
+
+def test_partial_adds_each_product_with_one_rounding():
+    fused = _chain(FMA_PIN_X, FMA_PIN_W, True)
+    rounded_first = _chain(FMA_PIN_X, FMA_PIN_W, False)
+    assert (fused, rounded_first) == (0x0181, 0x0182)    # the two readings differ here
+    x = np.array([FMA_PIN_X], dtype=np.uint16)
+    w = np.array([FMA_PIN_W], dtype=np.uint16)
+    p, _, _ = oracle.partials(1, x, w)
+    assert int(p[0, 0, 0]) == fused
 
 
 def test_partials_within_recursive_summation_bound():
