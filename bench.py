@@ -2,10 +2,15 @@
 workload (all partials, ring folds and residual adds) over one batch.
 
 Usage:
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
-                  [--variant auto|exact|tensor] [--staged] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME|all]
+                  [--variant auto|exact|tensor] [--staged] [--weights bf16|mxfp8]
+                  [--impl ours|reference]
 
-Prints ONE JSON line on rank 0. With --gpus N > 1 it runs under
+With the default --config all, the four benchmarked workloads run one after
+another (decode_n2, decode_n4_m32, decode_n8_m64, prefill_n4), each on its
+own freshly allocated buffers; the headline numbers are decode_n2's (the
+pages' worked decode example) and every workload's numbers are under
+"per_config". Prints ONE JSON line on rank 0. With --gpus N > 1 it runs under
 torch.distributed.run, one process per GPU; every rank runs an independent
 replica of the step (the N tensor-parallel ranks of the method are emulated
 inside each GPU), so there is no data-path collective and the scaling is weak.
@@ -16,6 +21,7 @@ from __future__ import annotations
 import argparse
 import dataclasses
 import datetime
+import gc
 import json
 import os
 import subprocess
@@ -29,11 +35,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import KIND_RESIDUAL, KIND_W, KIND_X, get_config, point_tensor  # noqa: E402
+from workloads import (KIND_RESIDUAL, KIND_W, KIND_X, get_config, point_tensor,  # noqa: E402
+                       point_tensor_rows)
 from workloads.configs import CONFIG_ORDER  # noqa: E402
 
 METRIC = "reconciliations/s & tokens/s on 1 B200; achieved HBM GB/s (TC util) vs peak"
-DEFAULT_CONFIG = "decode_n2"
+HEADLINE_CONFIG = "decode_n2"
+BENCH_CONFIGS = ["decode_n2", "decode_n4_m32", "decode_n8_m64", "prefill_n4"]
+TOL_MAX_ABS, TOL_REL_L2 = 2e-2, 5e-3      # acceptance tolerance against the oracle
 
 
 def _peaks():
@@ -54,15 +63,23 @@ def _peaks():
 # sources whose digest is recorded; a digest that no longer matches the
 # sources means the kernels changed since, and the traffic is reported null.
 PROFILED_TRAFFIC = {
-    # (workload, path): (bytes per call, kernel-source digest, profile summary)
-    ("decode_n2", "tensor"): (118179712, "6a43f336d1b1fa29", "profiles/tc_partial_decode_n2.md"),
+    # (workload, path): (bytes per call, kernel-source digest, the ncu capture)
+    ("decode_n2", "tensor"): (118179712, "6a43f336d1b1fa29",
+                              "ncu dram__bytes of tc_partial_kernel<32> (k-split, in-kernel fold) "
+                              "on decode_n2, one step"),
     ("decode_n4_m32", "tensor"): (119969664, "6a43f336d1b1fa29",
-                                  "profiles/tc_partial_ring_decode_n4_m32.md"),
+                                  "ncu dram__bytes of tc_partial_kernel<32> + ring_reduce_kernel "
+                                  "on decode_n4_m32, one step"),
     ("decode_n8_m64", "tensor"): (83670016, "6a43f336d1b1fa29",
-                                  "profiles/tc_partial_ring_decode_n8_m64.md"),
-    ("prefill_n4", "tensor"): (832162304, "6a43f336d1b1fa29", "profiles/tc2_partial_ring_prefill_n4.md"),
-    ("decode_n2", "exact-fused"): (117850112, "6a43f336d1b1fa29", "profiles/exact_partial_decode_n2.md"),
-    ("decode_n2", "mxfp8"): (61455872, "6a43f336d1b1fa29", "profiles/mx_reconcile_decode_n2.md"),
+                                  "ncu dram__bytes of tc_partial_kernel<64> + ring_reduce_kernel "
+                                  "on decode_n8_m64, one step"),
+    ("prefill_n4", "tensor"): (832162304, "6a43f336d1b1fa29",
+                               "ncu dram__bytes of tc2_partial_kernel + ring_reduce_kernel "
+                               "on prefill_n4, one step"),
+    ("decode_n2", "exact-fused"): (117850112, "6a43f336d1b1fa29",
+                                   "ncu dram__bytes of exact_partial_kernel<1> on decode_n2, one step"),
+    ("decode_n2", "mxfp8"): (61455872, "6a43f336d1b1fa29",
+                             "ncu dram__bytes of mx_reconcile_kernel<1> on decode_n2, one step"),
 }
 
 
@@ -253,6 +270,18 @@ class ClockSampler:
 
 # ------------------------------------------------------------------- oracle --
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(cfg, threads=None, target_s=12.0):
     """The oracle as it stands on this host's cores, on a bounded sample.
 
@@ -292,8 +321,92 @@ def cpu_baseline(cfg, threads=None, target_s=12.0):
         desc.append(f"{kind} point {p.index} (K={p.k}): {cols} of {cfg.hidden} output columns "
                     f"x {reps} runs")
     step_s = sum(per_kind[p.kind] for p in cfg.points)
-    return {"step_s": step_s, "cores": threads, "sample": "; ".join(desc) +
+    return {"step_s": step_s, "cores": threads, "cpu_model": _cpu_model(),
+            "sample": "; ".join(desc) +
             f"; step time extrapolated over {cfg.n_points} points ({measured:.1f} s measured)"}
+
+
+def _sample_cols(hidden, n_ranks, count, seed):
+    """Output columns checked at full size: both ends of every H/N chunk and a
+    seeded spread."""
+    hc = hidden // n_ranks
+    cols = {0, 1, hidden - 1, hidden - 2}
+    for c in range(n_ranks):
+        cols |= {c * hc, c * hc + 1, c * hc + hc - 1}
+    rng = np.random.default_rng(seed)
+    cols |= set(int(v) for v in rng.integers(0, hidden, count))
+    return np.array(sorted(c for c in cols if 0 <= c < hidden), dtype=np.int64)
+
+
+def oracle_parity(wl, threads=None):
+    """Parity of the outputs the timed graph wrote against the oracle, on
+    sampled columns of sampled points (the first and last point of each
+    projection kind; every token of each sampled column). Part of the CPU
+    leg, outside every timed region.
+
+    A partial is fragile when its fp64 value lies within 2^-19 * sum|x*w| of
+    a bf16 rounding boundary, where a summation order other than the
+    oracle's k-ascending fp32 chain may round it the other way; an output is
+    fragile when one of its N partials is. Reported: the largest absolute
+    error, the relative L2 error, the fragile partial and output counts, the
+    outputs that differ from the oracle (and how many of those are not
+    fragile: 0 is required), and the outputs beyond the 2e-2 absolute
+    tolerance (and how many of those are not fragile).
+    """
+    import oracle
+    cfg = wl.cfg
+    threads = threads or len(os.sched_getaffinity(0))
+    kinds = {}
+    for p in cfg.points:
+        kinds.setdefault(p.kind, []).append(p.index)
+    idx = sorted({v for lst in kinds.values() for v in (lst[0], lst[-1])})
+    cols = _sample_cols(cfg.hidden, cfg.n_ranks, 16 if cfg.tokens >= 1024 else 40,
+                        seed=len(cfg.name))
+    sq_err = sq_ref = 0.0
+    st = dict(max_abs=0.0, fragile_partials=0, fragile_outputs=0, outputs_differing=0,
+              differing_not_fragile=0, over_max_abs=0, over_max_abs_not_fragile=0,
+              sampled_outputs=0, sampled_partials=0)
+    t0 = time.perf_counter()
+    for i in idx:
+        p = cfg.points[i]
+        x = point_tensor(cfg, p, KIND_X).view(torch.int16).numpy().view(np.uint16)
+        w = point_tensor_rows(cfg, p, KIND_W, cols).view(torch.int16).numpy().view(np.uint16)
+        r = point_tensor(cfg, p, KIND_RESIDUAL).view(torch.int16).numpy().view(np.uint16)
+        r = np.ascontiguousarray(r[:, cols])
+        if wl.weights == "mxfp8":     # over the dequantised shards (a row quantises alone)
+            q, sc = oracle.mx_quantize(cfg.n_ranks, np.ascontiguousarray(w))
+            w = oracle.mx_dequant_bf16(cfg.n_ranks, q, sc)
+        ref = oracle.reconcile(cfg.n_ranks, cfg.hidden, x, np.ascontiguousarray(w), r, cols=cols,
+                               threads=threads)
+        got = wl.out(i)[:, torch.from_numpy(cols).to(wl.device)].cpu().view(torch.int16).numpy().view(np.uint16)
+        e = ref["pabs"] * 2.0 ** -19
+        frag = oracle.bf16_rne_f64(ref["p64"] - e) != oracle.bf16_rne_f64(ref["p64"] + e)
+        out_frag = frag.any(axis=0)
+        g64 = oracle.f32(got).astype(np.float64)
+        r64 = oracle.f32(ref["out"]).astype(np.float64)
+        diff = np.abs(g64 - r64)
+        differ = got != ref["out"]
+        over = diff > TOL_MAX_ABS
+        sq_err += float(np.sum((g64 - r64) ** 2))
+        sq_ref += float(np.sum(r64 ** 2))
+        st["max_abs"] = max(st["max_abs"], float(diff.max()))
+        st["fragile_partials"] += int(frag.sum())
+        st["fragile_outputs"] += int(out_frag.sum())
+        st["outputs_differing"] += int(differ.sum())
+        st["differing_not_fragile"] += int((differ & ~out_frag).sum())
+        st["over_max_abs"] += int(over.sum())
+        st["over_max_abs_not_fragile"] += int((over & ~out_frag).sum())
+        st["sampled_outputs"] += int(got.size)
+        st["sampled_partials"] += int(frag.size)
+    st["rel_l2"] = float(np.sqrt(sq_err / sq_ref)) if sq_ref > 0 else 0.0
+    st["within_tolerance"] = bool(st["rel_l2"] <= TOL_REL_L2 and st["max_abs"] <= TOL_MAX_ABS)
+    st["within_tolerance_except_fragile"] = bool(st["rel_l2"] <= TOL_REL_L2 and
+                                                 st["over_max_abs_not_fragile"] == 0 and
+                                                 st["differing_not_fragile"] == 0)
+    st["tolerance"] = {"max_abs": TOL_MAX_ABS, "rel_l2": TOL_REL_L2}
+    st["sample"] = (f"points {idx} x {len(cols)} output columns x {cfg.tokens} tokens; "
+                    f"oracle {time.perf_counter() - t0:.1f} s on {threads} threads")
+    return st
 
 
 # --------------------------------------------------------------------- main --
@@ -388,11 +501,33 @@ def _barrier(world):
         dist.barrier()
 
 
+def _config_keys(cfg, world, args, wl=None, staged_path=None):
+    """The `config` object of a bench line (the same keys on both arms)."""
+    d = {"workload": cfg.name, "n_ranks": cfg.n_ranks, "tokens": cfg.tokens,
+         "hidden": cfg.hidden, "points": cfg.n_points,
+         "weights": args.weights, "variant": args.variant,
+         "l2": "no flush: every step streams all points' distinct weights "
+               f"({cfg.weight_bytes() / 1e9:.2f} GB), larger than the 126 MB L2",
+         "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+    if wl is not None:
+        d["weights_gb_per_step"] = wl.weight_bytes_read() / 1e9
+        d["staged_partials"] = staged_path
+    return d
+
+
+def _configs_to_run(args):
+    names = BENCH_CONFIGS if args.config == "all" else [args.config]
+    if args.weights == "mxfp8":   # the fused MXFP8 kernel takes decode of at most 4 tokens
+        names = [n for n in names if get_config(n).tokens <= 4]
+    return names
+
+
 def run_reference(args, world, rank):
-    """The reference arm: the oracle timed on the host cores."""
+    """The reference arm: the oracle timed on the host cores, on the headline
+    workload (the first of the workloads the GPU arm runs)."""
     if rank != 0:
         return 0
-    cfg = get_config(args.config)
+    cfg = get_config(_configs_to_run(args)[0])
     for _ in range(args.warmup):
         cpu_baseline(cfg, target_s=1.0)
     times = []
@@ -408,10 +543,10 @@ def run_reference(args, world, rank):
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32-accumulate bf16", "data": "synthetic (seeded Philox)",
         "reconciliations_per_s": cfg.n_points / step_s,
-        "config": {"workload": cfg.name, "n_ranks": cfg.n_ranks, "tokens": cfg.tokens,
-                   "hidden": cfg.hidden, "points": cfg.n_points},
+        "config": _config_keys(cfg, world, args),
         "cpu_baseline": {"value": tok, "unit": "tokens/s", "cores": last["cores"],
-                         "kind": "oracle", "sample": last["sample"]},
+                         "cpu_model": last["cpu_model"], "kind": "oracle",
+                         "sample": last["sample"]},
         "e2e": {"value": tok, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -419,46 +554,16 @@ def run_reference(args, world, rank):
     return 0
 
 
-def main(argv=None):
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=CONFIG_ORDER)
-    ap.add_argument("--variant", default="auto", choices=["auto", "exact", "tensor"])
-    ap.add_argument("--staged", action="store_true")
-    ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp8"],
-                    help="mxfp8: MXFP8 weight shards (decode, at most 4 tokens)")
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-seconds", type=float, default=8.0)
-    ap.add_argument("--points", type=int, default=0,
-                    help="run only the first P points of the workload (small profiling cases)")
-    args = ap.parse_args(argv)
-    if args.warmup < 3:
-        ap.error("--warmup must be at least 3")
-
-    world, rank, local = _dist_env()
-    if world != args.gpus:
-        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    if args.impl == "reference":
-        return run_reference(args, world, rank)
-
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=device)
-
-    cfg = get_config(args.config)
+def run_config(name, args, device, world, rank, local, peaks):
+    """Times one workload (graph replays, eager calls, the end-to-end host
+    pipeline) and, on rank 0 of a single-GPU run, the CPU leg (oracle
+    baseline and parity). Returns its bench line (without the top-level
+    per_config object). Every buffer is released before it returns."""
+    cfg = get_config(name)
     if args.points:
         cfg = dataclasses.replace(cfg, layers=1, layer_points=cfg.layer_points)
         cfg.points[:] = cfg.points[:args.points]
-    if args.weights == "mxfp8" and cfg.tokens > 4:
-        ap.error("--weights mxfp8 takes decode workloads of at most 4 tokens")
     wl = Workload(cfg, device, variant=args.variant, staged=args.staged, weights=args.weights)
-    peaks = _peaks()
 
     graph = wl.capture()
     stream = torch.cuda.current_stream(device)
@@ -488,9 +593,6 @@ def main(argv=None):
     clocks = clk.summary()
 
     # ---- per-call durations outside a graph (for reference only) ---------
-    # Each call is the hot path of one point: the partial kernel (fused with the
-    # fold on the exact path) and, on staged paths, the ring fold kernel. Eager
-    # launches add host gaps between calls; the roofline uses the graph time.
     staged_path = (args.weights == "bf16" and
                    any(pl.workspace_bytes(cfg.tokens) for pl in wl.plans.values()))
     per_launch = []
@@ -507,10 +609,6 @@ def main(argv=None):
     call_ms_eager = np.mean(np.array(per_launch), axis=0)      # per point, ms
 
     # ---- end to end through the public API with host buffers -------------
-    # Every step: x and residual of all points host->device from pinned
-    # memory, one reconcile call per point through the C ABI (no graph), the
-    # outputs device->host; the points go in chunks on three streams so the
-    # copies of one chunk overlap the kernels of its neighbours.
     pipe = HostPipeline(wl, chunks=8)
     e2e_steps = max(3, min(args.steps, 10))
     for _ in range(2):
@@ -546,7 +644,6 @@ def main(argv=None):
     # dependent launch inside the graph. Its average duration is the graph's
     # device time over the timed region divided by the points per step.
     call_ms = step_ms / cfg.n_points
-    kern_bytes = step_bytes   # weights, activations, residual, output (+ staged partials)
     path = wl.path_name()
     one_kernel = wl.launches_per_step() == cfg.n_points
     kern_name = {
@@ -563,18 +660,18 @@ def main(argv=None):
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
     else:
-        achieved = kern_bytes / (step_ms * 1e-3) / 1e9
+        achieved = step_bytes / (step_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
-    roof["traffic"] = _profiled_traffic(cfg.name, wl.path_name())
+    roof["traffic"] = _profiled_traffic(cfg.name, path)
     roof["traffic_unit"] = "bytes per call (DRAM read + write, ncu), averaged over the points"
-    rec = PROFILED_TRAFFIC.get((cfg.name, wl.path_name()))
+    rec = PROFILED_TRAFFIC.get((cfg.name, path))
     roof["traffic_source"] = rec[2] if roof["traffic"] is not None else None
     roof["peak_source"] = peaks["source"] + " (burst: the step is timed alone)"
     roof["kernel"] = kern_name
     roof["call_ms_mean"] = call_ms
     roof["call_ms_mean_eager"] = float(np.mean(call_ms_eager))
-    roof["algorithmic_bytes_per_call"] = kern_bytes / cfg.n_points
+    roof["algorithmic_bytes_per_call"] = step_bytes / cfg.n_points
     roof["algorithmic_flops_per_call"] = flops / cfg.n_points
 
     line = {
@@ -586,14 +683,7 @@ def main(argv=None):
         "step_ms_stats": step_stats,
         "hbm_gbs_step": step_bytes / (step_ms * 1e-3) / 1e9,
         "tflops_step": flops / (step_ms * 1e-3) / 1e12,
-        "config": {"workload": cfg.name, "n_ranks": cfg.n_ranks, "tokens": cfg.tokens,
-                   "hidden": cfg.hidden, "points": cfg.n_points,
-                   "weights_gb_per_step": wl.weight_bytes_read() / 1e9,
-                   "weights": args.weights,
-                   "l2": "no flush: every step streams all points' distinct weights "
-                         f"({cfg.weight_bytes() / 1e9:.1f} GB), larger than the 126 MB L2",
-                   "variant": args.variant, "staged_partials": staged_path,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": _config_keys(cfg, world, args, wl, staged_path),
         "roofline": roof,
         "e2e": {"value": _job_rate(cfg.tokens, e2e_ms, world), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
@@ -602,11 +692,71 @@ def main(argv=None):
         "gpu_launches": wl.launches_per_step() * args.steps,
         "clocks": clocks,
     }
+    # ---- the CPU leg: oracle baseline and parity (rank 0, one GPU) -------
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(cfg)
+        line["parity"] = oracle_parity(wl)
+        cb = cpu_baseline(cfg, target_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": cfg.tokens / cb["step_s"], "unit": "tokens/s",
-                                "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"]}
-    del graph
+                                "cores": cb["cores"], "cpu_model": cb["cpu_model"],
+                                "kind": "oracle", "sample": cb["sample"]}
+    del graph, pipe, wl
+    gc.collect()
+    torch.cuda.empty_cache()
+    return line
+
+
+def _per_config_entry(line):
+    """The compact per-workload record under per_config."""
+    keep = ("value", "unit", "ms_per_step", "reconciliations_per_s", "step_ms_stats", "roofline",
+            "e2e", "gpu_launches", "clocks", "parity", "cpu_baseline", "config")
+    return {k: line[k] for k in keep if k in line}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="all", choices=["all"] + CONFIG_ORDER,
+                    help="one workload, or all four benchmarked ones (headline: decode_n2)")
+    ap.add_argument("--variant", default="auto", choices=["auto", "exact", "tensor"])
+    ap.add_argument("--staged", action="store_true")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp8"],
+                    help="mxfp8: MXFP8 weight shards (decode, at most 4 tokens)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the CPU leg (oracle baseline and parity)")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="oracle seconds of the CPU baseline per workload")
+    ap.add_argument("--ref-seconds", type=float, default=8.0)
+    ap.add_argument("--points", type=int, default=0,
+                    help="run only the first P points of each workload (small profiling cases)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    names = _configs_to_run(args)
+    if not names:
+        ap.error("--weights mxfp8 takes decode workloads of at most 4 tokens")
+
+    world, rank, local = _dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    peaks = _peaks()
+    lines = {name: run_config(name, args, device, world, rank, local, peaks) for name in names}
+    line = dict(lines[names[0]])
+    if len(names) > 1:
+        line["per_config"] = {name: _per_config_entry(lines[name]) for name in names}
+        line["headline"] = f"{names[0]} (the pages' worked decode example); every workload " \
+                           f"under per_config"
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

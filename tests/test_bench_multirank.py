@@ -41,7 +41,8 @@ def _rank_main(rank, world, port, q):
         mx = bench._max_over_ranks(step_ms, w, torch.device("cpu"))
         rate = bench._job_rate(1, mx, w)
         # reference arm: rank 0 alone does work; the others return at once
-        args = type("A", (), {"config": "tiny", "warmup": 3, "steps": 1, "ref_seconds": 0.1})()
+        args = type("A", (), {"config": "tiny", "warmup": 3, "steps": 1, "ref_seconds": 0.1,
+                              "weights": "bf16", "variant": "auto", "gpus": world})()
         ret = bench.run_reference(args, w, r) if r != 0 else None
         bench._barrier(w)
         q.put((rank, mx, rate, ret))

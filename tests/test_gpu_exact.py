@@ -120,3 +120,22 @@ def test_guard_zones_untouched(dev):
         assert torch.all(buf[:g].cpu() == sentinel) and torch.all(buf[g + n_in:].cpu() == sentinel)
     ref = oracle_point(n, h, x.cpu(), w.cpu(), r.cpu())
     assert np.array_equal(u16(out), ref["out"])
+
+
+def test_subnormal_product_added_with_one_rounding(dev):
+    """The oracle's pin of the accumulate step (a product below the fp32
+    normal range, added to the running sum with one rounding) on the exact
+    kernel: the partial, and with a zero residual the output, is 0x0181
+    (rounding the product first would give 0x0182)."""
+    import tensor_layer_reconciliation_b200 as tlr
+    from test_oracle_reconcile import FMA_PIN_W, FMA_PIN_X
+    n, m, k, h = 1, 1, 8, 8
+    xb = np.zeros((m, k), dtype=np.uint16)
+    wb = np.zeros((h, k), dtype=np.uint16)
+    xb[0, :4] = FMA_PIN_X
+    wb[0, :4] = FMA_PIN_W
+    x, w = from_u16(xb).to(dev), from_u16(wb).to(dev)
+    r = torch.zeros(m, h, dtype=torch.bfloat16, device=dev)
+    for staged in (False, True):
+        out, parts, _ = gpu_point(tlr.Plan(n, m, k, h), x, w, r, staged=staged)
+        assert int(parts[0, 0, 0]) == 0x0181 and int(out[0, 0]) == 0x0181

@@ -88,6 +88,39 @@ def test_noalloc_fused_path_needs_no_scratch():
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
 
 
+def test_noalloc_zero_tokens_tensor_plan():
+    """Zero tokens with the tensor-core variant chosen explicitly: nothing to
+    launch, TP_OK, and no work-size arithmetic on an empty token range."""
+    import tensor_layer_reconciliation_b200 as tlr
+    plan = tlr.Plan(4, 8, 1024, 512, variant="tensor")
+    st = tlr.tp_rowlinear_reconcile_noalloc(plan.handle, 0, 0, 0, 0, 0,
+                                            torch.cuda.current_stream().cuda_stream)
+    assert st == tlr.TP_OK
+    assert plan.launches(0) == 0 and plan.workspace_bytes(0) == 0
+
+
+def test_noalloc_staged_exact_twice():
+    """The exact variant with staged partials: its partials go through the
+    scratch array and a ring kernel; bit-identical to the workspace form."""
+    import tensor_layer_reconciliation_b200 as tlr
+    dev = torch.device("cuda")
+    n, m, k, h = 4, 3, 1024, 512
+    plan = tlr.Plan(n, m, k, h, variant="exact", staged=True)
+    assert plan.workspace_bytes(m) > 0
+    stream = torch.cuda.current_stream().cuda_stream
+    for call, seed in enumerate((41, 42)):
+        x, w, r = inputs(n, m, k, h, seed, dev)
+        wp = plan.pack_weights(w)
+        ref = plan.reconcile(x, wp, r)
+        out = torch.full((m, h), float("nan"), dtype=torch.bfloat16, device=dev)
+        st = tlr.tp_rowlinear_reconcile_noalloc(plan.handle, _ptr(x), _ptr(wp), _ptr(r), _ptr(out),
+                                                m, stream)
+        assert st == tlr.TP_OK
+        torch.cuda.synchronize()
+        assert plan.device_error_flags() == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), f"call {call}"
+
+
 def test_noalloc_refuses_more_than_its_scratch():
     import tensor_layer_reconciliation_b200 as tlr
     n, m, k, h = 4, 4096, 1024, 5120       # N*M*H*2 = 168 MB > 16 MiB
