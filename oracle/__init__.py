@@ -27,6 +27,11 @@ Functions and the passages they follow:
   all-reduce schemes (NVL72 hosting post, All-reduce section).
 * ``moe_combine_bytes`` -- per-rank bytes of an MoE combine: local weighted
   accumulation, then one all-reduce (NVL72 hosting post, MoE dispatch/combine).
+* ``mx_quantize`` / ``mx_dequant_bf16`` -- MXFP8 shards (OCP MX E4M3, E8M0 per
+  32 weights of a rank slice) for the NVL72 hosting post's MXFP8 weights.
+* ``nvfp4_quantize`` / ``nvfp4_dequant_bf16`` -- NVFP4 shards (E2M1, E4M3 per 16
+  weights, power-of-two second-level scale) for the TP=4-vs-TP=8 post's NVFP4
+  weights.
 
 Pins that tie each function to the pages or to mathematics (not to itself)
 live in ``tests/test_oracle_*.py``. Parity unpinned: the exact fp32 rounding of
@@ -98,6 +103,18 @@ def lib():
                                             ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                                             ctypes.c_int]
         L.orc_moe_combine_bytes.restype = ctypes.c_uint64
+        L.orc_e2m1_rne.argtypes = [ctypes.c_double]
+        L.orc_e2m1_rne.restype = ctypes.c_uint8
+        L.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+        L.orc_e2m1_value.restype = ctypes.c_double
+        L.orc_nvfp4_global_exp.argtypes = [ctypes.c_double]
+        L.orc_nvfp4_global_exp.restype = ctypes.c_int
+        L.orc_nvfp4_quantize.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, _U16P, _U8P, _U8P,
+                                         ctypes.POINTER(ctypes.c_int)]
+        L.orc_nvfp4_quantize.restype = ctypes.c_int
+        L.orc_nvfp4_dequant_bf16.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, _U8P, _U8P,
+                                             ctypes.c_int, _U16P]
+        L.orc_nvfp4_dequant_bf16.restype = ctypes.c_int
         L.orc_e4m3_rne.argtypes = [ctypes.c_double]
         L.orc_e4m3_rne.restype = ctypes.c_uint8
         L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
@@ -301,6 +318,49 @@ def moe_combine_bytes(scheme: str, n_ranks: int, tokens: int, hidden: int, elem_
     local_accumulate=False all-reduces each of the top_k expert slots apart."""
     return int(lib().orc_moe_combine_bytes(ALLREDUCE_SCHEMES[scheme], n_ranks, tokens, hidden,
                                            elem_bytes, top_k, int(bool(local_accumulate))))
+
+
+def e2m1_rne(v: float) -> int:
+    """E2M1 code (sign in bit 3) of the exact value v, nearest even, saturating at 6."""
+    return int(lib().orc_e2m1_rne(float(v)))
+
+
+def e2m1_value(code: int) -> float:
+    return float(lib().orc_e2m1_value(int(code)))
+
+
+def nvfp4_global_exp(amax: float) -> int:
+    return int(lib().orc_nvfp4_global_exp(float(amax)))
+
+
+def nvfp4_quantize(n_ranks: int, w_hk: np.ndarray):
+    """Linear weight [H, K] bf16 -> (q [N, H, K/N/2] uint8, two E2M1 codes per
+    byte (earlier k in the low nibble); scales [N, H, K/N/16] E4M3; g, the
+    second-level exponent)."""
+    w_hk = _u16(w_hk)
+    h, k = w_hk.shape
+    ks = k // n_ranks
+    q = np.zeros((n_ranks, h, ks // 2), dtype=np.uint8)
+    sc = np.zeros((n_ranks, h, ks // 16), dtype=np.uint8)
+    g = ctypes.c_int(0)
+    rc = lib().orc_nvfp4_quantize(n_ranks, h, k, _ptr(w_hk, _U16P), _ptr(q, _U8P), _ptr(sc, _U8P),
+                                  ctypes.byref(g))
+    if rc != ORC_OK:
+        raise OracleError(f"orc_nvfp4_quantize failed with {rc}")
+    return q, sc, g.value
+
+
+def nvfp4_dequant_bf16(n_ranks: int, q: np.ndarray, scales: np.ndarray, g: int) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    n, h, half = q.shape
+    k = 2 * half * n
+    w = np.empty((h, k), dtype=np.uint16)
+    rc = lib().orc_nvfp4_dequant_bf16(n_ranks, h, k, _ptr(q, _U8P), _ptr(scales, _U8P), int(g),
+                                      _ptr(w, _U16P))
+    if rc != ORC_OK:
+        raise OracleError(f"orc_nvfp4_dequant_bf16 failed with {rc}")
+    return w
 
 
 def cores() -> int:

@@ -31,6 +31,11 @@
  *      Linear weight to E4M3 codes with one E8M0 scale per 32 weights of a
  *      rank's slice, and back; a reconciliation over such shards is the
  *      point above over the dequantised weights (exact in bf16).
+ *   5. NVFP4 weight shards: E2M1 codes with one E4M3 scale per 16 weights
+ *      and a power-of-two second-level scale, and back (exact in bf16).
+ *   6. Byte models: the ring's 2(N-1)/N per rank, the naive, ring and switch
+ *      all-reduce schemes, and the MoE combine (local accumulation, then one
+ *      all-reduce).
  *
  * Build: plain C11, -ffp-contract=off (no fused multiply-add other than the
  * explicit fmaf), no fast-math, so every float operation is one IEEE
@@ -563,6 +568,133 @@ int orc_mx_dequant_bf16(int n_ranks, int64_t hidden, int64_t k, const uint8_t *q
                     return ORC_ERR_ARGS;
                 w_hk[h * k + (int64_t)r * ks + j] = b;
             }
+    return ORC_OK;
+}
+
+/* -------------------------------------------------- NVFP4 weight shards -- */
+/*
+ * 4-bit weights (the TP=4-vs-TP=8 post deploys NVFP4 weights with 16-bit
+ * activations; the post itself garbles the element format, so the format is
+ * NVIDIA's published NVFP4): each weight is an FP4 E2M1 value (sign, 2
+ * exponent bits, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6),
+ * every 16 consecutive weights along K inside one rank's slice share an FP8
+ * E4M3 block scale, and one second-level scale serves the whole tensor.
+ * Reading: the second-level scale is the power of two 2^g with g the
+ * smallest integer such that amax(W) / 2^g <= 6 * 448 (every block scale then
+ * fits E4M3; a power of two keeps every dequantised weight exact in bf16: at
+ * most 2 x 4 significant bits); an all-zero tensor takes g = 0.
+ *   block scale  b = E4M3 nearest to amax(block) / (6 * 2^g), ties to even
+ *   element      q = E2M1 nearest to w / (b * 2^g), ties to even,
+ *                    saturating at +-6; a block whose b is 0 stores zeros
+ *   value        q * b * 2^g
+ * Codes: sign in bit 3, magnitude index in bits 0-2. Two codes per byte,
+ * the earlier k in the low nibble.
+ */
+
+/* E2M1 code (0..15) of the exact value v, nearest even, saturating at 6. */
+uint8_t orc_e2m1_rne(double v)
+{
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    const uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    const double a = fabs(v);
+    if (a >= 6.0)
+        return sign | 7;
+    int lo = 0;
+    while (lo < 7 && mag[lo + 1] <= a)
+        ++lo;                                 /* mag[lo] <= a < mag[lo + 1] */
+    const double d_lo = a - mag[lo], d_hi = mag[lo + 1] - a;
+    int m = lo;
+    if (d_hi < d_lo || (d_hi == d_lo && (lo & 1)))
+        m = lo + 1;                           /* nearer, or a tie to the even index */
+    return sign | (uint8_t)m;
+}
+
+double orc_e2m1_value(uint8_t c)
+{
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    return (c & 0x8) ? -mag[c & 7] : mag[c & 7];
+}
+
+/* The second-level exponent g of a tensor whose largest magnitude is amax. */
+int orc_nvfp4_global_exp(double amax)
+{
+    if (amax == 0.0)
+        return 0;
+    int g = -200;
+    while (amax / ldexp(1.0, g) > 6.0 * 448.0)
+        ++g;
+    return g;
+}
+
+/* Linear weight [hidden][k] (bf16) -> per-rank NVFP4 shards:
+ *   q      [n_ranks][hidden][k/n_ranks/2] bytes, two E2M1 codes each
+ *   scales [n_ranks][hidden][k/n_ranks/16] E4M3 block scales
+ *   *g     the second-level exponent
+ * k/n_ranks must be a multiple of 16. */
+int orc_nvfp4_quantize(int n_ranks, int64_t hidden, int64_t k, const uint16_t *w_hk, uint8_t *q,
+                       uint8_t *scales, int *g_out)
+{
+    if (n_ranks < 1 || hidden < 0 || k < 0 || k % n_ranks != 0 || (k / n_ranks) % 16 != 0)
+        return ORC_ERR_ARGS;
+    double amax = 0.0;
+    for (int64_t i = 0; i < hidden * k; ++i) {
+        const double a = fabs((double)orc_f32(w_hk[i]));
+        if (a > amax)
+            amax = a;
+    }
+    const int g = orc_nvfp4_global_exp(amax);
+    const double two_g = ldexp(1.0, g);
+    const int64_t ks = k / n_ranks, nb = ks / 16;
+    for (int r = 0; r < n_ranks; ++r)
+        for (int64_t h = 0; h < hidden; ++h) {
+            const int64_t row = (int64_t)r * hidden + h;
+            for (int64_t b = 0; b < nb; ++b) {
+                const uint16_t *w = w_hk + h * k + (int64_t)r * ks + 16 * b;
+                double bmax = 0.0;
+                for (int i = 0; i < 16; ++i) {
+                    const double a = fabs((double)orc_f32(w[i]));
+                    if (a > bmax)
+                        bmax = a;
+                }
+                const uint8_t bs = orc_e4m3_rne(bmax / (6.0 * two_g));
+                scales[row * nb + b] = bs;
+                const double bval = orc_e4m3_value(bs);
+                for (int i = 0; i < 16; ++i) {
+                    const uint8_t c = bval == 0.0 ? 0 : orc_e2m1_rne((double)orc_f32(w[i]) / (bval * two_g));
+                    const int64_t j = 16 * b + i;           /* index within the row */
+                    uint8_t *dst = &q[row * (ks / 2) + j / 2];
+                    if (j % 2 == 0)
+                        *dst = c;
+                    else
+                        *dst = (uint8_t)(*dst | (c << 4));
+                }
+            }
+        }
+    *g_out = g;
+    return ORC_OK;
+}
+
+/* Dequantised NVFP4 shards back in the Linear layout [hidden][k] as bf16
+ * (exact; ORC_ERR_ARGS if a value leaves bf16's range). */
+int orc_nvfp4_dequant_bf16(int n_ranks, int64_t hidden, int64_t k, const uint8_t *q,
+                           const uint8_t *scales, int g, uint16_t *w_hk)
+{
+    if (n_ranks < 1 || hidden < 0 || k < 0 || k % n_ranks != 0 || (k / n_ranks) % 16 != 0)
+        return ORC_ERR_ARGS;
+    const int64_t ks = k / n_ranks, nb = ks / 16;
+    for (int r = 0; r < n_ranks; ++r)
+        for (int64_t h = 0; h < hidden; ++h) {
+            const int64_t row = (int64_t)r * hidden + h;
+            for (int64_t j = 0; j < ks; ++j) {
+                const uint8_t byte = q[row * (ks / 2) + j / 2];
+                const uint8_t c = (j % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+                const double v = ldexp(orc_e2m1_value(c) * orc_e4m3_value(scales[row * nb + j / 16]), g);
+                const uint16_t b = orc_bf16_rne_f64(v);
+                if ((double)orc_f32(b) != v)
+                    return ORC_ERR_ARGS;
+                w_hk[h * k + (int64_t)r * ks + j] = b;
+            }
+        }
     return ORC_OK;
 }
 

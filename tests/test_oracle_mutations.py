@@ -21,6 +21,7 @@ import test_oracle_reconcile as trc
 import test_oracle_ring as trg
 import test_oracle_allreduce as tar
 import test_oracle_mx as tmx
+import test_oracle_nvfp4 as tnv
 
 SRC = open(obuild.SRC).read()
 
@@ -84,6 +85,18 @@ MUTATIONS = {
     "combine_no_local_acc": ("const int64_t buffers = local_accumulate ? 1 : top_k;",
                              "const int64_t buffers = top_k;",
                              [tar.test_moe_combine_bytes_golden]),
+    # NVFP4: E2M1 ties go up instead of to the even index
+    "e2m1_half_up": ("    if (d_hi < d_lo || (d_hi == d_lo && (lo & 1)))",
+                     "    if (d_hi <= d_lo)",
+                     [lambda: [tnv.test_e2m1_midpoints_and_saturation(v, c)
+                               for v, c in ((0.25, 0), (1.25, 2), (2.5, 4))]]),
+    # NVFP4: no saturation at 6
+    "e2m1_no_saturation": ("    if (a >= 6.0)\n        return sign | 7;\n", "    if (a >= 12.0)\n        return sign | 7;\n",
+                           [lambda: tnv.test_e2m1_midpoints_and_saturation(6.5, 7)]),
+    # NVFP4: the second-level exponent one too large
+    "nvfp4_g_plus_one": ("    while (amax / ldexp(1.0, g) > 6.0 * 448.0)\n        ++g;\n    return g;",
+                         "    while (amax / ldexp(1.0, g) > 6.0 * 448.0)\n        ++g;\n    return g + 1;",
+                         [lambda: tnv.test_global_exponent_rule(0.1)]),
     # MXFP8: element rounding half away from zero instead of to even
     "e4m3_half_up": ("if (rem > 0.5 || (rem == 0.5 && fmod(m, 2.0) == 1.0))",
                      "if (rem >= 0.5)",
@@ -122,7 +135,8 @@ def test_pin_catches_mutation(name, monkeypatch):
     for fn in ("orc_bf16_rne", "orc_bf16_rne_f64", "orc_f32", "orc_bf16_rne_array",
                "orc_bf16_rne_f64_array", "orc_partials", "orc_ring", "orc_residual",
                "orc_reconcile", "orc_ring_bytes", "orc_allreduce_bytes", "orc_moe_combine_bytes",
-               "orc_e4m3_rne",
+               "orc_e4m3_rne", "orc_e2m1_rne", "orc_e2m1_value", "orc_nvfp4_global_exp",
+               "orc_nvfp4_quantize", "orc_nvfp4_dequant_bf16",
                "orc_e4m3_value", "orc_mx_quantize", "orc_mx_dequant_bf16"):
         f = getattr(mutant, fn)
         g = getattr(real, fn)
