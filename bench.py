@@ -132,7 +132,8 @@ class Workload:
         self.res_all = torch.empty(cfg.n_points * m * h, dtype=torch.bfloat16, device=device)
         self.out_all = torch.empty(cfg.n_points * m * h, dtype=torch.bfloat16, device=device)
         self.w_packed = []
-        ws_need = max(pl.workspace_bytes(m) for pl in self.plans.values())
+        ws_need = max({"mxfp8": pl.mxfp8_workspace_bytes, "nvfp4": pl.nvfp4_workspace_bytes}.get(
+            weights, pl.workspace_bytes)(m) for pl in self.plans.values())
         self.workspace = (torch.zeros(ws_need, dtype=torch.uint8, device=device)
                           if ws_need else None)   # counter head zero on first use
         for i, p in enumerate(cfg.points):
@@ -141,6 +142,8 @@ class Workload:
             w = point_tensor(cfg, p, KIND_W, device)
             if weights == "mxfp8":        # (E4M3 codes, E8M0 scales) per point
                 self.w_packed.append(self.plans[p.k].pack_weights_mxfp8(w))
+            elif weights == "nvfp4":      # (E2M1 code pairs, E4M3 block scales + g) per point
+                self.w_packed.append(self.plans[p.k].pack_weights_nvfp4(w))
             else:
                 self.w_packed.append(self.plans[p.k].pack_weights(w))
             del w
@@ -161,9 +164,10 @@ class Workload:
     def call(self, i, stream=None):
         """The reconciliation of point i through the public API."""
         plan = self.plans[self.cfg.points[i].k]
-        if self.weights == "mxfp8":
+        if self.weights in ("mxfp8", "nvfp4"):
             q, sc = self.w_packed[i]
-            plan.reconcile_mxfp8(self.x(i), q, sc, self.res(i), out=self.out(i), stream=stream)
+            fn = plan.reconcile_mxfp8 if self.weights == "mxfp8" else plan.reconcile_nvfp4
+            fn(self.x(i), q, sc, self.res(i), out=self.out(i), workspace=self.workspace, stream=stream)
         else:
             plan.reconcile(self.x(i), self.w_packed[i], self.res(i), out=self.out(i),
                            workspace=self.workspace, stream=stream)
@@ -175,24 +179,27 @@ class Workload:
 
     def weight_bytes_read(self):
         """Bytes of packed weights one step reads."""
-        if self.weights == "mxfp8":
+        if self.weights in ("mxfp8", "nvfp4"):
             return sum(q.numel() + sc.numel() for q, sc in self.w_packed)
         return self.cfg.weight_bytes()
 
     def path_name(self):
-        """Which kernels one call runs: 'tensor' (tensor-core partials, staged),
-        'exact-staged', 'exact-fused' or 'mxfp8' (MXFP8 shards, one fused kernel)."""
-        if self.weights == "mxfp8":
-            return "mxfp8"
+        """Which kernels one call runs: 'tensor' (tensor-core partials),
+        'exact-staged', 'exact-fused', 'mxfp8' or 'nvfp4' (quantised shards)."""
+        if self.weights in ("mxfp8", "nvfp4"):
+            return self.weights
         pl = next(iter(self.plans.values()))
         if pl.effective_variant(self.cfg.tokens) == "tensor":
             return "tensor"
         return "exact-staged" if pl.staged else "exact-fused"
 
     def launches_per_step(self):
-        if self.weights == "mxfp8":
-            return self.cfg.n_points
-        return sum(self.plans[p.k].launches(self.cfg.tokens) for p in self.cfg.points)
+        """Kernels one step launches (MXFP8 calls take the tensor-core path's
+        kernels: one where it folds on chip, two where a ring kernel follows)."""
+        m = self.cfg.tokens
+        if self.weights in ("mxfp8", "nvfp4"):
+            return sum(1 if self.workspace is None or m <= 2 else 2 for p in self.cfg.points)
+        return sum(self.plans[p.k].launches(m) for p in self.cfg.points)
 
     def capture(self):
         g = torch.cuda.CUDAGraph()
@@ -376,6 +383,10 @@ def oracle_parity(wl, threads=None):
         if wl.weights == "mxfp8":     # over the dequantised shards (a row quantises alone)
             q, sc = oracle.mx_quantize(cfg.n_ranks, np.ascontiguousarray(w))
             w = oracle.mx_dequant_bf16(cfg.n_ranks, q, sc)
+        elif wl.weights == "nvfp4":   # the tensor scale needs the whole weight's maximum
+            wfull = point_tensor(cfg, p, KIND_W).view(torch.int16).numpy().view(np.uint16)
+            q, sc, g = oracle.nvfp4_quantize(cfg.n_ranks, wfull)
+            w = np.ascontiguousarray(oracle.nvfp4_dequant_bf16(cfg.n_ranks, q, sc, g)[cols])
         ref = oracle.reconcile(cfg.n_ranks, cfg.hidden, x, np.ascontiguousarray(w), r, cols=cols,
                                threads=threads)
         got = wl.out(i)[:, torch.from_numpy(cols).to(wl.device)].cpu().view(torch.int16).numpy().view(np.uint16)
@@ -516,10 +527,7 @@ def _config_keys(cfg, world, args, wl=None, staged_path=None):
 
 
 def _configs_to_run(args):
-    names = BENCH_CONFIGS if args.config == "all" else [args.config]
-    if args.weights == "mxfp8":   # the fused MXFP8 kernel takes decode of at most 4 tokens
-        names = [n for n in names if get_config(n).tokens <= 4]
-    return names
+    return BENCH_CONFIGS if args.config == "all" else [args.config]
 
 
 def run_reference(args, world, rank):
@@ -593,8 +601,9 @@ def run_config(name, args, device, world, rank, local, peaks):
     clocks = clk.summary()
 
     # ---- per-call durations outside a graph (for reference only) ---------
-    staged_path = (args.weights == "bf16" and
-                   any(pl.workspace_bytes(cfg.tokens) for pl in wl.plans.values()))
+    # the calls stage partials (bf16 partials or fp32 k-parts) exactly when
+    # they need a workspace; the cluster fold and the exact fused kernel do not
+    staged_path = wl.workspace is not None
     per_launch = []
     for _ in range(2):
         evs = []
@@ -634,8 +643,8 @@ def run_config(name, args, device, world, rank, local, peaks):
     value = _job_rate(cfg.tokens, step_ms, world)
     recon = _job_rate(cfg.n_points, step_ms, world)
     step_bytes = cfg.algorithmic_bytes(staged_partials=staged_path)
-    if args.weights == "mxfp8":   # codes + scales in place of bf16 weights; nothing staged
-        step_bytes = (cfg.algorithmic_bytes(staged_partials=False) - cfg.weight_bytes()
+    if args.weights in ("mxfp8", "nvfp4"):   # codes + scales in place of bf16 weights
+        step_bytes = (cfg.algorithmic_bytes(staged_partials=staged_path) - cfg.weight_bytes()
                       + wl.weight_bytes_read())
     flops = cfg.flops()
     tensor_bound = cfg.tokens >= 1024
@@ -646,11 +655,19 @@ def run_config(name, args, device, world, rank, local, peaks):
     call_ms = step_ms / cfg.n_points
     path = wl.path_name()
     one_kernel = wl.launches_per_step() == cfg.n_points
+    fold_where = ("the N ranks of a tile in one cluster, ring fold through distributed shared memory"
+                  if wl.workspace is None else
+                  "k-split parts, ring fold by the CTA completing a tile")
     kern_name = {
-        "mxfp8": "reconciliation call: mx_reconcile_kernel (MXFP8 partials, ring fold, residual)",
+        "mxfp8": (f"reconciliation call: tc_partial_kernel, MXFP8 form (codes widened to bf16 "
+                  f"tiles on chip; {fold_where})" if one_kernel else
+                  "reconciliation call: tc_partial_kernel, MXFP8 form, then a ring fold kernel"),
+        "nvfp4": (f"reconciliation call: tc_partial_kernel, NVFP4 form (codes widened to bf16 "
+                  f"tiles on chip; {fold_where})" if one_kernel else
+                  "reconciliation call: tc_partial_kernel, NVFP4 form, then a ring fold kernel"),
         "exact-fused": "reconciliation call: exact_partial_kernel (partials, ring fold, residual)",
         "exact-staged": "reconciliation call: exact_partial_kernel then ring_reduce_kernel",
-        "tensor": ("reconciliation call: tc_partial_kernel (partials, in-kernel ring fold, residual)"
+        "tensor": (f"reconciliation call: tc_partial_kernel ({fold_where}; residual)"
                    if one_kernel else
                    "reconciliation call: tc_partial_kernel (tc2_partial_kernel on CTA pairs "
                    "from 129 tokens) then a ring fold kernel"),
@@ -721,8 +738,9 @@ def main(argv=None):
                     help="one workload, or all four benchmarked ones (headline: decode_n2)")
     ap.add_argument("--variant", default="auto", choices=["auto", "exact", "tensor"])
     ap.add_argument("--staged", action="store_true")
-    ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp8"],
-                    help="mxfp8: MXFP8 weight shards (decode, at most 4 tokens)")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp8", "nvfp4"],
+                    help="mxfp8: E4M3 codes, E8M0 scales per 32 weights; nvfp4: E2M1 codes, "
+                         "E4M3 scales per 16 weights, power-of-two tensor scale")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the CPU leg (oracle baseline and parity)")
@@ -735,8 +753,6 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     names = _configs_to_run(args)
-    if not names:
-        ap.error("--weights mxfp8 takes decode workloads of at most 4 tokens")
 
     world, rank, local = _dist_env()
     if world != args.gpus:

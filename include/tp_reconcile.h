@@ -210,39 +210,140 @@ TP_API uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int e
                        int64_t points);
 
 /* ---------------------------------------------------------------------
+ * The ring all-reduce as a protocol between ranks that each hold their own
+ * buffers: S2-S4 as N tensor-parallel GPUs run them ("Interconnects e
+ * clusters", 01 Conceito: a reduce-scatter and an all-gather of H/N-wide
+ * chunks; NVL72 hosting post, All-reduce section: each peer reduces one slice,
+ * then broadcasts it). Rank r pulls each chunk from its predecessor r-1 once
+ * the predecessor's step flag shows it written: reduce-scatter steps s =
+ * 0..N-2 fold chunk r-1-s into rank r's buffer (bf16 round-to-nearest-even
+ * per add, the received sum on the left), all-gather steps pass the reduced
+ * chunks on, and every rank adds the residual to every chunk. Every rank's
+ * output equals tp_ring_reduce's on the same partials, bit for bit.
+ * ------------------------------------------------------------------- */
+
+/* Bytes of one rank's workspace for tp_ring_allreduce_ranks: its step flags
+ * (one 32-bit flag per CTA of the rank, 256-byte rounded) first, then two
+ * [M][H] bf16 buffers (reduce-scatter, all-gather), each 256-byte rounded.
+ * 0 for a null plan or tokens outside 0..max_tokens. */
+TP_API size_t tp_ring_rank_workspace_bytes(const tp_plan* plan, int64_t tokens);
+
+/* Runs ranks first_rank .. first_rank + launch_ranks - 1 of the ring
+ * protocol in one launch on the current stream.
+ *   partials    [N] device pointers: rank r's partial [M][H] bf16
+ *   residual    [M][H] bf16 (the residual every rank adds)
+ *   outs        [N] device pointers: rank r's output [M][H] bf16
+ *   workspaces  [N] device pointers of tp_ring_rank_workspace_bytes each,
+ *               the flag block zeroed before the first call; every call
+ *               that completes leaves the flags equal again, so the same
+ *               workspaces serve any number of calls (after a call that set
+ *               the error bit, zero the flag blocks again)
+ *   wait_limit_ns  the bound of every wait on another rank's flag (0: 1 s);
+ *               a wait that runs out sets bit 1 of the device error word
+ *               (tp_device_error_flags) and that part of the rank stops
+ * The arrays are host arrays. On one GPU (all ranks in memory of this
+ * device) launch all N ranks at once: the launch is cooperative, so all their
+ * CTAs are resident together. With one GPU per rank, each process launches
+ * its own rank with the other ranks' buffers as peer pointers (peer memory is
+ * read with plain loads only). Launching only some ranks of a group whose
+ * other ranks never run makes their waits run out: a test of the bound.
+ * Checks: pointers non-null and 16-byte aligned, outputs and workspaces
+ * disjoint from each other and from the inputs, ranks within 0..N-1. */
+TP_API tp_status tp_ring_allreduce_ranks(const tp_plan* plan, const void* const* partials,
+                                         const void* residual, void* const* outs,
+                                         void* const* workspaces, int first_rank, int launch_ranks,
+                                         int64_t tokens, uint64_t wait_limit_ns, void* stream);
+
+/* ---------------------------------------------------------------------
  * MXFP8 weight shards. The NVL72 hosting post stores the MoE GEMM's weights
- * as MXFP8; the layout here is the OCP Microscaling v1.0 MXFP8 (E4M3)
- * format applied to each rank's slice: every 32 consecutive weights along
- * K share one E8M0 scale X = 2^s (byte s + 127), s = floor(log2 max|w|) - 8
- * clamped to [-127, 127] (-127 for an all-zero run), and each weight is the
- * E4M3 code nearest to w / X, ties to even, saturating at +-448. The
+ * as MXFP8; the format here is the OCP Microscaling v1.0 MXFP8 (E4M3)
+ * applied to each rank's slice: every 32 consecutive weights along K share
+ * one E8M0 scale X = 2^s (byte s + 127), s = floor(log2 max|w|) - 8 clamped
+ * to [-127, 127] (-127 for an all-zero run), and each weight is the E4M3
+ * code nearest to w / X, ties to even, saturating at +-448. The
  * reconciliation over such shards is S1-S4 over the dequantised weights
  * E4M3 * X, which are exact in bf16 for any run whose largest weight is at
- * least 2^-116.
+ * least 2^-116. Requires (K/N) % 64 == 0.
  * ------------------------------------------------------------------- */
 
 /* Sizes of the two shard buffers: q_bytes = H*K (one E4M3 code per weight,
- * [N][H][K/N]), scale_bytes = H*K/32 ([N][H][K/N/32]). TP_ERR_UNSUPPORTED
- * when K/N is not a multiple of 32; TP_ERR_INVALID for null arguments. */
+ * [N][H][K/N]), scale_bytes = H*K/32, laid out [N][K/N/64][H][2]: for each
+ * 64-column block of a rank slice, the scales of its two 32-weight runs for
+ * every row h in turn (the scales a 128-row tile needs for one block are
+ * contiguous). TP_ERR_UNSUPPORTED when K/N is not a multiple of 64;
+ * TP_ERR_INVALID for null arguments. */
 TP_API tp_status tp_plan_mxfp8_bytes(const tp_plan* plan, size_t* q_bytes, size_t* scale_bytes);
 
-/* S0 for MXFP8: Linear weight [H][K] bf16 -> w_q [N][H][K/N] codes and
- * w_scales [N][H][K/N/32] scales (device buffers of tp_plan_mxfp8_bytes'
- * sizes; w_hk and w_q 16-byte aligned; no overlap). Asynchronous on
- * `stream`; the result is identical, bit for bit, to the format's
- * definition above. */
+/* S0 for MXFP8: Linear weight [H][K] bf16 -> w_q codes and w_scales (device
+ * buffers of tp_plan_mxfp8_bytes' sizes and layouts; all 16-byte aligned; no
+ * overlap). Asynchronous on `stream`; the result is identical, bit for bit,
+ * to the format's definition above. */
 TP_API tp_status tp_pack_weights_mxfp8(const tp_plan* plan, const void* w_hk, void* w_q,
                                        void* w_scales, void* stream);
 
-/* S1-S4 for decode over MXFP8 shards, one kernel, no workspace:
- *   x, residual, out as in tp_rowlinear_reconcile; w_q, w_scales from
- *   tp_pack_weights_mxfp8; tokens 0 .. 4 (more: TP_ERR_UNSUPPORTED, the
- *   fused kernel streams the shards once for all tokens of a decode step).
- * Partials are fp32 sums rounded once to bf16, in an order of its own
- * (lanes of a warp split K), then folded in ring order with the residual. */
+/* Bytes of workspace tp_rowlinear_reconcile_mxfp8 needs for `tokens` tokens
+ * (0 when the call folds in clusters and stages nothing); the same layout
+ * and zeroing rule as tp_rowlinear_reconcile's workspace. Whatever the
+ * plan's variant, MXFP8 calls run on the tensor cores. 0 for a null plan or
+ * tokens <= 0. */
+TP_API size_t tp_plan_mxfp8_workspace_bytes(const tp_plan* plan, int64_t tokens);
+
+/* S1-S4 over MXFP8 shards, on the tensor cores:
+ *   x, residual, out, tokens as in tp_rowlinear_reconcile; w_q, w_scales
+ *   from tp_pack_weights_mxfp8; workspace of
+ *   tp_plan_mxfp8_workspace_bytes(plan, tokens) bytes (NULL when 0), zeroed
+ *   before its first use.
+ * Code tiles are widened to bf16 tiles in shared memory (E4M3 * 2^s, exact)
+ * and multiplied with the bf16 activations in fp32 on the tensor cores; the
+ * partials are rounded once to bf16 and folded in ring order with the
+ * residual, as for bf16 shards. TP_ERR_UNSUPPORTED when K/N is not a
+ * multiple of 64. */
 TP_API tp_status tp_rowlinear_reconcile_mxfp8(const tp_plan* plan, const void* x, const void* w_q,
                                               const void* w_scales, const void* residual,
-                                              void* out, int64_t tokens, void* stream);
+                                              void* out, int64_t tokens, void* workspace,
+                                              void* stream);
+
+/* ---------------------------------------------------------------------
+ * NVFP4 weight shards. The TP=4-vs-TP=8 post runs NVFP4 weights with
+ * 16-bit activations; the format is NVIDIA's NVFP4 applied to each rank's
+ * slice: FP4 E2M1 elements, one FP8 E4M3 block scale per 16 consecutive
+ * weights along K, and a second-level scale 2^g for the whole weight, g the
+ * smallest integer with max|W| / 2^g <= 6 * 448 (0 for an all-zero weight):
+ *   block scale b = E4M3 nearest to max|block| / (6 * 2^g), ties to even;
+ *   element     q = E2M1 nearest to w / (b * 2^g), ties to even, saturating
+ *                   at +-6 (0 where b is 0).
+ * (The second-level scale is a power of two so that every dequantised weight
+ * q * b * 2^g is exact in bf16.) The reconciliation over such shards is
+ * S1-S4 over the dequantised weights. Requires (K/N) % 64 == 0.
+ * ------------------------------------------------------------------- */
+
+/* Sizes of the two shard buffers: q_bytes = H*K/2 ([N][H][K/N/2], two E2M1
+ * codes a byte, the earlier k in bits 0-3); scale_bytes = H*K/16 + 16: the
+ * block scales laid out [N][K/N/64][H][4] (the four scales of each row for
+ * one 64-column block, row after row), then 16 bytes holding g (int32) and
+ * the weight's largest magnitude. TP_ERR_UNSUPPORTED when K/N is not a
+ * multiple of 64; TP_ERR_INVALID for null arguments. */
+TP_API tp_status tp_plan_nvfp4_bytes(const tp_plan* plan, size_t* q_bytes, size_t* scale_bytes);
+
+/* S0 for NVFP4: Linear weight [H][K] bf16 -> w_q codes and w_scales (device
+ * buffers of tp_plan_nvfp4_bytes' sizes; all 16-byte aligned; no overlap).
+ * Two kernels (the weight's largest magnitude, then the blocks), async on
+ * `stream`; identical, bit for bit, to the definition above. */
+TP_API tp_status tp_pack_weights_nvfp4(const tp_plan* plan, const void* w_hk, void* w_q,
+                                       void* w_scales, void* stream);
+
+/* Workspace of tp_rowlinear_reconcile_nvfp4 (as for MXFP8). */
+TP_API size_t tp_plan_nvfp4_workspace_bytes(const tp_plan* plan, int64_t tokens);
+
+/* S1-S4 over NVFP4 shards on the tensor cores, as
+ * tp_rowlinear_reconcile_mxfp8: code tiles widened to bf16 tiles in shared
+ * memory (E2M1 * block scale * 2^g, exact), multiplied with the bf16
+ * activations in fp32, partials rounded once to bf16 and folded in ring
+ * order with the residual. */
+TP_API tp_status tp_rowlinear_reconcile_nvfp4(const tp_plan* plan, const void* x, const void* w_q,
+                                              const void* w_scales, const void* residual,
+                                              void* out, int64_t tokens, void* workspace,
+                                              void* stream);
 
 /* All-reduce schemes of tp_allreduce_bytes. */
 typedef enum {
@@ -294,8 +395,9 @@ TP_API const char* tp_status_string(tp_status status);
 TP_API int tp_last_cuda_error(void);
 
 /* Reads, and with reset != 0 clears, the device-side error word of the
- * plan's device: bit 0 is set when a kernel's bounded wait on a pipeline
- * barrier ran out (the kernel then stops early, so its output is invalid;
+ * plan's device: bit 1 is set when a wait of tp_ring_allreduce_ranks on
+ * another rank's flag ran out; bit 0 is set when a kernel's bounded wait on a
+ * pipeline barrier ran out (the kernel then stops early, so its output is invalid;
  * copies or tensor-core operations it had in flight may not have finished
  * when it returned, so the context should be discarded, e.g. by
  * cudaDeviceReset, before results are trusted again). With reset != 0 and a

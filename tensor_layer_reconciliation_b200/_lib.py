@@ -24,7 +24,10 @@ EXPORTED = (
     "tp_pack_weights",
     "tp_rowlinear_reconcile", "tp_rowlinear_reconcile_noalloc", "tp_rowlinear_partials",
     "tp_ring_reduce", "tp_ring_bytes", "tp_allreduce_bytes", "tp_moe_combine_bytes",
-    "tp_plan_mxfp8_bytes", "tp_pack_weights_mxfp8", "tp_rowlinear_reconcile_mxfp8",
+    "tp_ring_rank_workspace_bytes", "tp_ring_allreduce_ranks",
+    "tp_plan_mxfp8_bytes", "tp_pack_weights_mxfp8", "tp_plan_mxfp8_workspace_bytes",
+    "tp_rowlinear_reconcile_mxfp8", "tp_plan_nvfp4_bytes", "tp_pack_weights_nvfp4",
+    "tp_plan_nvfp4_workspace_bytes", "tp_rowlinear_reconcile_nvfp4",
     "tp_plan_destroy", "tp_status_string", "tp_last_cuda_error", "tp_device_error_flags",
 )
 
@@ -73,13 +76,29 @@ def _load() -> ctypes.CDLL:
     L.tp_plan_mxfp8_bytes.restype = ctypes.c_int
     L.tp_pack_weights_mxfp8.argtypes = [vp, vp, vp, vp, vp]
     L.tp_pack_weights_mxfp8.restype = ctypes.c_int
-    L.tp_rowlinear_reconcile_mxfp8.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp]
+    L.tp_rowlinear_reconcile_mxfp8.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, vp]
+    L.tp_plan_mxfp8_workspace_bytes.argtypes = [vp, i64]
+    L.tp_plan_mxfp8_workspace_bytes.restype = sz
+    L.tp_plan_nvfp4_bytes.argtypes = [vp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.tp_plan_nvfp4_bytes.restype = ctypes.c_int
+    L.tp_pack_weights_nvfp4.argtypes = [vp, vp, vp, vp, vp]
+    L.tp_pack_weights_nvfp4.restype = ctypes.c_int
+    L.tp_plan_nvfp4_workspace_bytes.argtypes = [vp, i64]
+    L.tp_plan_nvfp4_workspace_bytes.restype = sz
+    L.tp_rowlinear_reconcile_nvfp4.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, vp]
+    L.tp_rowlinear_reconcile_nvfp4.restype = ctypes.c_int
     L.tp_rowlinear_reconcile_mxfp8.restype = ctypes.c_int
     L.tp_allreduce_bytes.argtypes = [ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int, i64]
     L.tp_allreduce_bytes.restype = ctypes.c_uint64
     L.tp_moe_combine_bytes.argtypes = [ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int, i64,
                                        ctypes.c_int]
     L.tp_moe_combine_bytes.restype = ctypes.c_uint64
+    L.tp_ring_rank_workspace_bytes.argtypes = [vp, i64]
+    L.tp_ring_rank_workspace_bytes.restype = sz
+    vpp = ctypes.POINTER(ctypes.c_void_p)
+    L.tp_ring_allreduce_ranks.argtypes = [vp, vpp, vp, vpp, vpp, ctypes.c_int, ctypes.c_int, i64,
+                                          ctypes.c_uint64, vp]
+    L.tp_ring_allreduce_ranks.restype = ctypes.c_int
     L.tp_plan_destroy.argtypes = [vp]
     L.tp_plan_destroy.restype = None
     L.tp_status_string.argtypes = [ctypes.c_int]
@@ -162,8 +181,33 @@ def tp_pack_weights_mxfp8(plan, w_hk: int, w_q: int, w_scales: int, stream: int)
 
 
 def tp_rowlinear_reconcile_mxfp8(plan, x: int, w_q: int, w_scales: int, residual: int, out: int,
-                                 tokens: int, stream: int) -> int:
-    return LIB.tp_rowlinear_reconcile_mxfp8(plan, x, w_q, w_scales, residual, out, tokens, stream)
+                                 tokens: int, workspace: int, stream: int) -> int:
+    return LIB.tp_rowlinear_reconcile_mxfp8(plan, x, w_q, w_scales, residual, out, tokens, workspace,
+                                            stream)
+
+
+def tp_plan_mxfp8_workspace_bytes(plan, tokens: int) -> int:
+    return LIB.tp_plan_mxfp8_workspace_bytes(plan, tokens)
+
+
+def tp_plan_nvfp4_bytes(plan):
+    q, sc = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    st = LIB.tp_plan_nvfp4_bytes(plan, ctypes.byref(q), ctypes.byref(sc))
+    return st, q.value, sc.value
+
+
+def tp_pack_weights_nvfp4(plan, w_hk: int, w_q: int, w_scales: int, stream: int) -> int:
+    return LIB.tp_pack_weights_nvfp4(plan, w_hk, w_q, w_scales, stream)
+
+
+def tp_plan_nvfp4_workspace_bytes(plan, tokens: int) -> int:
+    return LIB.tp_plan_nvfp4_workspace_bytes(plan, tokens)
+
+
+def tp_rowlinear_reconcile_nvfp4(plan, x: int, w_q: int, w_scales: int, residual: int, out: int,
+                                 tokens: int, workspace: int, stream: int) -> int:
+    return LIB.tp_rowlinear_reconcile_nvfp4(plan, x, w_q, w_scales, residual, out, tokens, workspace,
+                                            stream)
 
 
 TP_ALLREDUCE_RING, TP_ALLREDUCE_NAIVE, TP_ALLREDUCE_SWITCH = 0, 1, 2
@@ -178,6 +222,22 @@ def tp_moe_combine_bytes(scheme: int, n_ranks: int, tokens: int, hidden: int, el
                          top_k: int, local_accumulate: int = 1) -> int:
     return int(LIB.tp_moe_combine_bytes(scheme, n_ranks, tokens, hidden, elem_bytes, top_k,
                                         local_accumulate))
+
+
+def tp_ring_rank_workspace_bytes(plan, tokens: int) -> int:
+    return LIB.tp_ring_rank_workspace_bytes(plan, tokens)
+
+
+def tp_ring_allreduce_ranks(plan, partials, residual: int, outs, workspaces, first_rank: int,
+                            launch_ranks: int, tokens: int, wait_limit_ns: int, stream: int) -> int:
+    """partials, outs, workspaces: sequences of N device addresses (or None)."""
+    def arr(ptrs):
+        if ptrs is None:
+            return None
+        a = (ctypes.c_void_p * len(ptrs))(*[ctypes.c_void_p(int(v) if v else None) for v in ptrs])
+        return ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))
+    return LIB.tp_ring_allreduce_ranks(plan, arr(partials), residual, arr(outs), arr(workspaces),
+                                       first_rank, launch_ranks, tokens, wait_limit_ns, stream)
 
 
 def tp_ring_bytes(n_ranks: int, tokens: int, hidden: int, elem_bytes: int, points: int) -> int:

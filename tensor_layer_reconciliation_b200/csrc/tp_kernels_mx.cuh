@@ -1,14 +1,27 @@
-// MXFP8 weight shards: quantisation (S0) and the decode reconciliation over
-// them (S1-S4 in one kernel).
+// Quantised weight shards: the element and scale conversions and the
+// quantisation kernels (S0) of the two formats; the reconciliation over the
+// shards runs on the tensor cores (tp_kernels_tc.cuh, quantised forms).
 //
-// Format (the NVL72 hosting post's MXFP8 weights, laid out per the OCP
+// MXFP8 (the NVL72 hosting post's MXFP8 weights, laid out per the OCP
 // Microscaling v1.0 specification): each run of 32 consecutive weights
 // along K inside one rank's slice shares an E8M0 scale X = 2^s, stored as
 // the byte s + 127, with s = floor(log2 max|w|) - 8 clamped to [-127, 127]
 // (-127 for an all-zero run); each weight is the FP8 E4M3 code nearest to
 // w / X, ties to even, saturating at 448.
-//   q      [N][H][K/N] E4M3 codes      (K/N a multiple of 32)
-//   scales [N][H][K/N/32] E8M0 bytes
+//   q      [N][H][K/N] E4M3 codes                     (K/N a multiple of 64)
+//   scales [N][K/N/64][H][2] E8M0 bytes: for each 64-column block of a rank
+//          slice, the scales of its two 32-weight runs, row after row (the
+//          scales a 128-row tile needs for one block are 256 contiguous bytes)
+//
+// NVFP4 (the TP=4-vs-TP=8 post's NVFP4 weights, in NVIDIA's published
+// layout): E2M1 elements, one E4M3 block scale per 16 weights along K inside a
+// rank slice, and a second-level scale 2^g for the whole tensor, g the
+// smallest integer with max|W| / 2^g <= 6 * 448 (0 for an all-zero tensor):
+//   b = E4M3 nearest to max|block| / (6 * 2^g); q = E2M1 nearest to
+//   w / (b * 2^g), ties to even, saturating at 6 (zeros where b is 0).
+//   q      [N][H][K/N/2] bytes, two codes each, the earlier k in bits 0-3
+//   scales [N][K/N/64][H][4] E4M3 bytes (the four block scales of each row
+//          for one 64-column block), then 16 bytes: g (int32), max|W| bits
 #pragma once
 
 #include "tp_common.cuh"
@@ -16,8 +29,7 @@
 namespace tpr {
 
 constexpr int kMxBlock = 32;        // weights per shared scale
-constexpr int kMxMaxTokens = 4;     // decode token counts the fused kernel takes (MT = tokens)
-constexpr int kMxWarps = 4;         // output rows in flight per CTA (one per warp)
+constexpr int kMxPair = 64;         // columns whose two scales are stored together
 
 // Two f32 values -> two E4M3 codes, nearest even, saturating at +-448; the
 // code of `lo` in bits 0-7 of the result.
@@ -31,6 +43,13 @@ __device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
 __device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint16_t v) {
     uint32_t d;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(v));
+    return d;
+}
+
+// Two f32 values -> bf16x2, each rounded to nearest even; `lo` in bits 0-15.
+__device__ __forceinline__ uint32_t bf16x2_from_f32(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
 }
 
@@ -92,7 +111,8 @@ __global__ void __launch_bounds__(256)
         }
         int s = amax == 0 ? -127 : bf16_floor_log2(amax) - 8;
         s = max(-127, min(127, s));
-        scales[row * nb + b] = static_cast<uint8_t>(s + 127);
+        // [N][Ks/64][H][2]: run b is half b & 1 of 64-column block b >> 1
+        scales[((r * (nb >> 1) + (b >> 1)) * hidden + h) * 2 + (b & 1)] = static_cast<uint8_t>(s + 127);
         // w / 2^s = w * 2^-s: a power of two, exact unless it drops below the
         // f32 range, where the E4M3 code is a signed zero either way.
         const float inv = pow2_f32(-s);
@@ -110,169 +130,87 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// ---------------------------------------------------------------- S1-S4 --
-// One warp per output row h (grid-stride), all N ranks in turn. Lane i
-// takes the 32 consecutive codes of one scale block out of every 1024 (two
-// 16-byte loads: a warp load is 1024 contiguous bytes), two such chunks in
-// flight at a time. The codes become exact f32 values (E4M3 -> f16x2 ->
-// f32), the bf16 activations f32 pairs, and the 32 products of a chunk are
-// summed with packed f32x2 fused multiply-adds (two interleaved chains), the
-// chunk's sum scaled by 2^s into the lane's accumulator; lanes meet by
-// shuffles. The N partials of the row then fold in ring order from the
-// chunk's owner and meet the residual: nothing is staged. Codes of the first
-// chunks are loaded before griddepcontrol.wait. The summation order differs
-// from the oracle's k-ascending chain, so a partial can round to the other
-// bf16 neighbour where its exact value lies next to a rounding boundary.
-constexpr int kMxLaneChunk = kMxBlock;                 // codes per lane per step
-constexpr int kMxWarpStep = 32 * kMxLaneChunk;         // 1024 codes per warp step
+// ----------------------------------------------------------- S0, NVFP4 --
 
-struct MxParams {
-    int n_ranks;
-    int hidden;
-    int hc;          // H / N
-    int tokens;      // = MT, 1 .. kMxMaxTokens
-    int64_t k;       // K
-    int64_t ks;      // K / N
-    const uint16_t* x;       // [M][K]
-    const uint8_t* q;        // [N][H][Ks]
-    const uint8_t* scales;   // [N][H][Ks/32]
-    const uint16_t* residual;  // [M][H]
-    uint16_t* out;             // [M][H]
-};
-
-// d (f32x2) += a (f32x2) * b (f32x2), each lane of the pair rounded once.
-__device__ __forceinline__ void fma_f32x2(uint64_t& d, uint64_t a, uint64_t b) {
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
-}
-__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
-    return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+// Two f32 values -> two E2M1 codes, nearest even, saturating at +-6; the
+// code of `lo` in bits 0-3 of the result.
+__device__ __forceinline__ uint32_t e2m1x2_from_f32(float lo, float hi) {
+    uint32_t d;
+    asm("{\n\t.reg .b8 c;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c, %1, %2;\n\t"
+        "cvt.u32.u8 %0, c;\n\t}"
+        : "=r"(d)
+        : "f"(hi), "f"(lo));
+    return d;
 }
 
-// Sum of the 32 products of one chunk: codes in q0, q1 (32 bytes), the
-// activations' 32 bf16 at xp (64 bytes, 16-byte aligned).
-__device__ __forceinline__ float mx_chunk_dot(const uint4& q0, const uint4& q1, const uint16_t* xp) {
-    const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    const uint4* x4 = reinterpret_cast<const uint4*>(xp);
-    uint64_t s0 = 0, s1 = 0;   // two chains of f32x2 sums
+// The largest magnitude of the Linear weight (as a bf16 pattern without its
+// sign, which orders like the value) into *amax_bits (zero on entry).
+__global__ void __launch_bounds__(256)
+    nv_amax_kernel(const uint16_t* __restrict__ w, int64_t n_vec8, uint32_t* amax_bits) {
+    uint32_t m = 0;
+    for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n_vec8;
+         v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint4 q = ld_global_nc_v4(w + 8 * v);
+        const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint4 xv = __ldg(x4 + j);              // 8 activations: codes 8j .. 8j+7
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const uint32_t c = qw[2 * j + i];            // 4 codes
-            const uint32_t a = f16x2_from_e4m3x2(static_cast<uint16_t>(c & 0xFFFF));
-            const uint32_t b = f16x2_from_e4m3x2(static_cast<uint16_t>(c >> 16));
-            const uint64_t w01 = pack_f32x2(f16_lo_to_f32(a), f16_hi_to_f32(a));
-            const uint64_t w23 = pack_f32x2(f16_lo_to_f32(b), f16_hi_to_f32(b));
-            const uint32_t x01 = xw[2 * i], x23 = xw[2 * i + 1];
-            fma_f32x2(s0, pack_f32x2(bf16_lo(x01), bf16_hi(x01)), w01);
-            fma_f32x2(s1, pack_f32x2(bf16_lo(x23), bf16_hi(x23)), w23);
-        }
+        for (int i = 0; i < 4; ++i) m = max(m, max(wd[i] & 0x7FFFu, (wd[i] >> 16) & 0x7FFFu));
     }
-    const float a0 = __uint_as_float(static_cast<uint32_t>(s0));
-    const float a1 = __uint_as_float(static_cast<uint32_t>(s0 >> 32));
-    const float b0 = __uint_as_float(static_cast<uint32_t>(s1));
-    const float b1 = __uint_as_float(static_cast<uint32_t>(s1 >> 32));
-    return (a0 + a1) + (b0 + b1);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax_bits, m);
 }
 
-// One token: at most 56 registers, so 9 CTAs (36 warps) fit on an SM and a
-// 5120-row call runs in one wave on 148 SMs.
-template <int MT>
-__global__ void __launch_bounds__(kMxWarps * 32, MT == 1 ? 9 : 4)
-    mx_reconcile_kernel(const MxParams p) {
-    pdl_launch_dependents();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ks = static_cast<int>(p.ks);
-    const int nb = ks / kMxBlock;
-    bool waited = false;
-    for (int h = blockIdx.x * kMxWarps + warp; h < p.hidden; h += gridDim.x * kMxWarps) {
-        float part[kMaxRanks][MT];
-#pragma unroll
-        for (int r = 0; r < kMaxRanks; ++r)
-#pragma unroll
-            for (int m = 0; m < MT; ++m) part[r][m] = 0.0f;
-#pragma unroll 1
-        for (int r = 0; r < p.n_ranks; ++r) {
-            const int64_t row = static_cast<int64_t>(r) * p.hidden + h;
-            const uint8_t* qrow = p.q + row * ks;
-            const uint8_t* srow = p.scales + row * nb;
-            const uint16_t* xr = p.x + static_cast<int64_t>(r) * ks;
-            float acc[MT];
-#pragma unroll
-            for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
-            for (int k0 = lane * kMxLaneChunk; k0 < ks; k0 += 2 * kMxWarpStep) {
-                const int k1 = k0 + kMxWarpStep;
-                const bool has1 = k1 < ks;
-                const uint4* qa = reinterpret_cast<const uint4*>(qrow + k0);
-                const uint4 qa0 = ld_global_nc_v4(qa), qa1 = ld_global_nc_v4(qa + 1);
-                const uint32_t sa = srow[k0 / kMxBlock];
-                uint4 qb0 = make_uint4(0, 0, 0, 0), qb1 = qb0;
-                uint32_t sbb = 0;
-                if (has1) {
-                    const uint4* qb = reinterpret_cast<const uint4*>(qrow + k1);
-                    qb0 = ld_global_nc_v4(qb);
-                    qb1 = ld_global_nc_v4(qb + 1);
-                    sbb = srow[k1 / kMxBlock];
-                }
-                if (!waited) {
-                    pdl_wait();   // activations and residual follow the stream's order
-                    waited = true;
-                }
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    const uint16_t* xm = xr + static_cast<int64_t>(m) * p.k;
-                    acc[m] = fmaf(mx_chunk_dot(qa0, qa1, xm + k0), e8m0_to_f32(sa), acc[m]);
-                    if (has1) acc[m] = fmaf(mx_chunk_dot(qb0, qb1, xm + k1), e8m0_to_f32(sbb), acc[m]);
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
-                    acc[m] += __shfl_xor_sync(0xFFFFFFFFu, acc[m], off);
-            }
-#pragma unroll
-            for (int rr = 0; rr < kMaxRanks; ++rr)
-                if (rr == r)
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) part[rr][m] = acc[m];
-        }
-        if (!waited) {
-            pdl_wait();
-            waited = true;
-        }
-        // S2-S4: lane m folds token m's partials in ring order, adds the residual.
-        if (lane < MT) {
-            const int c = h / p.hc;
-            float pm[kMaxRanks];
-#pragma unroll
-            for (int rr = 0; rr < kMaxRanks; ++rr) {
-                pm[rr] = part[rr][0];
-#pragma unroll
-                for (int m = 1; m < MT; ++m)
-                    if (lane == m) pm[rr] = part[rr][m];
-            }
-            uint16_t s = 0;
-#pragma unroll
-            for (int i = 0; i < kMaxRanks; ++i) {
-                if (i < p.n_ranks) {
-                    int rr = c + i;
-                    if (rr >= p.n_ranks) rr -= p.n_ranks;
-                    float pv = pm[0];
-#pragma unroll
-                    for (int j = 1; j < kMaxRanks; ++j)
-                        if (j == rr) pv = pm[j];
-                    const uint16_t pb = f32_to_bf16_rne(pv);
-                    s = i == 0 ? pb : bf16_add(s, pb);
-                }
-            }
-            const size_t o = static_cast<size_t>(lane) * p.hidden + h;
-            p.out[o] = bf16_add(p.residual[o], s);
-        }
+// One thread per 16-weight block: the block scale from the block maximum,
+// then each weight divided by it (after the exact scaling by 2^-g) and
+// rounded. The quotients are rounded to fp32 first; an fp32 rounding cannot
+// carry a quotient of these few-bit operands onto or across an E4M3 or E2M1
+// rounding boundary, so the codes are those of the exact quotients.
+__global__ void __launch_bounds__(256)
+    pack_weights_nv_kernel(const uint16_t* __restrict__ w, uint8_t* __restrict__ q,
+                           uint8_t* __restrict__ scales, int* __restrict__ gexp,
+                           const uint32_t* __restrict__ amax_bits, int n_ranks, int hidden, int64_t k,
+                           int64_t ks) {
+    const uint32_t amax_b = *amax_bits;
+    // g: the smallest integer with amax <= 2688 * 2^g
+    int g = 0;
+    if (amax_b != 0) {
+        const int e = bf16_floor_log2(amax_b);                       // 2^e <= amax < 2^(e+1)
+        const float amax = bf16_bits_to_f32(amax_b);
+        g = e - 11;
+        if (amax > ldexpf(2688.0f, g)) g += 1;
     }
-    if (!waited) pdl_wait();
+    if (blockIdx.x == 0 && threadIdx.x == 0) *gexp = g;
+    const int64_t nb = ks / 16, nkb = ks / 64;
+    const int64_t total = static_cast<int64_t>(n_ranks) * hidden * nb;
+    for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
+         t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t b = t % nb;
+        const int64_t row = t / nb;              // r * H + h
+        const int64_t h = row % hidden;
+        const int64_t r = row / hidden;
+        const uint4* src = reinterpret_cast<const uint4*>(w + h * k + r * ks + b * 16);
+        const uint4 v0 = src[0], v1 = src[1];
+        const uint32_t wd[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint32_t bmax = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bmax = max(bmax, max(wd[i] & 0x7FFFu, (wd[i] >> 16) & 0x7FFFu));
+        // block scale: E4M3 nearest to bmax / (6 * 2^g) (at most 448 by the choice of g)
+        const float qs = __fdiv_rn(ldexpf(bf16_bits_to_f32(bmax), -g), 6.0f);
+        const uint32_t bs = e4m3x2_from_f32(qs, 0.0f) & 0xFFu;
+        scales[((r * nkb + (b >> 2)) * hidden + h) * 4 + (b & 3)] = static_cast<uint8_t>(bs);
+        const float bval = f16_lo_to_f32(f16x2_from_e4m3x2(static_cast<uint16_t>(bs)));
+        uint32_t out[2] = {0u, 0u};
+        if (bval != 0.0f) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {   // word i: weights 2i, 2i+1 -> one byte of codes
+                const float lo = __fdiv_rn(ldexpf(bf16_lo(wd[i]), -g), bval);
+                const float hi = __fdiv_rn(ldexpf(bf16_hi(wd[i]), -g), bval);
+                out[i >> 2] |= e2m1x2_from_f32(lo, hi) << (8 * (i & 3));
+            }
+        }
+        *reinterpret_cast<uint2*>(q + row * (ks / 2) + b * 8) = make_uint2(out[0], out[1]);
+    }
 }
 
 }  // namespace tpr

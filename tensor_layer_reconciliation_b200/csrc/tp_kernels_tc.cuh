@@ -33,19 +33,35 @@
 // ring kernel adds the parts in split order before the one rounding to bf16.
 // Units run token tile fastest, so CTAs working at the same time share each
 // weight tile through L2 (a tile of weights serves every token tile of a call).
-// Folding (S2-S4): for one or two tokens the CTA that stores the last of
-// the N * SPLITS parts of an (H tile, token tile) -- found with a per-tile
-// counter in the workspace -- folds that tile itself, each epilogue thread
-// one row h, so a call is one kernel and the next call's kernel waits on one
-// grid instead of two. For more tokens the fold stays a kernel of its own:
-// there the CTA that completes a tile would read N * SPLITS * 128 * BN
-// values behind its next accumulator (measured slower from 32 tokens up),
-// while a separate kernel spreads that work over the whole GPU.
+// Folding (S2-S4) inside this kernel, two ways:
+//  * cluster fold (no k-split): the N CTAs of a thread-block cluster are the
+//    N ranks of one (H tile, token tile). Each rounds its accumulator to a
+//    bf16 partial tile in its own shared memory; after an mbarrier handshake
+//    across the cluster each CTA folds BN/N of the tile's tokens, reading the
+//    N partials of every output through the cluster's shared window in ring
+//    order, and adds the residual. The partials never leave the chip and the
+//    fold work is spread over all N CTAs (CTAs of a cluster run at the same
+//    time, so the waits between them always end).
+//  * counter fold (one or two tokens with a k-split): the CTA that stores the
+//    last of the N * SPLITS parts of an (H tile, token tile) -- found with a
+//    per-tile counter in the workspace -- folds that tile, each epilogue
+//    thread one row h.
+// Otherwise (more tokens with a k-split) a ring kernel folds the stored parts.
+// Quantised weights (FMT = MXFP8 or NVFP4): the producer stages code tiles
+// (128 rows x 64 codes) and their scales instead of bf16 weight tiles; four
+// more warps (6-9) turn each code tile into the bf16 tile the MMA reads
+// (MXFP8: E4M3 * 2^s; NVFP4: E2M1 * E4M3 block scale * 2^g; exact in bf16
+// for the shards the formats' definitions allow), written in the same
+// 128-byte-swizzled K-major layout TMA gives the bf16 path, into one of two
+// converted slots; the MMA waits for its slot and frees it (and the stage,
+// whose activation tile it reads) when it is done. Everything after the MMA
+// -- the three epilogues -- is the same.
 // Accumulation order inside the tensor core is the hardware's; the partial
 // is the fp32 sum rounded once to bf16, like the oracle's, but only equal to
 // it where the two fp32 sums round to the same bf16 value.
 #pragma once
 
+#include "tp_kernels_mx.cuh"
 #include "tp_tcgen05.cuh"
 
 namespace tpr {
@@ -54,7 +70,30 @@ constexpr int kTcRows = 128;               // MMA M: weight rows per tile
 constexpr int kTcKBlock = 64;              // bf16 columns per staged block
 constexpr int kTcMaxStages = 8;
 constexpr int kTcThreads = 192;            // producer, MMA and 4 epilogue warps
+constexpr int kTcMxThreads = 320;          // quantised weights: + 4 converter warps
 constexpr uint32_t kTcATile = kTcRows * kTcKBlock * 2;  // 16 KB
+constexpr uint32_t kMxCodeTile = kTcRows * kTcKBlock;   // 8 KB of E4M3 codes
+constexpr uint32_t kMxScaleTile = kTcRows * 2;          // the 2 E8M0 scales of each row
+constexpr uint32_t kNvCodeTile = kTcRows * kTcKBlock / 2;  // 4 KB: two E2M1 codes a byte
+constexpr uint32_t kNvScaleTile = kTcRows * 4;             // the 4 E4M3 block scales of each row
+
+// Weight formats of the tensor-core kernel (a template parameter).
+constexpr int kFmtBf16 = 0;    // packed bf16 shards, staged by TMA as the MMA's A tiles
+constexpr int kFmtMxfp8 = 1;   // E4M3 codes + E8M0 scales per 32, widened on chip
+constexpr int kFmtNvfp4 = 2;   // E2M1 codes + E4M3 scales per 16 (x 2^g), widened on chip
+
+__host__ __device__ constexpr uint32_t fmt_code_tile(int fmt) {
+    return fmt == kFmtMxfp8 ? kMxCodeTile : fmt == kFmtNvfp4 ? kNvCodeTile : kTcATile;
+}
+__host__ __device__ constexpr uint32_t fmt_scale_tile(int fmt) {
+    return fmt == kFmtMxfp8 ? kMxScaleTile : fmt == kFmtNvfp4 ? kNvScaleTile : 0;
+}
+
+// What the epilogue does with each accumulator (a template parameter, so each
+// form compiles only its own epilogue):
+constexpr int kTcStore = 0;         // store the partials (or fp32 k-parts) for a ring kernel
+constexpr int kTcCounterFold = 1;   // store k-parts; the CTA that completes a tile folds it
+constexpr int kTcClusterFold = 2;   // fold on chip across the cluster's N CTAs
 
 struct TcParams {
     int n_ranks;   // N
@@ -68,20 +107,148 @@ struct TcParams {
     int stages;    // 2 .. kTcMaxStages
     uint16_t* partials;     // [N][M][H] bf16 (splits == 1)
     float* partials_f32;    // [splits][N][M][H] fp32 sums of each k part (splits > 1)
-    // In-kernel fold (S2-S4), few tokens only; fold == 0 leaves it to the ring kernel.
-    int fold;
+
     int hc;                       // H / N, the chunk each rank owns in the ring
     unsigned int* counters;       // [h_tiles][m_tiles] parts stored so far; zero between calls
     const uint16_t* residual;     // [M][H]
     uint16_t* out;                // [M][H]
+    const int* nv_gexp;           // NVFP4: the second-level exponent g
 };
 
-template <int BN>
-__global__ void __launch_bounds__(kTcThreads, 1)
+// Cluster fold of one (H tile, token tile): this CTA (rank `crank` of a
+// cluster of N = csize) folds tokens [crank * T, (crank + 1) * T) of the tile,
+// T = ceil(BN / N), all 128 rows, 8 columns (16 bytes) per thread step: the
+// N partial vectors are read from the CTAs' part_buf tiles ([BN][128] bf16)
+// in ring order from the chunk's owner, all loads before the first add, then
+// the residual is added and the output stored. et = epilogue thread, 0..127.
+__device__ __forceinline__ void cluster_fold_tile(const TcParams& p, const uint16_t* part_buf,
+                                                  uint32_t crank, int csize, int ht, int m0,
+                                                  int bn, int et) {
+    const int n = csize;
+    const int t_per = (bn + n - 1) / n;
+#pragma unroll 1
+    for (int v = et; v < t_per * (kTcRows / 8); v += 128) {
+        const int tt = static_cast<int>(crank) * t_per + (v >> 4);   // token in the tile
+        const int hv = (v & 15) * 8;                                 // row offset in the tile
+        const int m = m0 + tt;
+        const int h = ht * kTcRows + hv;
+        if (tt >= bn || m >= p.tokens || h >= p.hidden) continue;
+        const int c = h / p.hc;
+        const uint16_t* mine = part_buf + tt * kTcRows + hv;
+        uint4 pv[kMaxRanks];
+#pragma unroll
+        for (int i = 0; i < kMaxRanks; ++i) {
+            if (i < n) {
+                int rr = c + i;   // ring order: the chunk's owner first
+                if (rr >= n) rr -= n;
+                pv[i] = ld_dsmem_v4(mapa_shared(mine, static_cast<uint32_t>(rr)));
+            }
+        }
+        const size_t o = static_cast<size_t>(m) * p.hidden + h;
+        const uint4 rv = ld_global_nc_v4(p.residual + o);
+        uint4 sum = pv[0];
+#pragma unroll
+        for (int i = 1; i < kMaxRanks; ++i) {
+            if (i < n) {
+                sum.x = bf16x2_add(sum.x, pv[i].x);
+                sum.y = bf16x2_add(sum.y, pv[i].y);
+                sum.z = bf16x2_add(sum.z, pv[i].z);
+                sum.w = bf16x2_add(sum.w, pv[i].w);
+            }
+        }
+        uint4 out;
+        out.x = bf16x2_add(rv.x, sum.x);
+        out.y = bf16x2_add(rv.y, sum.y);
+        out.z = bf16x2_add(rv.z, sum.z);
+        out.w = bf16x2_add(rv.w, sum.w);
+        st_global_v4(p.out + o, out);
+    }
+}
+
+// Converts one row of a staged E4M3 code tile (64 codes, row-major, 64
+// bytes) with its two E8M0 scales into the row of a bf16 A tile in the
+// 128-byte-swizzled K-major layout (16-byte chunk q of row t at chunk
+// q ^ (t & 7)): each value is code * 2^s, computed in fp32 (exact) and
+// rounded to bf16 (exact for values bf16 holds). The row's four 16-code
+// chunks are visited starting at a row-dependent one, so the eight rows a
+// quarter-warp reads at once fall in different shared-memory banks.
+__device__ __forceinline__ void mx_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
+                                               uint8_t* a_row, int t) {
+    const float sc[2] = {e8m0_to_f32(scale_row[0]), e8m0_to_f32(scale_row[1])};
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        const int c = (cc + (t >> 1)) & 3;                 // codes 16c .. 16c+15
+        const uint4 q = *reinterpret_cast<const uint4*>(code_row + c * 16);
+        const float scale = sc[c >> 1];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t h01 = f16x2_from_e4m3x2(static_cast<uint16_t>(w[i] & 0xFFFF));
+            const uint32_t h23 = f16x2_from_e4m3x2(static_cast<uint16_t>(w[i] >> 16));
+            o[2 * i] = bf16x2_from_f32(f16_lo_to_f32(h01) * scale, f16_hi_to_f32(h01) * scale);
+            o[2 * i + 1] = bf16x2_from_f32(f16_lo_to_f32(h23) * scale, f16_hi_to_f32(h23) * scale);
+        }
+        const int q0 = (2 * c) ^ (t & 7), q1 = (2 * c + 1) ^ (t & 7);
+        *reinterpret_cast<uint4*>(a_row + q0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(a_row + q1 * 16) = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+// Two E2M1 codes (bits 0-3 and 4-7 of b) -> two exact f16 values as f16x2.
+__device__ __forceinline__ uint32_t f16x2_from_e2m1x2(uint32_t b) {
+    uint32_t d;
+    asm("{\n\t.reg .b8 c;\n\t"
+        "cvt.u8.u32 c, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+        : "=r"(d)
+        : "r"(b));
+    return d;
+}
+
+// NVFP4 row: 32 bytes of codes (64 E2M1 values, the earlier k in the low
+// nibble), the row's four E4M3 block scales (one per 16 values) and the
+// second-level factor 2^g -> the row of a bf16 A tile as in mx_convert_row.
+// The row's two 16-byte halves are read starting at a row-dependent one.
+__device__ __forceinline__ void nv_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
+                                               float two_g, uint8_t* a_row, int t) {
+    const uint32_t sw = *reinterpret_cast<const uint32_t*>(scale_row);
+    float sc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        sc[i] = f16_lo_to_f32(f16x2_from_e4m3x2(static_cast<uint16_t>((sw >> (8 * i)) & 0xFF))) * two_g;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int c = (hh + (t >> 2)) & 1;                 // codes 32c .. 32c+31
+        const uint4 q = *reinterpret_cast<const uint4*>(code_row + c * 16);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};        // 8 codes a word
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {                      // word i: codes 32c + 8i .. +7
+            const float scale = sc[2 * c + (i >> 1)];
+            uint32_t o[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t h2 = f16x2_from_e2m1x2((w[i] >> (8 * b)) & 0xFF);
+                o[b] = bf16x2_from_f32(f16_lo_to_f32(h2) * scale, f16_hi_to_f32(h2) * scale);
+            }
+            const int qc = (4 * c + i) ^ (t & 7);          // 16-byte chunk of 8 bf16 values
+            *reinterpret_cast<uint4*>(a_row + qc * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// Token tiles up to 64 run two CTAs per SM: at most 168 registers a thread
+// (96 with the converter warps).
+template <int BN, int MODE, int FMT>
+__global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, BN <= 64 ? 2 : 1)
     tc_partial_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                      const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
+                      const __grid_constant__ CUtensorMap tmap_x,
+                      const __grid_constant__ CUtensorMap tmap_s, const TcParams p) {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
     constexpr uint32_t kBTile = BN * kTcKBlock * 2;
+    constexpr bool MX = FMT != kFmtBf16;                        // converted on chip
+    constexpr uint32_t kWTile = fmt_code_tile(FMT);             // weight bytes staged per block
+    constexpr uint32_t kSTile = fmt_scale_tile(FMT);            // scale bytes staged per block
     constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
     constexpr uint32_t kIdesc = idesc_bf16_f32(kTcRows, BN);
 
@@ -89,24 +256,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int S = p.stages;
-    uint8_t* a_ring = smem;
-    uint8_t* b_ring = a_ring + static_cast<size_t>(S) * kTcATile;
-    uint64_t* full = reinterpret_cast<uint64_t*>(b_ring + static_cast<size_t>(S) * kBTile);
+    uint8_t* a_ring = smem;                                              // weight tiles (TMA)
+    uint8_t* b_ring = a_ring + static_cast<size_t>(S) * kWTile;         // activation tiles
+    uint8_t* a_cvt = b_ring + static_cast<size_t>(S) * kBTile;          // MX: 2 converted tiles
+    uint8_t* s_ring = a_cvt + (MX ? 2 * kTcATile : 0);                   // MX: scale tiles
+    uint64_t* full = reinterpret_cast<uint64_t*>(s_ring + static_cast<size_t>(S) * kSTile);
     uint64_t* empty = full + kTcMaxStages;
     uint64_t* acc_full = empty + kTcMaxStages;   // [2]
     uint64_t* acc_empty = acc_full + 2;          // [2]
     uint64_t* mma_done = acc_empty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* fold_ready = mma_done + 1;   // cluster fold: all N partial tiles written
+    uint64_t* fold_freed = fold_ready + 1; // cluster fold: all N CTAs done reading mine
+    uint64_t* cvt_full = fold_freed + 1;   // MX: [2] converted tile ready (4 warps)
+    uint64_t* cvt_empty = cvt_full + 2;    // MX: [2] converted tile read by the MMAs
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cvt_empty + 2);
+    // cluster fold: this CTA's bf16 partial tile, [BN tokens][128 rows]
+    uint16_t* part_buf = reinterpret_cast<uint16_t*>(
+        (reinterpret_cast<uintptr_t>(tmem_slot + 4) + 127) & ~static_cast<uintptr_t>(127));
     __shared__ int abort_flag;
     __shared__ int fold_mine;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nkb = (p.ks + kTcKBlock - 1) / kTcKBlock;
-    const int my_units = p.units > static_cast<int>(blockIdx.x)
-                             ? (p.units - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-                             : 0;
+    // Cluster fold: cluster c takes tiles c, c + clusters, ...; its CTA of rank
+    // r (in the cluster) computes rank r's partial of each.
+    constexpr bool kCluster = MODE == kTcClusterFold;
+    const int csize = kCluster ? p.n_ranks : 1;
+    const uint32_t crank = kCluster ? cluster_ctarank() : 0u;
+    const int cid = static_cast<int>(blockIdx.x) / csize;
+    const int n_clusters = static_cast<int>(gridDim.x) / csize;
+    const int tiles = p.h_tiles * p.m_tiles;
+    const int my_units =
+        kCluster ? (tiles > cid ? (tiles - 1 - cid) / n_clusters + 1 : 0)
+                       : (p.units > static_cast<int>(blockIdx.x)
+                              ? (p.units - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                              : 0);
     // unit index -> (rank, h tile, m tile, split); token tile fastest
     auto unit_of = [&](int lu, int& r, int& ht, int& mt, int& sp) {
+        if (kCluster) {
+            const int t = cid + lu * n_clusters;
+            mt = t % p.m_tiles;
+            ht = t / p.m_tiles;
+            r = static_cast<int>(crank);
+            sp = 0;
+            return;
+        }
         const int u = static_cast<int>(blockIdx.x) + lu * static_cast<int>(gridDim.x);
         mt = u % p.m_tiles;
         int t = u / p.m_tiles;
@@ -131,6 +325,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&acc_empty[b], 4);
         }
         mbar_init(mma_done, 1);
+        mbar_init(fold_ready, static_cast<uint32_t>(csize));
+        mbar_init(fold_freed, static_cast<uint32_t>(csize));
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&cvt_full[j], 4);
+            mbar_init(&cvt_empty[j], 1);
+        }
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -139,6 +339,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     tc_fence_before_sync();
     __syncthreads();
+    if (kCluster) cluster_sync_all();   // peers' barriers exist before any remote arrival
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
     pdl_launch_dependents();
@@ -148,7 +349,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tmap_w);
             tma_prefetch_desc(&tmap_x);
-            const uint32_t tx = kTcATile + kBTile;
+            if (MX) tma_prefetch_desc(&tmap_s);
+            const uint32_t tx = kWTile + kBTile + kSTile;
+            // The weights of one k-block (and, MX, their scales) into stage st.
+            auto load_w = [&](int st, int kb_, int ht_, int r_) {
+                tma_load_3d(a_ring + static_cast<size_t>(st) * kWTile, &tmap_w, &full[st],
+                            kb_ * kTcKBlock, ht_ * kTcRows, r_);
+                if (MX)   // MXFP8: 256 bytes from byte ht*256; NVFP4: 128 words from word ht*128
+                    tma_load_3d(s_ring + static_cast<size_t>(st) * kSTile, &tmap_s, &full[st],
+                                FMT == kFmtMxfp8 ? ht_ * kTcRows * 2 : ht_ * kTcRows, kb_, r_);
+            };
             // Walk (unit, k-block) in issue order.
             int lu = 0, kb = 0, kb_hi = 0, r = 0, ht = 0, mt = 0, sp = 0;
             auto enter_unit = [&]() {
@@ -168,8 +378,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int pre = 0;
             while (pre < S && lu < my_units) {
                 mbar_arrive_expect_tx(&full[pre], tx);
-                tma_load_3d(a_ring + static_cast<size_t>(pre) * kTcATile, &tmap_w, &full[pre],
-                            kb * kTcKBlock, ht * kTcRows, r);
+                load_w(pre, kb, ht, r);
                 pre_r[pre] = r;
                 pre_mt[pre] = mt;
                 pre_kb[pre] = kb;
@@ -190,8 +399,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
                 mbar_arrive_expect_tx(&full[s], tx);
-                tma_load_3d(a_ring + static_cast<size_t>(s) * kTcATile, &tmap_w, &full[s],
-                            kb * kTcKBlock, ht * kTcRows, r);
+                load_w(s, kb, ht, r);
                 tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, &full[s],
                             kb * kTcKBlock, r, mt * BN);
                 ++issued;
@@ -227,18 +435,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 bool ok = true;
                 for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
                     const int s = i % S;
-                    if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / S) & 1u)) {
+                    const int j = i & 1;   // MX: converted slot
+                    if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / S) & 1u) ||
+                        (MX && !mbar_wait_bounded(&cvt_full[j], static_cast<uint32_t>(i >> 1) & 1u))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint64_t ad = smem_desc_k128(a_ring + static_cast<size_t>(s) * kTcATile);
+                    const uint64_t ad = smem_desc_k128(MX ? a_cvt + static_cast<size_t>(j) * kTcATile
+                                                          : a_ring + static_cast<size_t>(s) * kTcATile);
                     const uint64_t bd = smem_desc_k128(b_ring + static_cast<size_t>(s) * kBTile);
 #pragma unroll
                     for (int kk = 0; kk < kTcKBlock / 16; ++kk)
                         umma_bf16(d, ad + 2ull * kk, bd + 2ull * kk, kIdesc,
                                   (kb != kb_lo) || (kk != 0));
                     umma_commit(&empty[s]);  // frees the stage when these MMAs finish
+                    if (MX) umma_commit(&cvt_empty[j]);   // and the converted slot
                 }
                 if (!ok) {
                     atomicExch(&abort_flag, 1);
@@ -251,6 +463,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             umma_commit(mma_done);
             if (!mbar_wait_bounded(mma_done, 0)) (void)mbar_wait_bounded(mma_done, 0);
         }
+    } else if (MX && warp >= 6) {
+        // ------------------------------------ converters (quantised weights) --
+        // Thread t converts row t of every staged code tile, in issue order.
+        const int t = static_cast<int>(threadIdx.x) - 192;
+        // NVFP4: the second-level factor 2^g, an exponent the packing stored
+        const float two_g = FMT == kFmtNvfp4 ? ldexpf(1.0f, *p.nv_gexp) : 1.0f;
+        int i = 0;
+        bool ok = true;
+        for (int lu = 0; lu < my_units && ok; ++lu) {
+            int r, ht, mt, sp, kb_lo, kb_hi;
+            unit_of(lu, r, ht, mt, sp);
+            split_range(sp, kb_lo, kb_hi);
+            for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
+                const int s = i % S, j = i & 1;
+                ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / S) & 1u) &&
+                     mbar_wait_bounded(&cvt_empty[j], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u);
+                if (!__all_sync(0xFFFFFFFFu, ok) ||
+                    *reinterpret_cast<volatile int*>(&abort_flag) != 0) {
+                    ok = false;
+                    atomicExch(&abort_flag, 1);
+                    break;
+                }
+                if (FMT == kFmtMxfp8)
+                    mx_convert_row(a_ring + static_cast<size_t>(s) * kWTile + t * kTcKBlock,
+                                   s_ring + static_cast<size_t>(s) * kSTile + t * 2,
+                                   a_cvt + static_cast<size_t>(j) * kTcATile + t * 128, t);
+                else
+                    nv_convert_row(a_ring + static_cast<size_t>(s) * kWTile + t * (kTcKBlock / 2),
+                                   s_ring + static_cast<size_t>(s) * kSTile + t * 4, two_g,
+                                   a_cvt + static_cast<size_t>(j) * kTcATile + t * 128, t);
+                // generic-proxy writes, read next by the tensor core (async proxy)
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cvt_full[j]);
+            }
+        }
     } else {
         // ---------------------------------------------------------- epilogue --
         const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -258,7 +506,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int lu = 0; lu < my_units; ++lu) {
             const int b = lu & 1;
             const uint32_t aph = static_cast<uint32_t>(lu >> 1) & 1u;
-            bool bad = !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&acc_full[b], aph));
+            bool ok = mbar_wait_bounded(&acc_full[b], aph);
+            // cluster fold: the peers have read the previous unit's partial tile
+            if (kCluster && lu > 0)
+                ok = mbar_wait_cluster_bounded(fold_freed, static_cast<uint32_t>(lu - 1) & 1u) && ok;
+            bool bad = !__all_sync(0xFFFFFFFFu, ok);
             if (bad) atomicExch(&abort_flag, 1);
             bad = bad || *reinterpret_cast<volatile int*>(&abort_flag) != 0;
             // The four epilogue warps leave together: one answer for all of them.
@@ -275,7 +527,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(b * BN + c0),
                                v);
-                if (h < p.hidden) {
+                if (kCluster) {
+                    // [token][row] in shared memory: lanes write 32 consecutive rows
+                    uint16_t* dst = part_buf + static_cast<size_t>(c0) * kTcRows + q * 32 + lane;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        dst[i * kTcRows] = f32_to_bf16_rne(__uint_as_float(v[i]));
+                } else if (h < p.hidden) {
                     if (p.splits == 1) {
                         uint16_t* dst = p.partials + static_cast<size_t>(r) * plane + h;
 #pragma unroll
@@ -299,7 +557,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[b]);
-            if (p.fold) {
+            if (kCluster) {
+                // Every CTA of the cluster has its partial tile in shared memory
+                // once each has arrived on everyone's fold_ready.
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                if (warp == 2 && lane == 0) {
+                    fence_acq_rel_cluster();
+                    for (int pr = 0; pr < csize; ++pr)
+                        mbar_arrive_cluster(mapa_shared(fold_ready, static_cast<uint32_t>(pr)));
+                }
+                if (!mbar_wait_cluster_bounded(fold_ready, static_cast<uint32_t>(lu) & 1u))
+                    atomicExch(&abort_flag, 1);
+                else
+                    cluster_fold_tile(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
+                // All reads of the peers' tiles are done: free them for the next unit.
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                if (warp == 2 && lane == 0) {
+                    fence_acq_rel_cluster();
+                    for (int pr = 0; pr < csize; ++pr)
+                        mbar_arrive_cluster(mapa_shared(fold_freed, static_cast<uint32_t>(pr)));
+                }
+            }
+            if (MODE == kTcCounterFold) {
                 // The CTA that stores the last of the N * SPLITS parts of this
                 // (H tile, token tile) folds the tile: ring order, residual add.
                 // Residual of this thread's row, loaded while the count goes round.
@@ -339,6 +618,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     tc_fence_before_sync();
     __syncthreads();
+    // Cluster fold: no CTA leaves while a peer may still read its shared
+    // memory or arrive on its barriers (every wait above is bounded, so every
+    // thread of the cluster gets here).
+    if (kCluster) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, kTmemCols);

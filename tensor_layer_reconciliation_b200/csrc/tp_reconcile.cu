@@ -14,6 +14,7 @@
 #include "tp_kernels_tc.cuh"
 #include "tp_kernels_tc2.cuh"
 #include "tp_kernels_mx.cuh"
+#include "tp_kernels_ring.cuh"
 #include "tp_reconcile.h"
 
 // Fixed scratch for tp_rowlinear_reconcile_noalloc: fold counters and the
@@ -166,20 +167,36 @@ tp_status encode_maps(const tp_plan* p, const ExactConfig& c, const void* x, con
     return TP_OK;
 }
 
+// Launch with programmatic dependent launch; cluster_x > 1 also groups the
+// CTAs in clusters of cluster_x (the grid is a multiple of it).
 template <typename Kern, typename... Args>
-cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                       Args... args) {
+cudaError_t launch_pdl_cluster(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                               int cluster_x, Args... args) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int na = 1;
+    if (cluster_x > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        na = 2;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+    return launch_pdl_cluster(kernel, grid, block, smem, stream, 1, args...);
 }
 
 tp_status launch_exact(const tp_plan* p, const void* x, const void* w, const void* residual,
@@ -221,6 +238,7 @@ tp_status launch_exact(const tp_plan* p, const void* x, const void* w, const voi
 
 struct TcConfig {
     int bn, stages, grid, units, h_tiles, m_tiles, splits;
+    bool cluster_fold;   // the N ranks of a tile on one cluster, folded on chip
     size_t smem;
 };
 
@@ -230,29 +248,47 @@ int tc_token_tile(int64_t tokens) {
     return tokens <= 32 ? 32 : tokens <= 64 ? 64 : tokens <= 128 ? 128 : 256;
 }
 
-TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split) {
+// allow_split: the call folds (S2-S4) in this library, so K may be split
+// across CTAs when there are fewer units than SMs; such calls without a split
+// and with a token tile of at most 128 fold on chip in clusters of N CTAs.
+TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt = tpr::kFmtBf16) {
     TcConfig c{};
     c.bn = tc_token_tile(tokens);
     c.h_tiles = static_cast<int>((p->hidden + tpr::kTcRows - 1) / tpr::kTcRows);
     c.m_tiles = static_cast<int>((tokens + c.bn - 1) / c.bn);
     const int base_units = p->n_ranks * c.h_tiles * c.m_tiles;
-    const size_t stage = tpr::kTcATile + static_cast<size_t>(c.bn) * tpr::kTcKBlock * 2;
-    const size_t fixed = (2 * tpr::kTcMaxStages + 5) * sizeof(uint64_t) + 16 + 1024;
     // Small token tiles stream weights: two CTAs per SM (about 100 KB each,
     // tensor memory 2 x 2*BN columns). Large tiles: one CTA per SM, deep ring.
     const bool two_per_sm = c.bn <= 64;
-    const size_t budget = std::min<size_t>(two_per_sm ? 110 * 1024 : 200 * 1024,
-                                           static_cast<size_t>(p->smem_optin));
-    c.stages = static_cast<int>(std::min<size_t>(tpr::kTcMaxStages, (budget - fixed) / stage));
-    c.smem = fixed + static_cast<size_t>(c.stages) * stage;
     const int slots = p->sm_count * (two_per_sm ? 2 : 1);
     // Fewer units than SMs: split K so every SM streams weights.
     const int nkb = static_cast<int>((p->ks + tpr::kTcKBlock - 1) / tpr::kTcKBlock);
     c.splits = 1;
     if (allow_split && base_units > 0 && base_units < p->sm_count)
         c.splits = std::max(1, std::min({slots / base_units, nkb, tpr::kMaxSplits}));
+    c.cluster_fold = allow_split && base_units > 0 && c.splits == 1 && c.bn <= 128;
+    // Quantised weights: a stage holds codes, scales and activations; two
+    // converted bf16 tiles sit beside the ring.
+    const bool quantised = fmt != tpr::kFmtBf16;
+    const size_t stage = tpr::fmt_code_tile(fmt) + tpr::fmt_scale_tile(fmt) +
+                         static_cast<size_t>(c.bn) * tpr::kTcKBlock * 2;
+    const size_t part_tile = c.cluster_fold ? static_cast<size_t>(c.bn) * tpr::kTcRows * 2 : 0;
+    const size_t fixed = (2 * tpr::kTcMaxStages + 11) * sizeof(uint64_t) + 16 + 128 + 1024 + part_tile +
+                         (quantised ? 2 * tpr::kTcATile : 0);
+    const size_t budget = std::min<size_t>(two_per_sm ? 110 * 1024 : 200 * 1024,
+                                           static_cast<size_t>(p->smem_optin));
+    c.stages = budget > fixed
+                   ? static_cast<int>(std::min<size_t>(tpr::kTcMaxStages, (budget - fixed) / stage))
+                   : 0;
+    c.smem = fixed + static_cast<size_t>(c.stages) * stage;
     c.units = base_units * c.splits;
-    c.grid = std::min(c.units, slots);
+    if (c.cluster_fold) {
+        // clusters of N CTAs, one per (H tile, token tile) at a time
+        const int tiles = c.h_tiles * c.m_tiles;
+        c.grid = p->n_ranks * std::max(1, std::min(tiles, slots / p->n_ranks));
+    } else {
+        c.grid = std::min(c.units, slots);
+    }
     return c;
 }
 
@@ -328,21 +364,140 @@ tp_status launch_tc2(const tp_plan* p, const void* x, const void* w, void* parti
     return e == cudaSuccess ? TP_OK : cuda_fail(e);
 }
 
-// fold: the kernel also runs S2-S4 (residual, out) for few tokens, counting
-// stored parts per H tile in `counters` (zero on entry, zero on return);
-// else a ring kernel must follow.
-tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partials, int64_t tokens,
-                    bool allow_split, bool fold, unsigned int* counters, const void* residual,
-                    void* out, cudaStream_t stream) {
-    const TcConfig c = tc_config(p, tokens, allow_split);
+// NVFP4 block-scale bytes (H*K/16); the second-level exponent g (int32)
+// follows them in the same buffer.
+size_t nv_scale_bytes(const tp_plan* p) {
+    return static_cast<size_t>(p->hidden) * static_cast<size_t>(p->k) / 16;
+}
+
+// Weights of a tensor-core call: packed bf16 shards, or MXFP8 codes with
+// their scales.
+struct TcWeights {
+    const void* w;        // [N][H][Ks] bf16; MXFP8 E4M3 codes; NVFP4 E2M1 code pairs
+    const void* scales;   // MXFP8 [N][Ks/64][H][2] E8M0; NVFP4 [N][Ks/64][H][4] E4M3 + g
+    int fmt;              // tpr::kFmt*
+};
+
+// MXFP8 codes [N][H][Ks] bytes, 128 rows x 64 codes per box (row-major in
+// shared memory), and their scales [N][Ks/64][H][2] bytes, the 256 bytes of a
+// 128-row tile per box (rows past H read as zero).
+tp_status encode_mx_maps(const tp_plan* p, const void* q, const void* scales, CUtensorMap* mq,
+                         CUtensorMap* ms) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc) return cuda_fail(g_encode_err);
+    const cuuint32_t estr[3] = {1, 1, 1};
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->ks), static_cast<cuuint64_t>(p->hidden),
+                                    static_cast<cuuint64_t>(p->n_ranks)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks),
+                                       static_cast<cuuint64_t>(p->hidden * p->ks)};
+        const cuuint32_t box[3] = {tpr::kTcKBlock, tpr::kTcRows, 1};
+        CUresult r = enc(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(q), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    }
+    {
+        const int64_t nkb = p->ks / tpr::kMxPair;
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(2 * p->hidden), static_cast<cuuint64_t>(nkb),
+                                    static_cast<cuuint64_t>(p->n_ranks)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(2 * p->hidden),
+                                       static_cast<cuuint64_t>(2 * p->hidden * nkb)};
+        const cuuint32_t box[3] = {tpr::kMxScaleTile, 1, 1};
+        CUresult r = enc(ms, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(scales), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    }
+    return TP_OK;
+}
+
+// NVFP4 code pairs [N][H][Ks/2] bytes, 128 rows x 32 bytes per box, and the
+// block scales [N][Ks/64][H][4] as 32-bit words, 128 words per box.
+tp_status encode_nv_maps(const tp_plan* p, const void* q, const void* scales, CUtensorMap* mq,
+                         CUtensorMap* ms) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc) return cuda_fail(g_encode_err);
+    const cuuint32_t estr[3] = {1, 1, 1};
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->ks / 2), static_cast<cuuint64_t>(p->hidden),
+                                    static_cast<cuuint64_t>(p->n_ranks)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks / 2),
+                                       static_cast<cuuint64_t>(p->hidden * p->ks / 2)};
+        const cuuint32_t box[3] = {tpr::kTcKBlock / 2, tpr::kTcRows, 1};
+        CUresult r = enc(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(q), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    }
+    {
+        const int64_t nkb = p->ks / tpr::kTcKBlock;
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->hidden), static_cast<cuuint64_t>(nkb),
+                                    static_cast<cuuint64_t>(p->n_ranks)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(4 * p->hidden),
+                                       static_cast<cuuint64_t>(4 * p->hidden * nkb)};
+        const cuuint32_t box[3] = {tpr::kTcRows, 1, 1};
+        CUresult r = enc(ms, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(scales), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    }
+    return TP_OK;
+}
+
+template <int BN, int MODE, int FMT>
+cudaError_t launch_tc_kernel(dim3 grid, size_t smem, cudaStream_t stream, int cluster_x,
+                             const CUtensorMap& mw, const CUtensorMap& mx, const CUtensorMap& ms,
+                             const tpr::TcParams& prm) {
+    return launch_pdl_cluster(tpr::tc_partial_kernel<BN, MODE, FMT>, grid,
+                              dim3(FMT != tpr::kFmtBf16 ? tpr::kTcMxThreads : tpr::kTcThreads), smem,
+                              stream, cluster_x, mw, mx, ms, prm);
+}
+
+// The instantiation for a token tile and an epilogue mode.
+template <int MX>
+cudaError_t dispatch_tc(int bn, int mode, dim3 grid, size_t smem, cudaStream_t st, int cl,
+                        const CUtensorMap& mw, const CUtensorMap& mx, const CUtensorMap& ms,
+                        const tpr::TcParams& prm) {
+    using namespace tpr;
+    if (mode == kTcClusterFold) {
+        if (bn == 32) return launch_tc_kernel<32, kTcClusterFold, MX>(grid, smem, st, cl, mw, mx, ms, prm);
+        if (bn == 64) return launch_tc_kernel<64, kTcClusterFold, MX>(grid, smem, st, cl, mw, mx, ms, prm);
+        return launch_tc_kernel<128, kTcClusterFold, MX>(grid, smem, st, cl, mw, mx, ms, prm);
+    }
+    if (mode == kTcCounterFold)   // at most two tokens: a 32-token tile
+        return launch_tc_kernel<32, kTcCounterFold, MX>(grid, smem, st, 1, mw, mx, ms, prm);
+    if (bn == 32) return launch_tc_kernel<32, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
+    if (bn == 64) return launch_tc_kernel<64, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
+    if (bn == 128) return launch_tc_kernel<128, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
+    return launch_tc_kernel<256, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
+}
+
+// allow_split (a reconciliation call): the kernel also runs S2-S4 (residual,
+// out) on chip when the configuration folds in clusters, or for few tokens
+// with `fold`, counting stored parts per H tile in `counters` (zero on entry,
+// zero on return); else a ring kernel must follow.
+tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* partials,
+                    int64_t tokens, bool allow_split, bool fold, unsigned int* counters,
+                    const void* residual, void* out, cudaStream_t stream) {
+    const TcConfig c = tc_config(p, tokens, allow_split, wt.fmt);
     if (c.stages < 2) return TP_ERR_UNSUPPORTED;
+    if (c.cluster_fold) fold = false;
     if (fold && (c.m_tiles != 1 || tokens > 2)) return TP_ERR_UNSUPPORTED;  // the kernel folds <= 2 rows
-    // Prefill-sized tiles without a k-split run on CTA pairs (2-SM MMA).
-    if (c.bn == tpr::kTc2Tokens && c.splits == 1 && !fold && p->sm_count >= 2)
-        return launch_tc2(p, x, w, partials, tokens, stream);
-    CUtensorMap mw, mx;
-    tp_status st = encode_tc_maps(p, c.bn, x, w, tokens, &mw, &mx);
+    // Prefill-sized bf16 tiles without a k-split run on CTA pairs (2-SM MMA).
+    if (wt.fmt == tpr::kFmtBf16 && c.bn == tpr::kTc2Tokens && c.splits == 1 && !fold && !c.cluster_fold &&
+        p->sm_count >= 2)
+        return launch_tc2(p, x, wt.w, partials, tokens, stream);
+    CUtensorMap mw, mx, ms;
+    tp_status st = encode_tc_maps(p, c.bn, x, wt.w, tokens, &mw, &mx);
     if (st != TP_OK) return st;
+    if (wt.fmt == tpr::kFmtMxfp8) {
+        if ((st = encode_mx_maps(p, wt.w, wt.scales, &mw, &ms)) != TP_OK) return st;
+    } else if (wt.fmt == tpr::kFmtNvfp4) {
+        if ((st = encode_nv_maps(p, wt.w, wt.scales, &mw, &ms)) != TP_OK) return st;
+    } else {
+        ms = mw;   // not read
+    }
     tpr::TcParams prm{};
     prm.n_ranks = p->n_ranks;
     prm.ks = static_cast<int>(p->ks);
@@ -355,19 +510,20 @@ tp_status launch_tc(const tp_plan* p, const void* x, const void* w, void* partia
     prm.stages = c.stages;
     prm.partials = static_cast<uint16_t*>(partials);
     prm.partials_f32 = static_cast<float*>(partials);
-    prm.fold = fold ? 1 : 0;
     prm.hc = static_cast<int>(p->hc);
     prm.counters = fold ? counters : nullptr;
     prm.residual = static_cast<const uint16_t*>(residual);
     prm.out = static_cast<uint16_t*>(out);
-    const dim3 grid(c.grid), block(tpr::kTcThreads);
-    cudaError_t e;
-    switch (c.bn) {
-        case 32: e = launch_pdl(tpr::tc_partial_kernel<32>, grid, block, c.smem, stream, mw, mx, prm); break;
-        case 64: e = launch_pdl(tpr::tc_partial_kernel<64>, grid, block, c.smem, stream, mw, mx, prm); break;
-        case 128: e = launch_pdl(tpr::tc_partial_kernel<128>, grid, block, c.smem, stream, mw, mx, prm); break;
-        default: e = launch_pdl(tpr::tc_partial_kernel<256>, grid, block, c.smem, stream, mw, mx, prm); break;
-    }
+    prm.nv_gexp = wt.fmt == tpr::kFmtNvfp4
+                      ? reinterpret_cast<const int*>(static_cast<const uint8_t*>(wt.scales) + nv_scale_bytes(p))
+                      : nullptr;
+    const int mode = c.cluster_fold ? tpr::kTcClusterFold : fold ? tpr::kTcCounterFold : tpr::kTcStore;
+    const int cl = c.cluster_fold ? p->n_ranks : 1;
+    const dim3 grid(c.grid);
+    const cudaError_t e =
+        wt.fmt == tpr::kFmtMxfp8   ? dispatch_tc<tpr::kFmtMxfp8>(c.bn, mode, grid, c.smem, stream, cl, mw, mx, ms, prm)
+        : wt.fmt == tpr::kFmtNvfp4 ? dispatch_tc<tpr::kFmtNvfp4>(c.bn, mode, grid, c.smem, stream, cl, mw, mx, ms, prm)
+                                   : dispatch_tc<tpr::kFmtBf16>(c.bn, mode, grid, c.smem, stream, cl, mw, mx, ms, prm);
     return e == cudaSuccess ? TP_OK : cuda_fail(e);
 }
 
@@ -394,18 +550,26 @@ tp_status launch_ring(const tp_plan* p, const void* partials, const void* residu
     return e == cudaSuccess ? TP_OK : cuda_fail(e);
 }
 
+#define TC_KERNELS(MX)                                                                   \
+    reinterpret_cast<const void*>(tpr::tc_partial_kernel<32, tpr::kTcStore, MX>),          \
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<64, tpr::kTcStore, MX>),      \
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<128, tpr::kTcStore, MX>),     \
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<256, tpr::kTcStore, MX>),     \
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<32, tpr::kTcCounterFold, MX>), \
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<32, tpr::kTcClusterFold, MX>), \
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<64, tpr::kTcClusterFold, MX>), \
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<128, tpr::kTcClusterFold, MX>)
+
 // Lets every exact kernel use the device's opt-in shared memory less its own
 // static shared memory; returns the smallest such dynamic allowance.
 cudaError_t set_kernel_attrs(int smem_optin, int* dyn_max) {
-    const void* kernels[9] = {reinterpret_cast<const void*>(tpr::exact_partial_kernel<1>),
-                              reinterpret_cast<const void*>(tpr::exact_partial_kernel<2>),
-                              reinterpret_cast<const void*>(tpr::exact_partial_kernel<4>),
-                              reinterpret_cast<const void*>(tpr::exact_partial_kernel<8>),
-                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<32>),
-                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<64>),
-                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<128>),
-                              reinterpret_cast<const void*>(tpr::tc_partial_kernel<256>),
-                              reinterpret_cast<const void*>(tpr::tc2_partial_kernel)};
+    const void* kernels[] = {
+        reinterpret_cast<const void*>(tpr::exact_partial_kernel<1>),
+        reinterpret_cast<const void*>(tpr::exact_partial_kernel<2>),
+        reinterpret_cast<const void*>(tpr::exact_partial_kernel<4>),
+        reinterpret_cast<const void*>(tpr::exact_partial_kernel<8>),
+        TC_KERNELS(tpr::kFmtBf16), TC_KERNELS(tpr::kFmtMxfp8), TC_KERNELS(tpr::kFmtNvfp4),
+        reinterpret_cast<const void*>(tpr::tc2_partial_kernel)};
     int lowest = smem_optin;
     for (const void* k : kernels) {
         cudaFuncAttributes fa{};
@@ -488,10 +652,18 @@ int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens) {
     return effective_variant(plan, tokens);
 }
 
-// The tensor path folds inside its partial kernel up to this many tokens.
+// The tensor path folds inside its partial kernel up to this many tokens
+// with a k-split (counter fold); without a split, at any token tile up to
+// 128, the kernel folds in clusters of N CTAs (cluster fold).
 constexpr int64_t kFoldMaxTokens = 2;
 
-static bool tc_folds(int64_t tokens) { return tokens <= kFoldMaxTokens; }
+static bool tc_cluster_folds(const tp_plan* plan, int64_t tokens) {
+    return tokens > 0 && tc_config(plan, tokens, true).cluster_fold;
+}
+
+static bool tc_folds(const tp_plan* plan, int64_t tokens) {
+    return tokens <= kFoldMaxTokens || tc_cluster_folds(plan, tokens);
+}
 
 // Fold counter block at the start of every workspace: one uint32 per
 // 128-row H tile, 256-byte rounded, reserved on every staged path so that
@@ -504,8 +676,10 @@ static size_t counter_block_bytes(const tp_plan* plan) {
 
 // Bytes of staged partials a call writes (0: none, the exact fused kernel).
 static size_t partial_bytes(const tp_plan* plan, int64_t tokens) {
-    if (effective_variant(plan, tokens) == TP_VARIANT_TENSOR)
-        return tc_partial_bytes(plan, tc_config(plan, tokens, true), tokens);
+    if (effective_variant(plan, tokens) == TP_VARIANT_TENSOR) {
+        const TcConfig c = tc_config(plan, tokens, true);
+        return c.cluster_fold ? 0 : tc_partial_bytes(plan, c, tokens);
+    }
     if (!plan->staged) return 0;
     return static_cast<size_t>(plan->n_ranks) * static_cast<size_t>(tokens) *
            static_cast<size_t>(plan->hidden) * 2;
@@ -521,7 +695,7 @@ size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens) {
 int tp_plan_launches(const tp_plan* plan, int64_t tokens) {
     if (!plan || tokens < 0) return -1;
     if (tokens == 0) return 0;
-    if (effective_variant(plan, tokens) == TP_VARIANT_TENSOR) return tc_folds(tokens) ? 1 : 2;
+    if (effective_variant(plan, tokens) == TP_VARIANT_TENSOR) return tc_folds(plan, tokens) ? 1 : 2;
     return plan->staged ? 2 : 1;
 }
 
@@ -568,6 +742,20 @@ static tp_status check_reconcile_args(const tp_plan* plan, const void* x, const 
     return TP_OK;
 }
 
+// S1-S4 on the tensor cores: one kernel that folds on chip (cluster fold, or
+// the counter fold for one or two tokens), else the partial kernel and a ring
+// kernel over the staged parts.
+static tp_status tensor_reconcile(const tp_plan* plan, const void* x, const TcWeights& wt,
+                                  const void* residual, void* out, int64_t tokens,
+                                  unsigned int* counters, void* partials, cudaStream_t s) {
+    const bool fold = tc_folds(plan, tokens);
+    tp_status st = launch_tc(plan, x, wt, partials, tokens, true, fold, counters, residual, out, s);
+    if (st != TP_OK || fold) return st;
+    const int splits = tc_config(plan, tokens, true).splits;
+    if (splits > 1) return launch_ring_splits(plan, partials, splits, residual, out, tokens, s);
+    return launch_ring(plan, partials, residual, out, tokens, s);
+}
+
 // S1-S4 with the fold counters and the staged partials given apart.
 static tp_status reconcile_launch(const tp_plan* plan, const void* x, const void* w_packed,
                                   const void* residual, void* out, int64_t tokens,
@@ -575,11 +763,8 @@ static tp_status reconcile_launch(const tp_plan* plan, const void* x, const void
     tp_status st = check_device(plan);
     if (st != TP_OK) return st;
     if (effective_variant(plan, tokens) == TP_VARIANT_TENSOR) {
-        const bool fold = tc_folds(tokens);
-        st = launch_tc(plan, x, w_packed, partials, tokens, true, fold, counters, residual, out, s);
-        if (st != TP_OK || fold) return st;
-        const int splits = tc_config(plan, tokens, true).splits;
-        if (splits > 1) return launch_ring_splits(plan, partials, splits, residual, out, tokens, s);
+        return tensor_reconcile(plan, x, TcWeights{w_packed, nullptr, tpr::kFmtBf16}, residual, out, tokens,
+                                counters, partials, s);
     } else {
         if (!plan->staged)
             return launch_exact(plan, x, w_packed, residual, out, nullptr, tokens, true, s);
@@ -637,7 +822,8 @@ tp_status tp_rowlinear_partials(const tp_plan* plan, const void* x, const void* 
     if ((st = check_device(plan)) != TP_OK) return st;
     const int variant = effective_variant(plan, tokens);
     if (variant == TP_VARIANT_TENSOR)
-        return launch_tc(plan, x, w_packed, partials, tokens, false, false, nullptr, nullptr,
+        return launch_tc(plan, x, TcWeights{w_packed, nullptr, tpr::kFmtBf16}, partials, tokens, false, false,
+                         nullptr, nullptr,
                          nullptr, static_cast<cudaStream_t>(stream));
     return launch_exact(plan, x, w_packed, nullptr, nullptr, partials, tokens, false,
                         static_cast<cudaStream_t>(stream));
@@ -669,17 +855,25 @@ uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_byt
 
 tp_status tp_plan_mxfp8_bytes(const tp_plan* plan, size_t* q_bytes, size_t* scale_bytes) {
     if (!plan || !q_bytes || !scale_bytes) return TP_ERR_INVALID;
-    if (plan->ks % tpr::kMxBlock != 0) return TP_ERR_UNSUPPORTED;
+    if (plan->ks % tpr::kMxPair != 0) return TP_ERR_UNSUPPORTED;
     *q_bytes = static_cast<size_t>(plan->hidden) * static_cast<size_t>(plan->k);
     *scale_bytes = *q_bytes / tpr::kMxBlock;
     return TP_OK;
 }
 
+size_t tp_plan_mxfp8_workspace_bytes(const tp_plan* plan, int64_t tokens) {
+    if (!plan || tokens <= 0) return 0;
+    const TcConfig c = tc_config(plan, tokens, true, tpr::kFmtMxfp8);
+    const size_t pb = c.cluster_fold ? 0 : tc_partial_bytes(plan, c, tokens);
+    if (pb == 0) return 0;
+    return (counter_block_bytes(plan) + pb + 255) / 256 * 256;
+}
+
 tp_status tp_pack_weights_mxfp8(const tp_plan* plan, const void* w_hk, void* w_q, void* w_scales,
                                 void* stream) {
     if (!plan || !w_hk || !w_q || !w_scales) return TP_ERR_INVALID;
-    if (plan->ks % tpr::kMxBlock != 0) return TP_ERR_UNSUPPORTED;
-    if (!aligned16(w_hk) || !aligned16(w_q)) return TP_ERR_ALIGN;
+    if (plan->ks % tpr::kMxPair != 0) return TP_ERR_UNSUPPORTED;
+    if (!aligned16(w_hk) || !aligned16(w_q) || !aligned16(w_scales)) return TP_ERR_ALIGN;
     const size_t wb = static_cast<size_t>(plan->hidden) * plan->k * 2;
     const size_t qb = wb / 2, sb = qb / tpr::kMxBlock;
     if (overlaps(w_hk, wb, w_q, qb) || overlaps(w_hk, wb, w_scales, sb) || overlaps(w_q, qb, w_scales, sb))
@@ -697,45 +891,182 @@ tp_status tp_pack_weights_mxfp8(const tp_plan* plan, const void* w_hk, void* w_q
 
 tp_status tp_rowlinear_reconcile_mxfp8(const tp_plan* plan, const void* x, const void* w_q,
                                        const void* w_scales, const void* residual, void* out,
-                                       int64_t tokens, void* stream) {
+                                       int64_t tokens, void* workspace, void* stream) {
     if (!plan) return TP_ERR_INVALID;
     if (tokens < 0 || tokens > plan->max_tokens) return TP_ERR_INVALID;
     if (tokens == 0) return TP_OK;
-    if (tokens > tpr::kMxMaxTokens || plan->ks % tpr::kMxBlock != 0) return TP_ERR_UNSUPPORTED;
+    if (plan->ks % tpr::kMxPair != 0) return TP_ERR_UNSUPPORTED;
     if (!x || !w_q || !w_scales || !residual || !out) return TP_ERR_INVALID;
-    if (!aligned16(x) || !aligned16(w_q) || !aligned16(residual) || !aligned16(out)) return TP_ERR_ALIGN;
+    if (!aligned16(x) || !aligned16(w_q) || !aligned16(w_scales) || !aligned16(residual) ||
+        !aligned16(out) || !aligned16(workspace))
+        return TP_ERR_ALIGN;
     const size_t mh = static_cast<size_t>(tokens) * plan->hidden * 2;
     const size_t xb = static_cast<size_t>(tokens) * plan->k * 2;
     const size_t qb = static_cast<size_t>(plan->hidden) * plan->k, sb = qb / tpr::kMxBlock;
+    const size_t ws = tp_plan_mxfp8_workspace_bytes(plan, tokens);
     if (overlaps(out, mh, x, xb) || overlaps(out, mh, w_q, qb) || overlaps(out, mh, w_scales, sb) ||
-        overlaps(out, mh, residual, mh))
+        overlaps(out, mh, residual, mh) || overlaps(out, mh, workspace, ws))
+        return TP_ERR_INVALID;
+    if (ws && !workspace) return TP_ERR_WORKSPACE;
+    tp_status st = check_device(plan);
+    if (st != TP_OK) return st;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    return tensor_reconcile(plan, x, TcWeights{w_q, w_scales, tpr::kFmtMxfp8}, residual, out, tokens,
+                            reinterpret_cast<unsigned int*>(base),
+                            ws ? base + counter_block_bytes(plan) : nullptr,
+                            static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------- NVFP4 weight shards --
+
+tp_status tp_plan_nvfp4_bytes(const tp_plan* plan, size_t* q_bytes, size_t* scale_bytes) {
+    if (!plan || !q_bytes || !scale_bytes) return TP_ERR_INVALID;
+    if (plan->ks % tpr::kTcKBlock != 0) return TP_ERR_UNSUPPORTED;
+    *q_bytes = static_cast<size_t>(plan->hidden) * static_cast<size_t>(plan->k) / 2;
+    *scale_bytes = nv_scale_bytes(plan) + 16;
+    return TP_OK;
+}
+
+size_t tp_plan_nvfp4_workspace_bytes(const tp_plan* plan, int64_t tokens) {
+    if (!plan || tokens <= 0) return 0;
+    const TcConfig c = tc_config(plan, tokens, true, tpr::kFmtNvfp4);
+    const size_t pb = c.cluster_fold ? 0 : tc_partial_bytes(plan, c, tokens);
+    if (pb == 0) return 0;
+    return (counter_block_bytes(plan) + pb + 255) / 256 * 256;
+}
+
+tp_status tp_pack_weights_nvfp4(const tp_plan* plan, const void* w_hk, void* w_q, void* w_scales,
+                                void* stream) {
+    if (!plan || !w_hk || !w_q || !w_scales) return TP_ERR_INVALID;
+    if (plan->ks % tpr::kTcKBlock != 0) return TP_ERR_UNSUPPORTED;
+    if (!aligned16(w_hk) || !aligned16(w_q) || !aligned16(w_scales)) return TP_ERR_ALIGN;
+    const size_t wb = static_cast<size_t>(plan->hidden) * plan->k * 2;
+    const size_t qb = wb / 4, sb = nv_scale_bytes(plan) + 16;
+    if (overlaps(w_hk, wb, w_q, qb) || overlaps(w_hk, wb, w_scales, sb) || overlaps(w_q, qb, w_scales, sb))
         return TP_ERR_INVALID;
     tp_status st = check_device(plan);
     if (st != TP_OK) return st;
-    tpr::MxParams prm{};
-    prm.n_ranks = plan->n_ranks;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* trailer = static_cast<uint8_t*>(w_scales) + nv_scale_bytes(plan);
+    cudaError_t e = cudaMemsetAsync(trailer, 0, 16, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    const int64_t nvec = plan->hidden * plan->k / 8;
+    const int64_t g1 = std::min<int64_t>((nvec + 255) / 256, static_cast<int64_t>(plan->sm_count) * 8);
+    tpr::nv_amax_kernel<<<static_cast<unsigned>(g1), 256, 0, s>>>(
+        static_cast<const uint16_t*>(w_hk), nvec, reinterpret_cast<uint32_t*>(trailer + 4));
+    const int64_t blocks_total = static_cast<int64_t>(plan->n_ranks) * plan->hidden * (plan->ks / 16);
+    const int64_t g2 = std::min<int64_t>((blocks_total + 255) / 256, static_cast<int64_t>(plan->sm_count) * 16);
+    tpr::pack_weights_nv_kernel<<<static_cast<unsigned>(g2), 256, 0, s>>>(
+        static_cast<const uint16_t*>(w_hk), static_cast<uint8_t*>(w_q), static_cast<uint8_t*>(w_scales),
+        reinterpret_cast<int*>(trailer), reinterpret_cast<const uint32_t*>(trailer + 4), plan->n_ranks,
+        static_cast<int>(plan->hidden), plan->k, plan->ks);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? TP_OK : cuda_fail(e);
+}
+
+tp_status tp_rowlinear_reconcile_nvfp4(const tp_plan* plan, const void* x, const void* w_q,
+                                       const void* w_scales, const void* residual, void* out,
+                                       int64_t tokens, void* workspace, void* stream) {
+    if (!plan) return TP_ERR_INVALID;
+    if (tokens < 0 || tokens > plan->max_tokens) return TP_ERR_INVALID;
+    if (tokens == 0) return TP_OK;
+    if (plan->ks % tpr::kTcKBlock != 0) return TP_ERR_UNSUPPORTED;
+    if (!x || !w_q || !w_scales || !residual || !out) return TP_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(w_q) || !aligned16(w_scales) || !aligned16(residual) ||
+        !aligned16(out) || !aligned16(workspace))
+        return TP_ERR_ALIGN;
+    const size_t mh = static_cast<size_t>(tokens) * plan->hidden * 2;
+    const size_t xb = static_cast<size_t>(tokens) * plan->k * 2;
+    const size_t qb = static_cast<size_t>(plan->hidden) * plan->k / 2, sb = nv_scale_bytes(plan) + 16;
+    const size_t ws = tp_plan_nvfp4_workspace_bytes(plan, tokens);
+    if (overlaps(out, mh, x, xb) || overlaps(out, mh, w_q, qb) || overlaps(out, mh, w_scales, sb) ||
+        overlaps(out, mh, residual, mh) || overlaps(out, mh, workspace, ws))
+        return TP_ERR_INVALID;
+    if (ws && !workspace) return TP_ERR_WORKSPACE;
+    tp_status st = check_device(plan);
+    if (st != TP_OK) return st;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    return tensor_reconcile(plan, x, TcWeights{w_q, w_scales, tpr::kFmtNvfp4}, residual, out, tokens,
+                            reinterpret_cast<unsigned int*>(base),
+                            ws ? base + counter_block_bytes(plan) : nullptr,
+                            static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------- ring protocol between ranks --
+
+// CTAs per rank of the ring protocol: the same for every call of a plan (the
+// step flags of a rank are one per CTA), and N of them fit on the device at once.
+static int ring_ctas_per_rank(const tp_plan* plan) {
+    return std::max(1, std::min(plan->sm_count / plan->n_ranks, 64));
+}
+
+static size_t ring_flag_bytes(const tp_plan* plan) {
+    return (static_cast<size_t>(ring_ctas_per_rank(plan)) * 4 + 255) / 256 * 256;
+}
+
+size_t tp_ring_rank_workspace_bytes(const tp_plan* plan, int64_t tokens) {
+    if (!plan || tokens < 0 || tokens > plan->max_tokens) return 0;
+    const size_t mh = static_cast<size_t>(tokens) * static_cast<size_t>(plan->hidden) * 2;
+    return ring_flag_bytes(plan) + 2 * ((mh + 255) / 256 * 256);
+}
+
+tp_status tp_ring_allreduce_ranks(const tp_plan* plan, const void* const* partials, const void* residual,
+                                  void* const* outs, void* const* workspaces, int first_rank,
+                                  int launch_ranks, int64_t tokens, uint64_t wait_limit_ns, void* stream) {
+    if (!plan || !partials || !outs || !workspaces) return TP_ERR_INVALID;
+    const int n = plan->n_ranks;
+    if (tokens < 0 || tokens > plan->max_tokens) return TP_ERR_INVALID;
+    if (first_rank < 0 || launch_ranks < 1 || first_rank + launch_ranks > n) return TP_ERR_INVALID;
+    if (tokens == 0) return TP_OK;
+    if (!residual) return TP_ERR_INVALID;
+    if (!aligned16(residual)) return TP_ERR_ALIGN;
+    const size_t mh = static_cast<size_t>(tokens) * static_cast<size_t>(plan->hidden) * 2;
+    const size_t ws = tp_ring_rank_workspace_bytes(plan, tokens);
+    for (int r = 0; r < n; ++r) {
+        if (!partials[r] || !outs[r] || !workspaces[r]) return TP_ERR_INVALID;
+        if (!aligned16(partials[r]) || !aligned16(outs[r]) || !aligned16(workspaces[r])) return TP_ERR_ALIGN;
+        for (int q = 0; q < n; ++q)
+            if (overlaps(outs[r], mh, partials[q], mh) || overlaps(outs[r], mh, workspaces[q], ws) ||
+                (q != r && overlaps(outs[r], mh, outs[q], mh)) ||
+                (q != r && overlaps(workspaces[r], ws, workspaces[q], ws)) ||
+                overlaps(workspaces[r], ws, partials[q], mh))
+                return TP_ERR_INVALID;
+        if (overlaps(outs[r], mh, residual, mh)) return TP_ERR_INVALID;
+    }
+    tp_status st = check_device(plan);
+    if (st != TP_OK) return st;
+    tpr::RingRanks rk{};
+    const size_t slot = (mh + 255) / 256 * 256;
+    for (int r = 0; r < n; ++r) {
+        uint8_t* w = static_cast<uint8_t*>(workspaces[r]);
+        rk.partial[r] = static_cast<const uint16_t*>(partials[r]);
+        rk.flags[r] = reinterpret_cast<uint32_t*>(w);
+        rk.work[r] = reinterpret_cast<uint16_t*>(w + ring_flag_bytes(plan));
+        rk.gather[r] = reinterpret_cast<uint16_t*>(w + ring_flag_bytes(plan) + slot);
+        rk.out[r] = static_cast<uint16_t*>(outs[r]);
+    }
+    tpr::RingParams prm{};
+    prm.n_ranks = n;
+    prm.first_rank = first_rank;
+    prm.ctas_per_rank = ring_ctas_per_rank(plan);
     prm.hidden = static_cast<int>(plan->hidden);
     prm.hc = static_cast<int>(plan->hc);
-    prm.tokens = static_cast<int>(tokens);
-    prm.k = plan->k;
-    prm.ks = plan->ks;
-    prm.x = static_cast<const uint16_t*>(x);
-    prm.q = static_cast<const uint8_t*>(w_q);
-    prm.scales = static_cast<const uint8_t*>(w_scales);
+    prm.tokens = tokens;
     prm.residual = static_cast<const uint16_t*>(residual);
-    prm.out = static_cast<uint16_t*>(out);
-    // one warp per output row (grid-stride beyond 32 CTAs per SM)
-    const int64_t grid = std::min<int64_t>((plan->hidden + tpr::kMxWarps - 1) / tpr::kMxWarps,
-                                           static_cast<int64_t>(plan->sm_count) * 32);
-    const dim3 g(static_cast<unsigned>(grid)), b(tpr::kMxWarps * 32);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    switch (tokens) {
-        case 1: e = launch_pdl(tpr::mx_reconcile_kernel<1>, g, b, 0, s, prm); break;
-        case 2: e = launch_pdl(tpr::mx_reconcile_kernel<2>, g, b, 0, s, prm); break;
-        case 3: e = launch_pdl(tpr::mx_reconcile_kernel<3>, g, b, 0, s, prm); break;
-        default: e = launch_pdl(tpr::mx_reconcile_kernel<4>, g, b, 0, s, prm); break;
-    }
+    prm.wait_limit_ns = wait_limit_ns ? wait_limit_ns : 1000000000ull;   // 1 s
+    // One launch for the ranks it runs; cooperative, so all their CTAs are
+    // resident together (a rank's CTAs wait on its predecessor's).
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(launch_ranks * prm.ctas_per_rank));
+    cfg.blockDim = dim3(tpr::kRingThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, tpr::ring_protocol_kernel, rk, prm);
     return e == cudaSuccess ? TP_OK : cuda_fail(e);
 }
 

@@ -141,6 +141,54 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                  : "memory");
 }
 
+// ------------------------------------------ cluster fold (distributed smem) --
+// The N CTAs of a cluster each hold one rank's partial tile in their shared
+// memory; a CTA reads its peers' tiles through the cluster's shared window.
+
+// Orders this thread's (and, after a CTA barrier, its CTA's) shared-memory
+// writes before later operations seen at cluster scope.
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+
+// As mbar_try_wait, with acquire at cluster scope: the writes that peer CTAs
+// made before their release-arrivals on this barrier are visible after it.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded like mbar_wait_bounded: gives up after kWaitLimitNs, sets the
+// device error word and returns false.
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_device_error, kErrWaitTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// 16 bytes of a CTA's shared memory, by their address in the cluster window.
+__device__ __forceinline__ uint4 ld_dsmem_v4(uint32_t cluster_addr) {
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(cluster_addr)
+                 : "memory");
+    return v;
+}
+
 // The leader CTA's copy of a barrier of this CTA: its shared::cta address with
 // the pair bit cleared (the form the paired TMA load and commit expect).
 __device__ __forceinline__ uint32_t pair_leader_addr(const void* p) {

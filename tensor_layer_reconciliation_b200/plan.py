@@ -147,10 +147,13 @@ class Plan:
             raise TPError(st, "tp_pack_weights_mxfp8")
         return q, sc
 
+    def mxfp8_workspace_bytes(self, tokens: int) -> int:
+        return _lib.tp_plan_mxfp8_workspace_bytes(self._h, tokens)
+
     def reconcile_mxfp8(self, x: torch.Tensor, w_q: torch.Tensor, w_scales: torch.Tensor,
                         residual: torch.Tensor, out: Optional[torch.Tensor] = None,
-                        stream=None) -> torch.Tensor:
-        """out [M, H] = residual + ring-ordered sum of x_r . dequant(W_r)^T (M <= 4)."""
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """out [M, H] = residual + ring-ordered sum of x_r . dequant(W_r)^T."""
         m = x.shape[0]
         if out is None:
             out = torch.empty(m, self.hidden, dtype=torch.bfloat16, device=x.device)
@@ -161,10 +164,69 @@ class Plan:
         px = _check(x, "x", (m, self.k))
         pr = _check(residual, "residual", (m, self.hidden))
         po = _check(out, "out", (m, self.hidden))
+        need = self.mxfp8_workspace_bytes(m)
+        pws = 0
+        if need:
+            if workspace is None:   # fold counters start at zero
+                workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+            if workspace.numel() * workspace.element_size() < need or workspace.device.type != "cuda":
+                raise ValueError("workspace too small")
+            pws = workspace.data_ptr()
         st = _lib.tp_rowlinear_reconcile_mxfp8(self._h, px, w_q.data_ptr(), w_scales.data_ptr(), pr, po,
-                                               m, _stream(stream))
+                                               m, pws, _stream(stream))
         if st != _lib.TP_OK:
             raise TPError(st, "tp_rowlinear_reconcile_mxfp8")
+        return out
+
+    # ---------------------------------------------------- NVFP4 shards --
+
+    def nvfp4_bytes(self):
+        """(code bytes, scale bytes) of this plan's NVFP4 shards."""
+        st, q, sc = _lib.tp_plan_nvfp4_bytes(self._h)
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_plan_nvfp4_bytes")
+        return q, sc
+
+    def nvfp4_workspace_bytes(self, tokens: int) -> int:
+        return _lib.tp_plan_nvfp4_workspace_bytes(self._h, tokens)
+
+    def pack_weights_nvfp4(self, w_hk: torch.Tensor, stream=None):
+        """Linear weight [H, K] -> (E2M1 code pairs, E4M3 block scales + g) as flat uint8 tensors."""
+        qb, sb = self.nvfp4_bytes()
+        q = torch.empty(qb, dtype=torch.uint8, device=w_hk.device)
+        sc = torch.empty(sb, dtype=torch.uint8, device=w_hk.device)
+        a = _check(w_hk, "w_hk", (self.hidden, self.k))
+        st = _lib.tp_pack_weights_nvfp4(self._h, a, q.data_ptr(), sc.data_ptr(), _stream(stream))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_pack_weights_nvfp4")
+        return q, sc
+
+    def reconcile_nvfp4(self, x: torch.Tensor, w_q: torch.Tensor, w_scales: torch.Tensor,
+                        residual: torch.Tensor, out: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """out [M, H] = residual + ring-ordered sum of x_r . dequant(W_r)^T (NVFP4 shards)."""
+        m = x.shape[0]
+        if out is None:
+            out = torch.empty(m, self.hidden, dtype=torch.bfloat16, device=x.device)
+        qb, sb = self.nvfp4_bytes()
+        for t, name, n in ((w_q, "w_q", qb), (w_scales, "w_scales", sb)):
+            if t.dtype != torch.uint8 or t.numel() != n or t.device.type != "cuda" or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CUDA uint8 tensor of {n} bytes")
+        px = _check(x, "x", (m, self.k))
+        pr = _check(residual, "residual", (m, self.hidden))
+        po = _check(out, "out", (m, self.hidden))
+        need = self.nvfp4_workspace_bytes(m)
+        pws = 0
+        if need:
+            if workspace is None:   # fold counters start at zero
+                workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+            if workspace.numel() * workspace.element_size() < need or workspace.device.type != "cuda":
+                raise ValueError("workspace too small")
+            pws = workspace.data_ptr()
+        st = _lib.tp_rowlinear_reconcile_nvfp4(self._h, px, w_q.data_ptr(), w_scales.data_ptr(), pr, po,
+                                               m, pws, _stream(stream))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_rowlinear_reconcile_nvfp4")
         return out
 
     def partials(self, x: torch.Tensor, w_packed: torch.Tensor,
@@ -194,6 +256,40 @@ class Plan:
         if st != _lib.TP_OK:
             raise TPError(st, "tp_ring_reduce")
         return out
+
+    def ring_rank_workspace_bytes(self, tokens: int) -> int:
+        return _lib.tp_ring_rank_workspace_bytes(self._h, tokens)
+
+    def ring_allreduce_ranks(self, partials, residual: torch.Tensor, outs=None, workspaces=None,
+                             first_rank: int = 0, launch_ranks: Optional[int] = None,
+                             wait_limit_ns: int = 0, stream=None):
+        """The ring all-reduce as a protocol between ranks with their own
+        buffers: partials and outs are N tensors [M, H] (one per rank),
+        workspaces N uint8 tensors of ring_rank_workspace_bytes (zeroed when
+        created here). Runs ranks first_rank .. first_rank + launch_ranks - 1
+        (default: all). Returns (outs, workspaces)."""
+        n = self.n_ranks
+        if len(partials) != n:
+            raise ValueError(f"need {n} partials")
+        m = partials[0].shape[0]
+        pp = [_check(t, f"partials[{i}]", (m, self.hidden)) for i, t in enumerate(partials)]
+        pr = _check(residual, "residual", (m, self.hidden))
+        if outs is None:
+            outs = [torch.empty(m, self.hidden, dtype=torch.bfloat16, device=residual.device)
+                    for _ in range(n)]
+        po = [_check(t, f"outs[{i}]", (m, self.hidden)) for i, t in enumerate(outs)]
+        need = self.ring_rank_workspace_bytes(m)
+        if workspaces is None:
+            workspaces = [torch.zeros(need, dtype=torch.uint8, device=residual.device) for _ in range(n)]
+        for i, w in enumerate(workspaces):
+            if w.device.type != "cuda" or w.numel() * w.element_size() < need:
+                raise ValueError(f"workspaces[{i}] too small")
+        st = _lib.tp_ring_allreduce_ranks(self._h, pp, pr, po, [w.data_ptr() for w in workspaces],
+                                          first_rank, n if launch_ranks is None else launch_ranks, m,
+                                          wait_limit_ns, _stream(stream))
+        if st != _lib.TP_OK:
+            raise TPError(st, "tp_ring_allreduce_ranks")
+        return outs, workspaces
 
     def device_error_flags(self, reset: bool = False) -> int:
         st, flags = _lib.tp_device_error_flags(self._h, int(reset))

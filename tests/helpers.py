@@ -117,3 +117,26 @@ def round_f32_exact(v: Fraction) -> Fraction:
         n += 1
     r = n * Fraction(2) ** q
     return -r if v < 0 else r
+
+
+def mx_scales_as_stored(sc):
+    """The oracle's MXFP8 scales [N][H][K/N/32] in the library's storage order
+    [N][K/N/64][H][2] (the two 32-weight runs of each 64-column block of a
+    rank slice, row after row), flattened. A permutation only."""
+    sc = np.asarray(sc)
+    n, h, nb = sc.shape
+    assert nb % 2 == 0
+    return np.ascontiguousarray(sc.reshape(n, h, nb // 2, 2).transpose(0, 2, 1, 3)).reshape(-1)
+
+
+def nv_scales_as_stored(sc, g, amax_bits):
+    """The oracle's NVFP4 block scales [N][H][K/N/16] and exponent g in the
+    library's storage order: [N][K/N/64][H][4], flattened, then 16 bytes
+    (g as int32, the weight's largest magnitude as bf16 bits in an int32,
+    8 zero bytes). A permutation and a packing only."""
+    sc = np.asarray(sc)
+    n, h, nb = sc.shape
+    assert nb % 4 == 0
+    body = np.ascontiguousarray(sc.reshape(n, h, nb // 4, 4).transpose(0, 2, 1, 3)).reshape(-1)
+    trailer = np.array([g, amax_bits, 0, 0], dtype=np.int32).view(np.uint8)
+    return np.concatenate([body, trailer])

@@ -81,12 +81,19 @@ def test_null_plan_everywhere():
     assert tlr.tp_plan_launches(None, 4) == -1
     assert tlr.tp_plan_mxfp8_bytes(None)[0] == INV
     assert tlr.tp_pack_weights_mxfp8(None, 16, 32, 48, 0) == INV
-    assert tlr.tp_rowlinear_reconcile_mxfp8(None, 16, 32, 48, 64, 80, 1, 0) == INV
+    assert tlr.tp_rowlinear_reconcile_mxfp8(None, 16, 32, 48, 64, 80, 1, 0, 0) == INV
+    assert tlr.tp_plan_mxfp8_workspace_bytes(None, 4) == 0
+    assert tlr.tp_plan_nvfp4_bytes(None)[0] == INV
+    assert tlr.tp_pack_weights_nvfp4(None, 16, 32, 48, 0) == INV
+    assert tlr.tp_plan_nvfp4_workspace_bytes(None, 4) == 0
+    assert tlr.tp_rowlinear_reconcile_nvfp4(None, 16, 32, 48, 64, 80, 1, 0, 0) == INV
     assert tlr.tp_pack_weights(None, 16, 32, 0) == INV
     assert tlr.tp_rowlinear_reconcile(None, 16, 32, 48, 64, 1, 0, 0) == INV
     assert tlr.tp_rowlinear_partials(None, 16, 32, 48, 1, 0) == INV
     assert tlr.tp_ring_reduce(None, 16, 32, 48, 1, 0) == INV
     assert tlr.tp_device_error_flags(None)[0] == INV
+    assert tlr.tp_ring_rank_workspace_bytes(None, 4) == 0
+    assert tlr.tp_ring_allreduce_ranks(None, [16, 32], 48, [64, 80], [96, 112], 0, 2, 1, 0, 0) == INV
     tlr.tp_plan_destroy(None)          # NULL-safe
 
 

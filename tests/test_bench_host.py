@@ -43,8 +43,8 @@ def test_configs_to_run():
     args = type("A", (), {"config": "all", "weights": "bf16"})()
     assert bench._configs_to_run(args) == bench.BENCH_CONFIGS
     assert bench.BENCH_CONFIGS[0] == bench.HEADLINE_CONFIG
-    args.weights = "mxfp8"
-    assert bench._configs_to_run(args) == ["decode_n2"]
+    args.weights = "mxfp8"                              # MXFP8 shards run every workload
+    assert bench._configs_to_run(args) == bench.BENCH_CONFIGS
     args.config, args.weights = "prefill_n4", "bf16"
     assert bench._configs_to_run(args) == ["prefill_n4"]
 

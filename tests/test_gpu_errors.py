@@ -4,7 +4,7 @@ around the buffers of every kernel path.
 Fault injection on the host: misaligned pointers (TP_ERR_ALIGN), an output
 that overlaps an input or the workspace (TP_ERR_INVALID), a missing workspace
 (TP_ERR_WORKSPACE), token counts outside [0, max_tokens] (TP_ERR_INVALID)
-and token counts the MXFP8 kernel has no form for (TP_ERR_UNSUPPORTED). Each
+and shard widths the MXFP8 path has no form for (TP_ERR_UNSUPPORTED). Each
 call must return its status with nothing launched: the output, filled with a
 sentinel beforehand, is unchanged after the stream has drained, and the
 device error word stays clear. The C ABI carries no workspace size, so a
@@ -168,22 +168,31 @@ def test_mxfp8_rejects_bad_arguments(setup):
     tlr, plan, x, wp, r, ws, dev = setup
     w = torch.randn(H, K, device=dev).to(torch.bfloat16)
     q, sc = plan.pack_weights_mxfp8(w)
+    need = plan.mxfp8_workspace_bytes(M)
+    assert need > 0
+    mws = torch.zeros(need, dtype=torch.uint8, device=dev)
     out = _sentinel(M * H + 8, dev)
     s = _stream()
     base = [x.data_ptr(), q.data_ptr(), sc.data_ptr(), r.data_ptr(), out.data_ptr()]
-    for i in (0, 1, 3, 4):                                # the scales need only byte alignment
+    for i in range(5):
         bad = list(base)
         bad[i] += 2
-        assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *bad, M, s) == tlr.TP_ERR_ALIGN, i
+        assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *bad, M, mws.data_ptr(), s) == tlr.TP_ERR_ALIGN, i
+    assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *base, M, mws.data_ptr() + 2, s) == tlr.TP_ERR_ALIGN
+    for i in (0, 1, 2, 3):                               # out overlapping x, codes, scales, residual
+        bad = list(base)
+        bad[4] = base[i]
+        assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *bad, M, mws.data_ptr(), s) == tlr.TP_ERR_INVALID, i
     bad = list(base)
-    bad[4] = x.data_ptr()
-    assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *bad, M, s) == tlr.TP_ERR_INVALID
-    bad = list(base)
-    bad[4] = q.data_ptr()
-    assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *bad, M, s) == tlr.TP_ERR_INVALID
-    assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *base, M + 1, s) == tlr.TP_ERR_INVALID
-    big = tlr.Plan(N, 8, K, H)
-    assert tlr.tp_rowlinear_reconcile_mxfp8(big.handle, *base, 5, s) == tlr.TP_ERR_UNSUPPORTED
+    bad[4] = mws.data_ptr()
+    assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *bad, M, mws.data_ptr(), s) == tlr.TP_ERR_INVALID
+    assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *base, M, 0, s) == tlr.TP_ERR_WORKSPACE
+    assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *base, M + 1, mws.data_ptr(), s) == tlr.TP_ERR_INVALID
+    assert tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, *base, -1, mws.data_ptr(), s) == tlr.TP_ERR_INVALID
+    # packing: misaligned or overlapping shard buffers
+    assert tlr.tp_pack_weights_mxfp8(plan.handle, w.data_ptr(), q.data_ptr() + 2, sc.data_ptr(), s) == tlr.TP_ERR_ALIGN
+    assert tlr.tp_pack_weights_mxfp8(plan.handle, w.data_ptr(), q.data_ptr(), sc.data_ptr() + 2, s) == tlr.TP_ERR_ALIGN
+    assert tlr.tp_pack_weights_mxfp8(plan.handle, w.data_ptr(), q.data_ptr(), q.data_ptr(), s) == tlr.TP_ERR_INVALID
     _untouched(out, plan)
 
 
@@ -225,7 +234,7 @@ def test_guard_zones_tensor_paths(n, m, k, h):
     assert plan.device_error_flags() == 0
 
 
-@pytest.mark.parametrize("n,m,k,h", [(2, 1, 2048, 512), (4, 4, 1024, 256)])
+@pytest.mark.parametrize("n,m,k,h", [(2, 1, 2048, 512), (4, 4, 1024, 256), (8, 64, 1024, 4096)])
 def test_guard_zones_mxfp8(n, m, k, h):
     import tensor_layer_reconciliation_b200 as tlr
     dev = torch.device("cuda")
@@ -234,8 +243,12 @@ def test_guard_zones_mxfp8(n, m, k, h):
     q, sc = plan.pack_weights_mxfp8(w)
     ref = plan.reconcile_mxfp8(x, q, sc, r)
     obuf, o = _guarded(m * h, dev)
-    plan.reconcile_mxfp8(x, q, sc, r, out=o.view(torch.bfloat16).view(m, h))
-    assert _guards_intact(obuf, m * h)
+    need = (plan.mxfp8_workspace_bytes(m) + 1) // 2
+    wbuf, ws = _guarded(need, dev)
+    ws.zero_()
+    plan.reconcile_mxfp8(x, q, sc, r, out=o.view(torch.bfloat16).view(m, h),
+                         workspace=ws if need else None)
+    assert _guards_intact(obuf, m * h) and _guards_intact(wbuf, need)
     assert torch.equal(o, ref.view(torch.int16).view(-1))
     # the shards themselves, packed into guarded buffers
     qb, sb = plan.mxfp8_bytes()

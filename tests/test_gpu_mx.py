@@ -17,7 +17,7 @@ import torch
 
 import oracle
 from gpu_util import inputs
-from helpers import from_u16, u16
+from helpers import from_u16, mx_scales_as_stored, u16
 from test_gpu_tensor import check_against_oracle
 
 pytestmark = pytest.mark.gpu
@@ -34,7 +34,7 @@ def _quantize_on_gpu(n, w):
     q, sc = plan.pack_weights_mxfp8(w)
     torch.cuda.synchronize()
     ks = k // n
-    return (q.cpu().numpy().reshape(n, h, ks), sc.cpu().numpy().reshape(n, h, ks // 32))
+    return q.cpu().numpy().reshape(n, h, ks), sc.cpu().numpy()
 
 
 @pytest.mark.parametrize("n,h,k,seed", [(1, 64, 256, 1), (2, 96, 1024, 2), (4, 128, 2048, 3),
@@ -44,7 +44,7 @@ def test_mx_quantize_gaussian_bit_exact(n, h, k, seed):
     _, w, _ = inputs(n, 1, k, h, seed, dev)
     q, sc = _quantize_on_gpu(n, w)
     q_ref, sc_ref = oracle.mx_quantize(n, u16(w))
-    assert np.array_equal(sc, sc_ref)
+    assert np.array_equal(sc, mx_scales_as_stored(sc_ref))
     assert np.array_equal(q, q_ref)
 
 
@@ -71,16 +71,20 @@ def test_mx_quantize_every_magnitude(amax_bits):
     w = np.ascontiguousarray(w.reshape(rows, per_row * 32))
     q, sc = _quantize_on_gpu(1, from_u16(w).cuda())
     q_ref, sc_ref = oracle.mx_quantize(1, w)
-    assert np.array_equal(sc, sc_ref)
+    assert np.array_equal(sc, mx_scales_as_stored(sc_ref))
     assert np.array_equal(q, q_ref)
 
 
 SHAPES = [             # N, M, K, H
-    (2, 1, 1024, 512),
-    (4, 2, 2048, 640),
-    (8, 3, 4096, 1024),
-    (1, 4, 512, 256),
+    (2, 1, 1024, 512),      # one token: K split, folded in the kernel
+    (4, 2, 2048, 640),      # two tokens, H % 128 != 0
+    (8, 3, 4096, 1024),     # three tokens: K split, fp32 parts, split ring kernel
+    (1, 4, 512, 256),       # N = 1
     (2, 1, 17408, 5120),    # the down-projection of the decode example, full size
+    (8, 64, 1024, 4096),    # 64 tokens, 256 units: fold on chip in clusters of 8
+    (3, 40, 768, 6504),     # clusters of 3, ragged H tile and tokens
+    (2, 300, 1024, 512),    # 256-token tiles with a K split: parts and the split ring kernel
+    (8, 300, 1024, 4224),   # 256-token tiles, no split: bf16 partials and the ring kernel
 ]
 IDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in SHAPES]
 
@@ -109,13 +113,12 @@ def test_mx_reconcile_against_oracle(shape):
 
 def test_mx_limits():
     import tensor_layer_reconciliation_b200 as tlr
-    dev = torch.device("cuda")
-    plan = _plan(2, 8, 1024, 256)
-    x, w, r = inputs(2, 5, 1024, 256, 5, dev)
-    q, sc = plan.pack_weights_mxfp8(w)
-    out = torch.empty(5, 256, dtype=torch.bfloat16, device=dev)
-    st = tlr.tp_rowlinear_reconcile_mxfp8(plan.handle, x.data_ptr(), q.data_ptr(), sc.data_ptr(),
-                                          r.data_ptr(), out.data_ptr(), 5, 0)
-    assert st == tlr.TP_ERR_UNSUPPORTED                  # five tokens: not a decode step here
     plan48 = _plan(2, 1, 96, 256)                        # K/N = 48: not whole 32-weight blocks
     assert tlr.tp_plan_mxfp8_bytes(plan48.handle)[0] == tlr.TP_ERR_UNSUPPORTED
+    plan96 = _plan(1, 1, 96, 256)                        # K/N = 96: 32-weight runs, not 64-column blocks
+    assert tlr.tp_plan_mxfp8_bytes(plan96.handle)[0] == tlr.TP_ERR_UNSUPPORTED
+    assert tlr.tp_rowlinear_reconcile_mxfp8(plan96.handle, 256, 512, 768, 1024, 1280, 1, 0,
+                                            0) == tlr.TP_ERR_UNSUPPORTED
+    plan = _plan(8, 64, 1024, 4096)
+    assert plan.mxfp8_workspace_bytes(64) == 0           # folds in clusters: nothing staged
+    assert _plan(2, 1, 1024, 512).mxfp8_workspace_bytes(1) > 0   # k-split parts and counters

@@ -52,6 +52,14 @@ SHAPES = [             # N, M, K, H
     (8, 512, 1024, 4096),   # prefill-sized: CTA pairs (2-SM MMA), 16 H-tile pairs, 2 token tiles
     (8, 300, 1024, 4224),   # CTA pairs, odd H-tile count (last pair half out of range), ragged tokens
     (1, 260, 512, 768),     # CTA pairs for the partials, N = 1, ragged second token tile
+    # units >= SMs, no k-split: the N ranks of a tile fold on chip in a cluster of N CTAs
+    (8, 64, 1024, 4096),    # clusters of 8, one tile each
+    (4, 32, 1024, 5120),    # clusters of 4
+    (3, 40, 768, 6504),     # clusters of 3 (tokens per CTA 22, 22, 20), ragged H tile and tokens
+    (2, 100, 512, 10240),   # 128-token tile, one CTA per SM: some clusters fold two tiles
+    (8, 64, 512, 8192),     # 64 tiles on 37 clusters: the shared partial tile is reused
+    (1, 16, 256, 19200),    # N = 1: a cluster of one CTA
+    (8, 1, 1024, 4096),     # one token without a k-split: cluster fold, not the counter fold
 ]
 IDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in SHAPES]
 
@@ -175,3 +183,16 @@ def test_fold_counters_return_to_zero():
             assert torch.equal(out.view(torch.int16), fresh.view(torch.int16))
             assert int(torch.count_nonzero(ws[:counter_bytes])) == 0
     assert plan.launches(3) == 2                       # from three tokens: a ring kernel follows
+
+
+def test_cluster_fold_needs_no_workspace():
+    """Without a k-split the N ranks of a tile fold on chip: one kernel per
+    call, no staged partials, so no workspace."""
+    import tensor_layer_reconciliation_b200 as tlr
+    for n, m, k, h in [(8, 64, 1024, 4096), (4, 32, 1024, 5120), (8, 1, 1024, 4096)]:
+        plan = tlr.Plan(n, m, k, h)
+        assert plan.launches(m) == 1 and plan.workspace_bytes(m) == 0, (n, m, k, h)
+        x, w, r = inputs(n, m, k, h, 5, torch.device("cuda"))
+        out = plan.reconcile(x, plan.pack_weights(w), r)
+        torch.cuda.synchronize()
+        assert out.shape == (m, h) and plan.device_error_flags() == 0
