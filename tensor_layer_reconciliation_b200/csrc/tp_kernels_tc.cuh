@@ -352,9 +352,11 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             if (MX) tma_prefetch_desc(&tmap_s);
             const uint32_t tx = kWTile + kBTile + kSTile;
             // The weights of one k-block (and, MX, their scales) into stage st.
+            // (NVFP4 code tiles hold two codes a byte: 32 bytes per 64-column block)
+            constexpr int kWCols = FMT == kFmtNvfp4 ? kTcKBlock / 2 : kTcKBlock;
             auto load_w = [&](int st, int kb_, int ht_, int r_) {
                 tma_load_3d(a_ring + static_cast<size_t>(st) * kWTile, &tmap_w, &full[st],
-                            kb_ * kTcKBlock, ht_ * kTcRows, r_);
+                            kb_ * kWCols, ht_ * kTcRows, r_);
                 if (MX)   // MXFP8: 256 bytes from byte ht*256; NVFP4: 128 words from word ht*128
                     tma_load_3d(s_ring + static_cast<size_t>(st) * kSTile, &tmap_s, &full[st],
                                 FMT == kFmtMxfp8 ? ht_ * kTcRows * 2 : ht_ * kTcRows, kb_, r_);
