@@ -34,12 +34,12 @@
 // Units run token tile fastest, so CTAs working at the same time share each
 // weight tile through L2 (a tile of weights serves every token tile of a call).
 // Folding (S2-S4) inside this kernel, two ways:
-//  * cluster fold (no k-split): the N CTAs of a thread-block cluster are the
-//    N ranks of one (H tile, token tile). Each rounds its accumulator to a
-//    bf16 partial tile in its own shared memory; after an mbarrier handshake
-//    across the cluster each CTA folds BN/N of the tile's tokens, reading the
-//    N partials of every output through the cluster's shared window in ring
-//    order, and adds the residual. The partials never leave the chip and the
+//  * cluster fold (N * SPLITS <= 8): the C = N * SPLITS CTAs of a thread-block
+//    cluster are the N ranks (and K parts) of one (H tile, token tile). Each
+//    keeps its accumulator (a bf16 partial, or an fp32 part sum) in its own
+//    shared memory; after an mbarrier handshake across the cluster each CTA
+//    folds 1/C of the tile's outputs, reading the parts of every output through
+//    the cluster's shared window in ring order, and adds the residual. The partials never leave the chip and the
 //    fold work is spread over all N CTAs (CTAs of a cluster run at the same
 //    time, so the waits between them always end).
 //  * counter fold (one or two tokens with a k-split): the CTA that stores the
@@ -115,53 +115,84 @@ struct TcParams {
     const int* nv_gexp;           // NVFP4: the second-level exponent g
 };
 
-// Cluster fold of one (H tile, token tile): this CTA (rank `crank` of a
-// cluster of N = csize) folds tokens [crank * T, (crank + 1) * T) of the tile,
-// T = ceil(BN / N), all 128 rows, 8 columns (16 bytes) per thread step: the
-// N partial vectors are read from the CTAs' part_buf tiles ([BN][128] bf16)
-// in ring order from the chunk's owner, all loads before the first add, then
-// the residual is added and the output stored. et = epilogue thread, 0..127.
-__device__ __forceinline__ void cluster_fold_tile(const TcParams& p, const uint16_t* part_buf,
+// Cluster fold of one (H tile, token tile). The cluster's C = N * SPLITS CTAs
+// hold, in shared memory, the tile's partial of rank q / SPLITS over K part
+// q % SPLITS (CTA q of the cluster): bf16 [T][128] when SPLITS == 1 (the
+// partial itself), fp32 [T][128] sums of the part otherwise (T = the tile's
+// tokens, at most BN). The tile's T x 16 vectors of 8 rows are shared out
+// evenly; for each, rank r's partial is the fp32 sum of its parts in split
+// (k-ascending) order rounded once to bf16, the N partials are added in ring
+// order from the chunk's owner (all loads before the first add), then the
+// residual, and the output is stored. et = epilogue thread, 0..127.
+// Eight ring adds at once (a on the left): bf16 round-to-nearest-even each.
+__device__ __forceinline__ uint4 bf16x8_add_tc(uint4 a, uint4 b) {
+    return make_uint4(bf16x2_add(a.x, b.x), bf16x2_add(a.y, b.y), bf16x2_add(a.z, b.z),
+                      bf16x2_add(a.w, b.w));
+}
+
+template <int SPLITS>
+__device__ __forceinline__ void cluster_fold_tile(const TcParams& p, const void* part_buf,
                                                   uint32_t crank, int csize, int ht, int m0,
                                                   int bn, int et) {
-    const int n = csize;
-    const int t_per = (bn + n - 1) / n;
+    const int n = p.n_ranks;
+    const int t_tile = min(bn, p.tokens - m0);                      // tokens of this tile
+    const int nv = t_tile * (kTcRows / 8);
+    const int v0 = static_cast<int>(crank) * nv / csize, v1 = (static_cast<int>(crank) + 1) * nv / csize;
 #pragma unroll 1
-    for (int v = et; v < t_per * (kTcRows / 8); v += 128) {
-        const int tt = static_cast<int>(crank) * t_per + (v >> 4);   // token in the tile
-        const int hv = (v & 15) * 8;                                 // row offset in the tile
+    for (int v = v0 + et; v < v1; v += 128) {
+        const int tt = v >> 4;                                      // token in the tile
+        const int hv = (v & 15) * 8;                                // row offset in the tile
         const int m = m0 + tt;
         const int h = ht * kTcRows + hv;
-        if (tt >= bn || m >= p.tokens || h >= p.hidden) continue;
+        if (h >= p.hidden) continue;
         const int c = h / p.hc;
-        const uint16_t* mine = part_buf + tt * kTcRows + hv;
-        uint4 pv[kMaxRanks];
+        uint4 sum;
+        if constexpr (SPLITS == 1) {
+            const uint16_t* mine = static_cast<const uint16_t*>(part_buf) + tt * kTcRows + hv;
+            uint4 pv[kMaxRanks];
 #pragma unroll
-        for (int i = 0; i < kMaxRanks; ++i) {
-            if (i < n) {
-                int rr = c + i;   // ring order: the chunk's owner first
+            for (int i = 0; i < kMaxRanks; ++i) {
+                if (i < n) {
+                    int rr = c + i;   // ring order: the chunk's owner first
+                    if (rr >= n) rr -= n;
+                    pv[i] = ld_dsmem_v4(mapa_shared(mine, static_cast<uint32_t>(rr)));
+                }
+            }
+            sum = pv[0];
+#pragma unroll
+            for (int i = 1; i < kMaxRanks; ++i)
+                if (i < n) sum = bf16x8_add_tc(sum, pv[i]);
+        } else {
+            static_assert(SPLITS >= 2 && SPLITS <= 4, "cluster of at most 8 CTAs");
+            // rank by rank in ring order (the parts of a rank loaded together)
+            const float* mine = static_cast<const float*>(part_buf) + tt * kTcRows + hv;
+#pragma unroll 1
+            for (int i = 0; i < n; ++i) {
+                int rr = c + i;
                 if (rr >= n) rr -= n;
-                pv[i] = ld_dsmem_v4(mapa_shared(mine, static_cast<uint32_t>(rr)));
+                uint4 a[SPLITS][2];
+#pragma unroll
+                for (int sp = 0; sp < SPLITS; ++sp) {
+                    const uint32_t base = mapa_shared(mine, static_cast<uint32_t>(rr * SPLITS + sp));
+                    a[sp][0] = ld_dsmem_v4(base);
+                    a[sp][1] = ld_dsmem_v4(base + 16);
+                }
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float((&a[0][e >> 2].x)[e & 3]);
+#pragma unroll
+                for (int sp = 1; sp < SPLITS; ++sp)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        f[e] = __fadd_rn(f[e], __uint_as_float((&a[sp][e >> 2].x)[e & 3]));
+                const uint4 pr = make_uint4(bf16x2_from_f32(f[0], f[1]), bf16x2_from_f32(f[2], f[3]),
+                                            bf16x2_from_f32(f[4], f[5]), bf16x2_from_f32(f[6], f[7]));
+                sum = i == 0 ? pr : bf16x8_add_tc(sum, pr);
             }
         }
         const size_t o = static_cast<size_t>(m) * p.hidden + h;
         const uint4 rv = ld_global_nc_v4(p.residual + o);
-        uint4 sum = pv[0];
-#pragma unroll
-        for (int i = 1; i < kMaxRanks; ++i) {
-            if (i < n) {
-                sum.x = bf16x2_add(sum.x, pv[i].x);
-                sum.y = bf16x2_add(sum.y, pv[i].y);
-                sum.z = bf16x2_add(sum.z, pv[i].z);
-                sum.w = bf16x2_add(sum.w, pv[i].w);
-            }
-        }
-        uint4 out;
-        out.x = bf16x2_add(rv.x, sum.x);
-        out.y = bf16x2_add(rv.y, sum.y);
-        out.z = bf16x2_add(rv.z, sum.z);
-        out.w = bf16x2_add(rv.w, sum.w);
-        st_global_v4(p.out + o, out);
+        st_global_v4(p.out + o, bf16x8_add_tc(rv, sum));
     }
 }
 
@@ -281,7 +312,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     // Cluster fold: cluster c takes tiles c, c + clusters, ...; its CTA of rank
     // r (in the cluster) computes rank r's partial of each.
     constexpr bool kCluster = MODE == kTcClusterFold;
-    const int csize = kCluster ? p.n_ranks : 1;
+    const int csize = kCluster ? p.n_ranks * p.splits : 1;
     const uint32_t crank = kCluster ? cluster_ctarank() : 0u;
     const int cid = static_cast<int>(blockIdx.x) / csize;
     const int n_clusters = static_cast<int>(gridDim.x) / csize;
@@ -293,12 +324,12 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                               : 0);
     // unit index -> (rank, h tile, m tile, split); token tile fastest
     auto unit_of = [&](int lu, int& r, int& ht, int& mt, int& sp) {
-        if (kCluster) {
+        if (kCluster) {   // CTA q of the cluster: rank q / SPLITS, K part q % SPLITS
             const int t = cid + lu * n_clusters;
             mt = t % p.m_tiles;
             ht = t / p.m_tiles;
-            r = static_cast<int>(crank);
-            sp = 0;
+            r = static_cast<int>(crank) / p.splits;
+            sp = static_cast<int>(crank) - r * p.splits;
             return;
         }
         const int u = static_cast<int>(blockIdx.x) + lu * static_cast<int>(gridDim.x);
@@ -530,11 +561,21 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                                    static_cast<uint32_t>(b * BN + c0),
                                v);
                 if (kCluster) {
-                    // [token][row] in shared memory: lanes write 32 consecutive rows
-                    uint16_t* dst = part_buf + static_cast<size_t>(c0) * kTcRows + q * 32 + lane;
+                    // [token][row] in shared memory, the tile's tokens only: lanes
+                    // write 32 consecutive rows; bf16 partials, or fp32 part sums
+                    const int t_tile = min(BN, p.tokens - m0);
+                    const int row = q * 32 + lane;
+                    if (p.splits == 1) {
+                        uint16_t* dst = part_buf + static_cast<size_t>(c0) * kTcRows + row;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        dst[i * kTcRows] = f32_to_bf16_rne(__uint_as_float(v[i]));
+                        for (int i = 0; i < 32; ++i)
+                            if (c0 + i < t_tile) dst[i * kTcRows] = f32_to_bf16_rne(__uint_as_float(v[i]));
+                    } else {
+                        float* dst = reinterpret_cast<float*>(part_buf) + static_cast<size_t>(c0) * kTcRows + row;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (c0 + i < t_tile) dst[i * kTcRows] = __uint_as_float(v[i]);
+                    }
                 } else if (h < p.hidden) {
                     if (p.splits == 1) {
                         uint16_t* dst = p.partials + static_cast<size_t>(r) * plane + h;
@@ -571,7 +612,11 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 if (!mbar_wait_cluster_bounded(fold_ready, static_cast<uint32_t>(lu) & 1u))
                     atomicExch(&abort_flag, 1);
                 else
-                    cluster_fold_tile(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
+                    // 1 .. 4 K parts, N * parts <= 8 (the host launches no other cluster fold)
+                    if (p.splits == 1) cluster_fold_tile<1>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
+                    else if (p.splits == 2) cluster_fold_tile<2>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
+                    else if (p.splits == 3) cluster_fold_tile<3>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
+                    else cluster_fold_tile<4>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
                 // All reads of the peers' tiles are done: free them for the next unit.
                 asm volatile("bar.sync 2, 128;" ::: "memory");
                 if (warp == 2 && lane == 0) {

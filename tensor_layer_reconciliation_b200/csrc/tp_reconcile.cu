@@ -249,8 +249,9 @@ int tc_token_tile(int64_t tokens) {
 }
 
 // allow_split: the call folds (S2-S4) in this library, so K may be split
-// across CTAs when there are fewer units than SMs; such calls without a split
-// and with a token tile of at most 128 fold on chip in clusters of N CTAs.
+// across CTAs when there are fewer units than SMs; calls with a token tile of
+// at most 128 whose N ranks x K parts make at most 8 CTAs (at most 4 parts)
+// fold on chip in clusters of those CTAs.
 TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt = tpr::kFmtBf16) {
     TcConfig c{};
     c.bn = tc_token_tile(tokens);
@@ -266,13 +267,19 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     c.splits = 1;
     if (allow_split && base_units > 0 && base_units < p->sm_count)
         c.splits = std::max(1, std::min({slots / base_units, nkb, tpr::kMaxSplits}));
-    c.cluster_fold = allow_split && base_units > 0 && c.splits == 1 && c.bn <= 128;
+    // cluster fold: the N ranks x K parts of a tile in one portable cluster
+    c.cluster_fold = allow_split && base_units > 0 && c.bn <= 128 && c.splits <= 4 &&
+                     p->n_ranks * c.splits <= 8;
     // Quantised weights: a stage holds codes, scales and activations; two
     // converted bf16 tiles sit beside the ring.
     const bool quantised = fmt != tpr::kFmtBf16;
     const size_t stage = tpr::fmt_code_tile(fmt) + tpr::fmt_scale_tile(fmt) +
                          static_cast<size_t>(c.bn) * tpr::kTcKBlock * 2;
-    const size_t part_tile = c.cluster_fold ? static_cast<size_t>(c.bn) * tpr::kTcRows * 2 : 0;
+    // the cluster fold's tile in shared memory: the tile's tokens x 128 rows,
+    // bf16 partials or fp32 part sums
+    const size_t part_tile = c.cluster_fold ? static_cast<size_t>(std::min<int64_t>(c.bn, tokens)) *
+                                                  tpr::kTcRows * (c.splits > 1 ? 4 : 2)
+                                            : 0;
     const size_t fixed = (2 * tpr::kTcMaxStages + 11) * sizeof(uint64_t) + 16 + 128 + 1024 + part_tile +
                          (quantised ? 2 * tpr::kTcATile : 0);
     const size_t budget = std::min<size_t>(two_per_sm ? 110 * 1024 : 200 * 1024,
@@ -283,9 +290,10 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     c.smem = fixed + static_cast<size_t>(c.stages) * stage;
     c.units = base_units * c.splits;
     if (c.cluster_fold) {
-        // clusters of N CTAs, one per (H tile, token tile) at a time
+        // clusters of N * splits CTAs, one per (H tile, token tile) at a time
         const int tiles = c.h_tiles * c.m_tiles;
-        c.grid = p->n_ranks * std::max(1, std::min(tiles, slots / p->n_ranks));
+        const int cl = p->n_ranks * c.splits;
+        c.grid = cl * std::max(1, std::min(tiles, slots / cl));
     } else {
         c.grid = std::min(c.units, slots);
     }
@@ -518,7 +526,7 @@ tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* 
                       ? reinterpret_cast<const int*>(static_cast<const uint8_t*>(wt.scales) + nv_scale_bytes(p))
                       : nullptr;
     const int mode = c.cluster_fold ? tpr::kTcClusterFold : fold ? tpr::kTcCounterFold : tpr::kTcStore;
-    const int cl = c.cluster_fold ? p->n_ranks : 1;
+    const int cl = c.cluster_fold ? p->n_ranks * c.splits : 1;
     const dim3 grid(c.grid);
     const cudaError_t e =
         wt.fmt == tpr::kFmtMxfp8   ? dispatch_tc<tpr::kFmtMxfp8>(c.bn, mode, grid, c.smem, stream, cl, mw, mx, ms, prm)
@@ -652,9 +660,10 @@ int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens) {
     return effective_variant(plan, tokens);
 }
 
-// The tensor path folds inside its partial kernel up to this many tokens
-// with a k-split (counter fold); without a split, at any token tile up to
-// 128, the kernel folds in clusters of N CTAs (cluster fold).
+// The tensor path folds inside its partial kernel: in clusters of the N ranks
+// x K parts of a tile when they make at most 8 CTAs and the token tile is at
+// most 128 (cluster fold), else up to this many tokens by the CTA completing
+// a tile (counter fold).
 constexpr int64_t kFoldMaxTokens = 2;
 
 static bool tc_cluster_folds(const tp_plan* plan, int64_t tokens) {

@@ -25,12 +25,13 @@ from helpers import u16
 pytestmark = pytest.mark.gpu
 
 TENSOR_SHAPES = [      # N, M, K, H
-    (2, 1, 2048, 512),      # one token: fold inside the partial kernel
+    (2, 1, 2048, 512),      # one token, 2 ranks x 8 parts: the counter fold
     (4, 3, 2048, 640),      # three tokens: k-split parts and the split ring kernel
     (4, 32, 1024, 512),     # 32 tokens, 16 units: k-split parts and the split ring kernel
     (8, 300, 1024, 4224),   # 300 tokens: CTA pairs and the ring kernel
     (8, 64, 1024, 4096),    # 64 tokens, 256 units: fold on chip in clusters of 8
     (3, 40, 768, 6504),     # clusters of 3, ragged last H tile and token tile
+    (2, 1, 5120, 5120),     # clusters of 2 ranks x 3 K parts (fp32 parts folded on chip)
 ]
 TIDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in TENSOR_SHAPES]
 

@@ -60,6 +60,11 @@ SHAPES = [             # N, M, K, H
     (8, 64, 512, 8192),     # 64 tiles on 37 clusters: the shared partial tile is reused
     (1, 16, 256, 19200),    # N = 1: a cluster of one CTA
     (8, 1, 1024, 4096),     # one token without a k-split: cluster fold, not the counter fold
+    # a k-split whose N ranks x parts make at most 8 CTAs: the cluster folds fp32 parts
+    (2, 1, 5120, 5120),     # the decode example's out-projection: 2 ranks x 3 parts
+    (4, 1, 4096, 4096),     # 4 ranks x 2 parts
+    (2, 3, 2048, 4096),     # 2 ranks x 4 parts, three tokens
+    (1, 1, 512, 10240),     # N = 1: 3 parts
 ]
 IDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in SHAPES]
 
@@ -186,10 +191,11 @@ def test_fold_counters_return_to_zero():
 
 
 def test_cluster_fold_needs_no_workspace():
-    """Without a k-split the N ranks of a tile fold on chip: one kernel per
-    call, no staged partials, so no workspace."""
+    """When the N ranks x K parts of a tile make at most 8 CTAs they fold on
+    chip in one cluster: one kernel per call, nothing staged, no workspace."""
     import tensor_layer_reconciliation_b200 as tlr
-    for n, m, k, h in [(8, 64, 1024, 4096), (4, 32, 1024, 5120), (8, 1, 1024, 4096)]:
+    for n, m, k, h in [(8, 64, 1024, 4096), (4, 32, 1024, 5120), (8, 1, 1024, 4096),
+                       (2, 1, 5120, 5120), (2, 3, 2048, 4096)]:
         plan = tlr.Plan(n, m, k, h)
         assert plan.launches(m) == 1 and plan.workspace_bytes(m) == 0, (n, m, k, h)
         x, w, r = inputs(n, m, k, h, 5, torch.device("cuda"))
