@@ -132,8 +132,9 @@ class Workload:
         self.res_all = torch.empty(cfg.n_points * m * h, dtype=torch.bfloat16, device=device)
         self.out_all = torch.empty(cfg.n_points * m * h, dtype=torch.bfloat16, device=device)
         self.w_packed = []
-        ws_need = max({"mxfp8": pl.mxfp8_workspace_bytes, "nvfp4": pl.nvfp4_workspace_bytes}.get(
-            weights, pl.workspace_bytes)(m) for pl in self.plans.values())
+        ws_fn = {"mxfp8": "mxfp8_workspace_bytes", "nvfp4": "nvfp4_workspace_bytes"}.get(
+            weights, "workspace_bytes")
+        ws_need = max(getattr(pl, ws_fn)(m) for pl in self.plans.values())
         self.workspace = (torch.zeros(ws_need, dtype=torch.uint8, device=device)
                           if ws_need else None)   # counter head zero on first use
         for i, p in enumerate(cfg.points):

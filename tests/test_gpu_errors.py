@@ -25,7 +25,7 @@ from gpu_util import inputs
 pytestmark = pytest.mark.gpu
 
 SENT = 0x7BCD
-N, M, K, H = 2, 4, 256, 128          # tensor-core path: a workspace is needed
+N, M, K, H = 4, 4, 1024, 128         # tensor cores, K split 4 ways, a ring kernel: a workspace
 
 
 @pytest.fixture(scope="module")

@@ -154,10 +154,10 @@ def test_tensor_gaussian_fragile_rule(shape):
 
 def test_auto_uses_tensor_cores():
     import tensor_layer_reconciliation_b200 as tlr
-    plan = tlr.Plan(2, 64, 256, 128)                   # AUTO
+    plan = tlr.Plan(2, 64, 4096, 1024)                 # AUTO
     assert plan.effective_variant(1) == "tensor"
     assert plan.effective_variant(64) == "tensor"
-    assert plan.workspace_bytes(1) > 0                 # tensor: staged partials
+    assert plan.workspace_bytes(1) > 0                 # tensor, 2 ranks x 8 K parts: counter fold
     plan.set_variant("exact")
     assert plan.effective_variant(1) == "exact"
     assert plan.workspace_bytes(1) == 0                # exact, fused: no workspace
