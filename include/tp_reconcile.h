@@ -92,18 +92,17 @@ TP_API tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, 
  *            ring fold and residual add (no workspace); 1 writes all N
  *            partials to the workspace and a separate ring kernel
  *            (tp_ring_reduce's) folds them. TENSOR (and AUTO) ignore it:
- *            they always write their partials to the workspace; with one
- *            or two tokens the partial kernel itself folds them (the CTA
- *            that stores the last part of a tile folds that tile), from
- *            three tokens up a ring kernel follows.
+ *            see tp_plan_launches and tp_plan_workspace_bytes for where
+ *            their partials go.
  * Call before the plan is shared between threads. */
 TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
 
 /* Bytes of workspace tp_rowlinear_reconcile needs for `tokens` tokens with
  * the plan's current setting; 0 when the partials stay on chip (EXACT, not
- * staged). The tensor-core variant always writes its partials to the
- * workspace, whether its own kernel folds them (one or two tokens) or a
- * ring kernel does: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of K
+ * staged; TENSOR folding across a cluster). Otherwise the tensor-core
+ * variant writes its partials to the workspace, whether its own kernel
+ * folds them (the CTA completing a tile, one or two tokens) or a ring
+ * kernel does: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of K
  * parts) when it splits K across CTAs to fill the SMs. Layout: a counter
  * block of one 32-bit counter per 128-row H tile (256-byte rounded; the
  * in-kernel fold counts stored parts there), then the partials. Rounded up
@@ -116,9 +115,11 @@ TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 TP_API int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens);
 
 /* Kernels one tp_rowlinear_reconcile call with `tokens` tokens launches under
- * the plan's current setting: 1 (EXACT not staged; TENSOR with 1 or 2 tokens,
- * which folds inside its partial kernel) or 2 (a partial kernel, then a ring
- * fold kernel); 0 for tokens = 0; -1 for a null plan or tokens < 0. */
+ * the plan's current setting: 1 (EXACT not staged; TENSOR when its partial
+ * kernel folds on chip: across a cluster of the N ranks x K parts of a tile
+ * when they make at most 8 CTAs and the token tile is at most 128, or by the
+ * CTA completing a tile for 1 or 2 tokens) or 2 (a partial kernel, then a
+ * ring fold kernel); 0 for tokens = 0; -1 for a null plan or tokens < 0. */
 TP_API int tp_plan_launches(const tp_plan* plan, int64_t tokens);
 
 /* Bytes of the packed weight buffer tp_pack_weights writes: N*H*(K/N)*2,
