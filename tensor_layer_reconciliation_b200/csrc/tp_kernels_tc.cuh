@@ -203,12 +203,16 @@ __device__ __forceinline__ void cluster_fold_tile(const TcParams& p, const void*
 // rounded to bf16 (exact for values bf16 holds). The row's four 16-code
 // chunks are visited starting at a row-dependent one, so the eight rows a
 // quarter-warp reads at once fall in different shared-memory banks.
+// NC = 4 converts the whole row; NC = 2 the half `part` (chunks 2part, 2part+1),
+// with the visiting order rotated by `rot` so that the rows a quarter-warp
+// reads at once fall in different banks.
+template <int NC>
 __device__ __forceinline__ void mx_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
-                                               uint8_t* a_row, int t) {
+                                               uint8_t* a_row, int t, int part, int rot) {
     const float sc[2] = {e8m0_to_f32(scale_row[0]), e8m0_to_f32(scale_row[1])};
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-        const int c = (cc + (t >> 1)) & 3;                 // codes 16c .. 16c+15
+    for (int cc = 0; cc < NC; ++cc) {
+        const int c = NC * part + ((cc + rot) & (NC - 1));  // codes 16c .. 16c+15
         const uint4 q = *reinterpret_cast<const uint4*>(code_row + c * 16);
         const float scale = sc[c >> 1];
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};
@@ -241,16 +245,18 @@ __device__ __forceinline__ uint32_t f16x2_from_e2m1x2(uint32_t b) {
 // nibble), the row's four E4M3 block scales (one per 16 values) and the
 // second-level factor 2^g -> the row of a bf16 A tile as in mx_convert_row.
 // The row's two 16-byte halves are read starting at a row-dependent one.
+// NH = 2 converts the whole row; NH = 1 the half `part`.
+template <int NH>
 __device__ __forceinline__ void nv_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
-                                               float two_g, uint8_t* a_row, int t) {
+                                               float two_g, uint8_t* a_row, int t, int part, int rot) {
     const uint32_t sw = *reinterpret_cast<const uint32_t*>(scale_row);
     float sc[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         sc[i] = f16_lo_to_f32(f16x2_from_e4m3x2(static_cast<uint16_t>((sw >> (8 * i)) & 0xFF))) * two_g;
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int c = (hh + (t >> 2)) & 1;                 // codes 32c .. 32c+31
+    for (int hh = 0; hh < NH; ++hh) {
+        const int c = NH == 2 ? ((hh + rot) & 1) : part;   // codes 32c .. 32c+31
         const uint4 q = *reinterpret_cast<const uint4*>(code_row + c * 16);
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};        // 8 codes a word
 #pragma unroll
@@ -345,6 +351,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         kb_lo = sp * nkb / p.splits;
         kb_hi = (sp + 1) * nkb / p.splits;
     };
+    // quantised weights, one unit: the 4 epilogue warps also convert (8 converter warps)
+    const bool cvt_helpers = MX && my_units == 1;
     if (threadIdx.x == 0) {
         abort_flag = 0;
         for (int s = 0; s < S; ++s) {
@@ -359,7 +367,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         mbar_init(fold_ready, static_cast<uint32_t>(csize));
         mbar_init(fold_freed, static_cast<uint32_t>(csize));
         for (int j = 0; j < 2; ++j) {
-            mbar_init(&cvt_full[j], 4);
+            mbar_init(&cvt_full[j], cvt_helpers ? 8 : 4);
             mbar_init(&cvt_empty[j], 1);
         }
         fence_barrier_init();
@@ -374,6 +382,50 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
     pdl_launch_dependents();
+
+    // Converter u (0 .. 127, or 0 .. 255 with the helpers) widens its share of
+    // every staged code tile, in issue order: row u (whole), or row u / 2 (half
+    // u % 2) with the helpers.
+    auto run_converters = [&](int u) {
+        if constexpr (MX) {
+            const float two_g = FMT == kFmtNvfp4 ? ldexpf(1.0f, *p.nv_gexp) : 1.0f;
+            const int row = cvt_helpers ? u >> 1 : u;
+            const int part = cvt_helpers ? u & 1 : 0;
+            int i = 0;
+            bool ok = true;
+            for (int lu = 0; lu < my_units && ok; ++lu) {
+                int r, ht, mt, sp, kb_lo, kb_hi;
+                unit_of(lu, r, ht, mt, sp);
+                split_range(sp, kb_lo, kb_hi);
+                for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
+                    const int s = i % S, j = i & 1;
+                    ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / S) & 1u) &&
+                         mbar_wait_bounded(&cvt_empty[j], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u);
+                    if (!__all_sync(0xFFFFFFFFu, ok) ||
+                        *reinterpret_cast<volatile int*>(&abort_flag) != 0) {
+                        ok = false;
+                        atomicExch(&abort_flag, 1);
+                        break;
+                    }
+                    const uint8_t* srow = s_ring + static_cast<size_t>(s) * kSTile;
+                    uint8_t* arow = a_cvt + static_cast<size_t>(j) * kTcATile + row * 128;
+                    if (FMT == kFmtMxfp8) {
+                        const uint8_t* crow = a_ring + static_cast<size_t>(s) * kWTile + row * kTcKBlock;
+                        if (cvt_helpers) mx_convert_row<2>(crow, srow + row * 2, arow, row, part, u >> 2);
+                        else mx_convert_row<4>(crow, srow + row * 2, arow, row, 0, row >> 1);
+                    } else {
+                        const uint8_t* crow = a_ring + static_cast<size_t>(s) * kWTile + row * (kTcKBlock / 2);
+                        if (cvt_helpers) nv_convert_row<1>(crow, srow + row * 4, two_g, arow, row, part, 0);
+                        else nv_convert_row<2>(crow, srow + row * 4, two_g, arow, row, 0, row >> 2);
+                    }
+                    // generic-proxy writes, read next by the tensor core (async proxy)
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if ((threadIdx.x & 31) == 0) mbar_arrive(&cvt_full[j]);
+                }
+            }
+        }
+    };
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer --
@@ -498,42 +550,12 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         }
     } else if (MX && warp >= 6) {
         // ------------------------------------ converters (quantised weights) --
-        // Thread t converts row t of every staged code tile, in issue order.
-        const int t = static_cast<int>(threadIdx.x) - 192;
-        // NVFP4: the second-level factor 2^g, an exponent the packing stored
-        const float two_g = FMT == kFmtNvfp4 ? ldexpf(1.0f, *p.nv_gexp) : 1.0f;
-        int i = 0;
-        bool ok = true;
-        for (int lu = 0; lu < my_units && ok; ++lu) {
-            int r, ht, mt, sp, kb_lo, kb_hi;
-            unit_of(lu, r, ht, mt, sp);
-            split_range(sp, kb_lo, kb_hi);
-            for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
-                const int s = i % S, j = i & 1;
-                ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / S) & 1u) &&
-                     mbar_wait_bounded(&cvt_empty[j], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u);
-                if (!__all_sync(0xFFFFFFFFu, ok) ||
-                    *reinterpret_cast<volatile int*>(&abort_flag) != 0) {
-                    ok = false;
-                    atomicExch(&abort_flag, 1);
-                    break;
-                }
-                if (FMT == kFmtMxfp8)
-                    mx_convert_row(a_ring + static_cast<size_t>(s) * kWTile + t * kTcKBlock,
-                                   s_ring + static_cast<size_t>(s) * kSTile + t * 2,
-                                   a_cvt + static_cast<size_t>(j) * kTcATile + t * 128, t);
-                else
-                    nv_convert_row(a_ring + static_cast<size_t>(s) * kWTile + t * (kTcKBlock / 2),
-                                   s_ring + static_cast<size_t>(s) * kSTile + t * 4, two_g,
-                                   a_cvt + static_cast<size_t>(j) * kTcATile + t * 128, t);
-                // generic-proxy writes, read next by the tensor core (async proxy)
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&cvt_full[j]);
-            }
-        }
+        run_converters(static_cast<int>(threadIdx.x) - 192);
     } else {
         // ---------------------------------------------------------- epilogue --
+        // A CTA with one unit has nothing for these warps until its MMAs end:
+        // they convert the second half of every code tile meanwhile.
+        if (MX && cvt_helpers) run_converters(static_cast<int>(threadIdx.x) - 64 + 128);
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         pdl_wait();  // the fold reads the residual and writes the output in stream order
         for (int lu = 0; lu < my_units; ++lu) {
