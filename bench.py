@@ -737,7 +737,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="all", choices=["all"] + CONFIG_ORDER,
                     help="one workload, or all four benchmarked ones (headline: decode_n2)")
-    ap.add_argument("--variant", default="auto", choices=["auto", "exact", "tensor"])
+    ap.add_argument("--variant", default="auto", choices=["auto", "exact", "tensor", "cluster"])
     ap.add_argument("--staged", action="store_true")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp8", "nvfp4"],
                     help="mxfp8: E4M3 codes, E8M0 scales per 32 weights; nvfp4: E2M1 codes, "

@@ -68,9 +68,20 @@ typedef enum {
 enum { TP_BF16 = 0 };
 
 typedef enum {
-    TP_VARIANT_AUTO = 0,   /* TENSOR (the fastest on B200 at every token count) */
-    TP_VARIANT_EXACT = 1,  /* CUDA cores, fp32 FMA chain per partial, k ascending */
-    TP_VARIANT_TENSOR = 2  /* tcgen05 tensor cores, fp32 accumulate in TMEM */
+    TP_VARIANT_AUTO = 0,    /* TENSOR (the fastest on B200 at every token count) */
+    TP_VARIANT_EXACT = 1,   /* CUDA cores, fp32 FMA chain per partial, k ascending */
+    TP_VARIANT_TENSOR = 2,  /* tcgen05 tensor cores, fp32 accumulate in TMEM; the
+                               partials go through the workspace (folded by the
+                               CTA completing a tile for 1-2 tokens, else by a
+                               ring kernel) */
+    TP_VARIANT_CLUSTER = 3  /* the TENSOR kernels, folding the ranks on chip where
+                               the N ranks x K parts of a tile make at most 8 CTAs
+                               (at most 4 parts) and the token tile is at most 128:
+                               one cluster of those CTAs, partials exchanged
+                               through distributed shared memory, no workspace.
+                               One kernel per call, but its CTAs stay until the
+                               whole cluster has folded: in a chain of calls
+                               slower than TENSOR on B200 */
 } tp_variant;
 
 /* Creates a plan for one projection shape.
@@ -110,7 +121,8 @@ TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
 TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 
 /* The partial kernel a call with `tokens` tokens runs under the plan's
- * current setting: TP_VARIANT_EXACT or TP_VARIANT_TENSOR (AUTO resolved).
+ * current setting: TP_VARIANT_EXACT or TP_VARIANT_TENSOR (AUTO and CLUSTER
+ * resolved; CLUSTER runs the tensor-core kernels).
  * Returns -1 for a null plan or tokens < 1. A query only; launches nothing. */
 TP_API int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens);
 

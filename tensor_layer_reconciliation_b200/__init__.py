@@ -9,7 +9,7 @@ include/tp_reconcile.h); this package only binds it.
 """
 
 from ._lib import (EXPORTED, LIB_PATH, TP_BF16, TP_ERR_ALIGN, TP_ERR_CUDA, TP_ERR_INVALID,
-                   TP_ERR_UNSUPPORTED, TP_ERR_WORKSPACE, TP_OK, TP_VARIANT_AUTO, TP_VARIANT_EXACT,
+                   TP_ERR_UNSUPPORTED, TP_ERR_WORKSPACE, TP_OK, TP_VARIANT_AUTO, TP_VARIANT_CLUSTER, TP_VARIANT_EXACT,
                    TP_VARIANT_TENSOR, TPError, tp_device_error_flags, tp_last_cuda_error,
                    tp_pack_weights, tp_plan_create, tp_plan_destroy, tp_plan_set_variant,
                    tp_allreduce_bytes, tp_moe_combine_bytes, tp_pack_weights_mxfp8,
@@ -34,5 +34,5 @@ __all__ = [
     "tp_plan_nvfp4_workspace_bytes", "tp_rowlinear_reconcile_nvfp4",
     "tp_plan_destroy", "tp_status_string", "tp_last_cuda_error", "tp_device_error_flags",
     "TP_OK", "TP_ERR_INVALID", "TP_ERR_ALIGN", "TP_ERR_UNSUPPORTED", "TP_ERR_WORKSPACE",
-    "TP_ERR_CUDA", "TP_BF16", "TP_VARIANT_AUTO", "TP_VARIANT_EXACT", "TP_VARIANT_TENSOR",
+    "TP_ERR_CUDA", "TP_BF16", "TP_VARIANT_AUTO", "TP_VARIANT_EXACT", "TP_VARIANT_TENSOR", "TP_VARIANT_CLUSTER",
 ]

@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libtp_reconcile.so")
 
 TP_OK, TP_ERR_INVALID, TP_ERR_ALIGN, TP_ERR_UNSUPPORTED, TP_ERR_WORKSPACE, TP_ERR_CUDA = range(6)
 TP_BF16 = 0
-TP_VARIANT_AUTO, TP_VARIANT_EXACT, TP_VARIANT_TENSOR = 0, 1, 2
+TP_VARIANT_AUTO, TP_VARIANT_EXACT, TP_VARIANT_TENSOR, TP_VARIANT_CLUSTER = 0, 1, 2, 3
 
 EXPORTED = (
     "tp_plan_create", "tp_plan_set_variant", "tp_plan_workspace_bytes", "tp_plan_kernel_variant", "tp_plan_launches",

@@ -130,10 +130,24 @@ __device__ __forceinline__ uint4 bf16x8_add_tc(uint4 a, uint4 b) {
                       bf16x2_add(a.w, b.w));
 }
 
+// The residual of this thread's first output vector of the cluster fold
+// (zero if it has none), loaded while the cluster's partial tiles are being
+// written, before the handshake.
+__device__ __forceinline__ uint4 cluster_fold_first_residual(const TcParams& p, uint32_t crank, int csize,
+                                                             int ht, int m0, int bn, int et) {
+    const int t_tile = min(bn, p.tokens - m0);
+    const int nv = t_tile * (kTcRows / 8);
+    const int v = static_cast<int>(crank) * nv / csize + et;
+    const int v1 = (static_cast<int>(crank) + 1) * nv / csize;
+    const int h = ht * kTcRows + (v & 15) * 8;
+    if (v >= v1 || h >= p.hidden) return make_uint4(0, 0, 0, 0);
+    return ld_global_nc_v4(p.residual + static_cast<size_t>(m0 + (v >> 4)) * p.hidden + h);
+}
+
 template <int SPLITS>
 __device__ __forceinline__ void cluster_fold_tile(const TcParams& p, const void* part_buf,
                                                   uint32_t crank, int csize, int ht, int m0,
-                                                  int bn, int et) {
+                                                  int bn, int et, uint4 first_res) {
     const int n = p.n_ranks;
     const int t_tile = min(bn, p.tokens - m0);                      // tokens of this tile
     const int nv = t_tile * (kTcRows / 8);
@@ -191,30 +205,28 @@ __device__ __forceinline__ void cluster_fold_tile(const TcParams& p, const void*
             }
         }
         const size_t o = static_cast<size_t>(m) * p.hidden + h;
-        const uint4 rv = ld_global_nc_v4(p.residual + o);
+        const uint4 rv = v == v0 + et ? first_res : ld_global_nc_v4(p.residual + o);
         st_global_v4(p.out + o, bf16x8_add_tc(rv, sum));
     }
 }
 
-// Converts one row of a staged E4M3 code tile (64 codes, row-major, 64
-// bytes) with its two E8M0 scales into the row of a bf16 A tile in the
-// 128-byte-swizzled K-major layout (16-byte chunk q of row t at chunk
-// q ^ (t & 7)): each value is code * 2^s, computed in fp32 (exact) and
-// rounded to bf16 (exact for values bf16 holds). The row's four 16-code
-// chunks are visited starting at a row-dependent one, so the eight rows a
-// quarter-warp reads at once fall in different shared-memory banks.
-// NC = 4 converts the whole row; NC = 2 the half `part` (chunks 2part, 2part+1),
-// with the visiting order rotated by `rot` so that the rows a quarter-warp
-// reads at once fall in different banks.
+// Converts one row of a staged E4M3 code tile (64 codes in a 64-byte row,
+// placed by TMA with the 64-byte swizzle: 16-byte chunk c of row t at chunk
+// c ^ ((t >> 1) & 3)) with its two E8M0 scales into the row of a bf16 A tile
+// in the 128-byte-swizzled K-major layout (chunk q of row t at q ^ (t & 7)):
+// each value is code * 2^s, computed in fp32 (exact) and rounded to bf16
+// (exact for values bf16 holds). With the two swizzles, the eight rows a
+// quarter-warp handles at once read and write eight different bank groups.
+// NC = 4 converts the whole row; NC = 2 its half `part` (chunks 2part, 2part+1).
 template <int NC>
 __device__ __forceinline__ void mx_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
-                                               uint8_t* a_row, int t, int part, int rot) {
-    const float sc[2] = {e8m0_to_f32(scale_row[0]), e8m0_to_f32(scale_row[1])};
+                                               uint8_t* a_row, int t, int part) {
+    const float s0 = e8m0_to_f32(scale_row[0]), s1 = e8m0_to_f32(scale_row[1]);
 #pragma unroll
     for (int cc = 0; cc < NC; ++cc) {
-        const int c = NC * part + ((cc + rot) & (NC - 1));  // codes 16c .. 16c+15
-        const uint4 q = *reinterpret_cast<const uint4*>(code_row + c * 16);
-        const float scale = sc[c >> 1];
+        const int c = NC == 4 ? cc : 2 * part + cc;          // codes 16c .. 16c+15
+        const uint4 q = *reinterpret_cast<const uint4*>(code_row + 16 * (c ^ ((t >> 1) & 3)));
+        const float scale = (NC == 4 ? cc >= 2 : part != 0) ? s1 : s0;
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};
         uint32_t o[8];
 #pragma unroll
@@ -242,13 +254,13 @@ __device__ __forceinline__ uint32_t f16x2_from_e2m1x2(uint32_t b) {
 }
 
 // NVFP4 row: 32 bytes of codes (64 E2M1 values, the earlier k in the low
-// nibble), the row's four E4M3 block scales (one per 16 values) and the
-// second-level factor 2^g -> the row of a bf16 A tile as in mx_convert_row.
-// The row's two 16-byte halves are read starting at a row-dependent one.
-// NH = 2 converts the whole row; NH = 1 the half `part`.
+// nibble; TMA's 32-byte swizzle puts half c of row t at half c ^ ((t >> 2) & 1)),
+// the row's four E4M3 block scales (one per 16 values) and the second-level
+// factor 2^g -> the row of a bf16 A tile as in mx_convert_row.
+// NH = 2 converts the whole row; NH = 1 its half `part`.
 template <int NH>
 __device__ __forceinline__ void nv_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
-                                               float two_g, uint8_t* a_row, int t, int part, int rot) {
+                                               float two_g, uint8_t* a_row, int t, int part) {
     const uint32_t sw = *reinterpret_cast<const uint32_t*>(scale_row);
     float sc[4];
 #pragma unroll
@@ -256,12 +268,15 @@ __device__ __forceinline__ void nv_convert_row(const uint8_t* code_row, const ui
         sc[i] = f16_lo_to_f32(f16x2_from_e4m3x2(static_cast<uint16_t>((sw >> (8 * i)) & 0xFF))) * two_g;
 #pragma unroll
     for (int hh = 0; hh < NH; ++hh) {
-        const int c = NH == 2 ? ((hh + rot) & 1) : part;   // codes 32c .. 32c+31
-        const uint4 q = *reinterpret_cast<const uint4*>(code_row + c * 16);
+        const int c = NH == 2 ? hh : part;                   // codes 32c .. 32c+31
+        const uint4 q = *reinterpret_cast<const uint4*>(code_row + 16 * (c ^ ((t >> 2) & 1)));
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};        // 8 codes a word
+        // the block scales of codes 32c .. 32c+15 and 32c+16 .. 32c+31
+        const float sa = NH == 2 ? sc[2 * hh] : (part ? sc[2] : sc[0]);
+        const float sb = NH == 2 ? sc[2 * hh + 1] : (part ? sc[3] : sc[1]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {                      // word i: codes 32c + 8i .. +7
-            const float scale = sc[2 * c + (i >> 1)];
+            const float scale = i < 2 ? sa : sb;
             uint32_t o[4];
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
@@ -411,12 +426,12 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                     uint8_t* arow = a_cvt + static_cast<size_t>(j) * kTcATile + row * 128;
                     if (FMT == kFmtMxfp8) {
                         const uint8_t* crow = a_ring + static_cast<size_t>(s) * kWTile + row * kTcKBlock;
-                        if (cvt_helpers) mx_convert_row<2>(crow, srow + row * 2, arow, row, part, u >> 2);
-                        else mx_convert_row<4>(crow, srow + row * 2, arow, row, 0, row >> 1);
+                        if (cvt_helpers) mx_convert_row<2>(crow, srow + row * 2, arow, row, part);
+                        else mx_convert_row<4>(crow, srow + row * 2, arow, row, 0);
                     } else {
                         const uint8_t* crow = a_ring + static_cast<size_t>(s) * kWTile + row * (kTcKBlock / 2);
-                        if (cvt_helpers) nv_convert_row<1>(crow, srow + row * 4, two_g, arow, row, part, 0);
-                        else nv_convert_row<2>(crow, srow + row * 4, two_g, arow, row, 0, row >> 2);
+                        if (cvt_helpers) nv_convert_row<1>(crow, srow + row * 4, two_g, arow, row, part);
+                        else nv_convert_row<2>(crow, srow + row * 4, two_g, arow, row, 0);
                     }
                     // generic-proxy writes, read next by the tensor core (async proxy)
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -625,6 +640,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             if (kCluster) {
                 // Every CTA of the cluster has its partial tile in shared memory
                 // once each has arrived on everyone's fold_ready.
+                const uint4 res0 = cluster_fold_first_residual(p, crank, csize, ht, m0, BN,
+                                                               static_cast<int>(threadIdx.x) - 64);
                 asm volatile("bar.sync 2, 128;" ::: "memory");
                 if (warp == 2 && lane == 0) {
                     fence_acq_rel_cluster();
@@ -635,10 +652,10 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                     atomicExch(&abort_flag, 1);
                 else
                     // 1 .. 4 K parts, N * parts <= 8 (the host launches no other cluster fold)
-                    if (p.splits == 1) cluster_fold_tile<1>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
-                    else if (p.splits == 2) cluster_fold_tile<2>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
-                    else if (p.splits == 3) cluster_fold_tile<3>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
-                    else cluster_fold_tile<4>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64);
+                    if (p.splits == 1) cluster_fold_tile<1>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64, res0);
+                    else if (p.splits == 2) cluster_fold_tile<2>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64, res0);
+                    else if (p.splits == 3) cluster_fold_tile<3>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64, res0);
+                    else cluster_fold_tile<4>(p, part_buf, crank, csize, ht, m0, BN, threadIdx.x - 64, res0);
                 // All reads of the peers' tiles are done: free them for the next unit.
                 asm volatile("bar.sync 2, 128;" ::: "memory");
                 if (warp == 2 && lane == 0) {

@@ -267,9 +267,10 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     c.splits = 1;
     if (allow_split && base_units > 0 && base_units < p->sm_count)
         c.splits = std::max(1, std::min({slots / base_units, nkb, tpr::kMaxSplits}));
-    // cluster fold: the N ranks x K parts of a tile in one portable cluster
-    c.cluster_fold = allow_split && base_units > 0 && c.bn <= 128 && c.splits <= 4 &&
-                     p->n_ranks * c.splits <= 8;
+    // cluster fold (the CLUSTER variant): the N ranks x K parts of a tile in
+    // one portable cluster
+    c.cluster_fold = allow_split && p->variant == TP_VARIANT_CLUSTER && base_units > 0 &&
+                     c.bn <= 128 && c.splits <= 4 && p->n_ranks * c.splits <= 8;
     // Quantised weights: a stage holds codes, scales and activations; two
     // converted bf16 tiles sit beside the ring.
     const bool quantised = fmt != tpr::kFmtBf16;
@@ -400,8 +401,10 @@ tp_status encode_mx_maps(const tp_plan* p, const void* q, const void* scales, CU
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks),
                                        static_cast<cuuint64_t>(p->hidden * p->ks)};
         const cuuint32_t box[3] = {tpr::kTcKBlock, tpr::kTcRows, 1};
+        // 64-byte swizzle: the converters' reads and their swizzled writes are
+        // both free of bank conflicts
         CUresult r = enc(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(q), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     }
@@ -433,8 +436,9 @@ tp_status encode_nv_maps(const tp_plan* p, const void* q, const void* scales, CU
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks / 2),
                                        static_cast<cuuint64_t>(p->hidden * p->ks / 2)};
         const cuuint32_t box[3] = {tpr::kTcKBlock / 2, tpr::kTcRows, 1};
+        // 32-byte swizzle, for the converters' banks (as for MXFP8)
         CUresult r = enc(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(q), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     }
@@ -637,7 +641,8 @@ tp_status tp_plan_create(tp_plan** out, int n_ranks, int64_t max_tokens, int64_t
 
 tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged) {
     if (!plan) return TP_ERR_INVALID;
-    if (variant != TP_VARIANT_AUTO && variant != TP_VARIANT_EXACT && variant != TP_VARIANT_TENSOR)
+    if (variant != TP_VARIANT_AUTO && variant != TP_VARIANT_EXACT && variant != TP_VARIANT_TENSOR &&
+        variant != TP_VARIANT_CLUSTER)
         return TP_ERR_INVALID;
     if (staged != 0 && staged != 1) return TP_ERR_INVALID;
     plan->variant = variant;
@@ -645,13 +650,16 @@ tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged) {
     return TP_OK;
 }
 
-// AUTO: the tensor cores (fastest at every token count measured on B200,
-// including single-token decode, where a 32-token tile is padded but the
-// point is bound by the weight stream). EXACT stays selectable: its partials
-// are the k-ascending fp32 sums bit for bit.
+// AUTO: the tensor cores with staged partials (fastest at every token count
+// measured on B200, including single-token decode, where a 32-token tile is
+// padded but the point is bound by the weight stream; in a chain of calls the
+// staged form beats the cluster fold, whose CTAs hold their SMs until the
+// whole cluster has folded). EXACT stays selectable: its partials are the
+// k-ascending fp32 sums bit for bit.
 static int effective_variant(const tp_plan* plan, int64_t tokens) {
     if (plan->variant == TP_VARIANT_AUTO)
         return tokens >= kTensorMinTokens ? TP_VARIANT_TENSOR : TP_VARIANT_EXACT;
+    if (plan->variant == TP_VARIANT_CLUSTER) return TP_VARIANT_TENSOR;   // the same kernels
     return plan->variant;
 }
 

@@ -15,7 +15,7 @@ from . import _lib
 from ._lib import TPError
 
 _VARIANTS = {"auto": _lib.TP_VARIANT_AUTO, "exact": _lib.TP_VARIANT_EXACT,
-             "tensor": _lib.TP_VARIANT_TENSOR}
+             "tensor": _lib.TP_VARIANT_TENSOR, "cluster": _lib.TP_VARIANT_CLUSTER}
 
 
 def _check(t: torch.Tensor, name: str, shape) -> int:

@@ -211,17 +211,19 @@ def _guards_intact(buf, numel):
     return bool(torch.all(buf[:GUARD] == SENT)) and bool(torch.all(buf[GUARD + numel:] == SENT))
 
 
-@pytest.mark.parametrize("n,m,k,h", [
-    (2, 1, 8192, 512),     # one token: K split across CTAs, folded in the kernel
-    (4, 3, 2048, 640),     # three tokens: K split, fp32 parts, ring kernel for parts
-    (8, 32, 1024, 4096),   # 32 tokens, 256 units (>= one per SM): no split, bf16 partials
-    (8, 300, 1024, 4224),  # CTA pairs (2-SM MMA), ragged token tile and H-tile pair
+@pytest.mark.parametrize("n,m,k,h,variant", [
+    (2, 1, 8192, 512, "auto"),      # one token: K split across CTAs, folded in the kernel
+    (4, 3, 2048, 640, "auto"),      # three tokens: K split, fp32 parts, ring kernel for parts
+    (8, 32, 1024, 4096, "auto"),    # 32 tokens, 256 units (>= one per SM): no split, bf16 partials
+    (8, 300, 1024, 4224, "auto"),   # CTA pairs (2-SM MMA), ragged token tile and H-tile pair
+    (8, 32, 1024, 4096, "cluster"), # folded on chip in clusters of 8
+    (2, 1, 5120, 5120, "cluster"),  # clusters of 2 ranks x 3 K parts
 ])
-def test_guard_zones_tensor_paths(n, m, k, h):
+def test_guard_zones_tensor_paths(n, m, k, h, variant):
     import tensor_layer_reconciliation_b200 as tlr
     dev = torch.device("cuda")
     x, w, r = inputs(n, m, k, h, 600 + m, dev)
-    plan = tlr.Plan(n, m, k, h)
+    plan = tlr.Plan(n, m, k, h, variant=variant)
     wp = plan.pack_weights(w)
     ref = plan.reconcile(x, wp, r)
     obuf, o = _guarded(m * h, dev)

@@ -81,20 +81,26 @@ SHAPES = [             # N, M, K, H
     (8, 3, 4096, 1024),     # three tokens: K split, fp32 parts, split ring kernel
     (1, 4, 512, 256),       # N = 1
     (2, 1, 17408, 5120),    # the down-projection of the decode example, full size
-    (8, 64, 1024, 4096),    # 64 tokens, 256 units: fold on chip in clusters of 8
-    (3, 40, 768, 6504),     # clusters of 3, ragged H tile and tokens
+    (8, 64, 1024, 4096),    # 64 tokens, 256 units: bf16 partials and the ring kernel
     (2, 300, 1024, 512),    # 256-token tiles with a K split: parts and the split ring kernel
     (8, 300, 1024, 4224),   # 256-token tiles, no split: bf16 partials and the ring kernel
 ]
-IDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in SHAPES]
+CLUSTER = [                 # the CLUSTER variant: ranks (x K parts) folded on chip
+    (8, 64, 1024, 4096),    # clusters of 8
+    (3, 40, 768, 6504),     # clusters of 3, ragged H tile and tokens
+    (2, 1, 5120, 5120),     # 2 ranks x 3 K parts
+]
+CASES = [("auto", s) for s in SHAPES] + [("cluster", s) for s in CLUSTER]
+IDS = [f"{v}-N{n}M{m}K{k}H{h}" for v, (n, m, k, h) in CASES]
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=IDS)
-def test_mx_reconcile_against_oracle(shape):
+@pytest.mark.parametrize("variant,shape", CASES, ids=IDS)
+def test_mx_reconcile_against_oracle(variant, shape):
+    import tensor_layer_reconciliation_b200 as tlr
     n, m, k, h = shape
     dev = torch.device("cuda")
     x, w, r = inputs(n, m, k, h, 900 + sum(shape), dev)
-    plan = _plan(n, m, k, h)
+    plan = tlr.Plan(n, m, k, h, variant=variant)
     q, sc = plan.pack_weights_mxfp8(w)
     out = plan.reconcile_mxfp8(x, q, sc, r)
     torch.cuda.synchronize()
@@ -119,6 +125,7 @@ def test_mx_limits():
     assert tlr.tp_plan_mxfp8_bytes(plan96.handle)[0] == tlr.TP_ERR_UNSUPPORTED
     assert tlr.tp_rowlinear_reconcile_mxfp8(plan96.handle, 256, 512, 768, 1024, 1280, 1, 0,
                                             0) == tlr.TP_ERR_UNSUPPORTED
-    plan = _plan(8, 64, 1024, 4096)
+    plan = tlr.Plan(8, 64, 1024, 4096, variant="cluster")
     assert plan.mxfp8_workspace_bytes(64) == 0           # folds in clusters: nothing staged
-    assert _plan(2, 1, 1024, 512).mxfp8_workspace_bytes(1) > 0   # k-split parts and counters
+    assert _plan(8, 64, 1024, 4096).mxfp8_workspace_bytes(64) > 0   # AUTO: staged partials
+    assert _plan(2, 1, 1024, 512).mxfp8_workspace_bytes(1) > 0      # k-split parts and counters

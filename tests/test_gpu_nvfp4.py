@@ -79,20 +79,22 @@ SHAPES = [             # N, M, K, H
     (2, 1, 1024, 512),      # one token: K split, folded in the kernel
     (4, 3, 2048, 640),      # three tokens: K split, fp32 parts, split ring kernel
     (2, 1, 17408, 5120),    # the down-projection of the decode example, full size
-    (8, 64, 1024, 4096),    # clusters of 8
-    (3, 40, 768, 6504),     # clusters of 3, ragged H tile and tokens
+    (8, 64, 1024, 4096),    # 256 units: bf16 partials and the ring kernel
     (8, 300, 1024, 4224),   # 256-token tiles: bf16 partials and the ring kernel
 ]
-IDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in SHAPES]
+CASES = [("auto", s) for s in SHAPES] + [("cluster", (8, 64, 1024, 4096)),
+                                          ("cluster", (3, 40, 768, 6504)),
+                                          ("cluster", (2, 1, 5120, 5120))]
+IDS = [f"{v}-N{n}M{m}K{k}H{h}" for v, (n, m, k, h) in CASES]
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=IDS)
-def test_nv_reconcile_against_oracle(shape):
+@pytest.mark.parametrize("variant,shape", CASES, ids=IDS)
+def test_nv_reconcile_against_oracle(variant, shape):
     import tensor_layer_reconciliation_b200 as tlr
     n, m, k, h = shape
     dev = torch.device("cuda")
     x, w, r = inputs(n, m, k, h, 950 + sum(shape), dev)
-    plan = tlr.Plan(n, m, k, h)
+    plan = tlr.Plan(n, m, k, h, variant=variant)
     q, sc = plan.pack_weights_nvfp4(w)
     out = plan.reconcile_nvfp4(x, q, sc, r)
     torch.cuda.synchronize()

@@ -24,16 +24,17 @@ from helpers import u16
 
 pytestmark = pytest.mark.gpu
 
-TENSOR_SHAPES = [      # N, M, K, H
-    (2, 1, 2048, 512),      # one token, 2 ranks x 8 parts: the counter fold
-    (4, 3, 2048, 640),      # three tokens: k-split parts and the split ring kernel
-    (4, 32, 1024, 512),     # 32 tokens, 16 units: k-split parts and the split ring kernel
-    (8, 300, 1024, 4224),   # 300 tokens: CTA pairs and the ring kernel
-    (8, 64, 1024, 4096),    # 64 tokens, 256 units: fold on chip in clusters of 8
-    (3, 40, 768, 6504),     # clusters of 3, ragged last H tile and token tile
-    (2, 1, 5120, 5120),     # clusters of 2 ranks x 3 K parts (fp32 parts folded on chip)
+TENSOR_SHAPES = [      # N, M, K, H, variant
+    (2, 1, 2048, 512, "auto"),        # one token, 2 ranks x 8 parts: the counter fold
+    (4, 3, 2048, 640, "auto"),        # three tokens: k-split parts and the split ring kernel
+    (4, 32, 1024, 512, "auto"),       # 32 tokens, 16 units: k-split parts and the split ring kernel
+    (8, 300, 1024, 4224, "auto"),     # 300 tokens: CTA pairs and the ring kernel
+    (8, 64, 1024, 4096, "auto"),      # 64 tokens, 256 units: bf16 partials and the ring kernel
+    (8, 64, 1024, 4096, "cluster"),   # the same folded on chip in clusters of 8
+    (3, 40, 768, 6504, "cluster"),    # clusters of 3, ragged last H tile and token tile
+    (2, 1, 5120, 5120, "cluster"),    # clusters of 2 ranks x 3 K parts (fp32 parts on chip)
 ]
-TIDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in TENSOR_SHAPES]
+TIDS = [f"{v}-N{n}M{m}K{k}H{h}" for n, m, k, h, v in TENSOR_SHAPES]
 
 
 def _plan(n, m, k, h, variant="auto"):
@@ -57,29 +58,29 @@ def _one_hot(m, k, cols, dev):
 
 @pytest.mark.parametrize("shape", TENSOR_SHAPES, ids=TIDS)
 def test_tensor_zero_x_gives_residual(shape):
-    n, m, k, h = shape
+    n, m, k, h, variant = shape
     dev = torch.device("cuda")
-    _, w, r = inputs(n, m, k, h, 41 + sum(shape), dev)
+    _, w, r = inputs(n, m, k, h, 41 + n + m + k + h, dev)
     x = torch.zeros(m, k, dtype=torch.bfloat16, device=dev)
-    assert np.array_equal(_run(_plan(n, m, k, h), x, w, r), u16(r))
+    assert np.array_equal(_run(_plan(n, m, k, h, variant), x, w, r), u16(r))
 
 
 @pytest.mark.parametrize("shape", TENSOR_SHAPES, ids=TIDS)
 def test_tensor_zero_w_gives_residual(shape):
-    n, m, k, h = shape
+    n, m, k, h, variant = shape
     dev = torch.device("cuda")
-    x, _, r = inputs(n, m, k, h, 43 + sum(shape), dev)
+    x, _, r = inputs(n, m, k, h, 43 + n + m + k + h, dev)
     w = torch.zeros(h, k, dtype=torch.bfloat16, device=dev)
-    assert np.array_equal(_run(_plan(n, m, k, h), x, w, r), u16(r))
+    assert np.array_equal(_run(_plan(n, m, k, h, variant), x, w, r), u16(r))
 
 
 @pytest.mark.parametrize("shape", TENSOR_SHAPES, ids=TIDS)
 def test_tensor_one_hot_x_bit_exact(shape):
-    n, m, k, h = shape
+    n, m, k, h, variant = shape
     dev = torch.device("cuda")
-    _, w, r = inputs(n, m, k, h, 47 + sum(shape), dev)
+    _, w, r = inputs(n, m, k, h, 47 + n + m + k + h, dev)
     x = _one_hot(m, k, [3, k - 1, k // 2 + 5], dev)      # columns in the first, last, middle rank
-    got = _run(_plan(n, m, k, h), x, w, r)
+    got = _run(_plan(n, m, k, h, variant), x, w, r)
     ref = oracle_point(n, h, x.cpu(), w.cpu(), r.cpu())
     assert np.array_equal(got, ref["out"])
 

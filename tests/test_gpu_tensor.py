@@ -52,26 +52,33 @@ SHAPES = [             # N, M, K, H
     (8, 512, 1024, 4096),   # prefill-sized: CTA pairs (2-SM MMA), 16 H-tile pairs, 2 token tiles
     (8, 300, 1024, 4224),   # CTA pairs, odd H-tile count (last pair half out of range), ragged tokens
     (1, 260, 512, 768),     # CTA pairs for the partials, N = 1, ragged second token tile
-    # units >= SMs, no k-split: the N ranks of a tile fold on chip in a cluster of N CTAs
+    (8, 64, 1024, 4096),    # 256 units, no split: bf16 partials and the ring kernel
+    (4, 32, 1024, 5120),
+    (8, 1, 1024, 4096),     # one token without a k-split: the counter fold over whole partials
+    (2, 1, 5120, 5120),     # the decode example's out-projection: 2 ranks x 3 parts, counter fold
+]
+# The CLUSTER variant: the N ranks (x K parts) of a tile fold on chip in one cluster.
+CLUSTER_SHAPES = [
     (8, 64, 1024, 4096),    # clusters of 8, one tile each
     (4, 32, 1024, 5120),    # clusters of 4
-    (3, 40, 768, 6504),     # clusters of 3 (tokens per CTA 22, 22, 20), ragged H tile and tokens
+    (3, 40, 768, 6504),     # clusters of 3, ragged H tile and tokens
     (2, 100, 512, 10240),   # 128-token tile, one CTA per SM: some clusters fold two tiles
     (8, 64, 512, 8192),     # 64 tiles on 37 clusters: the shared partial tile is reused
     (1, 16, 256, 19200),    # N = 1: a cluster of one CTA
-    (8, 1, 1024, 4096),     # one token without a k-split: cluster fold, not the counter fold
-    # a k-split whose N ranks x parts make at most 8 CTAs: the cluster folds fp32 parts
-    (2, 1, 5120, 5120),     # the decode example's out-projection: 2 ranks x 3 parts
+    (8, 1, 1024, 4096),     # one token, no split
+    (2, 1, 5120, 5120),     # 2 ranks x 3 K parts: fp32 parts folded on chip
     (4, 1, 4096, 4096),     # 4 ranks x 2 parts
     (2, 3, 2048, 4096),     # 2 ranks x 4 parts, three tokens
     (1, 1, 512, 10240),     # N = 1: 3 parts
+    (2, 1, 8192, 512),      # 8 parts: too many for a cluster, staged as TENSOR would
 ]
+CIDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in CLUSTER_SHAPES]
 IDS = [f"N{n}M{m}K{k}H{h}" for n, m, k, h in SHAPES]
 
 
-def _run(n, m, k, h, x, w, r):
+def _run(n, m, k, h, x, w, r, variant="tensor"):
     import tensor_layer_reconciliation_b200 as tlr
-    plan = tlr.Plan(n, m, k, h, variant="tensor")
+    plan = tlr.Plan(n, m, k, h, variant=variant)
     wp = plan.pack_weights(w)
     out = plan.reconcile(x, wp, r)
     parts = plan.partials(x, wp)
@@ -80,8 +87,10 @@ def _run(n, m, k, h, x, w, r):
     return u16(out), u16(parts)
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=IDS)
-def test_tensor_integer_exact(shape):
+@pytest.mark.parametrize("variant,shape", [("tensor", sh) for sh in SHAPES] +
+                         [("cluster", sh) for sh in CLUSTER_SHAPES],
+                         ids=[f"tensor-{i}" for i in IDS] + [f"cluster-{i}" for i in CIDS])
+def test_tensor_integer_exact(variant, shape):
     n, m, k, h = shape
     dev = torch.device("cuda")
     g = torch.Generator().manual_seed(sum(shape))
@@ -89,7 +98,7 @@ def test_tensor_integer_exact(shape):
     wi = torch.randint(-1, 2, (h, k), generator=g)
     ri = torch.randint(-8, 9, (m, h), generator=g)
     out, parts = _run(n, m, k, h, xi.to(dev, torch.bfloat16), wi.to(dev, torch.bfloat16),
-                      ri.to(dev, torch.bfloat16))
+                      ri.to(dev, torch.bfloat16), variant)
     ref = oracle_point(n, h, xi.to(torch.bfloat16), wi.to(torch.bfloat16), ri.to(torch.bfloat16))
     assert np.array_equal(parts, ref["partials"])
     assert np.array_equal(out, ref["out"])
@@ -140,12 +149,14 @@ def check_against_oracle(out, parts, ref, n, outputs_only=False):
     return int(frag.sum()), int(out_frag.sum()), float(diff.max()), float(rel_l2)
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=IDS)
-def test_tensor_gaussian_fragile_rule(shape):
+@pytest.mark.parametrize("variant,shape", [("tensor", sh) for sh in SHAPES] +
+                         [("cluster", sh) for sh in CLUSTER_SHAPES],
+                         ids=[f"tensor-{i}" for i in IDS] + [f"cluster-{i}" for i in CIDS])
+def test_tensor_gaussian_fragile_rule(variant, shape):
     n, m, k, h = shape
     dev = torch.device("cuda")
     x, w, r = inputs(n, m, k, h, 500 + sum(shape), dev)
-    out, parts = _run(n, m, k, h, x, w, r)
+    out, parts = _run(n, m, k, h, x, w, r, variant)
     ref = oracle_point(n, h, x.cpu(), w.cpu(), r.cpu())
     ref["res"] = u16(r)
     fp, fo, mx, rl2 = check_against_oracle(out, parts, ref, n)
@@ -191,13 +202,17 @@ def test_fold_counters_return_to_zero():
 
 
 def test_cluster_fold_needs_no_workspace():
-    """When the N ranks x K parts of a tile make at most 8 CTAs they fold on
-    chip in one cluster: one kernel per call, nothing staged, no workspace."""
+    """The CLUSTER variant: when the N ranks x K parts of a tile make at most 8
+    CTAs they fold on chip in one cluster: one kernel per call, nothing
+    staged, no workspace."""
     import tensor_layer_reconciliation_b200 as tlr
     for n, m, k, h in [(8, 64, 1024, 4096), (4, 32, 1024, 5120), (8, 1, 1024, 4096),
                        (2, 1, 5120, 5120), (2, 3, 2048, 4096)]:
-        plan = tlr.Plan(n, m, k, h)
+        plan = tlr.Plan(n, m, k, h, variant="cluster")
         assert plan.launches(m) == 1 and plan.workspace_bytes(m) == 0, (n, m, k, h)
+        assert plan.effective_variant(m) == "tensor"
+        auto = tlr.Plan(n, m, k, h)                      # AUTO stages its partials
+        assert auto.workspace_bytes(m) > 0 and auto.launches(m) == (1 if m <= 2 else 2)
         x, w, r = inputs(n, m, k, h, 5, torch.device("cuda"))
         out = plan.reconcile(x, plan.pack_weights(w), r)
         torch.cuda.synchronize()
