@@ -210,79 +210,130 @@ __device__ __forceinline__ void cluster_fold_tile(const TcParams& p, const void*
     }
 }
 
-// Converts one row of a staged E4M3 code tile (64 codes in a 64-byte row,
-// placed by TMA with the 64-byte swizzle: 16-byte chunk c of row t at chunk
-// c ^ ((t >> 1) & 3)) with its two E8M0 scales into the row of a bf16 A tile
-// in the 128-byte-swizzled K-major layout (chunk q of row t at q ^ (t & 7)):
-// each value is code * 2^s, computed in fp32 (exact) and rounded to bf16
-// (exact for values bf16 holds). With the two swizzles, the eight rows a
-// quarter-warp handles at once read and write eight different bank groups.
-// NC = 4 converts the whole row; NC = 2 its half `part` (chunks 2part, 2part+1).
-template <int NC>
+// Four E4M3 codes (one word, the earlier k in the low byte) times the scale
+// pair (f, f) (two f32 in 64 bits) -> two bf16x2 words: each code widened to
+// f16 (exact), then f32, multiplied (exact: 4 significant bits times a power
+// of two) and rounded to bf16 (exact for every value bf16 holds).
+__device__ __forceinline__ void e4m3x4_scaled_bf16(uint32_t w, uint64_t f2, uint32_t& o0, uint32_t& o1) {
+    asm("{\n\t"
+        ".reg .b16 c0, c1;\n\t.reg .b32 h, a, b;\n\t.reg .f16 h0, h1;\n\t.reg .b64 v;\n\t"
+        "mov.b32 {c0, c1}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h, c0;\n\t"
+        "mov.b32 {h0, h1}, h;\n\t"
+        "cvt.f32.f16 a, h0;\n\t"
+        "cvt.f32.f16 b, h1;\n\t"
+        "mov.b64 v, {a, b};\n\t"
+        "mul.rn.f32x2 v, v, %3;\n\t"
+        "mov.b64 {a, b}, v;\n\t"
+        "cvt.rn.bf16x2.f32 %0, b, a;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h, c1;\n\t"
+        "mov.b32 {h0, h1}, h;\n\t"
+        "cvt.f32.f16 a, h0;\n\t"
+        "cvt.f32.f16 b, h1;\n\t"
+        "mov.b64 v, {a, b};\n\t"
+        "mul.rn.f32x2 v, v, %3;\n\t"
+        "mov.b64 {a, b}, v;\n\t"
+        "cvt.rn.bf16x2.f32 %1, b, a;\n\t"
+        "}"
+        : "=r"(o0), "=r"(o1)
+        : "r"(w), "l"(f2));
+}
+
+// Eight E2M1 codes (one word: byte i holds codes 2i (bits 0-3) and 2i+1)
+// times (f, f) -> four bf16x2 words, as e4m3x4_scaled_bf16 (2 significant bits
+// times a 4-bit block scale times a power of two: exact in f32).
+__device__ __forceinline__ void e2m1x8_scaled_bf16(uint32_t w, uint64_t f2, uint32_t* o) {
+    asm("{\n\t"
+        ".reg .b8 c0, c1, c2, c3;\n\t.reg .b32 h, a, b;\n\t.reg .f16 h0, h1;\n\t.reg .b64 v;\n\t"
+        "mov.b32 {c0, c1, c2, c3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h, c0;\n\t"
+        "mov.b32 {h0, h1}, h;\n\t"
+        "cvt.f32.f16 a, h0;\n\t"
+        "cvt.f32.f16 b, h1;\n\t"
+        "mov.b64 v, {a, b};\n\t"
+        "mul.rn.f32x2 v, v, %5;\n\t"
+        "mov.b64 {a, b}, v;\n\t"
+        "cvt.rn.bf16x2.f32 %0, b, a;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h, c1;\n\t"
+        "mov.b32 {h0, h1}, h;\n\t"
+        "cvt.f32.f16 a, h0;\n\t"
+        "cvt.f32.f16 b, h1;\n\t"
+        "mov.b64 v, {a, b};\n\t"
+        "mul.rn.f32x2 v, v, %5;\n\t"
+        "mov.b64 {a, b}, v;\n\t"
+        "cvt.rn.bf16x2.f32 %1, b, a;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h, c2;\n\t"
+        "mov.b32 {h0, h1}, h;\n\t"
+        "cvt.f32.f16 a, h0;\n\t"
+        "cvt.f32.f16 b, h1;\n\t"
+        "mov.b64 v, {a, b};\n\t"
+        "mul.rn.f32x2 v, v, %5;\n\t"
+        "mov.b64 {a, b}, v;\n\t"
+        "cvt.rn.bf16x2.f32 %2, b, a;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h, c3;\n\t"
+        "mov.b32 {h0, h1}, h;\n\t"
+        "cvt.f32.f16 a, h0;\n\t"
+        "cvt.f32.f16 b, h1;\n\t"
+        "mov.b64 v, {a, b};\n\t"
+        "mul.rn.f32x2 v, v, %5;\n\t"
+        "mov.b64 {a, b}, v;\n\t"
+        "cvt.rn.bf16x2.f32 %3, b, a;\n\t"
+        "}"
+        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+        : "r"(w), "l"(f2));
+}
+
+// (f, f) as one 64-bit operand of the packed f32x2 multiply.
+__device__ __forceinline__ uint64_t f32_pair(float f) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(d) : "f"(f));
+    return d;
+}
+
+// Widens row t of a staged E4M3 code tile (64 codes in a 64-byte row, placed
+// by TMA with the 64-byte swizzle: 16-byte chunk c of row t at chunk
+// c ^ ((t >> 1) & 3)), with its two E8M0 scales (codes 0-31, 32-63), into row
+// t of a bf16 A tile in the 128-byte-swizzled K-major layout (chunk q of row
+// t at q ^ (t & 7)). With the two swizzles the eight rows a quarter-warp
+// handles at once read and write eight different bank groups.
 __device__ __forceinline__ void mx_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
-                                               uint8_t* a_row, int t, int part) {
-    const float s0 = e8m0_to_f32(scale_row[0]), s1 = e8m0_to_f32(scale_row[1]);
+                                               uint8_t* a_row, int t) {
+    const uint32_t sb = *reinterpret_cast<const uint16_t*>(scale_row);
+    const uint64_t f0 = f32_pair(e8m0_to_f32(sb & 0xFFu)), f1 = f32_pair(e8m0_to_f32(sb >> 8));
 #pragma unroll
-    for (int cc = 0; cc < NC; ++cc) {
-        const int c = NC == 4 ? cc : 2 * part + cc;          // codes 16c .. 16c+15
+    for (int c = 0; c < 4; ++c) {                            // codes 16c .. 16c+15
         const uint4 q = *reinterpret_cast<const uint4*>(code_row + 16 * (c ^ ((t >> 1) & 3)));
-        const float scale = (NC == 4 ? cc >= 2 : part != 0) ? s1 : s0;
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        const uint64_t f = c < 2 ? f0 : f1;
         uint32_t o[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t h01 = f16x2_from_e4m3x2(static_cast<uint16_t>(w[i] & 0xFFFF));
-            const uint32_t h23 = f16x2_from_e4m3x2(static_cast<uint16_t>(w[i] >> 16));
-            o[2 * i] = bf16x2_from_f32(f16_lo_to_f32(h01) * scale, f16_hi_to_f32(h01) * scale);
-            o[2 * i + 1] = bf16x2_from_f32(f16_lo_to_f32(h23) * scale, f16_hi_to_f32(h23) * scale);
-        }
+        e4m3x4_scaled_bf16(q.x, f, o[0], o[1]);
+        e4m3x4_scaled_bf16(q.y, f, o[2], o[3]);
+        e4m3x4_scaled_bf16(q.z, f, o[4], o[5]);
+        e4m3x4_scaled_bf16(q.w, f, o[6], o[7]);
         const int q0 = (2 * c) ^ (t & 7), q1 = (2 * c + 1) ^ (t & 7);
         *reinterpret_cast<uint4*>(a_row + q0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<uint4*>(a_row + q1 * 16) = make_uint4(o[4], o[5], o[6], o[7]);
     }
 }
 
-// Two E2M1 codes (bits 0-3 and 4-7 of b) -> two exact f16 values as f16x2.
-__device__ __forceinline__ uint32_t f16x2_from_e2m1x2(uint32_t b) {
-    uint32_t d;
-    asm("{\n\t.reg .b8 c;\n\t"
-        "cvt.u8.u32 c, %1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
-        : "=r"(d)
-        : "r"(b));
-    return d;
-}
-
 // NVFP4 row: 32 bytes of codes (64 E2M1 values, the earlier k in the low
 // nibble; TMA's 32-byte swizzle puts half c of row t at half c ^ ((t >> 2) & 1)),
 // the row's four E4M3 block scales (one per 16 values) and the second-level
-// factor 2^g -> the row of a bf16 A tile as in mx_convert_row.
-// NH = 2 converts the whole row; NH = 1 its half `part`.
-template <int NH>
+// factor 2^g -> row t of a bf16 A tile as in mx_convert_row.
 __device__ __forceinline__ void nv_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
-                                               float two_g, uint8_t* a_row, int t, int part) {
+                                               float two_g, uint8_t* a_row, int t) {
     const uint32_t sw = *reinterpret_cast<const uint32_t*>(scale_row);
-    float sc[4];
+    const uint32_t h01 = f16x2_from_e4m3x2(static_cast<uint16_t>(sw & 0xFFFFu));
+    const uint32_t h23 = f16x2_from_e4m3x2(static_cast<uint16_t>(sw >> 16));
+    const uint64_t f[4] = {f32_pair(f16_lo_to_f32(h01) * two_g), f32_pair(f16_hi_to_f32(h01) * two_g),
+                           f32_pair(f16_lo_to_f32(h23) * two_g), f32_pair(f16_hi_to_f32(h23) * two_g)};
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        sc[i] = f16_lo_to_f32(f16x2_from_e4m3x2(static_cast<uint16_t>((sw >> (8 * i)) & 0xFF))) * two_g;
-#pragma unroll
-    for (int hh = 0; hh < NH; ++hh) {
-        const int c = NH == 2 ? hh : part;                   // codes 32c .. 32c+31
+    for (int c = 0; c < 2; ++c) {                            // codes 32c .. 32c+31
         const uint4 q = *reinterpret_cast<const uint4*>(code_row + 16 * (c ^ ((t >> 2) & 1)));
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};        // 8 codes a word
-        // the block scales of codes 32c .. 32c+15 and 32c+16 .. 32c+31
-        const float sa = NH == 2 ? sc[2 * hh] : (part ? sc[2] : sc[0]);
-        const float sb = NH == 2 ? sc[2 * hh + 1] : (part ? sc[3] : sc[1]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {                      // word i: codes 32c + 8i .. +7
-            const float scale = i < 2 ? sa : sb;
+        for (int i = 0; i < 4; ++i) {                      // word i: codes 32c + 8i .. +7, block 2c + i/2
             uint32_t o[4];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const uint32_t h2 = f16x2_from_e2m1x2((w[i] >> (8 * b)) & 0xFF);
-                o[b] = bf16x2_from_f32(f16_lo_to_f32(h2) * scale, f16_hi_to_f32(h2) * scale);
-            }
+            e2m1x8_scaled_bf16(w[i], f[2 * c + (i >> 1)], o);
             const int qc = (4 * c + i) ^ (t & 7);          // 16-byte chunk of 8 bf16 values
             *reinterpret_cast<uint4*>(a_row + qc * 16) = make_uint4(o[0], o[1], o[2], o[3]);
         }
@@ -382,7 +433,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         mbar_init(fold_ready, static_cast<uint32_t>(csize));
         mbar_init(fold_freed, static_cast<uint32_t>(csize));
         for (int j = 0; j < 2; ++j) {
-            mbar_init(&cvt_full[j], cvt_helpers ? 8 : 4);
+            mbar_init(&cvt_full[j], 4);
             mbar_init(&cvt_empty[j], 1);
         }
         fence_barrier_init();
@@ -398,45 +449,49 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     const uint32_t tmem_base = *tmem_slot;
     pdl_launch_dependents();
 
-    // Converter u (0 .. 127, or 0 .. 255 with the helpers) widens its share of
-    // every staged code tile, in issue order: row u (whole), or row u / 2 (half
-    // u % 2) with the helpers.
-    auto run_converters = [&](int u) {
+    // Converters: thread `row` of a group of four warps widens row `row` of
+    // the staged code tiles in issue order (k-block i into converted slot
+    // i % 2). With the helpers (a CTA with one unit) the epilogue warps form a
+    // second group: group g then takes the k-blocks with i % 2 == g.
+    auto run_converters = [&](int row, int group) {
         if constexpr (MX) {
             const float two_g = FMT == kFmtNvfp4 ? ldexpf(1.0f, *p.nv_gexp) : 1.0f;
-            const int row = cvt_helpers ? u >> 1 : u;
-            const int part = cvt_helpers ? u & 1 : 0;
-            int i = 0;
+            int i = 0, s = 0;
+            uint32_t ph = 0;   // parity of full[s] for k-block i
             bool ok = true;
             for (int lu = 0; lu < my_units && ok; ++lu) {
                 int r, ht, mt, sp, kb_lo, kb_hi;
                 unit_of(lu, r, ht, mt, sp);
                 split_range(sp, kb_lo, kb_hi);
-                for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
-                    const int s = i % S, j = i & 1;
-                    ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / S) & 1u) &&
-                         mbar_wait_bounded(&cvt_empty[j], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u);
-                    if (!__all_sync(0xFFFFFFFFu, ok) ||
-                        *reinterpret_cast<volatile int*>(&abort_flag) != 0) {
-                        ok = false;
-                        atomicExch(&abort_flag, 1);
-                        break;
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
+                    const int j = i & 1;
+                    if (!cvt_helpers || j == group) {
+                        ok = mbar_wait_bounded(&full[s], ph) &&
+                             mbar_wait_bounded(&cvt_empty[j], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u);
+                        if (!__all_sync(0xFFFFFFFFu, ok) ||
+                            *reinterpret_cast<volatile int*>(&abort_flag) != 0) {
+                            ok = false;
+                            atomicExch(&abort_flag, 1);
+                            break;
+                        }
+                        const uint8_t* srow = s_ring + static_cast<size_t>(s) * kSTile;
+                        uint8_t* arow = a_cvt + static_cast<size_t>(j) * kTcATile + row * 128;
+                        if (FMT == kFmtMxfp8)
+                            mx_convert_row(a_ring + static_cast<size_t>(s) * kWTile + row * kTcKBlock,
+                                           srow + row * 2, arow, row);
+                        else
+                            nv_convert_row(a_ring + static_cast<size_t>(s) * kWTile + row * (kTcKBlock / 2),
+                                           srow + row * 4, two_g, arow, row);
+                        // generic-proxy writes, read next by the tensor core (async proxy)
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        __syncwarp();
+                        if ((threadIdx.x & 31) == 0) mbar_arrive(&cvt_full[j]);
                     }
-                    const uint8_t* srow = s_ring + static_cast<size_t>(s) * kSTile;
-                    uint8_t* arow = a_cvt + static_cast<size_t>(j) * kTcATile + row * 128;
-                    if (FMT == kFmtMxfp8) {
-                        const uint8_t* crow = a_ring + static_cast<size_t>(s) * kWTile + row * kTcKBlock;
-                        if (cvt_helpers) mx_convert_row<2>(crow, srow + row * 2, arow, row, part);
-                        else mx_convert_row<4>(crow, srow + row * 2, arow, row, 0);
-                    } else {
-                        const uint8_t* crow = a_ring + static_cast<size_t>(s) * kWTile + row * (kTcKBlock / 2);
-                        if (cvt_helpers) nv_convert_row<1>(crow, srow + row * 4, two_g, arow, row, part);
-                        else nv_convert_row<2>(crow, srow + row * 4, two_g, arow, row, 0);
+                    ++i;
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
                     }
-                    // generic-proxy writes, read next by the tensor core (async proxy)
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
-                    if ((threadIdx.x & 31) == 0) mbar_arrive(&cvt_full[j]);
                 }
             }
         }
@@ -460,50 +515,56 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                                 FMT == kFmtMxfp8 ? ht_ * kTcRows * 2 : ht_ * kTcRows, kb_, r_);
             };
             // Walk (unit, k-block) in issue order.
-            int lu = 0, kb = 0, kb_hi = 0, r = 0, ht = 0, mt = 0, sp = 0;
-            auto enter_unit = [&]() {
-                if (lu < my_units) {
-                    unit_of(lu, r, ht, mt, sp);
-                    split_range(sp, kb, kb_hi);
+            struct Cursor {
+                int lu, kb, kb_hi, r, ht, mt, sp;
+            };
+            auto enter_unit = [&](Cursor& c) {
+                if (c.lu < my_units) {
+                    unit_of(c.lu, c.r, c.ht, c.mt, c.sp);
+                    split_range(c.sp, c.kb, c.kb_hi);
                 }
             };
-            auto advance = [&]() {
-                if (++kb == kb_hi) {
-                    ++lu;
-                    enter_unit();
+            auto advance = [&](Cursor& c) {
+                if (++c.kb == c.kb_hi) {
+                    ++c.lu;
+                    enter_unit(c);
                 }
             };
-            enter_unit();
-            int pre_r[kTcMaxStages], pre_mt[kTcMaxStages], pre_kb[kTcMaxStages];
+            Cursor cur{0, 0, 0, 0, 0, 0, 0};
+            enter_unit(cur);
             int pre = 0;
-            while (pre < S && lu < my_units) {
+            while (pre < S && cur.lu < my_units) {
                 mbar_arrive_expect_tx(&full[pre], tx);
-                load_w(pre, kb, ht, r);
-                pre_r[pre] = r;
-                pre_mt[pre] = mt;
-                pre_kb[pre] = kb;
+                load_w(pre, cur.kb, cur.ht, cur.r);
                 ++pre;
-                advance();
+                advance(cur);
             }
             pdl_wait();  // activations may be produced by the previous kernel
-            for (int i = 0; i < pre; ++i)
-                tma_load_3d(b_ring + static_cast<size_t>(i) * kBTile, &tmap_x, &full[i],
-                            pre_kb[i] * kTcKBlock, pre_r[i], pre_mt[i] * BN);
+            {
+                // the same first positions again, for their activation blocks
+                Cursor c0{0, 0, 0, 0, 0, 0, 0};
+                enter_unit(c0);
+                for (int i = 0; i < pre; ++i) {
+                    tma_load_3d(b_ring + static_cast<size_t>(i) * kBTile, &tmap_x, &full[i],
+                                c0.kb * kTcKBlock, c0.r, c0.mt * BN);
+                    advance(c0);
+                }
+            }
             int issued = pre;
             int s = pre % S;
             uint32_t phase = pre >= S ? 1u : 0u;   // parity of slot s's next fill
-            while (lu < my_units) {
+            while (cur.lu < my_units) {
                 if (!mbar_wait_bounded(&empty[s], phase ^ 1u)) {
                     atomicExch(&abort_flag, 1);
                     break;
                 }
                 if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
                 mbar_arrive_expect_tx(&full[s], tx);
-                load_w(s, kb, ht, r);
+                load_w(s, cur.kb, cur.ht, cur.r);
                 tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, &full[s],
-                            kb * kTcKBlock, r, mt * BN);
+                            cur.kb * kTcKBlock, cur.r, cur.mt * BN);
                 ++issued;
-                advance();
+                advance(cur);
                 if (++s == S) {
                     s = 0;
                     phase ^= 1u;
@@ -519,7 +580,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     } else if (warp == 1) {
         // --------------------------------------------------------- MMA issue --
         if (lane == 0) {
-            int i = 0;
+            int i = 0, s = 0;
+            uint32_t ph = 0;   // parity of full[s] for k-block i
             for (int lu = 0; lu < my_units; ++lu) {
                 const int b = lu & 1;
                 const uint32_t aph = static_cast<uint32_t>(lu >> 1) & 1u;
@@ -534,9 +596,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 split_range(sp, kb_lo, kb_hi);
                 bool ok = true;
                 for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
-                    const int s = i % S;
                     const int j = i & 1;   // MX: converted slot
-                    if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(i / S) & 1u) ||
+                    if (!mbar_wait_bounded(&full[s], ph) ||
                         (MX && !mbar_wait_bounded(&cvt_full[j], static_cast<uint32_t>(i >> 1) & 1u))) {
                         ok = false;
                         break;
@@ -551,6 +612,10 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                                   (kb != kb_lo) || (kk != 0));
                     umma_commit(&empty[s]);  // frees the stage when these MMAs finish
                     if (MX) umma_commit(&cvt_empty[j]);   // and the converted slot
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (!ok) {
                     atomicExch(&abort_flag, 1);
@@ -565,12 +630,12 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         }
     } else if (MX && warp >= 6) {
         // ------------------------------------ converters (quantised weights) --
-        run_converters(static_cast<int>(threadIdx.x) - 192);
+        run_converters(static_cast<int>(threadIdx.x) - 192, 0);
     } else {
         // ---------------------------------------------------------- epilogue --
         // A CTA with one unit has nothing for these warps until its MMAs end:
-        // they convert the second half of every code tile meanwhile.
-        if (MX && cvt_helpers) run_converters(static_cast<int>(threadIdx.x) - 64 + 128);
+        // they widen every other code tile meanwhile.
+        if (MX && cvt_helpers) run_converters(static_cast<int>(threadIdx.x) - 64, 1);
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         pdl_wait();  // the fold reads the residual and writes the output in stream order
         for (int lu = 0; lu < my_units; ++lu) {

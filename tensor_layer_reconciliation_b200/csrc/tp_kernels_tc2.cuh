@@ -134,24 +134,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             };
             const int row0 = static_cast<int>(rank) * kTcRows;
             const int tok0 = static_cast<int>(rank) * kTc2HalfTokens;
-            int pre_r[kTc2MaxStages], pre_mt[kTc2MaxStages], pre_kb[kTc2MaxStages];
             int pre = 0;
             while (pre < S && lu < my_units) {
                 if (leader) mbar_arrive_expect_tx(&full[pre], tx_pair);
                 tma_load_3d_pair(a_ring + static_cast<size_t>(pre) * kTcATile, &tmap_w,
                                  pair_leader_addr(&full[pre]), kb * kTcKBlock,
                                  hp * 2 * kTcRows + row0, r);
-                pre_r[pre] = r;
-                pre_mt[pre] = mt;
-                pre_kb[pre] = kb;
                 ++pre;
                 advance();
             }
             pdl_wait();  // activations may be produced by the previous kernel
-            for (int i = 0; i < pre; ++i)
-                tma_load_3d_pair(b_ring + static_cast<size_t>(i) * kTc2BTile, &tmap_x,
-                                 pair_leader_addr(&full[i]), pre_kb[i] * kTcKBlock, pre_r[i],
-                                 pre_mt[i] * kTc2Tokens + tok0);
+            {
+                // the same first positions again, for their activation blocks
+                int r0 = 0, hp0 = 0, mt0 = 0, lu0 = 0, kb0 = 0;
+                unit_of(0, r0, hp0, mt0);
+                for (int i = 0; i < pre; ++i) {
+                    tma_load_3d_pair(b_ring + static_cast<size_t>(i) * kTc2BTile, &tmap_x,
+                                     pair_leader_addr(&full[i]), kb0 * kTcKBlock, r0,
+                                     mt0 * kTc2Tokens + tok0);
+                    if (++kb0 == nkb) {
+                        kb0 = 0;
+                        if (++lu0 < my_units) unit_of(lu0, r0, hp0, mt0);
+                    }
+                }
+            }
             int issued = pre;
             int s = pre % S;
             uint32_t phase = pre >= S ? 1u : 0u;
