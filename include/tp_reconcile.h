@@ -115,9 +115,9 @@ TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
  * folds them (the CTA completing a tile, one or two tokens) or a ring
  * kernel does: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of K
  * parts) when it splits K across CTAs to fill the SMs. Layout: a counter
- * block of one 32-bit counter per 128-row H tile (256-byte rounded; the
- * in-kernel fold counts stored parts there), then the partials. Rounded up
- * to 256 in all. Returns 0 for a null plan or tokens <= 0. */
+ * block of two 32-bit counters per 128-row H tile (256-byte rounded; the
+ * in-kernel fold counts the tile's parts there: tickets taken, parts
+ * stored), then the partials. Rounded up to 256 in all. Returns 0 for a null plan or tokens <= 0. */
 TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 
 /* The partial kernel a call with `tokens` tokens runs under the plan's
@@ -181,9 +181,9 @@ TP_API tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, cons
  * once per device when a plan is created on it, so this call does no set-up
  * of its own and allocates nothing.
  *  - Returns TP_ERR_WORKSPACE, launching nothing, when the call needs more
- *    scratch than that: staged partials above 16 MiB - 4 KiB (N*M*H*2
+ *    scratch than that: staged partials above 16 MiB - 8 KiB (N*M*H*2
  *    bytes, or splits*N*M*H*4; e.g. N=8, M=64, H=4096 needs 4 MiB), or
- *    H > 131072 (the first 4 KiB hold the fold counters of every plan).
+ *    H > 131072 (the first 8 KiB hold the fold counters of every plan).
  *  - Every call, from every plan and thread on a device, shares the one
  *    array, which keeps the last call's partials; each call writes every
  *    partial it reads. The fold counters at its start are zero when the

@@ -273,6 +273,28 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// `bytes` (a multiple of 16) from the 16-byte aligned global address into L2
+// only: no shared memory, no completion to wait for. L2 is where global
+// memory is kept coherent, so a line prefetched before another kernel writes
+// it is updated in place by that write.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Counter handshake between the CTAs of one grid. red_release_add: this
+// CTA's earlier writes (ordered before the calling thread by a barrier) are
+// visible at gpu scope before the addition. ld_acquire_gpu: reads after it
+// (and, through a barrier, the CTA's reads) see what the releases covered.
+__device__ __forceinline__ void red_release_add(unsigned int* p, unsigned int v) {
+    asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v)
+                 : "memory");
+}
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // --------------------------------------------- programmatic dependent launch --
 
 // Blocks until the grids this one depends on have completed and their memory

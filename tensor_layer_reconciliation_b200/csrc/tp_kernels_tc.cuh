@@ -109,7 +109,9 @@ struct TcParams {
     float* partials_f32;    // [splits][N][M][H] fp32 sums of each k part (splits > 1)
 
     int hc;                       // H / N, the chunk each rank owns in the ring
-    unsigned int* counters;       // [h_tiles][m_tiles] parts stored so far; zero between calls
+    unsigned int* counters;       // [2][h_tiles * m_tiles]: tickets taken, parts stored; zero between calls
+    const uint16_t* x;            // [M][K] activations (for the L2 prefetch)
+    int64_t k;                    // K
     const uint16_t* residual;     // [M][H]
     uint16_t* out;                // [M][H]
     const int* nv_gexp;           // NVFP4: the second-level exponent g
@@ -539,6 +541,21 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 ++pre;
                 advance(cur);
             }
+            // The activation rows of the first stages into L2 as well (the
+            // first unit's tokens, the K range of those stages): coherent there
+            // even if the previous kernel writes them, and close when the wait
+            // returns.
+            if (pre > 0) {
+                Cursor c0{0, 0, 0, 0, 0, 0, 0};
+                enter_unit(c0);
+                const int64_t k_lo = static_cast<int64_t>(c0.kb) * kTcKBlock;
+                const int64_t k_hi = min(static_cast<int64_t>(min(c0.kb + pre, c0.kb_hi)) * kTcKBlock,
+                                         static_cast<int64_t>(p.ks));
+                const int m_end = min(p.tokens, (c0.mt + 1) * BN);
+                for (int m = c0.mt * BN; m < m_end; ++m)
+                    bulk_prefetch_l2(p.x + m * p.k + static_cast<int64_t>(c0.r) * p.ks + k_lo,
+                                     static_cast<uint32_t>((k_hi - k_lo) * 2));
+            }
             pdl_wait();  // activations may be produced by the previous kernel
             {
                 // the same first positions again, for their activation blocks
@@ -656,6 +673,10 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             const int h = ht * kTcRows + q * 32 + lane;
             const int m0 = mt * BN;
             const size_t plane = static_cast<size_t>(p.tokens) * p.hidden;
+            // Counter fold: this CTA's place among the parts of its tile, taken
+            // now so the round trip overlaps the stores below.
+            unsigned int ticket = 0;
+            if (MODE == kTcCounterFold && threadIdx.x == 64) ticket = atomicAdd(p.counters + ht * p.m_tiles + mt, 1u);
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
@@ -730,24 +751,40 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 }
             }
             if (MODE == kTcCounterFold) {
-                // The CTA that stores the last of the N * SPLITS parts of this
-                // (H tile, token tile) folds the tile: ring order, residual add.
-                // Residual of this thread's row, loaded while the count goes round.
-                uint16_t res[2] = {0, 0};
+                // The CTA holding the last ticket of this (H tile, token tile)
+                // folds it once every other part is stored: ring order, residual
+                // add. The others count their stored part and leave.
+                uint16_t res[2] = {0, 0};   // this thread's residual, loaded meanwhile
                 if (h < p.hidden)
                     for (int m = m0, i = 0; m < p.tokens && i < 2; ++m, ++i)
                         res[i] = p.residual[static_cast<size_t>(m) * p.hidden + h];
-                __threadfence();  // this thread's parts are visible before the count
-                asm volatile("bar.sync 2, 128;" ::: "memory");
-                unsigned int* cnt = p.counters + ht * p.m_tiles + mt;
-                if (warp == 2 && lane == 0)
-                    fold_mine = atomicAdd(cnt, 1u) == static_cast<unsigned int>(p.n_ranks * p.splits - 1);
+                unsigned int* tickets = p.counters + ht * p.m_tiles + mt;
+                unsigned int* stored = tickets + p.h_tiles * p.m_tiles;
+                const unsigned int last = static_cast<unsigned int>(p.n_ranks * p.splits - 1);
+                asm volatile("bar.sync 2, 128;" ::: "memory");   // this CTA's part is stored
+                if (threadIdx.x == 64) {
+                    int mine = ticket == last;
+                    if (!mine) {
+                        red_release_add(stored, 1u);
+                    } else if (ld_acquire_gpu(stored) != last) {
+                        const uint64_t t0 = globaltimer_ns();
+                        while (ld_acquire_gpu(stored) != last) {
+                            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                                atomicOr(&g_device_error, kErrWaitTimeout);
+                                atomicExch(&abort_flag, 1);
+                                mine = 0;
+                                break;
+                            }
+                        }
+                    }
+                    fold_mine = mine;
+                }
                 asm volatile("bar.sync 2, 128;" ::: "memory");
                 if (fold_mine) {
-                    __threadfence();  // the other CTAs' parts, counted above, are read after it
                     if (h < p.hidden) {
                         const int c = h / p.hc;
-                        // at most two tokens here (m_tiles == 1, tokens <= 2)
+                        // at most two tokens here (m_tiles == 1, tokens <= 2); this
+                        // CTA's own part is read back by the thread that stored it
                         for (int m = m0, i = 0; m < p.tokens && i < 2; ++m, ++i) {
                             const size_t off = static_cast<size_t>(m) * p.hidden + h;
                             const uint16_t sum =
@@ -761,7 +798,10 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                             p.out[off] = bf16_add(res[i], sum);
                         }
                     }
-                    if (warp == 2 && lane == 0) atomicExch(cnt, 0u);  // zero for the next call
+                    if (threadIdx.x == 64) {   // zero for the next call
+                        *tickets = 0u;
+                        *stored = 0u;
+                    }
                 }
             }
         }

@@ -23,7 +23,7 @@
 // kNoAllocCounterBytes hold the counters of every plan (zero-initialised,
 // left zero by each call), the rest the partials.
 constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB
-constexpr size_t kNoAllocCounterBytes = 4096;       // 1024 H tiles: H <= 131072
+constexpr size_t kNoAllocCounterBytes = 8192;       // 2 x 1024 H tiles: H <= 131072
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 struct tp_plan {
@@ -526,6 +526,8 @@ tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* 
     prm.counters = fold ? counters : nullptr;
     prm.residual = static_cast<const uint16_t*>(residual);
     prm.out = static_cast<uint16_t*>(out);
+    prm.x = static_cast<const uint16_t*>(x);
+    prm.k = p->k;
     prm.nv_gexp = wt.fmt == tpr::kFmtNvfp4
                       ? reinterpret_cast<const int*>(static_cast<const uint8_t*>(wt.scales) + nv_scale_bytes(p))
                       : nullptr;
@@ -682,13 +684,13 @@ static bool tc_folds(const tp_plan* plan, int64_t tokens) {
     return tokens <= kFoldMaxTokens || tc_cluster_folds(plan, tokens);
 }
 
-// Fold counter block at the start of every workspace: one uint32 per
-// 128-row H tile, 256-byte rounded, reserved on every staged path so that
-// calls of other variants or token counts sharing the workspace leave the
-// counters alone.
+// Fold counter block at the start of every workspace: two uint32 per
+// 128-row H tile (tickets taken, parts stored), 256-byte rounded, reserved
+// on every staged path so that calls of other variants or token counts
+// sharing the workspace leave the counters alone.
 static size_t counter_block_bytes(const tp_plan* plan) {
     const size_t tiles = static_cast<size_t>((plan->hidden + tpr::kTcRows - 1) / tpr::kTcRows);
-    return (tiles * 4 + 255) / 256 * 256;
+    return (2 * tiles * 4 + 255) / 256 * 256;
 }
 
 // Bytes of staged partials a call writes (0: none, the exact fused kernel).
