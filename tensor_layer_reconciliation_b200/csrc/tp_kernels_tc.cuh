@@ -68,7 +68,7 @@ namespace tpr {
 
 constexpr int kTcRows = 128;               // MMA M: weight rows per tile
 constexpr int kTcKBlock = 64;              // bf16 columns per staged block
-constexpr int kTcMaxStages = 8;
+constexpr int kTcMaxStages = 12;
 constexpr int kTcThreads = 192;            // producer, MMA and 4 epilogue warps
 constexpr int kTcMxThreads = 320;          // quantised weights: + 4 converter warps
 constexpr uint32_t kTcATile = kTcRows * kTcKBlock * 2;  // 16 KB
@@ -105,6 +105,7 @@ struct TcParams {
     int splits;    // k-splits per (rank, h tile, m tile)
     int units;     // N * h_tiles * m_tiles * splits
     int stages;    // 2 .. kTcMaxStages
+    int x_rows;    // token rows of x staged per block: BN, or 8 (one swizzle atom) for at most 8 tokens
     uint16_t* partials;     // [N][M][H] bf16 (splits == 1)
     float* partials_f32;    // [splits][N][M][H] fp32 sums of each k part (splits > 1)
 
@@ -350,7 +351,12 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                       const __grid_constant__ CUtensorMap tmap_x,
                       const __grid_constant__ CUtensorMap tmap_s, const TcParams p) {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
-    constexpr uint32_t kBTile = BN * kTcKBlock * 2;
+    // Activation rows staged per block: the whole BN-row tile, or, for at most
+    // eight tokens, one 8-row swizzle atom that every 8-row group of the MMA's
+    // B operand reads (descriptor stride 0): rows 8.. of the product repeat
+    // rows 0..7 in accumulator columns nobody reads.
+    const uint32_t kBTile = static_cast<uint32_t>(p.x_rows) * kTcKBlock * 2;
+    const bool x_atom = p.x_rows < BN;
     constexpr bool MX = FMT != kFmtBf16;                        // converted on chip
     constexpr uint32_t kWTile = fmt_code_tile(FMT);             // weight bytes staged per block
     constexpr uint32_t kSTile = fmt_scale_tile(FMT);            // scale bytes staged per block
@@ -622,7 +628,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                     tc_fence_after_sync();
                     const uint64_t ad = smem_desc_k128(MX ? a_cvt + static_cast<size_t>(j) * kTcATile
                                                           : a_ring + static_cast<size_t>(s) * kTcATile);
-                    const uint64_t bd = smem_desc_k128(b_ring + static_cast<size_t>(s) * kBTile);
+                    uint64_t bd = smem_desc_k128(b_ring + static_cast<size_t>(s) * kBTile);
+                    if (x_atom) bd &= ~(0x3FFFull << 32);   // stride between 8-row groups: 0
 #pragma unroll
                     for (int kk = 0; kk < kTcKBlock / 16; ++kk)
                         umma_bf16(d, ad + 2ull * kk, bd + 2ull * kk, kIdesc,

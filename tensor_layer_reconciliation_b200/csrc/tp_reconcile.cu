@@ -237,7 +237,7 @@ tp_status launch_exact(const tp_plan* p, const void* x, const void* w, const voi
 // -------------------------------------------------------- tensor variant --
 
 struct TcConfig {
-    int bn, stages, grid, units, h_tiles, m_tiles, splits;
+    int bn, stages, grid, units, h_tiles, m_tiles, splits, x_rows;
     bool cluster_fold;   // the N ranks of a tile on one cluster, folded on chip
     size_t smem;
 };
@@ -274,8 +274,10 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     // Quantised weights: a stage holds codes, scales and activations; two
     // converted bf16 tiles sit beside the ring.
     const bool quantised = fmt != tpr::kFmtBf16;
+    // at most 8 tokens: one 8-row atom of x a block instead of the BN-row tile
+    c.x_rows = tokens <= 8 && c.m_tiles == 1 ? 8 : c.bn;
     const size_t stage = tpr::fmt_code_tile(fmt) + tpr::fmt_scale_tile(fmt) +
-                         static_cast<size_t>(c.bn) * tpr::kTcKBlock * 2;
+                         static_cast<size_t>(c.x_rows) * tpr::kTcKBlock * 2;
     // the cluster fold's tile in shared memory: the tile's tokens x 128 rows,
     // bf16 partials or fp32 part sums
     const size_t part_tile = c.cluster_fold ? static_cast<size_t>(std::min<int64_t>(c.bn, tokens)) *
@@ -501,7 +503,7 @@ tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* 
         p->sm_count >= 2)
         return launch_tc2(p, x, wt.w, partials, tokens, stream);
     CUtensorMap mw, mx, ms;
-    tp_status st = encode_tc_maps(p, c.bn, x, wt.w, tokens, &mw, &mx);
+    tp_status st = encode_tc_maps(p, c.x_rows, x, wt.w, tokens, &mw, &mx);
     if (st != TP_OK) return st;
     if (wt.fmt == tpr::kFmtMxfp8) {
         if ((st = encode_mx_maps(p, wt.w, wt.scales, &mw, &ms)) != TP_OK) return st;
@@ -520,6 +522,7 @@ tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* 
     prm.splits = c.splits;
     prm.units = c.units;
     prm.stages = c.stages;
+    prm.x_rows = c.x_rows;
     prm.partials = static_cast<uint16_t*>(partials);
     prm.partials_f32 = static_cast<float*>(partials);
     prm.hc = static_cast<int>(p->hc);
