@@ -513,18 +513,15 @@ def _barrier(world):
         dist.barrier()
 
 
-def _config_keys(cfg, world, args, wl=None, staged_path=None):
-    """The `config` object of a bench line (the same keys on both arms)."""
-    d = {"workload": cfg.name, "n_ranks": cfg.n_ranks, "tokens": cfg.tokens,
-         "hidden": cfg.hidden, "points": cfg.n_points,
-         "weights": args.weights, "variant": args.variant,
-         "l2": "no flush: every step streams all points' distinct weights "
-               f"({cfg.weight_bytes() / 1e9:.2f} GB), larger than the 126 MB L2",
-         "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
-    if wl is not None:
-        d["weights_gb_per_step"] = wl.weight_bytes_read() / 1e9
-        d["staged_partials"] = staged_path
-    return d
+def _config_keys(cfg, world, args):
+    """The `config` object of a bench line: the same keys and values on both
+    arms (what the library's own path does goes under `path` instead)."""
+    return {"workload": cfg.name, "n_ranks": cfg.n_ranks, "tokens": cfg.tokens,
+            "hidden": cfg.hidden, "points": cfg.n_points,
+            "weights": args.weights, "variant": args.variant,
+            "l2": "no flush: every step streams all points' distinct weights "
+                  f"({cfg.weight_bytes() / 1e9:.2f} GB), larger than the 126 MB L2",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 def _configs_to_run(args):
@@ -668,10 +665,12 @@ def run_config(name, args, device, world, rank, local, peaks):
                   "reconciliation call: tc_partial_kernel, NVFP4 form, then a ring fold kernel"),
         "exact-fused": "reconciliation call: exact_partial_kernel (partials, ring fold, residual)",
         "exact-staged": "reconciliation call: exact_partial_kernel then ring_reduce_kernel",
-        "tensor": (f"reconciliation call: tc_partial_kernel ({fold_where}; residual)"
+        "tensor": ("reconciliation call: tc2_partial_kernel on CTA pairs (partials staged; the CTA "
+                   "storing a half tile's last rank folds it: ring order, residual)"
+                   if one_kernel and cfg.tokens > 128 else
+                   f"reconciliation call: tc_partial_kernel ({fold_where}; residual)"
                    if one_kernel else
-                   "reconciliation call: tc_partial_kernel (tc2_partial_kernel on CTA pairs "
-                   "from 129 tokens) then a ring fold kernel"),
+                   "reconciliation call: tc_partial_kernel then a ring fold kernel"),
     }[path]
     if tensor_bound:
         achieved = flops / (step_ms * 1e-3) / 1e12
@@ -701,7 +700,8 @@ def run_config(name, args, device, world, rank, local, peaks):
         "step_ms_stats": step_stats,
         "hbm_gbs_step": step_bytes / (step_ms * 1e-3) / 1e9,
         "tflops_step": flops / (step_ms * 1e-3) / 1e12,
-        "config": _config_keys(cfg, world, args, wl, staged_path),
+        "config": _config_keys(cfg, world, args),
+        "path": {"weights_gb_per_step": wl.weight_bytes_read() / 1e9, "staged_partials": staged_path},
         "roofline": roof,
         "e2e": {"value": _job_rate(cfg.tokens, e2e_ms, world), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
@@ -726,7 +726,7 @@ def run_config(name, args, device, world, rank, local, peaks):
 def _per_config_entry(line):
     """The compact per-workload record under per_config."""
     keep = ("value", "unit", "ms_per_step", "reconciliations_per_s", "step_ms_stats", "roofline",
-            "e2e", "gpu_launches", "clocks", "parity", "cpu_baseline", "config")
+            "e2e", "gpu_launches", "clocks", "parity", "cpu_baseline", "config", "path")
     return {k: line[k] for k in keep if k in line}
 
 

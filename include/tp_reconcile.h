@@ -112,12 +112,14 @@ TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
  * the plan's current setting; 0 when the partials stay on chip (EXACT, not
  * staged; TENSOR folding across a cluster). Otherwise the tensor-core
  * variant writes its partials to the workspace, whether its own kernel
- * folds them (the CTA completing a tile, one or two tokens) or a ring
- * kernel does: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of K
- * parts) when it splits K across CTAs to fill the SMs. Layout: a counter
- * block of two 32-bit counters per 128-row H tile (256-byte rounded; the
- * in-kernel fold counts the tile's parts there: tickets taken, parts
- * stored), then the partials. Rounded up to 256 in all. Returns 0 for a null plan or tokens <= 0. */
+ * folds them (one or two tokens: the CTA holding a tile's last ticket; more
+ * than 128 tokens on CTA pairs: the CTA storing a half tile's last rank) or
+ * a ring kernel does: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of
+ * K parts) when it splits K across CTAs to fill the SMs. Layout: a counter
+ * block (256-byte rounded) of two 32-bit counters per 128-row H tile
+ * (tickets taken, parts stored), or, if more, two per 256-row x 256-token
+ * tile of max_tokens (ranks stored per half tile), then the partials.
+ * Rounded up to 256 in all. Returns 0 for a null plan or tokens <= 0. */
 TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 
 /* The partial kernel a call with `tokens` tokens runs under the plan's
@@ -128,10 +130,11 @@ TP_API int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens);
 
 /* Kernels one tp_rowlinear_reconcile call with `tokens` tokens launches under
  * the plan's current setting: 1 (EXACT not staged; TENSOR when its partial
- * kernel folds on chip: across a cluster of the N ranks x K parts of a tile
- * when they make at most 8 CTAs and the token tile is at most 128, or by the
- * CTA completing a tile for 1 or 2 tokens) or 2 (a partial kernel, then a
- * ring fold kernel); 0 for tokens = 0; -1 for a null plan or tokens < 0. */
+ * kernel also folds: for 1 or 2 tokens, for more than 128 tokens on CTA
+ * pairs, and with CLUSTER across a cluster of the N ranks x K parts of a
+ * tile when they make at most 8 CTAs and the token tile is at most 128) or
+ * 2 (a partial kernel, then a ring fold kernel: TENSOR at 3 to 128 tokens);
+ * 0 for tokens = 0; -1 for a null plan or tokens < 0. */
 TP_API int tp_plan_launches(const tp_plan* plan, int64_t tokens);
 
 /* Bytes of the packed weight buffer tp_pack_weights writes: N*H*(K/N)*2,

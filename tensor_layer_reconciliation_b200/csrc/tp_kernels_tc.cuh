@@ -52,8 +52,8 @@
 // more warps (6-9) turn each code tile into the bf16 tile the MMA reads
 // (MXFP8: E4M3 * 2^s; NVFP4: E2M1 * E4M3 block scale * 2^g; exact in bf16
 // for the shards the formats' definitions allow), written in the same
-// 128-byte-swizzled K-major layout TMA gives the bf16 path, into one of two
-// converted slots; the MMA waits for its slot and frees it (and the stage,
+// 128-byte-swizzled K-major layout TMA gives the bf16 path, into one of
+// kCvtSlots converted slots; the MMA waits for its slot and frees it (and the stage,
 // whose activation tile it reads) when it is done. Everything after the MMA
 // -- the three epilogues -- is the same.
 // Accumulation order inside the tensor core is the hardware's; the partial
@@ -72,6 +72,9 @@ constexpr int kTcMaxStages = 12;
 constexpr int kTcThreads = 192;            // producer, MMA and 4 epilogue warps
 constexpr int kTcMxThreads = 320;          // quantised weights: + 4 converter warps
 constexpr uint32_t kTcATile = kTcRows * kTcKBlock * 2;  // 16 KB
+// Quantised forms: converted bf16 tiles in flight between the converters and
+// the MMAs (k-block i goes to slot i % kCvtSlots).
+constexpr int kCvtSlots = 3;
 constexpr uint32_t kMxCodeTile = kTcRows * kTcKBlock;   // 8 KB of E4M3 codes
 constexpr uint32_t kMxScaleTile = kTcRows * 2;          // the 2 E8M0 scales of each row
 constexpr uint32_t kNvCodeTile = kTcRows * kTcKBlock / 2;  // 4 KB: two E2M1 codes a byte
@@ -369,8 +372,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     const int S = p.stages;
     uint8_t* a_ring = smem;                                              // weight tiles (TMA)
     uint8_t* b_ring = a_ring + static_cast<size_t>(S) * kWTile;         // activation tiles
-    uint8_t* a_cvt = b_ring + static_cast<size_t>(S) * kBTile;          // MX: 2 converted tiles
-    uint8_t* s_ring = a_cvt + (MX ? 2 * kTcATile : 0);                   // MX: scale tiles
+    uint8_t* a_cvt = b_ring + static_cast<size_t>(S) * kBTile;          // MX: converted tiles
+    uint8_t* s_ring = a_cvt + (MX ? kCvtSlots * kTcATile : 0);           // MX: scale tiles
     uint64_t* full = reinterpret_cast<uint64_t*>(s_ring + static_cast<size_t>(S) * kSTile);
     uint64_t* empty = full + kTcMaxStages;
     uint64_t* acc_full = empty + kTcMaxStages;   // [2]
@@ -378,9 +381,9 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     uint64_t* mma_done = acc_empty + 2;
     uint64_t* fold_ready = mma_done + 1;   // cluster fold: all N partial tiles written
     uint64_t* fold_freed = fold_ready + 1; // cluster fold: all N CTAs done reading mine
-    uint64_t* cvt_full = fold_freed + 1;   // MX: [2] converted tile ready (4 warps)
-    uint64_t* cvt_empty = cvt_full + 2;    // MX: [2] converted tile read by the MMAs
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cvt_empty + 2);
+    uint64_t* cvt_full = fold_freed + 1;           // MX: [kCvtSlots] converted tile ready (4 warps)
+    uint64_t* cvt_empty = cvt_full + kCvtSlots;    // MX: [kCvtSlots] converted tile read by the MMAs
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cvt_empty + kCvtSlots);
     // cluster fold: this CTA's bf16 partial tile, [BN tokens][128 rows]
     uint16_t* part_buf = reinterpret_cast<uint16_t*>(
         (reinterpret_cast<uintptr_t>(tmem_slot + 4) + 127) & ~static_cast<uintptr_t>(127));
@@ -440,7 +443,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         mbar_init(mma_done, 1);
         mbar_init(fold_ready, static_cast<uint32_t>(csize));
         mbar_init(fold_freed, static_cast<uint32_t>(csize));
-        for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < kCvtSlots; ++j) {
             mbar_init(&cvt_full[j], 4);
             mbar_init(&cvt_empty[j], 1);
         }
@@ -459,23 +462,21 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
 
     // Converters: thread `row` of a group of four warps widens row `row` of
     // the staged code tiles in issue order (k-block i into converted slot
-    // i % 2). With the helpers (a CTA with one unit) the epilogue warps form a
-    // second group: group g then takes the k-blocks with i % 2 == g.
+    // i % kCvtSlots). With the helpers (a CTA with one unit) the epilogue warps
+    // form a second group: group g then takes the k-blocks with i % 2 == g.
     auto run_converters = [&](int row, int group) {
         if constexpr (MX) {
             const float two_g = FMT == kFmtNvfp4 ? ldexpf(1.0f, *p.nv_gexp) : 1.0f;
-            int i = 0, s = 0;
-            uint32_t ph = 0;   // parity of full[s] for k-block i
+            int i = 0, s = 0, j = 0;
+            uint32_t ph = 0, jph = 0;   // parities of full[s] and of slot j's use for k-block i
             bool ok = true;
             for (int lu = 0; lu < my_units && ok; ++lu) {
                 int r, ht, mt, sp, kb_lo, kb_hi;
                 unit_of(lu, r, ht, mt, sp);
                 split_range(sp, kb_lo, kb_hi);
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                    const int j = i & 1;
-                    if (!cvt_helpers || j == group) {
-                        ok = mbar_wait_bounded(&full[s], ph) &&
-                             mbar_wait_bounded(&cvt_empty[j], (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u);
+                    if (!cvt_helpers || (i & 1) == group) {
+                        ok = mbar_wait_bounded(&full[s], ph) && mbar_wait_bounded(&cvt_empty[j], jph ^ 1u);
                         if (!__all_sync(0xFFFFFFFFu, ok) ||
                             *reinterpret_cast<volatile int*>(&abort_flag) != 0) {
                             ok = false;
@@ -499,6 +500,10 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
+                    }
+                    if (++j == kCvtSlots) {
+                        j = 0;
+                        jph ^= 1u;
                     }
                 }
             }
@@ -603,8 +608,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     } else if (warp == 1) {
         // --------------------------------------------------------- MMA issue --
         if (lane == 0) {
-            int i = 0, s = 0;
-            uint32_t ph = 0;   // parity of full[s] for k-block i
+            int i = 0, s = 0, j = 0;
+            uint32_t ph = 0, jph = 0;   // parities of full[s] and (MX) of converted slot j
             for (int lu = 0; lu < my_units; ++lu) {
                 const int b = lu & 1;
                 const uint32_t aph = static_cast<uint32_t>(lu >> 1) & 1u;
@@ -619,9 +624,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 split_range(sp, kb_lo, kb_hi);
                 bool ok = true;
                 for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
-                    const int j = i & 1;   // MX: converted slot
-                    if (!mbar_wait_bounded(&full[s], ph) ||
-                        (MX && !mbar_wait_bounded(&cvt_full[j], static_cast<uint32_t>(i >> 1) & 1u))) {
+                    if (!mbar_wait_bounded(&full[s], ph) || (MX && !mbar_wait_bounded(&cvt_full[j], jph))) {
                         ok = false;
                         break;
                     }
@@ -639,6 +642,10 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
+                    }
+                    if (++j == kCvtSlots) {
+                        j = 0;
+                        jph ^= 1u;
                     }
                 }
                 if (!ok) {

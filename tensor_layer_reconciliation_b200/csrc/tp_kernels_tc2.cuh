@@ -28,7 +28,11 @@
 //   warps 2-5  epilogue of this CTA's 128 rows: tcgen05.ld, one rounding to
 //              bf16 per partial, stores to [N][M][H]; then an arrival on the
 //              leader's "accumulator empty" barrier (8 arrivals: 4 warps x 2
-//              CTAs) so the leader may reuse the accumulator.
+//              CTAs) so the leader may reuse the accumulator. With `fold`,
+//              the CTA that stores the last of the N ranks' partials of its
+//              128 rows x 256 tokens (a counter per half tile) folds them
+//              there (S2-S4: ring order, residual, output) while the leader
+//              already multiplies the next unit.
 // Units run token tile fastest (CTAs working at the same time share weight
 // tiles through L2). Two accumulators of 256 fp32 columns fill the 512
 // tensor-memory columns, so the epilogue of one unit overlaps the next
@@ -56,7 +60,56 @@ struct Tc2Params {
     int units;     // N * h_pairs * m_tiles
     int stages;    // 2 .. kTc2MaxStages
     uint16_t* partials;  // [N][M][H] bf16
+    int fold;                     // fold in the epilogue (else a ring kernel follows)
+    int hc;                       // H / N
+    unsigned int* counters;       // [h_pairs * m_tiles][2] parts stored per half tile; zero between calls
+    const uint16_t* residual;     // [M][H]
+    uint16_t* out;                // [M][H]
 };
+
+// S2-S4 of one half tile (128 rows from h0, tokens m0 .. m1-1) from the
+// staged partials, by the 128 epilogue threads (et): 16-byte vectors of 8
+// rows, V of them in flight per thread, each folded in ring order from its
+// chunk's owner (all N loads before the first add), the residual added.
+template <int V>
+__device__ __forceinline__ void tc2_fold_half(const Tc2Params& p, int h0, int m0, int m1, int et) {
+    const size_t plane = static_cast<size_t>(p.tokens) * p.hidden;
+    const int total = (m1 - m0) * (kTcRows / 8);
+    for (int v0 = et; v0 < total; v0 += V * 128) {
+        uint4 pv[V][kMaxRanks], rv[V];
+        size_t off[V];
+        int c[V];
+        bool ok[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            const int v = v0 + j * 128;
+            const int m = m0 + v / (kTcRows / 8);
+            const int h = h0 + (v % (kTcRows / 8)) * 8;
+            ok[j] = v < total && h < p.hidden;
+            off[j] = static_cast<size_t>(m) * p.hidden + h;
+            c[j] = h / p.hc;
+            if (ok[j]) {
+#pragma unroll
+                for (int i = 0; i < kMaxRanks; ++i)
+                    if (i < p.n_ranks) {
+                        int rr = c[j] + i;
+                        if (rr >= p.n_ranks) rr -= p.n_ranks;
+                        pv[j][i] = __ldcg(reinterpret_cast<const uint4*>(p.partials + rr * plane + off[j]));
+                    }
+                rv[j] = ld_global_nc_v4(p.residual + off[j]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            if (!ok[j]) continue;
+            uint4 sum = pv[j][0];
+#pragma unroll
+            for (int i = 1; i < kMaxRanks; ++i)
+                if (i < p.n_ranks) sum = bf16x8_add_tc(sum, pv[j][i]);
+            st_global_v4(p.out + off[j], bf16x8_add_tc(rv[j], sum));
+        }
+    }
+}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     tc2_partial_kernel(const __grid_constant__ CUtensorMap tmap_w,
@@ -77,6 +130,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     uint64_t* mma_done = acc_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     __shared__ int abort_flag;
+    __shared__ int fold_mine;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();          // 0: leader, 1: peer
@@ -269,6 +323,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty[b]);
+            if (p.fold) {
+                // This CTA's 128 rows of the tile are stored: count them; the
+                // CTA storing the N-th rank's folds those rows of the tile.
+                unsigned int* cnt = p.counters + (hp * p.m_tiles + mt) * 2 + static_cast<int>(rank);
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                if (threadIdx.x == 64) {
+                    __threadfence();   // this CTA's stores (ordered by the barrier) before the count
+                    const unsigned int prev = atomicAdd(cnt, 1u);
+                    fold_mine = prev == static_cast<unsigned int>(p.n_ranks - 1);
+                    if (fold_mine) __threadfence();   // the other ranks' stores, counted, before the loads
+                }
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                if (fold_mine) {
+                    const int h0 = hp * 2 * kTcRows + static_cast<int>(rank) * kTcRows;
+                    const int m1 = min(p.tokens, m0 + kTc2Tokens);
+                    const int et = static_cast<int>(threadIdx.x) - 64;
+                    if (p.n_ranks <= 4) tc2_fold_half<4>(p, h0, m0, m1, et);
+                    else tc2_fold_half<2>(p, h0, m0, m1, et);
+                    if (threadIdx.x == 64) *cnt = 0u;   // zero for the next call
+                }
+            }
         }
     }
 

@@ -283,8 +283,8 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     const size_t part_tile = c.cluster_fold ? static_cast<size_t>(std::min<int64_t>(c.bn, tokens)) *
                                                   tpr::kTcRows * (c.splits > 1 ? 4 : 2)
                                             : 0;
-    const size_t fixed = (2 * tpr::kTcMaxStages + 11) * sizeof(uint64_t) + 16 + 128 + 1024 + part_tile +
-                         (quantised ? 2 * tpr::kTcATile : 0);
+    const size_t fixed = (2 * tpr::kTcMaxStages + 7 + 2 * tpr::kCvtSlots) * sizeof(uint64_t) + 16 + 128 +
+                         1024 + part_tile + (quantised ? tpr::kCvtSlots * tpr::kTcATile : 0);
     const size_t budget = std::min<size_t>(two_per_sm ? 110 * 1024 : 200 * 1024,
                                            static_cast<size_t>(p->smem_optin));
     c.stages = budget > fixed
@@ -344,10 +344,18 @@ size_t tc_partial_bytes(const tp_plan* p, const TcConfig& c, int64_t tokens) {
            static_cast<size_t>(p->hidden) * (c.splits > 1 ? 4u * c.splits : 2u);
 }
 
+// Calls that run on CTA pairs: bf16 shards, prefill-sized token tiles, no
+// k-split, not the cluster fold.
+bool tc2_path(const tp_plan* p, const TcConfig& c, int fmt) {
+    return fmt == tpr::kFmtBf16 && c.bn == tpr::kTc2Tokens && c.splits == 1 && !c.cluster_fold &&
+           p->sm_count >= 2;
+}
+
 // The partials [N][M][H] of a prefill-sized call on CTA pairs: units of
 // (rank, 256 rows of H, 256 tokens), two CTAs per unit, one per SM.
 tp_status launch_tc2(const tp_plan* p, const void* x, const void* w, void* partials, int64_t tokens,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, bool fold = false, unsigned int* counters = nullptr,
+                     const void* residual = nullptr, void* out = nullptr) {
     const int h_pairs = static_cast<int>((p->hidden + 2 * tpr::kTcRows - 1) / (2 * tpr::kTcRows));
     const int m_tiles = static_cast<int>((tokens + tpr::kTc2Tokens - 1) / tpr::kTc2Tokens);
     const int units = p->n_ranks * h_pairs * m_tiles;
@@ -370,6 +378,11 @@ tp_status launch_tc2(const tp_plan* p, const void* x, const void* w, void* parti
     prm.units = units;
     prm.stages = stages;
     prm.partials = static_cast<uint16_t*>(partials);
+    prm.fold = fold ? 1 : 0;
+    prm.hc = static_cast<int>(p->hc);
+    prm.counters = fold ? counters : nullptr;
+    prm.residual = static_cast<const uint16_t*>(residual);
+    prm.out = static_cast<uint16_t*>(out);
     cudaError_t e = launch_pdl(tpr::tc2_partial_kernel, dim3(static_cast<unsigned>(2 * pairs)),
                                dim3(tpr::kTcThreads), smem, stream, mw, mx, prm);
     return e == cudaSuccess ? TP_OK : cuda_fail(e);
@@ -497,11 +510,11 @@ tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* 
     const TcConfig c = tc_config(p, tokens, allow_split, wt.fmt);
     if (c.stages < 2) return TP_ERR_UNSUPPORTED;
     if (c.cluster_fold) fold = false;
+    // Prefill-sized bf16 tiles without a k-split run on CTA pairs (2-SM MMA),
+    // which fold in their epilogue with `fold`.
+    if (tc2_path(p, c, wt.fmt))
+        return launch_tc2(p, x, wt.w, partials, tokens, stream, fold, counters, residual, out);
     if (fold && (c.m_tiles != 1 || tokens > 2)) return TP_ERR_UNSUPPORTED;  // the kernel folds <= 2 rows
-    // Prefill-sized bf16 tiles without a k-split run on CTA pairs (2-SM MMA).
-    if (wt.fmt == tpr::kFmtBf16 && c.bn == tpr::kTc2Tokens && c.splits == 1 && !fold && !c.cluster_fold &&
-        p->sm_count >= 2)
-        return launch_tc2(p, x, wt.w, partials, tokens, stream);
     CUtensorMap mw, mx, ms;
     tp_status st = encode_tc_maps(p, c.x_rows, x, wt.w, tokens, &mw, &mx);
     if (st != TP_OK) return st;
@@ -674,17 +687,20 @@ int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens) {
 }
 
 // The tensor path folds inside its partial kernel: in clusters of the N ranks
-// x K parts of a tile when they make at most 8 CTAs and the token tile is at
-// most 128 (cluster fold), else up to this many tokens by the CTA completing
-// a tile (counter fold).
+// x K parts of a tile (the CLUSTER variant), up to this many tokens by the
+// CTA holding a tile's last ticket (counter fold), and on CTA pairs (bf16
+// prefill) by the CTA storing a half tile's last rank; other calls stage
+// their partials for a ring kernel.
 constexpr int64_t kFoldMaxTokens = 2;
 
 static bool tc_cluster_folds(const tp_plan* plan, int64_t tokens) {
     return tokens > 0 && tc_config(plan, tokens, true).cluster_fold;
 }
 
-static bool tc_folds(const tp_plan* plan, int64_t tokens) {
-    return tokens <= kFoldMaxTokens || tc_cluster_folds(plan, tokens);
+static bool tc_folds(const tp_plan* plan, int64_t tokens, int fmt = tpr::kFmtBf16) {
+    if (tokens <= kFoldMaxTokens) return true;
+    const TcConfig c = tc_config(plan, tokens, true, fmt);
+    return c.cluster_fold || tc2_path(plan, c, fmt);
 }
 
 // Fold counter block at the start of every workspace: two uint32 per
@@ -693,7 +709,10 @@ static bool tc_folds(const tp_plan* plan, int64_t tokens) {
 // sharing the workspace leave the counters alone.
 static size_t counter_block_bytes(const tp_plan* plan) {
     const size_t tiles = static_cast<size_t>((plan->hidden + tpr::kTcRows - 1) / tpr::kTcRows);
-    return (2 * tiles * 4 + 255) / 256 * 256;
+    // CTA pairs: one counter per half tile (128 rows x 256 tokens)
+    const size_t pair_words = 2 * static_cast<size_t>((plan->hidden + 2 * tpr::kTcRows - 1) / (2 * tpr::kTcRows)) *
+                              static_cast<size_t>((plan->max_tokens + tpr::kTc2Tokens - 1) / tpr::kTc2Tokens);
+    return (std::max(2 * tiles, pair_words) * 4 + 255) / 256 * 256;
 }
 
 // Bytes of staged partials a call writes (0: none, the exact fused kernel).
@@ -770,7 +789,7 @@ static tp_status check_reconcile_args(const tp_plan* plan, const void* x, const 
 static tp_status tensor_reconcile(const tp_plan* plan, const void* x, const TcWeights& wt,
                                   const void* residual, void* out, int64_t tokens,
                                   unsigned int* counters, void* partials, cudaStream_t s) {
-    const bool fold = tc_folds(plan, tokens);
+    const bool fold = tc_folds(plan, tokens, wt.fmt);
     tp_status st = launch_tc(plan, x, wt, partials, tokens, true, fold, counters, residual, out, s);
     if (st != TP_OK || fold) return st;
     const int splits = tc_config(plan, tokens, true).splits;

@@ -187,8 +187,8 @@ def test_fold_counters_return_to_zero():
         assert plan.launches(m) == 1                   # partials and fold in one kernel
         need = plan.workspace_bytes(m)
         ws = torch.zeros(need, dtype=torch.uint8, device=dev)
-        h_tiles = (h + 127) // 128
-        counter_bytes = (h_tiles * 4 + 255) // 256 * 256
+        h_tiles = (h + 127) // 128                     # tickets and stored parts per tile
+        counter_bytes = (2 * h_tiles * 4 + 255) // 256 * 256
         for seed in (31, 32, 33):
             x, w, r = inputs(n, m, k, h, seed + 10 * m, dev)
             wp = plan.pack_weights(w)
@@ -199,6 +199,30 @@ def test_fold_counters_return_to_zero():
             assert torch.equal(out.view(torch.int16), fresh.view(torch.int16))
             assert int(torch.count_nonzero(ws[:counter_bytes])) == 0
     assert plan.launches(3) == 2                       # from three tokens: a ring kernel follows
+
+
+def test_pair_fold_counters_return_to_zero():
+    """Prefill-sized calls on CTA pairs fold in their epilogue: one kernel a
+    call; the CTA storing a half tile's last rank folds it and sets its count
+    back to zero, so one zeroed workspace serves many calls."""
+    import tensor_layer_reconciliation_b200 as tlr
+    dev = torch.device("cuda")
+    n, m, k, h = 8, 300, 1024, 4224
+    plan = tlr.Plan(n, m, k, h)                        # AUTO
+    assert plan.launches(m) == 1
+    need = plan.workspace_bytes(m)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+    pair_words = 2 * ((h + 255) // 256) * ((m + 255) // 256)
+    counter_bytes = (max(2 * ((h + 127) // 128), pair_words) * 4 + 255) // 256 * 256
+    for seed in (41, 42):
+        x, w, r = inputs(n, m, k, h, seed, dev)
+        wp = plan.pack_weights(w)
+        out = plan.reconcile(x, wp, r, workspace=ws)
+        fresh = plan.reconcile(x, wp, r)               # its own zeroed workspace
+        torch.cuda.synchronize()
+        assert plan.device_error_flags() == 0
+        assert torch.equal(out.view(torch.int16), fresh.view(torch.int16))
+        assert int(torch.count_nonzero(ws[:counter_bytes])) == 0
 
 
 def test_cluster_fold_needs_no_workspace():
