@@ -430,6 +430,11 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     };
     // quantised weights, one unit: the 4 epilogue warps also convert (8 converter warps)
     const bool cvt_helpers = MX && my_units == 1;
+    // Store form, one unit: the epilogue stages the bf16 partial tile in the
+    // stage ring (idle once the unit's last MMA is done) and stores whole
+    // 16-byte vectors instead of one 2-byte value per token and row.
+    const bool stage_tile = MODE == kTcStore && p.splits == 1 && my_units == 1 && p.tokens > 2 &&
+                            static_cast<uint32_t>(BN) * kTcRows * 2 <= static_cast<uint32_t>(S) * (kWTile + kBTile);
     if (threadIdx.x == 0) {
         abort_flag = 0;
         for (int s = 0; s < S; ++s) {
@@ -713,6 +718,13 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                         for (int i = 0; i < 32; ++i)
                             if (c0 + i < t_tile) dst[i * kTcRows] = __uint_as_float(v[i]);
                     }
+                } else if (stage_tile) {
+                    // [token][128 rows] in the (now idle) stage ring: lanes write
+                    // 32 consecutive rows of one token
+                    uint16_t* dst = reinterpret_cast<uint16_t*>(a_ring) + static_cast<size_t>(c0) * kTcRows +
+                                    q * 32 + lane;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) dst[i * kTcRows] = f32_to_bf16_rne(__uint_as_float(v[i]));
                 } else if (h < p.hidden) {
                     if (p.splits == 1) {
                         uint16_t* dst = p.partials + static_cast<size_t>(r) * plane + h;
@@ -737,6 +749,22 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[b]);
+            if (stage_tile) {
+                // the tile's token rows, 16 bytes a store
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                const int t_tile = min(BN, p.tokens - m0);
+                const int et = static_cast<int>(threadIdx.x) - 64;
+                const uint8_t* tile = a_ring;
+                for (int idx = et; idx < t_tile * (kTcRows / 8); idx += 128) {
+                    const int m = idx / (kTcRows / 8);
+                    const int hh = ht * kTcRows + (idx % (kTcRows / 8)) * 8;
+                    if (hh < p.hidden)
+                        st_global_v4(p.partials + static_cast<size_t>(r) * plane +
+                                         static_cast<size_t>(m0 + m) * p.hidden + hh,
+                                     *reinterpret_cast<const uint4*>(tile + static_cast<size_t>(m) * kTcRows * 2 +
+                                                                     (idx % (kTcRows / 8)) * 16));
+                }
+            }
             if (kCluster) {
                 // Every CTA of the cluster has its partial tile in shared memory
                 // once each has arrived on everyone's fold_ready.

@@ -70,13 +70,13 @@ struct Tc2Params {
 // S2-S4 of one half tile (128 rows from h0, tokens m0 .. m1-1) from the
 // staged partials, by the 128 epilogue threads (et): 16-byte vectors of 8
 // rows, V of them in flight per thread, each folded in ring order from its
-// chunk's owner (all N loads before the first add), the residual added.
-template <int V>
+// chunk's owner (all N <= NR loads before the first add), the residual added.
+template <int V, int NR>
 __device__ __forceinline__ void tc2_fold_half(const Tc2Params& p, int h0, int m0, int m1, int et) {
     const size_t plane = static_cast<size_t>(p.tokens) * p.hidden;
     const int total = (m1 - m0) * (kTcRows / 8);
     for (int v0 = et; v0 < total; v0 += V * 128) {
-        uint4 pv[V][kMaxRanks], rv[V];
+        uint4 pv[V][NR], rv[V];
         size_t off[V];
         int c[V];
         bool ok[V];
@@ -90,7 +90,7 @@ __device__ __forceinline__ void tc2_fold_half(const Tc2Params& p, int h0, int m0
             c[j] = h / p.hc;
             if (ok[j]) {
 #pragma unroll
-                for (int i = 0; i < kMaxRanks; ++i)
+                for (int i = 0; i < NR; ++i)
                     if (i < p.n_ranks) {
                         int rr = c[j] + i;
                         if (rr >= p.n_ranks) rr -= p.n_ranks;
@@ -104,7 +104,7 @@ __device__ __forceinline__ void tc2_fold_half(const Tc2Params& p, int h0, int m0
             if (!ok[j]) continue;
             uint4 sum = pv[j][0];
 #pragma unroll
-            for (int i = 1; i < kMaxRanks; ++i)
+            for (int i = 1; i < NR; ++i)
                 if (i < p.n_ranks) sum = bf16x8_add_tc(sum, pv[j][i]);
             st_global_v4(p.out + off[j], bf16x8_add_tc(rv[j], sum));
         }
@@ -339,8 +339,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
                     const int h0 = hp * 2 * kTcRows + static_cast<int>(rank) * kTcRows;
                     const int m1 = min(p.tokens, m0 + kTc2Tokens);
                     const int et = static_cast<int>(threadIdx.x) - 64;
-                    if (p.n_ranks <= 4) tc2_fold_half<4>(p, h0, m0, m1, et);
-                    else tc2_fold_half<2>(p, h0, m0, m1, et);
+                    if (p.n_ranks <= 4) tc2_fold_half<4, 4>(p, h0, m0, m1, et);
+                    else tc2_fold_half<2, kMaxRanks>(p, h0, m0, m1, et);
                     if (threadIdx.x == 64) *cnt = 0u;   // zero for the next call
                 }
             }

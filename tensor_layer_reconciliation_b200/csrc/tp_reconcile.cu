@@ -693,10 +693,6 @@ int tp_plan_kernel_variant(const tp_plan* plan, int64_t tokens) {
 // their partials for a ring kernel.
 constexpr int64_t kFoldMaxTokens = 2;
 
-static bool tc_cluster_folds(const tp_plan* plan, int64_t tokens) {
-    return tokens > 0 && tc_config(plan, tokens, true).cluster_fold;
-}
-
 static bool tc_folds(const tp_plan* plan, int64_t tokens, int fmt = tpr::kFmtBf16) {
     if (tokens <= kFoldMaxTokens) return true;
     const TcConfig c = tc_config(plan, tokens, true, fmt);
