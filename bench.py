@@ -64,22 +64,22 @@ def _peaks():
 # sources means the kernels changed since, and the traffic is reported null.
 PROFILED_TRAFFIC = {
     # (workload, path): (bytes per call, kernel-source digest, the ncu capture)
-    ("decode_n2", "tensor"): (118179712, "6a43f336d1b1fa29",
-                              "ncu dram__bytes of tc_partial_kernel<32> (k-split, in-kernel fold) "
-                              "on decode_n2, one step"),
-    ("decode_n4_m32", "tensor"): (119969664, "6a43f336d1b1fa29",
-                                  "ncu dram__bytes of tc_partial_kernel<32> + ring_reduce_kernel "
-                                  "on decode_n4_m32, one step"),
-    ("decode_n8_m64", "tensor"): (83670016, "6a43f336d1b1fa29",
-                                  "ncu dram__bytes of tc_partial_kernel<64> + ring_reduce_kernel "
-                                  "on decode_n8_m64, one step"),
-    ("prefill_n4", "tensor"): (832162304, "6a43f336d1b1fa29",
-                               "ncu dram__bytes of tc2_partial_kernel + ring_reduce_kernel "
-                               "on prefill_n4, one step"),
-    ("decode_n2", "exact-fused"): (117850112, "6a43f336d1b1fa29",
-                                   "ncu dram__bytes of exact_partial_kernel<1> on decode_n2, one step"),
-    ("decode_n2", "mxfp8"): (61455872, "6a43f336d1b1fa29",
-                             "ncu dram__bytes of mx_reconcile_kernel<1> on decode_n2, one step"),
+    ("decode_n2", "tensor"): (118238720, "8afd34ef1960e26e",
+        "ncu dram__bytes of tc_partial_kernel<32> (counter fold) on decode_n2, one call per point kind"),
+    ("decode_n4_m32", "tensor"): (120671104, "8afd34ef1960e26e",
+        "ncu dram__bytes of tc_partial_kernel<32> + ring_reduce_kernel on decode_n4_m32, one call per point kind"),
+    ("decode_n8_m64", "tensor"): (83176320, "8afd34ef1960e26e",
+        "ncu dram__bytes of tc_partial_kernel<64> + ring_reduce_kernel on decode_n8_m64, one call per point kind"),
+    ("prefill_n4", "tensor"): (897310208, "8afd34ef1960e26e",
+        "ncu dram__bytes of tc2_partial_kernel (fold in the epilogue) on prefill_n4, one call per point kind"),
+    ("decode_n2", "exact-fused"): (118017280, "8afd34ef1960e26e",
+        "ncu dram__bytes of exact_partial_kernel<1> on decode_n2, one call per point kind"),
+    ("decode_n2", "mxfp8"): (63567872, "8afd34ef1960e26e",
+        "ncu dram__bytes of tc_partial_kernel<32> MXFP8 form on decode_n2, one call per point kind"),
+    ("decode_n2", "nvfp4"): (32577536, "8afd34ef1960e26e",
+        "ncu dram__bytes of tc_partial_kernel<32> NVFP4 form on decode_n2, one call per point kind"),
+    ("decode_n2", "tensor-cluster"): (118124672, "8afd34ef1960e26e",
+        "ncu dram__bytes of tc_partial_kernel<32> cluster fold on decode_n2, one call per point kind"),
 }
 
 
@@ -186,12 +186,13 @@ class Workload:
 
     def path_name(self):
         """Which kernels one call runs: 'tensor' (tensor-core partials),
-        'exact-staged', 'exact-fused', 'mxfp8' or 'nvfp4' (quantised shards)."""
+        'tensor-cluster' (the CLUSTER variant), 'exact-staged', 'exact-fused',
+        'mxfp8' or 'nvfp4' (quantised shards)."""
         if self.weights in ("mxfp8", "nvfp4"):
             return self.weights
         pl = next(iter(self.plans.values()))
         if pl.effective_variant(self.cfg.tokens) == "tensor":
-            return "tensor"
+            return "tensor-cluster" if pl.variant == "cluster" else "tensor"
         return "exact-staged" if pl.staged else "exact-fused"
 
     def launches_per_step(self):
@@ -671,6 +672,8 @@ def run_config(name, args, device, world, rank, local, peaks):
                    f"reconciliation call: tc_partial_kernel ({fold_where}; residual)"
                    if one_kernel else
                    "reconciliation call: tc_partial_kernel then a ring fold kernel"),
+        "tensor-cluster": ("reconciliation call: tc_partial_kernel, CLUSTER variant (the N ranks x K parts "
+                           "of a tile in one cluster, ring fold through distributed shared memory; residual)"),
     }[path]
     if tensor_bound:
         achieved = flops / (step_ms * 1e-3) / 1e12
