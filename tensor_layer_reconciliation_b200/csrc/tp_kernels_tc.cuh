@@ -51,11 +51,11 @@
 // (128 rows x 64 codes) and their scales instead of bf16 weight tiles; four
 // more warps (6-9) turn each code tile into the bf16 tile the MMA reads
 // (MXFP8: E4M3 * 2^s; NVFP4: E2M1 * E4M3 block scale * 2^g; exact in bf16
-// for the shards the formats' definitions allow), written in the same
-// 128-byte-swizzled K-major layout TMA gives the bf16 path, into one of
-// kCvtSlots converted slots; the MMA waits for its slot and frees it (and the stage,
-// whose activation tile it reads) when it is done. Everything after the MMA
-// -- the three epilogues -- is the same.
+// for the shards the formats' definitions allow), each thread one row, into
+// one of the converted slots in tensor memory beside the accumulators (a row
+// a lane, two bf16 a column); the MMA reads A from there, waits for its slot
+// and frees it (and the stage, whose activation tile it reads) when it is
+// done. Everything after the MMA -- the three epilogues -- is the same.
 // Accumulation order inside the tensor core is the hardware's; the partial
 // is the fp32 sum rounded once to bf16, like the oracle's, but only equal to
 // it where the two fp32 sums round to the same bf16 value.
@@ -68,13 +68,14 @@ namespace tpr {
 
 constexpr int kTcRows = 128;               // MMA M: weight rows per tile
 constexpr int kTcKBlock = 64;              // bf16 columns per staged block
-constexpr int kTcMaxStages = 12;
+constexpr int kTcMaxStages = 16;
 constexpr int kTcThreads = 192;            // producer, MMA and 4 epilogue warps
 constexpr int kTcMxThreads = 320;          // quantised weights: + 4 converter warps
 constexpr uint32_t kTcATile = kTcRows * kTcKBlock * 2;  // 16 KB
 // Quantised forms: converted bf16 tiles in flight between the converters and
-// the MMAs (k-block i goes to slot i % kCvtSlots).
-constexpr int kCvtSlots = 3;
+// the MMAs live in tensor memory beside the accumulators (k-block i goes to
+// slot i % slots; at most kCvtSlotsMax slots).
+constexpr int kCvtSlotsMax = 8;
 constexpr uint32_t kMxCodeTile = kTcRows * kTcKBlock;   // 8 KB of E4M3 codes
 constexpr uint32_t kMxScaleTile = kTcRows * 2;          // the 2 E8M0 scales of each row
 constexpr uint32_t kNvCodeTile = kTcRows * kTcKBlock / 2;  // 4 KB: two E2M1 codes a byte
@@ -298,35 +299,37 @@ __device__ __forceinline__ uint64_t f32_pair(float f) {
 
 // Widens row t of a staged E4M3 code tile (64 codes in a 64-byte row, placed
 // by TMA with the 64-byte swizzle: 16-byte chunk c of row t at chunk
-// c ^ ((t >> 1) & 3)), with its two E8M0 scales (codes 0-31, 32-63), into row
-// t of a bf16 A tile in the 128-byte-swizzled K-major layout (chunk q of row
-// t at q ^ (t & 7)). With the two swizzles the eight rows a quarter-warp
-// handles at once read and write eight different bank groups.
+// c ^ ((t >> 1) & 3)), with its two E8M0 scales (codes 0-31, 32-63), into
+// this thread's lane of a bf16 A tile in tensor memory: 32 columns from
+// taddr, two values a column, k ascending. With the swizzle the eight rows a
+// quarter-warp reads at once lie in eight different bank groups.
 __device__ __forceinline__ void mx_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
-                                               uint8_t* a_row, int t) {
+                                               uint32_t taddr, int t) {
     const uint32_t sb = *reinterpret_cast<const uint16_t*>(scale_row);
-    const uint64_t f0 = f32_pair(e8m0_to_f32(sb & 0xFFu)), f1 = f32_pair(e8m0_to_f32(sb >> 8));
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {                            // codes 16c .. 16c+15
-        const uint4 q = *reinterpret_cast<const uint4*>(code_row + 16 * (c ^ ((t >> 1) & 3)));
-        const uint64_t f = c < 2 ? f0 : f1;
-        uint32_t o[8];
-        e4m3x4_scaled_bf16(q.x, f, o[0], o[1]);
-        e4m3x4_scaled_bf16(q.y, f, o[2], o[3]);
-        e4m3x4_scaled_bf16(q.z, f, o[4], o[5]);
-        e4m3x4_scaled_bf16(q.w, f, o[6], o[7]);
-        const int q0 = (2 * c) ^ (t & 7), q1 = (2 * c + 1) ^ (t & 7);
-        *reinterpret_cast<uint4*>(a_row + q0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
-        *reinterpret_cast<uint4*>(a_row + q1 * 16) = make_uint4(o[4], o[5], o[6], o[7]);
+    for (int half = 0; half < 2; ++half) {                   // codes 32half .. 32half+31
+        const uint64_t f = f32_pair(e8m0_to_f32(half ? sb >> 8 : sb & 0xFFu));
+        uint32_t o[16];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;                     // codes 16c .. 16c+15
+            const uint4 q = *reinterpret_cast<const uint4*>(code_row + 16 * (c ^ ((t >> 1) & 3)));
+            e4m3x4_scaled_bf16(q.x, f, o[8 * cc + 0], o[8 * cc + 1]);
+            e4m3x4_scaled_bf16(q.y, f, o[8 * cc + 2], o[8 * cc + 3]);
+            e4m3x4_scaled_bf16(q.z, f, o[8 * cc + 4], o[8 * cc + 5]);
+            e4m3x4_scaled_bf16(q.w, f, o[8 * cc + 6], o[8 * cc + 7]);
+        }
+        tmem_st_16cols(taddr + 16 * half, o);
     }
 }
 
 // NVFP4 row: 32 bytes of codes (64 E2M1 values, the earlier k in the low
 // nibble; TMA's 32-byte swizzle puts half c of row t at half c ^ ((t >> 2) & 1)),
 // the row's four E4M3 block scales (one per 16 values) and the second-level
-// factor 2^g -> row t of a bf16 A tile as in mx_convert_row.
+// factor 2^g -> this thread's lane of a bf16 A tile in tensor memory, as in
+// mx_convert_row.
 __device__ __forceinline__ void nv_convert_row(const uint8_t* code_row, const uint8_t* scale_row,
-                                               float two_g, uint8_t* a_row, int t) {
+                                               float two_g, uint32_t taddr, int t) {
     const uint32_t sw = *reinterpret_cast<const uint32_t*>(scale_row);
     const uint32_t h01 = f16x2_from_e4m3x2(static_cast<uint16_t>(sw & 0xFFFFu));
     const uint32_t h23 = f16x2_from_e4m3x2(static_cast<uint16_t>(sw >> 16));
@@ -336,13 +339,17 @@ __device__ __forceinline__ void nv_convert_row(const uint8_t* code_row, const ui
     for (int c = 0; c < 2; ++c) {                            // codes 32c .. 32c+31
         const uint4 q = *reinterpret_cast<const uint4*>(code_row + 16 * (c ^ ((t >> 2) & 1)));
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};        // 8 codes a word
+        uint32_t o[16];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {                      // word i: codes 32c + 8i .. +7, block 2c + i/2
-            uint32_t o[4];
-            e2m1x8_scaled_bf16(w[i], f[2 * c + (i >> 1)], o);
-            const int qc = (4 * c + i) ^ (t & 7);          // 16-byte chunk of 8 bf16 values
-            *reinterpret_cast<uint4*>(a_row + qc * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+            uint32_t oo[4];
+            e2m1x8_scaled_bf16(w[i], f[2 * c + (i >> 1)], oo);
+            o[4 * i + 0] = oo[0];
+            o[4 * i + 1] = oo[1];
+            o[4 * i + 2] = oo[2];
+            o[4 * i + 3] = oo[3];
         }
+        tmem_st_16cols(taddr + 16 * c, o);
     }
 }
 
@@ -363,7 +370,14 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     constexpr bool MX = FMT != kFmtBf16;                        // converted on chip
     constexpr uint32_t kWTile = fmt_code_tile(FMT);             // weight bytes staged per block
     constexpr uint32_t kSTile = fmt_scale_tile(FMT);            // scale bytes staged per block
-    constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
+    // Tensor memory: two accumulators of BN columns; the quantised forms add
+    // their converted A slots (32 columns each: 128 rows x 64 bf16) after them,
+    // within 256 columns a CTA when two share an SM.
+    constexpr int kSlots = !MX ? 1 : BN <= 32 ? 6 : BN <= 64 ? 4 : 8;
+    constexpr uint32_t kSlotCol0 = 2 * BN;
+    constexpr uint32_t kTmemCols = MX ? (BN <= 64 ? 256u : 512u) : (2 * BN < 32 ? 32u : 2u * BN);
+    static_assert(!MX || (BN <= 128 && kSlotCol0 + 32 * kSlots <= kTmemCols && kSlots <= kCvtSlotsMax),
+                  "converted slots fit in tensor memory");
     constexpr uint32_t kIdesc = idesc_bf16_f32(kTcRows, BN);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -372,8 +386,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     const int S = p.stages;
     uint8_t* a_ring = smem;                                              // weight tiles (TMA)
     uint8_t* b_ring = a_ring + static_cast<size_t>(S) * kWTile;         // activation tiles
-    uint8_t* a_cvt = b_ring + static_cast<size_t>(S) * kBTile;          // MX: converted tiles
-    uint8_t* s_ring = a_cvt + (MX ? kCvtSlots * kTcATile : 0);           // MX: scale tiles
+    uint8_t* s_ring = b_ring + static_cast<size_t>(S) * kBTile;          // MX: scale tiles
     uint64_t* full = reinterpret_cast<uint64_t*>(s_ring + static_cast<size_t>(S) * kSTile);
     uint64_t* empty = full + kTcMaxStages;
     uint64_t* acc_full = empty + kTcMaxStages;   // [2]
@@ -381,9 +394,9 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     uint64_t* mma_done = acc_empty + 2;
     uint64_t* fold_ready = mma_done + 1;   // cluster fold: all N partial tiles written
     uint64_t* fold_freed = fold_ready + 1; // cluster fold: all N CTAs done reading mine
-    uint64_t* cvt_full = fold_freed + 1;           // MX: [kCvtSlots] converted tile ready (4 warps)
-    uint64_t* cvt_empty = cvt_full + kCvtSlots;    // MX: [kCvtSlots] converted tile read by the MMAs
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cvt_empty + kCvtSlots);
+    uint64_t* cvt_full = fold_freed + 1;              // MX: [kSlots] converted tile ready (4 warps)
+    uint64_t* cvt_empty = cvt_full + kCvtSlotsMax;    // MX: [kSlots] converted tile read by the MMAs
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cvt_empty + kCvtSlotsMax);
     // cluster fold: this CTA's bf16 partial tile, [BN tokens][128 rows]
     uint16_t* part_buf = reinterpret_cast<uint16_t*>(
         (reinterpret_cast<uintptr_t>(tmem_slot + 4) + 127) & ~static_cast<uintptr_t>(127));
@@ -448,7 +461,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         mbar_init(mma_done, 1);
         mbar_init(fold_ready, static_cast<uint32_t>(csize));
         mbar_init(fold_freed, static_cast<uint32_t>(csize));
-        for (int j = 0; j < kCvtSlots; ++j) {
+        for (int j = 0; j < kSlots; ++j) {
             mbar_init(&cvt_full[j], 4);
             mbar_init(&cvt_empty[j], 1);
         }
@@ -465,11 +478,13 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     const uint32_t tmem_base = *tmem_slot;
     pdl_launch_dependents();
 
-    // Converters: thread `row` of a group of four warps widens row `row` of
-    // the staged code tiles in issue order (k-block i into converted slot
-    // i % kCvtSlots). With the helpers (a CTA with one unit) the epilogue warps
-    // form a second group: group g then takes the k-blocks with i % 2 == g.
-    auto run_converters = [&](int row, int group) {
+    // Converters: a group of four warps, one per tensor-memory lane quarter;
+    // thread `row` (its lane) widens row `row` of the staged code tiles in
+    // issue order (k-block i into converted slot i % kSlots). With the helpers
+    // (a CTA with one unit) the epilogue warps form a second group: group g
+    // then takes the k-blocks with i % 2 == g.
+    auto run_converters = [&](int group) {
+        const int row = 32 * (warp & 3) + lane;
         if constexpr (MX) {
             const float two_g = FMT == kFmtNvfp4 ? ldexpf(1.0f, *p.nv_gexp) : 1.0f;
             int i = 0, s = 0, j = 0;
@@ -489,24 +504,26 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                             break;
                         }
                         const uint8_t* srow = s_ring + static_cast<size_t>(s) * kSTile;
-                        uint8_t* arow = a_cvt + static_cast<size_t>(j) * kTcATile + row * 128;
+                        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
+                                               kSlotCol0 + 32u * static_cast<uint32_t>(j);
                         if (FMT == kFmtMxfp8)
                             mx_convert_row(a_ring + static_cast<size_t>(s) * kWTile + row * kTcKBlock,
-                                           srow + row * 2, arow, row);
+                                           srow + row * 2, taddr, row);
                         else
                             nv_convert_row(a_ring + static_cast<size_t>(s) * kWTile + row * (kTcKBlock / 2),
-                                           srow + row * 4, two_g, arow, row);
-                        // generic-proxy writes, read next by the tensor core (async proxy)
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                                           srow + row * 4, two_g, taddr, row);
+                        // the tensor-memory stores are done before the MMA may read them
+                        tmem_st_wait();
+                        tc_fence_before_sync();
                         __syncwarp();
-                        if ((threadIdx.x & 31) == 0) mbar_arrive(&cvt_full[j]);
+                        if (lane == 0) mbar_arrive(&cvt_full[j]);
                     }
                     ++i;
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
                     }
-                    if (++j == kCvtSlots) {
+                    if (++j == kSlots) {
                         j = 0;
                         jph ^= 1u;
                     }
@@ -634,21 +651,27 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint64_t ad = smem_desc_k128(MX ? a_cvt + static_cast<size_t>(j) * kTcATile
-                                                          : a_ring + static_cast<size_t>(s) * kTcATile);
                     uint64_t bd = smem_desc_k128(b_ring + static_cast<size_t>(s) * kBTile);
                     if (x_atom) bd &= ~(0x3FFFull << 32);   // stride between 8-row groups: 0
+                    if constexpr (MX) {
+                        // A: the converted tile in tensor memory, 8 columns per 16 of K
+                        const uint32_t at = tmem_base + kSlotCol0 + 32u * static_cast<uint32_t>(j);
 #pragma unroll
-                    for (int kk = 0; kk < kTcKBlock / 16; ++kk)
-                        umma_bf16(d, ad + 2ull * kk, bd + 2ull * kk, kIdesc,
-                                  (kb != kb_lo) || (kk != 0));
+                        for (int kk = 0; kk < kTcKBlock / 16; ++kk)
+                            umma_bf16_ta(d, at + 8u * kk, bd + 2ull * kk, kIdesc, (kb != kb_lo) || (kk != 0));
+                    } else {
+                        const uint64_t ad = smem_desc_k128(a_ring + static_cast<size_t>(s) * kTcATile);
+#pragma unroll
+                        for (int kk = 0; kk < kTcKBlock / 16; ++kk)
+                            umma_bf16(d, ad + 2ull * kk, bd + 2ull * kk, kIdesc, (kb != kb_lo) || (kk != 0));
+                    }
                     umma_commit(&empty[s]);  // frees the stage when these MMAs finish
                     if (MX) umma_commit(&cvt_empty[j]);   // and the converted slot
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
                     }
-                    if (++j == kCvtSlots) {
+                    if (++j == kSlots) {
                         j = 0;
                         jph ^= 1u;
                     }
@@ -666,12 +689,12 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         }
     } else if (MX && warp >= 6) {
         // ------------------------------------ converters (quantised weights) --
-        run_converters(static_cast<int>(threadIdx.x) - 192, 0);
+        run_converters(0);
     } else {
         // ---------------------------------------------------------- epilogue --
         // A CTA with one unit has nothing for these warps until its MMAs end:
         // they widen every other code tile meanwhile.
-        if (MX && cvt_helpers) run_converters(static_cast<int>(threadIdx.x) - 64, 1);
+        if (MX && cvt_helpers) run_converters(1);
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         pdl_wait();  // the fold reads the residual and writes the output in stream order
         for (int lu = 0; lu < my_units; ++lu) {

@@ -255,6 +255,9 @@ int tc_token_tile(int64_t tokens) {
 TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt = tpr::kFmtBf16) {
     TcConfig c{};
     c.bn = tc_token_tile(tokens);
+    // quantised forms: token tiles up to 128 (their converted slots share
+    // tensor memory with the accumulators)
+    if (fmt != tpr::kFmtBf16) c.bn = std::min(c.bn, 128);
     c.h_tiles = static_cast<int>((p->hidden + tpr::kTcRows - 1) / tpr::kTcRows);
     c.m_tiles = static_cast<int>((tokens + c.bn - 1) / c.bn);
     const int base_units = p->n_ranks * c.h_tiles * c.m_tiles;
@@ -271,10 +274,9 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     // one portable cluster
     c.cluster_fold = allow_split && p->variant == TP_VARIANT_CLUSTER && base_units > 0 &&
                      c.bn <= 128 && c.splits <= 4 && p->n_ranks * c.splits <= 8;
-    // Quantised weights: a stage holds codes, scales and activations; two
-    // converted bf16 tiles sit beside the ring.
-    const bool quantised = fmt != tpr::kFmtBf16;
-    // at most 8 tokens: one 8-row atom of x a block instead of the BN-row tile
+    // Quantised weights: a stage holds codes, scales and activations (the
+    // converted bf16 tiles live in tensor memory).
+    // At most 8 tokens: one 8-row atom of x a block instead of the BN-row tile
     c.x_rows = tokens <= 8 && c.m_tiles == 1 ? 8 : c.bn;
     const size_t stage = tpr::fmt_code_tile(fmt) + tpr::fmt_scale_tile(fmt) +
                          static_cast<size_t>(c.x_rows) * tpr::kTcKBlock * 2;
@@ -283,8 +285,8 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     const size_t part_tile = c.cluster_fold ? static_cast<size_t>(std::min<int64_t>(c.bn, tokens)) *
                                                   tpr::kTcRows * (c.splits > 1 ? 4 : 2)
                                             : 0;
-    const size_t fixed = (2 * tpr::kTcMaxStages + 7 + 2 * tpr::kCvtSlots) * sizeof(uint64_t) + 16 + 128 +
-                         1024 + part_tile + (quantised ? tpr::kCvtSlots * tpr::kTcATile : 0);
+    const size_t fixed = (2 * tpr::kTcMaxStages + 7 + 2 * tpr::kCvtSlotsMax) * sizeof(uint64_t) + 16 + 128 +
+                         1024 + part_tile;
     const size_t budget = std::min<size_t>(two_per_sm ? 110 * 1024 : 200 * 1024,
                                            static_cast<size_t>(p->smem_optin));
     c.stages = budget > fixed
@@ -496,8 +498,12 @@ cudaError_t dispatch_tc(int bn, int mode, dim3 grid, size_t smem, cudaStream_t s
         return launch_tc_kernel<32, kTcCounterFold, MX>(grid, smem, st, 1, mw, mx, ms, prm);
     if (bn == 32) return launch_tc_kernel<32, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
     if (bn == 64) return launch_tc_kernel<64, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
-    if (bn == 128) return launch_tc_kernel<128, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
-    return launch_tc_kernel<256, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
+    if constexpr (MX != kFmtBf16) {   // quantised forms: token tiles up to 128
+        return launch_tc_kernel<128, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
+    } else {
+        if (bn == 128) return launch_tc_kernel<128, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
+        return launch_tc_kernel<256, kTcStore, MX>(grid, smem, st, 1, mw, mx, ms, prm);
+    }
 }
 
 // allow_split (a reconciliation call): the kernel also runs S2-S4 (residual,
@@ -584,7 +590,6 @@ tp_status launch_ring(const tp_plan* p, const void* partials, const void* residu
     reinterpret_cast<const void*>(tpr::tc_partial_kernel<32, tpr::kTcStore, MX>),          \
         reinterpret_cast<const void*>(tpr::tc_partial_kernel<64, tpr::kTcStore, MX>),      \
         reinterpret_cast<const void*>(tpr::tc_partial_kernel<128, tpr::kTcStore, MX>),     \
-        reinterpret_cast<const void*>(tpr::tc_partial_kernel<256, tpr::kTcStore, MX>),     \
         reinterpret_cast<const void*>(tpr::tc_partial_kernel<32, tpr::kTcCounterFold, MX>), \
         reinterpret_cast<const void*>(tpr::tc_partial_kernel<32, tpr::kTcClusterFold, MX>), \
         reinterpret_cast<const void*>(tpr::tc_partial_kernel<64, tpr::kTcClusterFold, MX>), \
@@ -599,6 +604,7 @@ cudaError_t set_kernel_attrs(int smem_optin, int* dyn_max) {
         reinterpret_cast<const void*>(tpr::exact_partial_kernel<4>),
         reinterpret_cast<const void*>(tpr::exact_partial_kernel<8>),
         TC_KERNELS(tpr::kFmtBf16), TC_KERNELS(tpr::kFmtMxfp8), TC_KERNELS(tpr::kFmtNvfp4),
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<256, tpr::kTcStore, tpr::kFmtBf16>),
         reinterpret_cast<const void*>(tpr::tc2_partial_kernel)};
     int lowest = smem_optin;
     for (const void* k : kernels) {
