@@ -396,7 +396,10 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     uint64_t* fold_freed = fold_ready + 1; // cluster fold: all N CTAs done reading mine
     uint64_t* cvt_full = fold_freed + 1;              // MX: [kSlots] converted tile ready (4 warps)
     uint64_t* cvt_empty = cvt_full + kCvtSlotsMax;    // MX: [kSlots] converted tile read by the MMAs
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cvt_empty + kCvtSlotsMax);
+    // MX: [S] a stage's activation block landed (its codes and scales land on
+    // full[s], so the converters need not wait for the dependency)
+    uint64_t* full_x = cvt_empty + kCvtSlotsMax;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full_x + kTcMaxStages);
     // cluster fold: this CTA's bf16 partial tile, [BN tokens][128 rows]
     uint16_t* part_buf = reinterpret_cast<uint16_t*>(
         (reinterpret_cast<uintptr_t>(tmem_slot + 4) + 127) & ~static_cast<uintptr_t>(127));
@@ -452,6 +455,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         abort_flag = 0;
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&full_x[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -538,7 +542,9 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             tma_prefetch_desc(&tmap_w);
             tma_prefetch_desc(&tmap_x);
             if (MX) tma_prefetch_desc(&tmap_s);
-            const uint32_t tx = kWTile + kBTile + kSTile;
+            // bytes landing on full[s]: the whole stage, or (MX) codes and scales
+            // only, the activation block then counting on full_x[s]
+            const uint32_t tx = MX ? kWTile + kSTile : kWTile + kBTile + kSTile;
             // The weights of one k-block (and, MX, their scales) into stage st.
             // (NVFP4 code tiles hold two codes a byte: 32 bytes per 64-column block)
             constexpr int kWCols = FMT == kFmtNvfp4 ? kTcKBlock / 2 : kTcKBlock;
@@ -595,7 +601,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 Cursor c0{0, 0, 0, 0, 0, 0, 0};
                 enter_unit(c0);
                 for (int i = 0; i < pre; ++i) {
-                    tma_load_3d(b_ring + static_cast<size_t>(i) * kBTile, &tmap_x, &full[i],
+                    if (MX) mbar_arrive_expect_tx(&full_x[i], kBTile);
+                    tma_load_3d(b_ring + static_cast<size_t>(i) * kBTile, &tmap_x, MX ? &full_x[i] : &full[i],
                                 c0.kb * kTcKBlock, c0.r, c0.mt * BN);
                     advance(c0);
                 }
@@ -611,7 +618,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
                 mbar_arrive_expect_tx(&full[s], tx);
                 load_w(s, cur.kb, cur.ht, cur.r);
-                tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, &full[s],
+                if (MX) mbar_arrive_expect_tx(&full_x[s], kBTile);
+                tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, MX ? &full_x[s] : &full[s],
                             cur.kb * kTcKBlock, cur.r, cur.mt * BN);
                 ++issued;
                 advance(cur);
@@ -625,7 +633,9 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             // results are then invalid and the context should be discarded.
             const int first = issued > S ? issued - S : 0;
             for (int i = first; i < issued; ++i)
-                if (!mbar_wait_bounded(&full[i % S], static_cast<uint32_t>(i / S) & 1u)) break;
+                if (!mbar_wait_bounded(&full[i % S], static_cast<uint32_t>(i / S) & 1u) ||
+                    (MX && !mbar_wait_bounded(&full_x[i % S], static_cast<uint32_t>(i / S) & 1u)))
+                    break;
         }
     } else if (warp == 1) {
         // --------------------------------------------------------- MMA issue --
@@ -646,7 +656,9 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 split_range(sp, kb_lo, kb_hi);
                 bool ok = true;
                 for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
-                    if (!mbar_wait_bounded(&full[s], ph) || (MX && !mbar_wait_bounded(&cvt_full[j], jph))) {
+                    // MX: the converters consumed the codes; the MMA needs the activations
+                    if (!mbar_wait_bounded(MX ? &full_x[s] : &full[s], ph) ||
+                        (MX && !mbar_wait_bounded(&cvt_full[j], jph))) {
                         ok = false;
                         break;
                     }

@@ -285,7 +285,7 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     const size_t part_tile = c.cluster_fold ? static_cast<size_t>(std::min<int64_t>(c.bn, tokens)) *
                                                   tpr::kTcRows * (c.splits > 1 ? 4 : 2)
                                             : 0;
-    const size_t fixed = (2 * tpr::kTcMaxStages + 7 + 2 * tpr::kCvtSlotsMax) * sizeof(uint64_t) + 16 + 128 +
+    const size_t fixed = (3 * tpr::kTcMaxStages + 7 + 2 * tpr::kCvtSlotsMax) * sizeof(uint64_t) + 16 + 128 +
                          1024 + part_tile;
     const size_t budget = std::min<size_t>(two_per_sm ? 110 * 1024 : 200 * 1024,
                                            static_cast<size_t>(p->smem_optin));
