@@ -115,11 +115,15 @@ TP_API tp_status tp_plan_set_variant(tp_plan* plan, int variant, int staged);
  * folds them (one or two tokens: the CTA holding a tile's last ticket; more
  * than 128 tokens on CTA pairs: the CTA storing a half tile's last rank) or
  * a ring kernel does: N*M*H*2 bytes (bf16), or splits*N*M*H*4 (fp32 sums of
- * K parts) when it splits K across CTAs to fill the SMs. Layout: a counter
- * block (256-byte rounded) of two 32-bit counters per 128-row H tile
- * (tickets taken, parts stored), or, if more, two per 256-row x 256-token
- * tile of max_tokens (ranks stored per half tile), then the partials.
- * Rounded up to 256 in all. Returns 0 for a null plan or tokens <= 0. */
+ * K parts) when it splits K across CTAs to fill the SMs; one or two tokens
+ * store each part with its call's tag in one 8-byte word (N*M*H*8, or
+ * splits*N*M*H*8).
+ * Layout: a counter block (256-byte rounded) of 32-bit words -- per 128-row
+ * H tile a ticket count (zero between calls) and a fold count (one more each
+ * call), then per 256-row x 256-token tile of max_tokens two rank counts
+ * (zero between calls) -- then the partials. Rounded up to 256 in all.
+ * Returns 0 for a null plan or tokens <= 0. A workspace a call left with a
+ * device error flag set must be zeroed again before its next use. */
 TP_API size_t tp_plan_workspace_bytes(const tp_plan* plan, int64_t tokens);
 
 /* The partial kernel a call with `tokens` tokens runs under the plan's
@@ -190,9 +194,10 @@ TP_API tp_status tp_rowlinear_reconcile(const tp_plan* plan, const void* x, cons
  *  - Every call, from every plan and thread on a device, shares the one
  *    array, which keeps the last call's partials; each call writes every
  *    partial it reads. The fold counters at its start are zero when the
- *    library is loaded and every call that sets no device error flag leaves
- *    them zero; after one that does, this entry point may give wrong results
- *    until tp_device_error_flags with reset != 0 clears them. Calls whose kernels overlap
+ *    library is loaded; every call that sets no device error flag leaves the
+ *    ticket counts at zero (and each tile's fold count one higher); after one
+ *    that does, this entry point may give wrong results until
+ *    tp_device_error_flags with reset != 0 clears the whole array. Calls whose kernels overlap
  *    on the GPU (different streams without ordering between them) race on
  *    the array and give wrong results: order them on one stream.
  * The pages describe no counterpart of this entry point. */

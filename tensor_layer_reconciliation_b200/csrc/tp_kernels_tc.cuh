@@ -111,10 +111,10 @@ struct TcParams {
     int stages;    // 2 .. kTcMaxStages
     int x_rows;    // token rows of x staged per block: BN, or 8 (one swizzle atom) for at most 8 tokens
     uint16_t* partials;     // [N][M][H] bf16 (splits == 1)
-    float* partials_f32;    // [splits][N][M][H] fp32 sums of each k part (splits > 1)
+    float* partials_f32;    // [splits][N][M][H] fp32 sums of each k part (splits > 1); the 64-bit tagged parts of the counter fold
 
     int hc;                       // H / N, the chunk each rank owns in the ring
-    unsigned int* counters;       // [2][h_tiles * m_tiles]: tickets taken, parts stored; zero between calls
+    unsigned int* counters;       // [2][h_tiles * m_tiles]: tickets taken (zero between calls), folds done
     const uint16_t* x;            // [M][K] activations (for the L2 prefetch)
     int64_t k;                    // K
     const uint16_t* residual;     // [M][H]
@@ -351,6 +351,114 @@ __device__ __forceinline__ void nv_convert_row(const uint8_t* code_row, const ui
         }
         tmem_st_16cols(taddr + 16 * c, o);
     }
+}
+
+// Counter fold: K parts carry the tag of their call (the tile's fold count
+// + 1) in the same 64-bit word -- the fp32 part, or the bf16 partial when K is
+// not split, in the low half, the tag in the high half -- so the CTA folding
+// a tile reads them without waiting for a count: a part whose tag is not yet
+// this call's is read again (bounded). Word-sized stores and loads are
+// single-copy atomic, so a part is never seen half-written.
+__device__ __forceinline__ uint64_t ld_cg_u64(const uint64_t* p) {
+    return __ldcg(reinterpret_cast<const unsigned long long*>(p));
+}
+// The low half of a tagged part once its tag is `tag` (read again until then).
+__device__ __forceinline__ bool tagged_part(const uint64_t* p, uint32_t tag, uint32_t& v) {
+    uint64_t w = ld_cg_u64(p);
+    if (static_cast<uint32_t>(w >> 32) != tag) {
+        const uint64_t t0 = globaltimer_ns();
+        while (static_cast<uint32_t>((w = ld_cg_u64(p)) >> 32) != tag)
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(&g_device_error, kErrWaitTimeout);
+                return false;
+            }
+    }
+    v = static_cast<uint32_t>(w);
+    return true;
+}
+
+// S2-S3 of one output element from tagged parts: rank r's partial is the sum
+// of its SPLITS fp32 parts in split (k) order rounded once to bf16 (or its
+// bf16 partial when SPLITS == 1); the N partials are added in ring order
+// from the chunk's owner c. All loads are issued before the first check
+// (up to 16 of them at once; more go a rank at a time).
+__device__ __forceinline__ bool fold_tagged(const TcParams& p, size_t plane, size_t off, int c, uint32_t tag,
+                                            uint16_t& out) {
+    const int n = p.n_ranks, splits = p.splits;
+    bool ok = true;
+    uint16_t s = 0;
+    const uint64_t* parts = reinterpret_cast<const uint64_t*>(p.partials_f32);
+    if (splits == 1) {   // bf16 partials
+        uint64_t w[kMaxRanks];
+#pragma unroll
+        for (int i = 0; i < kMaxRanks; ++i)
+            if (i < n) {
+                int rr = c + i;
+                if (rr >= n) rr -= n;
+                w[i] = ld_cg_u64(parts + static_cast<size_t>(rr) * plane + off);
+            }
+#pragma unroll
+        for (int i = 0; i < kMaxRanks; ++i)
+            if (i < n) {
+                uint32_t v = static_cast<uint32_t>(w[i]);
+                if (static_cast<uint32_t>(w[i] >> 32) != tag) {
+                    int rr = c + i;
+                    if (rr >= n) rr -= n;
+                    ok = tagged_part(parts + static_cast<size_t>(rr) * plane + off, tag, v) && ok;
+                }
+                s = i == 0 ? static_cast<uint16_t>(v) : bf16_add(s, static_cast<uint16_t>(v));
+            }
+        out = s;
+        return ok;
+    }
+    if (n * splits <= 16) {
+        uint64_t w[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < n * splits) {
+                const int i = j / splits, sp = j - i * splits;
+                int rr = c + i;
+                if (rr >= n) rr -= n;
+                w[j] = ld_cg_u64(parts + (static_cast<size_t>(sp) * n + rr) * plane + off);
+            }
+        float f = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < n * splits) {
+                const int i = j / splits, sp = j - i * splits;
+                uint32_t vb = static_cast<uint32_t>(w[j]);
+                if (static_cast<uint32_t>(w[j] >> 32) != tag) {
+                    int rr = c + i;
+                    if (rr >= n) rr -= n;
+                    ok = tagged_part(parts + (static_cast<size_t>(sp) * n + rr) * plane + off, tag, vb) && ok;
+                }
+                const float v = __uint_as_float(vb);
+                f = sp == 0 ? v : __fadd_rn(f, v);
+                if (sp == splits - 1) {
+                    const uint16_t pr = f32_to_bf16_rne(f);
+                    s = i == 0 ? pr : bf16_add(s, pr);
+                }
+            }
+        out = s;
+        return ok;
+    }
+#pragma unroll 1
+    for (int i = 0; i < n; ++i) {
+        int rr = c + i;
+        if (rr >= n) rr -= n;
+        float f = 0.0f;
+#pragma unroll 1
+        for (int sp = 0; sp < splits; ++sp) {
+            uint32_t vb = 0;
+            ok = tagged_part(parts + (static_cast<size_t>(sp) * n + rr) * plane + off, tag, vb) && ok;
+            const float v = __uint_as_float(vb);
+            f = sp == 0 ? v : __fadd_rn(f, v);
+        }
+        const uint16_t pr = f32_to_bf16_rne(f);
+        s = i == 0 ? pr : bf16_add(s, pr);
+    }
+    out = s;
+    return ok;
 }
 
 // Token tiles up to 64 run two CTAs per SM: at most 168 registers a thread
@@ -729,8 +837,13 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             const size_t plane = static_cast<size_t>(p.tokens) * p.hidden;
             // Counter fold: this CTA's place among the parts of its tile, taken
             // now so the round trip overlaps the stores below.
-            unsigned int ticket = 0;
-            if (MODE == kTcCounterFold && threadIdx.x == 64) ticket = atomicAdd(p.counters + ht * p.m_tiles + mt, 1u);
+            unsigned int ticket = 0, tag = 0;
+            if (MODE == kTcCounterFold) {
+                if (threadIdx.x == 64) ticket = atomicAdd(p.counters + ht * p.m_tiles + mt, 1u);
+                // this call's tag: the tile's folds so far + 1 (the previous
+                // call's fold is complete: the epilogue waited for the dependency)
+                tag = __ldcg(p.counters + p.h_tiles * p.m_tiles + ht * p.m_tiles + mt) + 1u;
+            }
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
@@ -760,9 +873,33 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                                     q * 32 + lane;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) dst[i * kTcRows] = f32_to_bf16_rne(__uint_as_float(v[i]));
+                } else if (MODE == kTcCounterFold) {
+                    if (h < p.hidden) {
+                        if (p.splits == 1) {   // (bf16, tag) words [N][M][H]
+                            uint64_t* dst = reinterpret_cast<uint64_t*>(p.partials_f32) + static_cast<size_t>(r) * plane + h;
+#pragma unroll
+                            for (int i = 0; i < 2; ++i) {   // at most two tokens
+                                const int m = m0 + c0 + i;
+                                if (m < p.tokens)
+                                    dst[static_cast<size_t>(m) * p.hidden] =
+                                        (static_cast<uint64_t>(tag) << 32) | f32_to_bf16_rne(__uint_as_float(v[i]));
+                            }
+                        } else {               // (fp32, tag) words [splits][N][M][H]
+                            uint64_t* dst = reinterpret_cast<uint64_t*>(p.partials_f32) +
+                                            (static_cast<size_t>(sp) * p.n_ranks + r) * plane + h;
+#pragma unroll
+                            for (int i = 0; i < 2; ++i) {
+                                const int m = m0 + c0 + i;
+                                if (m < p.tokens)
+                                    dst[static_cast<size_t>(m) * p.hidden] =
+                                        (static_cast<uint64_t>(tag) << 32) | v[i];
+                            }
+                        }
+                    }
                 } else if (h < p.hidden) {
                     if (p.splits == 1) {
                         uint16_t* dst = p.partials + static_cast<size_t>(r) * plane + h;
+
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
                             const int m = m0 + c0 + i;
@@ -829,55 +966,33 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             }
             if (MODE == kTcCounterFold) {
                 // The CTA holding the last ticket of this (H tile, token tile)
-                // folds it once every other part is stored: ring order, residual
-                // add. The others count their stored part and leave.
+                // folds it: ring order, residual add. Its parts are read by tag,
+                // so the other CTAs leave as soon as their parts are stored.
                 uint16_t res[2] = {0, 0};   // this thread's residual, loaded meanwhile
                 if (h < p.hidden)
                     for (int m = m0, i = 0; m < p.tokens && i < 2; ++m, ++i)
                         res[i] = p.residual[static_cast<size_t>(m) * p.hidden + h];
                 unsigned int* tickets = p.counters + ht * p.m_tiles + mt;
-                unsigned int* stored = tickets + p.h_tiles * p.m_tiles;
-                const unsigned int last = static_cast<unsigned int>(p.n_ranks * p.splits - 1);
-                asm volatile("bar.sync 2, 128;" ::: "memory");   // this CTA's part is stored
-                if (threadIdx.x == 64) {
-                    int mine = ticket == last;
-                    if (!mine) {
-                        red_release_add(stored, 1u);
-                    } else if (ld_acquire_gpu(stored) != last) {
-                        const uint64_t t0 = globaltimer_ns();
-                        while (ld_acquire_gpu(stored) != last) {
-                            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                                atomicOr(&g_device_error, kErrWaitTimeout);
-                                atomicExch(&abort_flag, 1);
-                                mine = 0;
-                                break;
-                            }
-                        }
-                    }
-                    fold_mine = mine;
-                }
+                unsigned int* folds = tickets + p.h_tiles * p.m_tiles;
+                if (threadIdx.x == 64) fold_mine = ticket == static_cast<unsigned int>(p.n_ranks * p.splits - 1);
                 asm volatile("bar.sync 2, 128;" ::: "memory");
                 if (fold_mine) {
+                    bool ok = true;
                     if (h < p.hidden) {
                         const int c = h / p.hc;
                         // at most two tokens here (m_tiles == 1, tokens <= 2); this
-                        // CTA's own part is read back by the thread that stored it
+                        // thread's own part it stored itself
                         for (int m = m0, i = 0; m < p.tokens && i < 2; ++m, ++i) {
                             const size_t off = static_cast<size_t>(m) * p.hidden + h;
-                            const uint16_t sum =
-                                p.splits == 1
-                                    ? ring_fold_bf16<true>(p.partials, p.n_ranks, plane, off, c)
-                                : p.n_ranks * p.splits <= 16
-                                    ? ring_fold_f32_parts16<true>(p.partials_f32, p.splits,
-                                                                  p.n_ranks, plane, off, c)
-                                    : ring_fold_f32_parts_by_rank<true>(p.partials_f32, p.splits,
-                                                                        p.n_ranks, plane, off, c);
+                            uint16_t sum = 0;
+                            ok = fold_tagged(p, plane, off, c, tag, sum) && ok;
                             p.out[off] = bf16_add(res[i], sum);
                         }
                     }
-                    if (threadIdx.x == 64) {   // zero for the next call
+                    if (!ok) atomicExch(&abort_flag, 1);
+                    if (threadIdx.x == 64) {   // for the next call
+                        *folds = tag;
                         *tickets = 0u;
-                        *stored = 0u;
                     }
                 }
             }

@@ -239,6 +239,7 @@ tp_status launch_exact(const tp_plan* p, const void* x, const void* w, const voi
 struct TcConfig {
     int bn, stages, grid, units, h_tiles, m_tiles, splits, x_rows;
     bool cluster_fold;   // the N ranks of a tile on one cluster, folded on chip
+    bool splits_allowed; // a reconciliation call (the kernel may fold; K may be split)
     size_t smem;
 };
 
@@ -254,6 +255,7 @@ int tc_token_tile(int64_t tokens) {
 // fold on chip in clusters of those CTAs.
 TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt = tpr::kFmtBf16) {
     TcConfig c{};
+    c.splits_allowed = allow_split;
     c.bn = tc_token_tile(tokens);
     // quantised forms: token tiles up to 128 (their converted slots share
     // tensor memory with the accumulators)
@@ -342,8 +344,11 @@ tp_status encode_tc_maps(const tp_plan* p, int x_box_tokens, const void* x, cons
 // The tensor-core partials: bf16 [N][M][H] when the units are not split, or
 // fp32 k-part sums [splits][N][M][H] (allow_split) for the ring kernel to add.
 size_t tc_partial_bytes(const tp_plan* p, const TcConfig& c, int64_t tokens) {
-    return static_cast<size_t>(p->n_ranks) * static_cast<size_t>(tokens) *
-           static_cast<size_t>(p->hidden) * (c.splits > 1 ? 4u * c.splits : 2u);
+    // the counter fold (a reconciliation of one or two tokens) stores its
+    // parts with their call's tag: 8 bytes a part
+    const bool tagged = c.splits_allowed && tokens <= 2 && !c.cluster_fold;
+    const size_t elem = tagged ? 8u * c.splits : c.splits > 1 ? 4u * c.splits : 2u;
+    return static_cast<size_t>(p->n_ranks) * static_cast<size_t>(tokens) * static_cast<size_t>(p->hidden) * elem;
 }
 
 // Calls that run on CTA pairs: bf16 shards, prefill-sized token tiles, no
@@ -519,7 +524,9 @@ tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* 
     // Prefill-sized bf16 tiles without a k-split run on CTA pairs (2-SM MMA),
     // which fold in their epilogue with `fold`.
     if (tc2_path(p, c, wt.fmt))
-        return launch_tc2(p, x, wt.w, partials, tokens, stream, fold, counters, residual, out);
+        return launch_tc2(p, x, wt.w, partials, tokens, stream, fold,
+                          counters ? counters + 2 * c.h_tiles : nullptr,   // after the counter fold's words
+                          residual, out);
     if (fold && (c.m_tiles != 1 || tokens > 2)) return TP_ERR_UNSUPPORTED;  // the kernel folds <= 2 rows
     CUtensorMap mw, mx, ms;
     tp_status st = encode_tc_maps(p, c.x_rows, x, wt.w, tokens, &mw, &mx);
@@ -709,12 +716,15 @@ static bool tc_folds(const tp_plan* plan, int64_t tokens, int fmt = tpr::kFmtBf1
 // 128-row H tile (tickets taken, parts stored), 256-byte rounded, reserved
 // on every staged path so that calls of other variants or token counts
 // sharing the workspace leave the counters alone.
+static size_t counter_tiles(const tp_plan* plan) {
+    return static_cast<size_t>((plan->hidden + tpr::kTcRows - 1) / tpr::kTcRows);
+}
 static size_t counter_block_bytes(const tp_plan* plan) {
-    const size_t tiles = static_cast<size_t>((plan->hidden + tpr::kTcRows - 1) / tpr::kTcRows);
-    // CTA pairs: one counter per half tile (128 rows x 256 tokens)
+    // CTA pairs: one counter per half tile (128 rows x 256 tokens), after the
+    // counter fold's tickets and fold counts
     const size_t pair_words = 2 * static_cast<size_t>((plan->hidden + 2 * tpr::kTcRows - 1) / (2 * tpr::kTcRows)) *
                               static_cast<size_t>((plan->max_tokens + tpr::kTc2Tokens - 1) / tpr::kTc2Tokens);
-    return (std::max(2 * tiles, pair_words) * 4 + 255) / 256 * 256;
+    return ((2 * counter_tiles(plan) + pair_words) * 4 + 255) / 256 * 256;
 }
 
 // Bytes of staged partials a call writes (0: none, the exact fused kernel).
@@ -1163,8 +1173,9 @@ tp_status tp_device_error_flags(const tp_plan* plan, uint32_t* flags, int reset)
         if ((e = cudaMemcpyToSymbol(tpr::g_device_error, &zero, sizeof zero)) != cudaSuccess)
             return cuda_fail(e);
         // A call that ran out of a wait may have left fold counters of the
-        // no-alloc scratch above zero; clear them (device idle: synchronised above).
-        if (v != 0 && (e = cudaMemset(plan->noalloc_scratch, 0, kNoAllocCounterBytes)) != cudaSuccess)
+        // no-alloc scratch above zero and parts of any tag in it; clear it all
+        // (device idle: synchronised above).
+        if (v != 0 && (e = cudaMemset(plan->noalloc_scratch, 0, kNoAllocScratchBytes)) != cudaSuccess)
             return cuda_fail(e);
     }
     *flags = v;

@@ -177,8 +177,9 @@ def test_auto_uses_tensor_cores():
 
 def test_fold_counters_return_to_zero():
     """One zeroed workspace serves many calls: the in-kernel fold (one or two
-    tokens) counts stored parts per tile in the workspace's first bytes and
-    the folding CTA sets each count back to zero."""
+    tokens) hands out tickets per tile in the workspace's first words (the
+    folding CTA sets them back to zero) and counts each tile's folds in the
+    next ones (the tag its parts carry the next call)."""
     import tensor_layer_reconciliation_b200 as tlr
     dev = torch.device("cuda")
     n, k, h = 4, 4096, 640
@@ -187,9 +188,8 @@ def test_fold_counters_return_to_zero():
         assert plan.launches(m) == 1                   # partials and fold in one kernel
         need = plan.workspace_bytes(m)
         ws = torch.zeros(need, dtype=torch.uint8, device=dev)
-        h_tiles = (h + 127) // 128                     # tickets and stored parts per tile
-        counter_bytes = (2 * h_tiles * 4 + 255) // 256 * 256
-        for seed in (31, 32, 33):
+        h_tiles = (h + 127) // 128                     # tickets, then folds done, per tile
+        for call, seed in enumerate((31, 32, 33)):
             x, w, r = inputs(n, m, k, h, seed + 10 * m, dev)
             wp = plan.pack_weights(w)
             out = plan.reconcile(x, wp, r, workspace=ws)
@@ -197,7 +197,9 @@ def test_fold_counters_return_to_zero():
             torch.cuda.synchronize()
             assert plan.device_error_flags() == 0
             assert torch.equal(out.view(torch.int16), fresh.view(torch.int16))
-            assert int(torch.count_nonzero(ws[:counter_bytes])) == 0
+            words = ws[:8 * h_tiles].view(torch.int32).cpu()
+            assert int(torch.count_nonzero(words[:h_tiles])) == 0          # tickets
+            assert torch.equal(words[h_tiles:2 * h_tiles], torch.full((h_tiles,), call + 1, dtype=torch.int32))
     assert plan.launches(3) == 2                       # from three tokens: a ring kernel follows
 
 
@@ -213,7 +215,7 @@ def test_pair_fold_counters_return_to_zero():
     need = plan.workspace_bytes(m)
     ws = torch.zeros(need, dtype=torch.uint8, device=dev)
     pair_words = 2 * ((h + 255) // 256) * ((m + 255) // 256)
-    counter_bytes = (max(2 * ((h + 127) // 128), pair_words) * 4 + 255) // 256 * 256
+    counter_bytes = ((2 * ((h + 127) // 128) + pair_words) * 4 + 255) // 256 * 256
     for seed in (41, 42):
         x, w, r = inputs(n, m, k, h, seed, dev)
         wp = plan.pack_weights(w)
