@@ -288,11 +288,13 @@ TP_API tp_status tp_ring_allreduce_ranks(const tp_plan* plan, const void* const*
  * ------------------------------------------------------------------- */
 
 /* Sizes of the two shard buffers: q_bytes = H*K (one E4M3 code per weight,
- * [N][H][K/N]), scale_bytes = H*K/32, laid out [N][K/N/64][H][2]: for each
- * 64-column block of a rank slice, the scales of its two 32-weight runs for
- * every row h in turn (the scales a 128-row tile needs for one block are
- * contiguous). TP_ERR_UNSUPPORTED when K/N is not a multiple of 64;
- * TP_ERR_INVALID for null arguments. */
+ * [N][H][K/N]), scale_bytes = N * ceil(H/128) * ceil(K/N/128) * 512: the
+ * E8M0 scales in 512-byte chunks [N][ceil(H/128)][ceil(K/N/128)], one per
+ * rank, 128-row tile and 128 columns (four 32-weight runs) of a rank slice;
+ * row t of the tile, run j of the four at byte 16 (t % 32) + 4 (t / 32) + j
+ * of the chunk (the order in which the block-scaled MMA reads scales from
+ * tensor memory); rows past H and runs past K/N hold 0. TP_ERR_UNSUPPORTED
+ * when K/N is not a multiple of 64; TP_ERR_INVALID for null arguments. */
 TP_API tp_status tp_plan_mxfp8_bytes(const tp_plan* plan, size_t* q_bytes, size_t* scale_bytes);
 
 /* S0 for MXFP8: Linear weight [H][K] bf16 -> w_q codes and w_scales (device
@@ -314,9 +316,15 @@ TP_API size_t tp_plan_mxfp8_workspace_bytes(const tp_plan* plan, int64_t tokens)
  *   from tp_pack_weights_mxfp8; workspace of
  *   tp_plan_mxfp8_workspace_bytes(plan, tokens) bytes (NULL when 0), zeroed
  *   before its first use.
- * Code tiles are widened to bf16 tiles in shared memory (E4M3 * 2^s, exact)
- * and multiplied with the bf16 activations in fp32 on the tensor cores; the
- * partials are rounded once to bf16 and folded in ring order with the
+ * More than 8 tokens: code tiles are widened to bf16 tiles in tensor memory
+ * (E4M3 * 2^s, exact) and multiplied with the bf16 activations in fp32 on
+ * the tensor cores. At most 8 tokens: the codes and scales go to the
+ * block-scaled MMA (kind::mxf8f6f4) as stored, and each 32-value run of the
+ * activations is split on chip into two E4M3 terms with E8M0 scales,
+ * x = 2^e1 q1 + 2^e2 q2 with e1 = floor(log2 max|run|) - 7: exact for every
+ * x of at least 2^(e1 - 6), within 2^(e1 - 14) below that (plus 2^-137 for
+ * runs whose remainders fall below 2^-119). Either way the partials are
+ * fp32 sums rounded once to bf16 and folded in ring order with the
  * residual, as for bf16 shards. TP_ERR_UNSUPPORTED when K/N is not a
  * multiple of 64. */
 TP_API tp_status tp_rowlinear_reconcile_mxfp8(const tp_plan* plan, const void* x, const void* w_q,

@@ -9,9 +9,11 @@
 // (-127 for an all-zero run); each weight is the FP8 E4M3 code nearest to
 // w / X, ties to even, saturating at 448.
 //   q      [N][H][K/N] E4M3 codes                     (K/N a multiple of 64)
-//   scales [N][K/N/64][H][2] E8M0 bytes: for each 64-column block of a rank
-//          slice, the scales of its two 32-weight runs, row after row (the
-//          scales a 128-row tile needs for one block are 256 contiguous bytes)
+//   scales [N][ceil(H/128)][ceil(K/N/128)][512] E8M0 bytes: one 512-byte chunk
+//          holds the scales of a 128-row tile for four 32-weight runs (128
+//          columns): row t of the tile, run j at byte 16 (t % 32) + 4 (t / 32)
+//          + j -- the order in which the block-scaled MMA reads them from
+//          tensor memory; rows past H and runs past K/N hold 0
 //
 // NVFP4 (the TP=4-vs-TP=8 post's NVFP4 weights, in NVIDIA's published
 // layout): E2M1 elements, one E4M3 block scale per 16 weights along K inside a
@@ -29,7 +31,16 @@
 namespace tpr {
 
 constexpr int kMxBlock = 32;        // weights per shared scale
-constexpr int kMxPair = 64;         // columns whose two scales are stored together
+constexpr int kMxPair = 64;         // K/N is a multiple of this
+constexpr int kMxChunk = 512;       // scale bytes of a 128-row tile x 128 columns
+constexpr int kMxChunkCols = 128;   // columns a scale chunk covers
+
+// Byte of the scale of run b (32 columns) of row h of rank r in the chunked
+// scale array (h_tiles = ceil(H/128), kg = ceil(K/N/128)).
+__host__ __device__ constexpr int64_t mx_scale_index(int64_t r, int64_t h, int64_t b, int64_t h_tiles,
+                                                     int64_t kg) {
+    return ((r * h_tiles + h / 128) * kg + b / 4) * kMxChunk + (h % 32) * 16 + ((h % 128) / 32) * 4 + b % 4;
+}
 
 // Two f32 values -> two E4M3 codes, nearest even, saturating at +-448; the
 // code of `lo` in bits 0-7 of the result.
@@ -111,8 +122,8 @@ __global__ void __launch_bounds__(256)
         }
         int s = amax == 0 ? -127 : bf16_floor_log2(amax) - 8;
         s = max(-127, min(127, s));
-        // [N][Ks/64][H][2]: run b is half b & 1 of 64-column block b >> 1
-        scales[((r * (nb >> 1) + (b >> 1)) * hidden + h) * 2 + (b & 1)] = static_cast<uint8_t>(s + 127);
+        scales[mx_scale_index(r, h, b, (hidden + 127) / 128, (ks + kMxChunkCols - 1) / kMxChunkCols)] =
+            static_cast<uint8_t>(s + 127);
         // w / 2^s = w * 2^-s: a power of two, exact unless it drops below the
         // f32 range, where the E4M3 code is a signed zero either way.
         const float inv = pow2_f32(-s);

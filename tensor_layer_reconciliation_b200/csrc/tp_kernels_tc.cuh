@@ -77,7 +77,7 @@ constexpr uint32_t kTcATile = kTcRows * kTcKBlock * 2;  // 16 KB
 // slot i % slots; at most kCvtSlotsMax slots).
 constexpr int kCvtSlotsMax = 8;
 constexpr uint32_t kMxCodeTile = kTcRows * kTcKBlock;   // 8 KB of E4M3 codes
-constexpr uint32_t kMxScaleTile = kTcRows * 2;          // the 2 E8M0 scales of each row
+constexpr uint32_t kMxScaleTile = kMxChunk;             // the scale chunk holding the block's scales
 constexpr uint32_t kNvCodeTile = kTcRows * kTcKBlock / 2;  // 4 KB: two E2M1 codes a byte
 constexpr uint32_t kNvScaleTile = kTcRows * 4;             // the 4 E4M3 block scales of each row
 
@@ -85,12 +85,55 @@ constexpr uint32_t kNvScaleTile = kTcRows * 4;             // the 4 E4M3 block s
 constexpr int kFmtBf16 = 0;    // packed bf16 shards, staged by TMA as the MMA's A tiles
 constexpr int kFmtMxfp8 = 1;   // E4M3 codes + E8M0 scales per 32, widened on chip
 constexpr int kFmtNvfp4 = 2;   // E2M1 codes + E4M3 scales per 16 (x 2^g), widened on chip
+constexpr int kFmtMxfp8Bs = 3; // MXFP8 codes read by the block-scaled MMA (at most 8 tokens)
+
+// Block-scaled MXFP8 form. The codes and their E8M0 scales go to the tensor
+// cores as stored (tcgen05.mma kind::mxf8f6f4, one scale per 32 values of K
+// on each side), 128 columns of K a stage. The bf16 activations are split on
+// chip into two E4M3 terms with E8M0 scales of their own, one pair per 32
+// values of K: x = 2^e1 q1 + 2^e2 q2, e1 = floor(log2 max|x|) - 7 (so the
+// run's largest value over 2^e1 lies in [128, 256): nothing saturates), q1
+// the E4M3 value nearest x / 2^e1, and q2 the same for the remainder
+// x - 2^e1 q1 under its own maximum. A bf16 value has 8 significant bits; q1
+// takes the leading 4 and the remainder fits the 4 of q2 whenever q1 is a
+// normal E4M3 value, so every x at least 2^(e1 - 6) (about 2^-13 of its run's
+// maximum) is split exactly; a smaller one is off by at most 2^(e1 - 14).
+// The MMA's B operand holds q1 of token t in row t and q2 in row 8 + t; the
+// epilogue adds accumulator columns t and 8 + t in fp32.
+// The split activations have a ring of their own (kBsXSlots slots, apart
+// from the code stages), so the splits run ahead of the MMAs whenever the
+// codes come late. A slot first receives the bf16 block of x by TMA ([8
+// tokens][128] bf16, 2 KB, no swizzle); the splitting warps read it into
+// registers and then write the B tile and its scale chunk over it.
+constexpr int kBsXSlots = 8;                              // <= kCvtSlotsMax
+constexpr int kBsXLead = 4;                               // blocks of x loaded ahead of the split
+constexpr uint32_t kBsBRows = 16;                         // MMA N: 8 tokens x 2 terms
+constexpr uint32_t kBsXTile = 8 * kMxChunkCols * 2;       // the bf16 activation block
+constexpr uint32_t kBsSfbOff = kBsBRows * 128;            // B scale chunk after the B tile
+constexpr uint32_t kBsBTile = 3 * 1024;                   // B tile + scale chunk, 1024-aligned
+constexpr uint32_t kBsCodeTile = kTcRows * kMxChunkCols;  // 16 KB of E4M3 codes
+// The four K = 32 steps of a stage alternate between this many accumulators
+// (16 columns each, within the unit's 32), summed by the epilogue: MMAs into
+// different accumulators do not wait on one another's results.
+constexpr int kBsAccs = 2;
 
 __host__ __device__ constexpr uint32_t fmt_code_tile(int fmt) {
-    return fmt == kFmtMxfp8 ? kMxCodeTile : fmt == kFmtNvfp4 ? kNvCodeTile : kTcATile;
+    return fmt == kFmtMxfp8 ? kMxCodeTile
+           : fmt == kFmtNvfp4 ? kNvCodeTile
+           : fmt == kFmtMxfp8Bs ? kBsCodeTile
+                                : kTcATile;
 }
 __host__ __device__ constexpr uint32_t fmt_scale_tile(int fmt) {
-    return fmt == kFmtMxfp8 ? kMxScaleTile : fmt == kFmtNvfp4 ? kNvScaleTile : 0;
+    return fmt == kFmtMxfp8 || fmt == kFmtMxfp8Bs ? kMxScaleTile : fmt == kFmtNvfp4 ? kNvScaleTile : 0;
+}
+// Columns of K one stage holds.
+__host__ __device__ constexpr int fmt_k_block(int fmt) {
+    return fmt == kFmtMxfp8Bs ? kMxChunkCols : kTcKBlock;
+}
+// Activation bytes of one stage: x_rows rows of the block, or (block-scaled
+// form) the split B tile with its scale chunk.
+__host__ __device__ constexpr uint32_t fmt_b_tile(int fmt, int x_rows) {
+    return fmt == kFmtMxfp8Bs ? kBsBTile : static_cast<uint32_t>(x_rows) * kTcKBlock * 2;
 }
 
 // What the epilogue does with each accumulator (a template parameter, so each
@@ -120,6 +163,8 @@ struct TcParams {
     const uint16_t* residual;     // [M][H]
     uint16_t* out;                // [M][H]
     const int* nv_gexp;           // NVFP4: the second-level exponent g
+    const uint8_t* mx_scales;     // MXFP8: chunked E8M0 scales [N][h_tiles][mx_kg][512]
+    int mx_kg;                    // MXFP8: ceil(K/N / 128), scale chunks per row tile
 };
 
 // Cluster fold of one (H tile, token tile). The cluster's C = N * SPLITS CTAs
@@ -463,6 +508,70 @@ __device__ __forceinline__ bool fold_tagged(const TcParams& p, size_t plane, siz
 
 // Token tiles up to 64 run two CTAs per SM: at most 168 registers a thread
 // (96 with the converter warps).
+// E8M0 exponent of a split term under run maximum a: floor(log2 a) - 7,
+// at least -127 (a = 0 or below the f32 normal range gives -127).
+__device__ __forceinline__ int split_exp(float a) {
+    return max(-127, static_cast<int>((__float_as_uint(a) >> 23) & 0xFFu) - 134);
+}
+
+// Block-scaled form, one 32-value run of the activations: lane 4t + part of
+// a converter warp holds x[t][8 part .. 8 part + 7] of the run (bf16 in v,
+// zeros past the tokens or K/N); the four lanes of token t hold the whole
+// run. Writes q1 to row t and q2 to row 8 + t of the B tile `bt` (rows of
+// 128 bytes with the 128-byte swizzle: 16-byte chunk c of row n at chunk
+// c ^ (n % 8)), columns 32 run + 8 part .. + 7, and the exponents' E8M0
+// bytes to the scale chunk after the tile (row n, byte `run`).
+__device__ __forceinline__ void x_split_run(uint4 v, uint8_t* bt, int t, int run, int part) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        y[2 * i] = bf16_lo(w[i]);
+        y[2 * i + 1] = bf16_hi(w[i]);
+    }
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(y[i]));
+    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+    const int e1 = split_exp(a);
+    const float inv1 = pow2_f32(-e1), sc1 = pow2_f32(e1);
+    // q1, and the remainder (exact: both sides carry at most 8 significant
+    // bits within a few binades of each other)
+    uint32_t q1[2], q2[2];
+    float rem[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint16_t c = e4m3x2_from_f32(y[2 * i] * inv1, y[2 * i + 1] * inv1);
+        const uint32_t h = f16x2_from_e4m3x2(c);
+        rem[2 * i] = y[2 * i] - f16_lo_to_f32(h) * sc1;
+        rem[2 * i + 1] = y[2 * i + 1] - f16_hi_to_f32(h) * sc1;
+        if (i & 1) q1[i >> 1] |= static_cast<uint32_t>(c) << 16;
+        else q1[i >> 1] = c;
+    }
+    float b = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b = fmaxf(b, fabsf(rem[i]));
+    b = fmaxf(b, __shfl_xor_sync(0xFFFFFFFFu, b, 1));
+    b = fmaxf(b, __shfl_xor_sync(0xFFFFFFFFu, b, 2));
+    const int e2 = split_exp(b);
+    const float inv2 = pow2_f32(-e2);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint16_t c = e4m3x2_from_f32(rem[2 * i] * inv2, rem[2 * i + 1] * inv2);
+        if (i & 1) q2[i >> 1] |= static_cast<uint32_t>(c) << 16;
+        else q2[i >> 1] = c;
+    }
+    const int chunk = 2 * run + (part >> 1);
+    const int off = ((chunk ^ (t & 7)) << 4) + (part & 1) * 8;
+    *reinterpret_cast<uint2*>(bt + t * 128 + off) = make_uint2(q1[0], q1[1]);
+    *reinterpret_cast<uint2*>(bt + (8 + t) * 128 + off) = make_uint2(q2[0], q2[1]);
+    if (part == 0) {
+        bt[kBsSfbOff + t * 16 + run] = static_cast<uint8_t>(e1 + 127);
+        bt[kBsSfbOff + (8 + t) * 16 + run] = static_cast<uint8_t>(e2 + 127);
+    }
+}
+
 template <int BN, int MODE, int FMT>
 __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, BN <= 64 ? 2 : 1)
     tc_partial_kernel(const __grid_constant__ CUtensorMap tmap_w,
@@ -473,9 +582,14 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     // eight tokens, one 8-row swizzle atom that every 8-row group of the MMA's
     // B operand reads (descriptor stride 0): rows 8.. of the product repeat
     // rows 0..7 in accumulator columns nobody reads.
-    const uint32_t kBTile = static_cast<uint32_t>(p.x_rows) * kTcKBlock * 2;
-    const bool x_atom = p.x_rows < BN;
-    constexpr bool MX = FMT != kFmtBf16;                        // converted on chip
+    constexpr bool BS = FMT == kFmtMxfp8Bs;                     // block-scaled MMA on the codes
+    static_assert(!BS || BN == 32, "block-scaled form: a 32-column accumulator, at most 8 tokens");
+    static_assert(!BS || (kBsAccs >= 1 && kBsAccs * 16 <= BN && 4 % kBsAccs == 0), "accumulators fit the unit's columns");
+    static_assert(kBsXSlots <= kCvtSlotsMax && kBsXSlots <= kTcMaxStages && kBsXLead < kBsXSlots, "split ring");
+    const uint32_t kBTile = fmt_b_tile(FMT, p.x_rows);
+    const bool x_atom = !BS && p.x_rows < BN;
+    constexpr bool MX = FMT == kFmtMxfp8 || FMT == kFmtNvfp4;   // converted on chip
+    constexpr int KB = fmt_k_block(FMT);                        // columns of K a stage holds
     constexpr uint32_t kWTile = fmt_code_tile(FMT);             // weight bytes staged per block
     constexpr uint32_t kSTile = fmt_scale_tile(FMT);            // scale bytes staged per block
     // Tensor memory: two accumulators of BN columns; the quantised forms add
@@ -483,9 +597,14 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     // within 256 columns a CTA when two share an SM.
     constexpr int kSlots = !MX ? 1 : BN <= 32 ? 6 : BN <= 64 ? 4 : 8;
     constexpr uint32_t kSlotCol0 = 2 * BN;
-    constexpr uint32_t kTmemCols = MX ? (BN <= 64 ? 256u : 512u) : (2 * BN < 32 ? 32u : 2u * BN);
+    // The block-scaled form adds, per stage, the A and B scales (4 columns
+    // each) after them: a stage's copies never overwrite scales the previous
+    // stages' MMAs may still read.
+    constexpr uint32_t kTmemCols = MX ? (BN <= 64 ? 256u : 512u) : BS ? 256u : (2 * BN < 32 ? 32u : 2u * BN);
     static_assert(!MX || (BN <= 128 && kSlotCol0 + 32 * kSlots <= kTmemCols && kSlots <= kCvtSlotsMax),
                   "converted slots fit in tensor memory");
+    constexpr uint32_t kSfaCol = 2 * BN, kSfbCol = 2 * BN + 4;   // + 8 per stage
+    static_assert(!BS || kSfbCol + 8 * (kTcMaxStages - 1) + 4 <= kTmemCols, "block scales fit in tensor memory");
     constexpr uint32_t kIdesc = idesc_bf16_f32(kTcRows, BN);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -494,7 +613,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     const int S = p.stages;
     uint8_t* a_ring = smem;                                              // weight tiles (TMA)
     uint8_t* b_ring = a_ring + static_cast<size_t>(S) * kWTile;         // activation tiles
-    uint8_t* s_ring = b_ring + static_cast<size_t>(S) * kBTile;          // MX: scale tiles
+    // activation slots: one per stage, or (BS) the split ring's
+    uint8_t* s_ring = b_ring + static_cast<size_t>(BS ? kBsXSlots : S) * kBTile;   // scale tiles
     uint64_t* full = reinterpret_cast<uint64_t*>(s_ring + static_cast<size_t>(S) * kSTile);
     uint64_t* empty = full + kTcMaxStages;
     uint64_t* acc_full = empty + kTcMaxStages;   // [2]
@@ -503,11 +623,15 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     uint64_t* fold_ready = mma_done + 1;   // cluster fold: all N partial tiles written
     uint64_t* fold_freed = fold_ready + 1; // cluster fold: all N CTAs done reading mine
     uint64_t* cvt_full = fold_freed + 1;              // MX: [kSlots] converted tile ready (4 warps)
-    uint64_t* cvt_empty = cvt_full + kCvtSlotsMax;    // MX: [kSlots] converted tile read by the MMAs
+    uint64_t* cvt_empty = cvt_full + kCvtSlotsMax;    // MX: [kSlots] converted tile read by the MMAs;
+                                                      // BS: [kBsXSlots] split slot read by the MMAs
     // MX: [S] a stage's activation block landed (its codes and scales land on
     // full[s], so the converters need not wait for the dependency)
     uint64_t* full_x = cvt_empty + kCvtSlotsMax;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full_x + kTcMaxStages);
+    // BS: full_x [kBsXSlots] split slot written (4 warps); x_full [kBsXSlots]
+    // its bf16 activation block landed
+    uint64_t* x_full = full_x + kTcMaxStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_full + kTcMaxStages);
     // cluster fold: this CTA's bf16 partial tile, [BN tokens][128 rows]
     uint16_t* part_buf = reinterpret_cast<uint16_t*>(
         (reinterpret_cast<uintptr_t>(tmem_slot + 4) + 127) & ~static_cast<uintptr_t>(127));
@@ -515,7 +639,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     __shared__ int fold_mine;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nkb = (p.ks + kTcKBlock - 1) / kTcKBlock;
+    const int nkb = (p.ks + KB - 1) / KB;
     // Cluster fold: cluster c takes tiles c, c + clusters, ...; its CTA of rank
     // r (in the cluster) computes rank r's partial of each.
     constexpr bool kCluster = MODE == kTcClusterFold;
@@ -563,8 +687,11 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         abort_flag = 0;
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&full_x[s], 1);
             mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < kTcMaxStages; ++s) {   // (BS: split slots, up to kBsXSlots)
+            mbar_init(&full_x[s], BS ? 4 : 1);       // BS: the four splitting warps
+            mbar_init(&x_full[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -573,7 +700,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         mbar_init(mma_done, 1);
         mbar_init(fold_ready, static_cast<uint32_t>(csize));
         mbar_init(fold_freed, static_cast<uint32_t>(csize));
-        for (int j = 0; j < kSlots; ++j) {
+        for (int j = 0; j < (BS ? kBsXSlots : kSlots); ++j) {
             mbar_init(&cvt_full[j], 4);
             mbar_init(&cvt_empty[j], 1);
         }
@@ -619,8 +746,9 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
                                                kSlotCol0 + 32u * static_cast<uint32_t>(j);
                         if (FMT == kFmtMxfp8)
+                            // row's two scales of this 64-column block in the chunk
                             mx_convert_row(a_ring + static_cast<size_t>(s) * kWTile + row * kTcKBlock,
-                                           srow + row * 2, taddr, row);
+                                           srow + (row & 31) * 16 + (row >> 5) * 4 + 2 * (kb & 1), taddr, row);
                         else
                             nv_convert_row(a_ring + static_cast<size_t>(s) * kWTile + row * (kTcKBlock / 2),
                                            srow + row * 4, two_g, taddr, row);
@@ -644,24 +772,123 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         }
     };
 
+    // Block-scaled form: converter warp 6 + run splits run `run` (32 columns)
+    // of every k-block's 128 activation columns, for the (at most 8) tokens,
+    // into split slot i % kBsXSlots (B tile and scale chunk). The bf16 block
+    // lands in the slot by TMA (x_full), issued by lane 0 of warp 6
+    // kBsXSlots - kBsXLead blocks ahead of the split once the MMAs that read
+    // the slot's previous split are done; each lane takes its 16 bytes into
+    // registers, and once all four warps have theirs (one barrier, which
+    // also makes the decision to give up common to them) the split
+    // overwrites the block.
+    auto run_x_split = [&]() {
+        if constexpr (BS) {
+            const int run = warp - 6;
+            const int t = lane >> 2, part = lane & 3;
+            const bool issuer = warp == 6 && lane == 0;
+            // the scale chunks' bytes no split writes (rows 16.., columns 1..)
+            // are never read by the MMA: zero them once all the same
+            for (int j = 0; j < kBsXSlots; ++j)
+                *reinterpret_cast<uint32_t*>(b_ring + static_cast<size_t>(j) * kBTile + kBsSfbOff +
+                                             4 * (32 * run + lane)) = 0u;
+            // (unit, k-block) walk in issue order, for the loads
+            struct XCursor {
+                int lu, kb, kb_hi, r, mt;
+            };
+            auto x_enter = [&](XCursor& c) {
+                if (c.lu < my_units) {
+                    int ht, sp;
+                    unit_of(c.lu, c.r, ht, c.mt, sp);
+                    split_range(sp, c.kb, c.kb_hi);
+                }
+            };
+            auto x_advance = [&](XCursor& c) {
+                if (++c.kb == c.kb_hi) {
+                    ++c.lu;
+                    x_enter(c);
+                }
+            };
+            int n = 0;   // k-blocks of this CTA
+            for (int lu = 0; lu < my_units; ++lu) {
+                int r, ht, mt, sp, kb_lo, kb_hi;
+                unit_of(lu, r, ht, mt, sp);
+                split_range(sp, kb_lo, kb_hi);
+                n += kb_hi - kb_lo;
+            }
+            XCursor ld{0, 0, 0, 0, 0};
+            x_enter(ld);
+            int issued = 0;
+            auto issue_x = [&]() {   // the next block of the walk into its slot
+                const int j = issued % kBsXSlots;
+                mbar_arrive_expect_tx(&x_full[j], kBsXTile);
+                tma_load_3d(b_ring + static_cast<size_t>(j) * kBTile, &tmap_x, &x_full[j], ld.kb * KB, ld.r,
+                            ld.mt * BN);
+                x_advance(ld);
+                ++issued;
+            };
+            asm volatile("bar.sync 3, 128;" ::: "memory");   // zeroed before any load lands
+            if (issuer) {
+                pdl_wait();  // activations may be produced by the previous kernel
+                while (issued < n && issued < kBsXSlots - kBsXLead) issue_x();
+            }
+            bool ok = true;
+            int i = 0;
+            for (; i < n; ++i) {
+                const int j = i % kBsXSlots;
+                const uint32_t ph = static_cast<uint32_t>(i / kBsXSlots) & 1u;
+                ok = mbar_wait_bounded(&x_full[j], ph);
+                uint8_t* bt = b_ring + static_cast<size_t>(j) * kBTile;
+                const uint4 v = *reinterpret_cast<const uint4*>(bt + t * (kMxChunkCols * 2) + (run * 32 + part * 8) * 2);
+                if (bar_sync_any(3, 128, !ok || *reinterpret_cast<volatile int*>(&abort_flag) != 0)) {
+                    ok = false;
+                    atomicExch(&abort_flag, 1);
+                    break;
+                }
+                x_split_run(v, bt, t, run, part);
+                fence_proxy_async_smem();   // the tensor core reads them through the async proxy
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_x[j]);
+                // refill: the block kBsXSlots - kBsXLead ahead, into the slot
+                // of block i - kBsXLead once the MMAs have read that split
+                if (issuer && issued < n) {
+                    const int prev = issued - kBsXSlots;   // the slot's previous block
+                    if (prev < 0 || mbar_wait_bounded(&cvt_empty[issued % kBsXSlots],
+                                                      static_cast<uint32_t>(prev / kBsXSlots) & 1u))
+                        issue_x();
+                    else
+                        atomicExch(&abort_flag, 1);
+                }
+            }
+            // blocks still landing (after an abort): wait for them (bounded)
+            if (issuer)
+                for (int k = i; k < issued; ++k)
+                    if (!mbar_wait_bounded(&x_full[k % kBsXSlots], static_cast<uint32_t>(k / kBsXSlots) & 1u)) break;
+        }
+    };
+
     if (warp == 0) {
         // ---------------------------------------------------------- producer --
         if (lane == 0) {
             tma_prefetch_desc(&tmap_w);
             tma_prefetch_desc(&tmap_x);
-            if (MX) tma_prefetch_desc(&tmap_s);
-            // bytes landing on full[s]: the whole stage, or (MX) codes and scales
-            // only, the activation block then counting on full_x[s]
-            const uint32_t tx = MX ? kWTile + kSTile : kWTile + kBTile + kSTile;
-            // The weights of one k-block (and, MX, their scales) into stage st.
+            if (FMT == kFmtNvfp4) tma_prefetch_desc(&tmap_s);
+            // bytes landing on full[s]: the whole stage, or (quantised) codes and
+            // scales only, the activation block then counting on full_x[s]
+            const uint32_t tx = (MX || BS) ? kWTile + kSTile : kWTile + kBTile + kSTile;
+            // The weights of one k-block (and their scales) into stage st.
             // (NVFP4 code tiles hold two codes a byte: 32 bytes per 64-column block)
-            constexpr int kWCols = FMT == kFmtNvfp4 ? kTcKBlock / 2 : kTcKBlock;
+            constexpr int kWCols = FMT == kFmtNvfp4 ? kTcKBlock / 2 : KB;
             auto load_w = [&](int st, int kb_, int ht_, int r_) {
                 tma_load_3d(a_ring + static_cast<size_t>(st) * kWTile, &tmap_w, &full[st],
                             kb_ * kWCols, ht_ * kTcRows, r_);
-                if (MX)   // MXFP8: 256 bytes from byte ht*256; NVFP4: 128 words from word ht*128
-                    tma_load_3d(s_ring + static_cast<size_t>(st) * kSTile, &tmap_s, &full[st],
-                                FMT == kFmtMxfp8 ? ht_ * kTcRows * 2 : ht_ * kTcRows, kb_, r_);
+                if (FMT == kFmtNvfp4)   // 128 words from word ht*128
+                    tma_load_3d(s_ring + static_cast<size_t>(st) * kSTile, &tmap_s, &full[st], ht_ * kTcRows,
+                                kb_, r_);
+                else if (FMT == kFmtMxfp8 || BS)   // the 512-byte chunk holding the block's scales
+                    bulk_load(s_ring + static_cast<size_t>(st) * kSTile,
+                              p.mx_scales + ((static_cast<int64_t>(r_) * p.h_tiles + ht_) * p.mx_kg +
+                                             kb_ * KB / kMxChunkCols) * kMxChunk,
+                              kMxChunk, &full[st]);
             };
             // Walk (unit, k-block) in issue order.
             struct Cursor {
@@ -695,8 +922,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             if (pre > 0) {
                 Cursor c0{0, 0, 0, 0, 0, 0, 0};
                 enter_unit(c0);
-                const int64_t k_lo = static_cast<int64_t>(c0.kb) * kTcKBlock;
-                const int64_t k_hi = min(static_cast<int64_t>(min(c0.kb + pre, c0.kb_hi)) * kTcKBlock,
+                const int64_t k_lo = static_cast<int64_t>(c0.kb) * KB;
+                const int64_t k_hi = min(static_cast<int64_t>(min(c0.kb + pre, c0.kb_hi)) * KB,
                                          static_cast<int64_t>(p.ks));
                 const int m_end = min(p.tokens, (c0.mt + 1) * BN);
                 for (int m = c0.mt * BN; m < m_end; ++m)
@@ -704,7 +931,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                                      static_cast<uint32_t>((k_hi - k_lo) * 2));
             }
             pdl_wait();  // activations may be produced by the previous kernel
-            {
+            if (!BS) {   // (the block-scaled form's splitting warps load their own)
                 // the same first positions again, for their activation blocks
                 Cursor c0{0, 0, 0, 0, 0, 0, 0};
                 enter_unit(c0);
@@ -726,9 +953,11 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
                 mbar_arrive_expect_tx(&full[s], tx);
                 load_w(s, cur.kb, cur.ht, cur.r);
-                if (MX) mbar_arrive_expect_tx(&full_x[s], kBTile);
-                tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, MX ? &full_x[s] : &full[s],
-                            cur.kb * kTcKBlock, cur.r, cur.mt * BN);
+                if (!BS) {
+                    if (MX) mbar_arrive_expect_tx(&full_x[s], kBTile);
+                    tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, MX ? &full_x[s] : &full[s],
+                                cur.kb * kTcKBlock, cur.r, cur.mt * BN);
+                }
                 ++issued;
                 advance(cur);
                 if (++s == S) {
@@ -765,13 +994,15 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 bool ok = true;
                 for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
                     // MX: the converters consumed the codes; the MMA needs the activations
+                    // BS: the codes and scales, then split slot j
                     if (!mbar_wait_bounded(MX ? &full_x[s] : &full[s], ph) ||
-                        (MX && !mbar_wait_bounded(&cvt_full[j], jph))) {
+                        (MX && !mbar_wait_bounded(&cvt_full[j], jph)) ||
+                        (BS && !mbar_wait_bounded(&full_x[j], jph))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    uint64_t bd = smem_desc_k128(b_ring + static_cast<size_t>(s) * kBTile);
+                    uint64_t bd = smem_desc_k128(b_ring + static_cast<size_t>(BS ? j : s) * kBTile);
                     if (x_atom) bd &= ~(0x3FFFull << 32);   // stride between 8-row groups: 0
                     if constexpr (MX) {
                         // A: the converted tile in tensor memory, 8 columns per 16 of K
@@ -779,6 +1010,22 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
 #pragma unroll
                         for (int kk = 0; kk < kTcKBlock / 16; ++kk)
                             umma_bf16_ta(d, at + 8u * kk, bd + 2ull * kk, kIdesc, (kb != kb_lo) || (kk != 0));
+                    } else if constexpr (BS) {
+                        // the stage's two scale chunks into its own tensor-memory
+                        // columns (in issue order with the MMAs)
+                        const uint32_t sfa = tmem_base + kSfaCol + 8u * static_cast<uint32_t>(s);
+                        const uint32_t sfb = tmem_base + kSfbCol + 8u * static_cast<uint32_t>(s);
+                        tmem_cp_32x128b_x4(sfa, smem_desc_rows16(s_ring + static_cast<size_t>(s) * kSTile));
+                        tmem_cp_32x128b_x4(sfb, smem_desc_rows16(b_ring + static_cast<size_t>(j) * kBTile + kBsSfbOff));
+                        const uint64_t ad = smem_desc_k128(a_ring + static_cast<size_t>(s) * kWTile);
+                        // K = 32 a step (32 bytes of each row); step kk reads scale
+                        // byte kk and goes to accumulator kk % kBsAccs
+#pragma unroll
+                        for (int kk = 0; kk < KB / 32; ++kk)
+                            umma_mxf8(d + kBsBRows * static_cast<uint32_t>(kk % kBsAccs), ad + 2ull * kk, bd + 2ull * kk,
+                                      idesc_mxf8_f32(kTcRows, kBsBRows, kk),
+                                      (static_cast<uint32_t>(kk) << 30) | sfa, (static_cast<uint32_t>(kk) << 30) | sfb,
+                                      (kb != kb_lo) || (kk >= kBsAccs));
                     } else {
                         const uint64_t ad = smem_desc_k128(a_ring + static_cast<size_t>(s) * kTcATile);
 #pragma unroll
@@ -786,12 +1033,12 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                             umma_bf16(d, ad + 2ull * kk, bd + 2ull * kk, kIdesc, (kb != kb_lo) || (kk != 0));
                     }
                     umma_commit(&empty[s]);  // frees the stage when these MMAs finish
-                    if (MX) umma_commit(&cvt_empty[j]);   // and the converted slot
+                    if (MX || BS) umma_commit(&cvt_empty[j]);   // and the converted (split) slot
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
                     }
-                    if (++j == kSlots) {
+                    if (++j == (BS ? kBsXSlots : kSlots)) {
                         j = 0;
                         jph ^= 1u;
                     }
@@ -807,9 +1054,10 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             umma_commit(mma_done);
             if (!mbar_wait_bounded(mma_done, 0)) (void)mbar_wait_bounded(mma_done, 0);
         }
-    } else if (MX && warp >= 6) {
+    } else if ((MX || BS) && warp >= 6) {
         // ------------------------------------ converters (quantised weights) --
-        run_converters(0);
+        if constexpr (BS) run_x_split();
+        else run_converters(0);
     } else {
         // ---------------------------------------------------------- epilogue --
         // A CTA with one unit has nothing for these warps until its MMAs end:
@@ -820,6 +1068,19 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         for (int lu = 0; lu < my_units; ++lu) {
             const int b = lu & 1;
             const uint32_t aph = static_cast<uint32_t>(lu >> 1) & 1u;
+            int r, ht, mt, sp;
+            unit_of(lu, r, ht, mt, sp);
+            // Counter fold: this CTA's place among the parts of its tile, taken
+            // before the accumulator is ready (the tags, not the tickets, say
+            // which parts have landed: the ticket only elects the CTA that
+            // folds), so the round trip overlaps the MMAs.
+            unsigned int ticket = 0, tag = 0;
+            if (MODE == kTcCounterFold) {
+                if (threadIdx.x == 64) ticket = atomicAdd(p.counters + ht * p.m_tiles + mt, 1u);
+                // this call's tag: the tile's folds so far + 1 (the previous
+                // call's fold is complete: the epilogue waited for the dependency)
+                tag = __ldcg(p.counters + p.h_tiles * p.m_tiles + ht * p.m_tiles + mt) + 1u;
+            }
             bool ok = mbar_wait_bounded(&acc_full[b], aph);
             // cluster fold: the peers have read the previous unit's partial tile
             if (kCluster && lu > 0)
@@ -830,26 +1091,25 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             // The four epilogue warps leave together: one answer for all of them.
             if (bar_sync_any(2, 128, bad)) break;
             tc_fence_after_sync();
-            int r, ht, mt, sp;
-            unit_of(lu, r, ht, mt, sp);
             const int h = ht * kTcRows + q * 32 + lane;
             const int m0 = mt * BN;
             const size_t plane = static_cast<size_t>(p.tokens) * p.hidden;
-            // Counter fold: this CTA's place among the parts of its tile, taken
-            // now so the round trip overlaps the stores below.
-            unsigned int ticket = 0, tag = 0;
-            if (MODE == kTcCounterFold) {
-                if (threadIdx.x == 64) ticket = atomicAdd(p.counters + ht * p.m_tiles + mt, 1u);
-                // this call's tag: the tile's folds so far + 1 (the previous
-                // call's fold is complete: the epilogue waited for the dependency)
-                tag = __ldcg(p.counters + p.h_tiles * p.m_tiles + ht * p.m_tiles + mt) + 1u;
-            }
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(b * BN + c0),
                                v);
+                if constexpr (BS) {   // token i's two activation terms in each accumulator
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float f = __fadd_rn(__uint_as_float(v[i]), __uint_as_float(v[i + 8]));
+#pragma unroll
+                        for (int a = 1; a < kBsAccs; ++a)
+                            f = __fadd_rn(f, __fadd_rn(__uint_as_float(v[16 * a + i]), __uint_as_float(v[16 * a + i + 8])));
+                        v[i] = __float_as_uint(f);
+                    }
+                }
                 if (kCluster) {
                     // [token][row] in shared memory, the tile's tokens only: lanes
                     // write 32 consecutive rows; bf16 partials, or fp32 part sums

@@ -237,6 +237,7 @@ tp_status launch_exact(const tp_plan* p, const void* x, const void* w, const voi
 // -------------------------------------------------------- tensor variant --
 
 struct TcConfig {
+    int fmt;   // the kernel's form (tpr::kFmt*): MXFP8 for at most 8 tokens is block-scaled
     int bn, stages, grid, units, h_tiles, m_tiles, splits, x_rows;
     bool cluster_fold;   // the N ranks of a tile on one cluster, folded on chip
     bool splits_allowed; // a reconciliation call (the kernel may fold; K may be split)
@@ -256,6 +257,10 @@ int tc_token_tile(int64_t tokens) {
 TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt = tpr::kFmtBf16) {
     TcConfig c{};
     c.splits_allowed = allow_split;
+    // MXFP8 for at most 8 tokens: the codes go to the block-scaled MMA as
+    // stored and the activations are split into two E4M3 terms on chip
+    if (fmt == tpr::kFmtMxfp8 && tokens <= 8) fmt = tpr::kFmtMxfp8Bs;
+    c.fmt = fmt;
     c.bn = tc_token_tile(tokens);
     // quantised forms: token tiles up to 128 (their converted slots share
     // tensor memory with the accumulators)
@@ -268,7 +273,8 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     const bool two_per_sm = c.bn <= 64;
     const int slots = p->sm_count * (two_per_sm ? 2 : 1);
     // Fewer units than SMs: split K so every SM streams weights.
-    const int nkb = static_cast<int>((p->ks + tpr::kTcKBlock - 1) / tpr::kTcKBlock);
+    const int kblock = tpr::fmt_k_block(fmt);
+    const int nkb = static_cast<int>((p->ks + kblock - 1) / kblock);
     c.splits = 1;
     if (allow_split && base_units > 0 && base_units < p->sm_count)
         c.splits = std::max(1, std::min({slots / base_units, nkb, tpr::kMaxSplits}));
@@ -280,15 +286,17 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     // converted bf16 tiles live in tensor memory).
     // At most 8 tokens: one 8-row atom of x a block instead of the BN-row tile
     c.x_rows = tokens <= 8 && c.m_tiles == 1 ? 8 : c.bn;
+    // (the block-scaled form's split activations have a ring of their own)
+    const bool split_ring = fmt == tpr::kFmtMxfp8Bs;
     const size_t stage = tpr::fmt_code_tile(fmt) + tpr::fmt_scale_tile(fmt) +
-                         static_cast<size_t>(c.x_rows) * tpr::kTcKBlock * 2;
+                         (split_ring ? 0 : tpr::fmt_b_tile(fmt, c.x_rows));
     // the cluster fold's tile in shared memory: the tile's tokens x 128 rows,
     // bf16 partials or fp32 part sums
     const size_t part_tile = c.cluster_fold ? static_cast<size_t>(std::min<int64_t>(c.bn, tokens)) *
                                                   tpr::kTcRows * (c.splits > 1 ? 4 : 2)
                                             : 0;
-    const size_t fixed = (3 * tpr::kTcMaxStages + 7 + 2 * tpr::kCvtSlotsMax) * sizeof(uint64_t) + 16 + 128 +
-                         1024 + part_tile;
+    const size_t fixed = (4 * tpr::kTcMaxStages + 7 + 2 * tpr::kCvtSlotsMax) * sizeof(uint64_t) + 16 + 128 +
+                         1024 + part_tile + (split_ring ? tpr::kBsXSlots * tpr::kBsBTile : 0);
     const size_t budget = std::min<size_t>(two_per_sm ? 110 * 1024 : 200 * 1024,
                                            static_cast<size_t>(p->smem_optin));
     c.stages = budget > fixed
@@ -310,7 +318,7 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
 // x_box_tokens: token rows of one activation box (the 1-SM kernel's BN, or
 // the half tile a CTA of a pair stages).
 tp_status encode_tc_maps(const tp_plan* p, int x_box_tokens, const void* x, const void* w,
-                         int64_t tokens, CUtensorMap* mw, CUtensorMap* mx) {
+                         int64_t tokens, CUtensorMap* mw, CUtensorMap* mx, bool x_block_scaled = false) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
     if (!enc) return cuda_fail(g_encode_err);
     const cuuint32_t estr[3] = {1, 1, 1};
@@ -327,14 +335,19 @@ tp_status encode_tc_maps(const tp_plan* p, int x_box_tokens, const void* x, cons
         if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     }
     {
-        // Activations [M][N][Ks]: {Ks, N, M}, BN token rows x 64 columns of one rank.
+        // Activations [M][N][Ks]: {Ks, N, M}, BN token rows x 64 columns of one
+        // rank (128-byte swizzle, the MMA's B tiles), or for the block-scaled
+        // form 8 token rows x 128 columns unswizzled (the splitting warps' input).
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->ks), static_cast<cuuint64_t>(p->n_ranks),
                                     static_cast<cuuint64_t>(tokens)};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks) * 2,
                                        static_cast<cuuint64_t>(p->k) * 2};
-        const cuuint32_t box[3] = {tpr::kTcKBlock, 1, static_cast<cuuint32_t>(x_box_tokens)};
+        const cuuint32_t box[3] = {x_block_scaled ? static_cast<cuuint32_t>(tpr::kMxChunkCols)
+                                                  : static_cast<cuuint32_t>(tpr::kTcKBlock),
+                                   1, static_cast<cuuint32_t>(x_box_tokens)};
         CUresult r = enc(mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides,
-                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         x_block_scaled ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     }
@@ -405,44 +418,29 @@ size_t nv_scale_bytes(const tp_plan* p) {
 // their scales.
 struct TcWeights {
     const void* w;        // [N][H][Ks] bf16; MXFP8 E4M3 codes; NVFP4 E2M1 code pairs
-    const void* scales;   // MXFP8 [N][Ks/64][H][2] E8M0; NVFP4 [N][Ks/64][H][4] E4M3 + g
+    const void* scales;   // MXFP8 [N][H/128][Ks/128][512] E8M0 chunks; NVFP4 [N][Ks/64][H][4] E4M3 + g
     int fmt;              // tpr::kFmt*
 };
 
-// MXFP8 codes [N][H][Ks] bytes, 128 rows x 64 codes per box (row-major in
-// shared memory), and their scales [N][Ks/64][H][2] bytes, the 256 bytes of a
-// 128-row tile per box (rows past H read as zero).
-tp_status encode_mx_maps(const tp_plan* p, const void* q, const void* scales, CUtensorMap* mq,
-                         CUtensorMap* ms) {
+// MXFP8 codes [N][H][Ks] bytes, 128 rows per box: 64 codes with the 64-byte
+// swizzle for the converters (their reads and swizzled writes are then free
+// of bank conflicts), or 128 codes with the 128-byte swizzle the block-scaled
+// MMA reads. (The scales travel by plain bulk copies of their chunks.)
+tp_status encode_mx_maps(const tp_plan* p, const void* q, bool block_scaled, CUtensorMap* mq) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
     if (!enc) return cuda_fail(g_encode_err);
     const cuuint32_t estr[3] = {1, 1, 1};
-    {
-        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->ks), static_cast<cuuint64_t>(p->hidden),
-                                    static_cast<cuuint64_t>(p->n_ranks)};
-        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks),
-                                       static_cast<cuuint64_t>(p->hidden * p->ks)};
-        const cuuint32_t box[3] = {tpr::kTcKBlock, tpr::kTcRows, 1};
-        // 64-byte swizzle: the converters' reads and their swizzled writes are
-        // both free of bank conflicts
-        CUresult r = enc(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(q), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
-    }
-    {
-        const int64_t nkb = p->ks / tpr::kMxPair;
-        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(2 * p->hidden), static_cast<cuuint64_t>(nkb),
-                                    static_cast<cuuint64_t>(p->n_ranks)};
-        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(2 * p->hidden),
-                                       static_cast<cuuint64_t>(2 * p->hidden * nkb)};
-        const cuuint32_t box[3] = {tpr::kMxScaleTile, 1, 1};
-        CUresult r = enc(ms, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(scales), dims, strides,
-                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
-    }
-    return TP_OK;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(p->ks), static_cast<cuuint64_t>(p->hidden),
+                                static_cast<cuuint64_t>(p->n_ranks)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(p->ks), static_cast<cuuint64_t>(p->hidden * p->ks)};
+    const cuuint32_t box[3] = {block_scaled ? static_cast<cuuint32_t>(tpr::kMxChunkCols)
+                                            : static_cast<cuuint32_t>(tpr::kTcKBlock),
+                               tpr::kTcRows, 1};
+    CUresult r = enc(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(q), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     block_scaled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? TP_OK : cuda_fail(cudaErrorInvalidValue);
 }
 
 // NVFP4 code pairs [N][H][Ks/2] bytes, 128 rows x 32 bytes per box, and the
@@ -488,6 +486,18 @@ cudaError_t launch_tc_kernel(dim3 grid, size_t smem, cudaStream_t stream, int cl
                               stream, cluster_x, mw, mx, ms, prm);
 }
 
+// The block-scaled MXFP8 form (at most 8 tokens, one 32-column tile) for an
+// epilogue mode.
+cudaError_t dispatch_tc_bs(int mode, dim3 grid, size_t smem, cudaStream_t st, int cl, const CUtensorMap& mw,
+                           const CUtensorMap& mx, const CUtensorMap& ms, const tpr::TcParams& prm) {
+    using namespace tpr;
+    if (mode == kTcClusterFold)
+        return launch_tc_kernel<32, kTcClusterFold, kFmtMxfp8Bs>(grid, smem, st, cl, mw, mx, ms, prm);
+    if (mode == kTcCounterFold)
+        return launch_tc_kernel<32, kTcCounterFold, kFmtMxfp8Bs>(grid, smem, st, 1, mw, mx, ms, prm);
+    return launch_tc_kernel<32, kTcStore, kFmtMxfp8Bs>(grid, smem, st, 1, mw, mx, ms, prm);
+}
+
 // The instantiation for a token tile and an epilogue mode.
 template <int MX>
 cudaError_t dispatch_tc(int bn, int mode, dim3 grid, size_t smem, cudaStream_t st, int cl,
@@ -523,16 +533,17 @@ tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* 
     if (c.cluster_fold) fold = false;
     // Prefill-sized bf16 tiles without a k-split run on CTA pairs (2-SM MMA),
     // which fold in their epilogue with `fold`.
-    if (tc2_path(p, c, wt.fmt))
+    if (tc2_path(p, c, c.fmt))
         return launch_tc2(p, x, wt.w, partials, tokens, stream, fold,
                           counters ? counters + 2 * c.h_tiles : nullptr,   // after the counter fold's words
                           residual, out);
     if (fold && (c.m_tiles != 1 || tokens > 2)) return TP_ERR_UNSUPPORTED;  // the kernel folds <= 2 rows
     CUtensorMap mw, mx, ms;
-    tp_status st = encode_tc_maps(p, c.x_rows, x, wt.w, tokens, &mw, &mx);
+    tp_status st = encode_tc_maps(p, c.x_rows, x, wt.w, tokens, &mw, &mx, c.fmt == tpr::kFmtMxfp8Bs);
     if (st != TP_OK) return st;
-    if (wt.fmt == tpr::kFmtMxfp8) {
-        if ((st = encode_mx_maps(p, wt.w, wt.scales, &mw, &ms)) != TP_OK) return st;
+    if (c.fmt == tpr::kFmtMxfp8 || c.fmt == tpr::kFmtMxfp8Bs) {
+        if ((st = encode_mx_maps(p, wt.w, c.fmt == tpr::kFmtMxfp8Bs, &mw)) != TP_OK) return st;
+        ms = mw;   // not read
     } else if (wt.fmt == tpr::kFmtNvfp4) {
         if ((st = encode_nv_maps(p, wt.w, wt.scales, &mw, &ms)) != TP_OK) return st;
     } else {
@@ -557,6 +568,8 @@ tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* 
     prm.out = static_cast<uint16_t*>(out);
     prm.x = static_cast<const uint16_t*>(x);
     prm.k = p->k;
+    prm.mx_scales = wt.fmt == tpr::kFmtMxfp8 ? static_cast<const uint8_t*>(wt.scales) : nullptr;
+    prm.mx_kg = static_cast<int>((p->ks + tpr::kMxChunkCols - 1) / tpr::kMxChunkCols);
     prm.nv_gexp = wt.fmt == tpr::kFmtNvfp4
                       ? reinterpret_cast<const int*>(static_cast<const uint8_t*>(wt.scales) + nv_scale_bytes(p))
                       : nullptr;
@@ -564,8 +577,9 @@ tp_status launch_tc(const tp_plan* p, const void* x, const TcWeights& wt, void* 
     const int cl = c.cluster_fold ? p->n_ranks * c.splits : 1;
     const dim3 grid(c.grid);
     const cudaError_t e =
-        wt.fmt == tpr::kFmtMxfp8   ? dispatch_tc<tpr::kFmtMxfp8>(c.bn, mode, grid, c.smem, stream, cl, mw, mx, ms, prm)
-        : wt.fmt == tpr::kFmtNvfp4 ? dispatch_tc<tpr::kFmtNvfp4>(c.bn, mode, grid, c.smem, stream, cl, mw, mx, ms, prm)
+        c.fmt == tpr::kFmtMxfp8Bs  ? dispatch_tc_bs(mode, grid, c.smem, stream, cl, mw, mx, ms, prm)
+        : c.fmt == tpr::kFmtMxfp8  ? dispatch_tc<tpr::kFmtMxfp8>(c.bn, mode, grid, c.smem, stream, cl, mw, mx, ms, prm)
+        : c.fmt == tpr::kFmtNvfp4  ? dispatch_tc<tpr::kFmtNvfp4>(c.bn, mode, grid, c.smem, stream, cl, mw, mx, ms, prm)
                                    : dispatch_tc<tpr::kFmtBf16>(c.bn, mode, grid, c.smem, stream, cl, mw, mx, ms, prm);
     return e == cudaSuccess ? TP_OK : cuda_fail(e);
 }
@@ -611,6 +625,9 @@ cudaError_t set_kernel_attrs(int smem_optin, int* dyn_max) {
         reinterpret_cast<const void*>(tpr::exact_partial_kernel<4>),
         reinterpret_cast<const void*>(tpr::exact_partial_kernel<8>),
         TC_KERNELS(tpr::kFmtBf16), TC_KERNELS(tpr::kFmtMxfp8), TC_KERNELS(tpr::kFmtNvfp4),
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<32, tpr::kTcStore, tpr::kFmtMxfp8Bs>),
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<32, tpr::kTcCounterFold, tpr::kFmtMxfp8Bs>),
+        reinterpret_cast<const void*>(tpr::tc_partial_kernel<32, tpr::kTcClusterFold, tpr::kFmtMxfp8Bs>),
         reinterpret_cast<const void*>(tpr::tc_partial_kernel<256, tpr::kTcStore, tpr::kFmtBf16>),
         reinterpret_cast<const void*>(tpr::tc2_partial_kernel)};
     int lowest = smem_optin;
@@ -804,7 +821,7 @@ static tp_status tensor_reconcile(const tp_plan* plan, const void* x, const TcWe
     const bool fold = tc_folds(plan, tokens, wt.fmt);
     tp_status st = launch_tc(plan, x, wt, partials, tokens, true, fold, counters, residual, out, s);
     if (st != TP_OK || fold) return st;
-    const int splits = tc_config(plan, tokens, true).splits;
+    const int splits = tc_config(plan, tokens, true, wt.fmt).splits;
     if (splits > 1) return launch_ring_splits(plan, partials, splits, residual, out, tokens, s);
     return launch_ring(plan, partials, residual, out, tokens, s);
 }
@@ -906,11 +923,19 @@ uint64_t tp_ring_bytes(int n_ranks, int64_t tokens, int64_t hidden, int elem_byt
 
 // ---------------------------------------------------- MXFP8 weight shards --
 
+// Scale bytes of an MXFP8 shard set: one 512-byte chunk per rank, 128-row
+// tile and 128 columns of a rank slice.
+size_t mx_scale_bytes(const tp_plan* p) {
+    const int64_t h_tiles = (p->hidden + 127) / 128;
+    const int64_t kg = (p->ks + tpr::kMxChunkCols - 1) / tpr::kMxChunkCols;
+    return static_cast<size_t>(p->n_ranks) * h_tiles * kg * tpr::kMxChunk;
+}
+
 tp_status tp_plan_mxfp8_bytes(const tp_plan* plan, size_t* q_bytes, size_t* scale_bytes) {
     if (!plan || !q_bytes || !scale_bytes) return TP_ERR_INVALID;
     if (plan->ks % tpr::kMxPair != 0) return TP_ERR_UNSUPPORTED;
     *q_bytes = static_cast<size_t>(plan->hidden) * static_cast<size_t>(plan->k);
-    *scale_bytes = *q_bytes / tpr::kMxBlock;
+    *scale_bytes = mx_scale_bytes(plan);
     return TP_OK;
 }
 
@@ -928,11 +953,14 @@ tp_status tp_pack_weights_mxfp8(const tp_plan* plan, const void* w_hk, void* w_q
     if (plan->ks % tpr::kMxPair != 0) return TP_ERR_UNSUPPORTED;
     if (!aligned16(w_hk) || !aligned16(w_q) || !aligned16(w_scales)) return TP_ERR_ALIGN;
     const size_t wb = static_cast<size_t>(plan->hidden) * plan->k * 2;
-    const size_t qb = wb / 2, sb = qb / tpr::kMxBlock;
+    const size_t qb = wb / 2, sb = mx_scale_bytes(plan);
     if (overlaps(w_hk, wb, w_q, qb) || overlaps(w_hk, wb, w_scales, sb) || overlaps(w_q, qb, w_scales, sb))
         return TP_ERR_INVALID;
     tp_status st = check_device(plan);
     if (st != TP_OK) return st;
+    // the chunks' padding (rows past H, runs past K/N) reads as scale 2^-127
+    cudaError_t me = cudaMemsetAsync(w_scales, 0, sb, static_cast<cudaStream_t>(stream));
+    if (me != cudaSuccess) return cuda_fail(me);
     const int64_t blocks_total = static_cast<int64_t>(plan->n_ranks) * plan->hidden * (plan->ks / tpr::kMxBlock);
     const int64_t grid = std::min<int64_t>((blocks_total + 255) / 256, static_cast<int64_t>(plan->sm_count) * 16);
     tpr::pack_weights_mx_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
@@ -955,7 +983,7 @@ tp_status tp_rowlinear_reconcile_mxfp8(const tp_plan* plan, const void* x, const
         return TP_ERR_ALIGN;
     const size_t mh = static_cast<size_t>(tokens) * plan->hidden * 2;
     const size_t xb = static_cast<size_t>(tokens) * plan->k * 2;
-    const size_t qb = static_cast<size_t>(plan->hidden) * plan->k, sb = qb / tpr::kMxBlock;
+    const size_t qb = static_cast<size_t>(plan->hidden) * plan->k, sb = mx_scale_bytes(plan);
     const size_t ws = tp_plan_mxfp8_workspace_bytes(plan, tokens);
     if (overlaps(out, mh, x, xb) || overlaps(out, mh, w_q, qb) || overlaps(out, mh, w_scales, sb) ||
         overlaps(out, mh, residual, mh) || overlaps(out, mh, workspace, ws))

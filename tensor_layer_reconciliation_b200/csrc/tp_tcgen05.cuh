@@ -94,6 +94,32 @@ __device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, u
         : "memory");
 }
 
+// Block-scaled MMA, kind::mxf8f6f4 with E4M3 A and B and E8M0 scales, one per
+// 32 values of K (one K = 32 step): D[tmem] (+)= sum over k of
+// (A[m][k] * SA[m]) * (B[n][k] * SB[n]). The scales are read from tensor
+// memory: row m's from lane m of column sfa_tmem + m / 32, column n's from
+// lane n of column sfb_tmem + n / 32, byte `sf_id` of the 32-bit cell (the
+// layout tcgen05.cp .32x128b.warpx4 writes); the instruction descriptor
+// carries the same byte index (idesc_mxf8_f32).
+__device__ __forceinline__ void umma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Copies a 32-row x 16-byte shared-memory tile (descriptor `sdesc`) into 4
+// columns of tensor memory from column taddr, once into each 32-lane
+// quarter: lane 32q + r, column taddr + c <- bytes 16r + 4c .. 16r + 4c + 3.
+// Asynchronous, in issue order with this thread's MMAs.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrives once on the mbarrier when every MMA this thread issued so far has
 // completed (and their shared-memory reads are done).
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -124,6 +150,29 @@ __device__ __forceinline__ uint64_t smem_desc_k128(const void* tile) {
     d |= 1ull << 46;                    // version
     d |= 2ull << 61;                    // 128-byte swizzle
     return d;
+}
+
+// Descriptor of a 32-row x 16-byte shared-memory tile, rows 16 bytes apart
+// (no swizzle: 8-row core matrices of 128 contiguous bytes, 128 bytes apart
+// in the stride dimension; one core matrix wide, so the leading offset is
+// not used), the source of tmem_cp_32x128b_x4.
+__device__ __forceinline__ uint64_t smem_desc_rows16(const void* tile) {
+    const uint64_t addr = static_cast<uint64_t>(smem_u32(tile));
+    uint64_t d = (addr >> 4) & 0x3FFFull;
+    d |= (128ull >> 4) << 16;           // LBO (unused)
+    d |= (128ull >> 4) << 32;           // SBO
+    d |= 1ull << 46;                    // version
+    return d;                           // layout 0: no swizzle
+}
+
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4.block_scale with E4M3
+// A and B (format 0), fp32 D, both K-major, E8M0 scales:
+//   bits 4-5 B scale byte, bits 7-9 / 10-12 A / B format (0 = E4M3),
+//   bits 17-22 N >> 3, bit 23 scale format (1 = E8M0), bits 24-28 M >> 4,
+//   bits 29-30 A scale byte, bit 31 K size (0: K = 32).
+__host__ __device__ constexpr uint32_t idesc_mxf8_f32(int m, int n, int sf_id) {
+    return (static_cast<uint32_t>(sf_id) << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(m >> 4) << 24) | (static_cast<uint32_t>(sf_id) << 29);
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B, fp32 D,

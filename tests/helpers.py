@@ -120,13 +120,46 @@ def round_f32_exact(v: Fraction) -> Fraction:
 
 
 def mx_scales_as_stored(sc):
-    """The oracle's MXFP8 scales [N][H][K/N/32] in the library's storage order
-    [N][K/N/64][H][2] (the two 32-weight runs of each 64-column block of a
-    rank slice, row after row), flattened. A permutation only."""
-    sc = np.asarray(sc)
+    """The oracle's MXFP8 scales [N][H][K/N/32] in the library's storage order,
+    flattened: [N][ceil(H/128)][ceil(K/N/128)] chunks of 512 bytes, row t of a
+    128-row tile and run j (of the chunk's four 32-column runs) at byte
+    16 (t % 32) + 4 (t // 32) + j; zeros where rows pass H or runs pass K/N.
+    A permutation plus padding only."""
+    sc = np.asarray(sc, dtype=np.uint8)
     n, h, nb = sc.shape
-    assert nb % 2 == 0
-    return np.ascontiguousarray(sc.reshape(n, h, nb // 2, 2).transpose(0, 2, 1, 3)).reshape(-1)
+    ht, kg = (h + 127) // 128, (nb + 3) // 4
+    pad = np.zeros((n, ht * 128, kg * 4), dtype=np.uint8)
+    pad[:, :h, :nb] = sc
+    # (rank, tile, t // 32, t % 32, chunk, j) -> (rank, tile, chunk, t % 32, t // 32, j)
+    return np.ascontiguousarray(pad.reshape(n, ht, 4, 32, kg, 4).transpose(0, 1, 4, 3, 2, 5)).reshape(-1)
+
+
+def x_split_exponent(amax):
+    """E8M0 exponent e1 of the block-scaled form's first activation term for
+    32-value runs with largest magnitude amax: floor(log2 amax) - 7, at
+    least -127."""
+    a = np.asarray(amax, dtype=np.float64)
+    _, e = np.frexp(np.where(a > 0, a, 1.0))
+    return np.where(a > 0, np.maximum(e - 1 - 7, -127), -127).astype(np.int64)
+
+
+def x_split_error_bound(n, x_u16, w_u16):
+    """Bound on how far the block-scaled MXFP8 form's partials [N][M][H] can
+    move from the exact products by splitting each activation into two E4M3
+    terms (x = 2^e1 q1 + 2^e2 q2 per 32-value run of a rank slice): an x below
+    2^(e1 - 6) may be off by 2^(e1 - 14), any x by at most 2^-137 (runs so
+    small that the second term's exponent stops at -127); each error is
+    weighted by |w|. x [M][K], w [H][K] as bf16 bit patterns."""
+    from oracle import f32
+    x = f32(np.asarray(x_u16, dtype=np.uint16)).astype(np.float64)
+    w = np.abs(f32(np.asarray(w_u16, dtype=np.uint16)).astype(np.float64))
+    m, k = x.shape
+    ks = k // n
+    runs = np.abs(x).reshape(m, n, ks // 32, 32)
+    e1 = x_split_exponent(runs.max(axis=3))[..., None]
+    err = np.where(runs < np.ldexp(1.0, e1 - 6), np.ldexp(1.0, e1 - 14), 0.0) + 2.0 ** -137
+    err = err.reshape(m, n, ks)
+    return np.stack([err[:, r, :] @ w[:, r * ks:(r + 1) * ks].T for r in range(n)])
 
 
 def nv_scales_as_stored(sc, g, amax_bits):
