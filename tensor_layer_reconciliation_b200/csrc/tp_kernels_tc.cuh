@@ -100,13 +100,10 @@ constexpr int kFmtMxfp8Bs = 3; // MXFP8 codes read by the block-scaled MMA (at m
 // maximum) is split exactly; a smaller one is off by at most 2^(e1 - 14).
 // The MMA's B operand holds q1 of token t in row t and q2 in row 8 + t; the
 // epilogue adds accumulator columns t and 8 + t in fp32.
-// The split activations have a ring of their own (kBsXSlots slots, apart
-// from the code stages), so the splits run ahead of the MMAs whenever the
-// codes come late. A slot first receives the bf16 block of x by TMA ([8
-// tokens][128] bf16, 2 KB, no swizzle); the splitting warps read it into
-// registers and then write the B tile and its scale chunk over it.
-constexpr int kBsXSlots = 8;                              // <= kCvtSlotsMax
-constexpr int kBsXLead = 4;                               // blocks of x loaded ahead of the split
+// A stage's activation slot first receives the bf16 block of x by TMA ([8
+// tokens][128] bf16, 2 KB, no swizzle; a barrier of its own, x_full); the
+// splitting warps read it into registers and then write the B tile and its
+// scale chunk over it.
 constexpr uint32_t kBsBRows = 16;                         // MMA N: 8 tokens x 2 terms
 constexpr uint32_t kBsXTile = 8 * kMxChunkCols * 2;       // the bf16 activation block
 constexpr uint32_t kBsSfbOff = kBsBRows * 128;            // B scale chunk after the B tile
@@ -585,7 +582,6 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     constexpr bool BS = FMT == kFmtMxfp8Bs;                     // block-scaled MMA on the codes
     static_assert(!BS || BN == 32, "block-scaled form: a 32-column accumulator, at most 8 tokens");
     static_assert(!BS || (kBsAccs >= 1 && kBsAccs * 16 <= BN && 4 % kBsAccs == 0), "accumulators fit the unit's columns");
-    static_assert(kBsXSlots <= kCvtSlotsMax && kBsXSlots <= kTcMaxStages && kBsXLead < kBsXSlots, "split ring");
     const uint32_t kBTile = fmt_b_tile(FMT, p.x_rows);
     const bool x_atom = !BS && p.x_rows < BN;
     constexpr bool MX = FMT == kFmtMxfp8 || FMT == kFmtNvfp4;   // converted on chip
@@ -613,8 +609,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     const int S = p.stages;
     uint8_t* a_ring = smem;                                              // weight tiles (TMA)
     uint8_t* b_ring = a_ring + static_cast<size_t>(S) * kWTile;         // activation tiles
-    // activation slots: one per stage, or (BS) the split ring's
-    uint8_t* s_ring = b_ring + static_cast<size_t>(BS ? kBsXSlots : S) * kBTile;   // scale tiles
+    uint8_t* s_ring = b_ring + static_cast<size_t>(S) * kBTile;          // scale tiles
     uint64_t* full = reinterpret_cast<uint64_t*>(s_ring + static_cast<size_t>(S) * kSTile);
     uint64_t* empty = full + kTcMaxStages;
     uint64_t* acc_full = empty + kTcMaxStages;   // [2]
@@ -623,13 +618,12 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     uint64_t* fold_ready = mma_done + 1;   // cluster fold: all N partial tiles written
     uint64_t* fold_freed = fold_ready + 1; // cluster fold: all N CTAs done reading mine
     uint64_t* cvt_full = fold_freed + 1;              // MX: [kSlots] converted tile ready (4 warps)
-    uint64_t* cvt_empty = cvt_full + kCvtSlotsMax;    // MX: [kSlots] converted tile read by the MMAs;
-                                                      // BS: [kBsXSlots] split slot read by the MMAs
+    uint64_t* cvt_empty = cvt_full + kCvtSlotsMax;    // MX: [kSlots] converted tile read by the MMAs
     // MX: [S] a stage's activation block landed (its codes and scales land on
     // full[s], so the converters need not wait for the dependency)
     uint64_t* full_x = cvt_empty + kCvtSlotsMax;
-    // BS: full_x [kBsXSlots] split slot written (4 warps); x_full [kBsXSlots]
-    // its bf16 activation block landed
+    // BS: full_x [S] a stage's split activations written (4 warps); x_full
+    // [S] its bf16 activation block landed
     uint64_t* x_full = full_x + kTcMaxStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_full + kTcMaxStages);
     // cluster fold: this CTA's bf16 partial tile, [BN tokens][128 rows]
@@ -689,7 +683,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int s = 0; s < kTcMaxStages; ++s) {   // (BS: split slots, up to kBsXSlots)
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full_x[s], BS ? 4 : 1);       // BS: the four splitting warps
             mbar_init(&x_full[s], 1);
         }
@@ -700,7 +694,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         mbar_init(mma_done, 1);
         mbar_init(fold_ready, static_cast<uint32_t>(csize));
         mbar_init(fold_freed, static_cast<uint32_t>(csize));
-        for (int j = 0; j < (BS ? kBsXSlots : kSlots); ++j) {
+        for (int j = 0; j < kSlots; ++j) {
             mbar_init(&cvt_full[j], 4);
             mbar_init(&cvt_empty[j], 1);
         }
@@ -773,96 +767,47 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
     };
 
     // Block-scaled form: converter warp 6 + run splits run `run` (32 columns)
-    // of every k-block's 128 activation columns, for the (at most 8) tokens,
-    // into split slot i % kBsXSlots (B tile and scale chunk). The bf16 block
-    // lands in the slot by TMA (x_full), issued by lane 0 of warp 6
-    // kBsXSlots - kBsXLead blocks ahead of the split once the MMAs that read
-    // the slot's previous split are done; each lane takes its 16 bytes into
-    // registers, and once all four warps have theirs (one barrier, which
-    // also makes the decision to give up common to them) the split
-    // overwrites the block.
+    // of every stage's 128 activation columns, for the (at most 8) tokens,
+    // into the stage's B tile and its scale chunk: the bf16 block lands in
+    // the stage's slot by TMA (x_full), each lane takes its 16 bytes into
+    // registers, and once all four warps have theirs (one barrier, which also
+    // makes the decision to give up common to them) the split overwrites it.
     auto run_x_split = [&]() {
         if constexpr (BS) {
             const int run = warp - 6;
             const int t = lane >> 2, part = lane & 3;
-            const bool issuer = warp == 6 && lane == 0;
             // the scale chunks' bytes no split writes (rows 16.., columns 1..)
             // are never read by the MMA: zero them once all the same
-            for (int j = 0; j < kBsXSlots; ++j)
-                *reinterpret_cast<uint32_t*>(b_ring + static_cast<size_t>(j) * kBTile + kBsSfbOff +
+            for (int s = 0; s < S; ++s)
+                *reinterpret_cast<uint32_t*>(b_ring + static_cast<size_t>(s) * kBTile + kBsSfbOff +
                                              4 * (32 * run + lane)) = 0u;
-            // (unit, k-block) walk in issue order, for the loads
-            struct XCursor {
-                int lu, kb, kb_hi, r, mt;
-            };
-            auto x_enter = [&](XCursor& c) {
-                if (c.lu < my_units) {
-                    int ht, sp;
-                    unit_of(c.lu, c.r, ht, c.mt, sp);
-                    split_range(sp, c.kb, c.kb_hi);
-                }
-            };
-            auto x_advance = [&](XCursor& c) {
-                if (++c.kb == c.kb_hi) {
-                    ++c.lu;
-                    x_enter(c);
-                }
-            };
-            int n = 0;   // k-blocks of this CTA
-            for (int lu = 0; lu < my_units; ++lu) {
+            asm volatile("bar.sync 3, 128;" ::: "memory");   // zeroed before any split
+            int s = 0;
+            uint32_t ph = 0;   // parity of stage s's use
+            bool ok = true;
+            for (int lu = 0; lu < my_units && ok; ++lu) {
                 int r, ht, mt, sp, kb_lo, kb_hi;
                 unit_of(lu, r, ht, mt, sp);
                 split_range(sp, kb_lo, kb_hi);
-                n += kb_hi - kb_lo;
-            }
-            XCursor ld{0, 0, 0, 0, 0};
-            x_enter(ld);
-            int issued = 0;
-            auto issue_x = [&]() {   // the next block of the walk into its slot
-                const int j = issued % kBsXSlots;
-                mbar_arrive_expect_tx(&x_full[j], kBsXTile);
-                tma_load_3d(b_ring + static_cast<size_t>(j) * kBTile, &tmap_x, &x_full[j], ld.kb * KB, ld.r,
-                            ld.mt * BN);
-                x_advance(ld);
-                ++issued;
-            };
-            asm volatile("bar.sync 3, 128;" ::: "memory");   // zeroed before any load lands
-            if (issuer) {
-                pdl_wait();  // activations may be produced by the previous kernel
-                while (issued < n && issued < kBsXSlots - kBsXLead) issue_x();
-            }
-            bool ok = true;
-            int i = 0;
-            for (; i < n; ++i) {
-                const int j = i % kBsXSlots;
-                const uint32_t ph = static_cast<uint32_t>(i / kBsXSlots) & 1u;
-                ok = mbar_wait_bounded(&x_full[j], ph);
-                uint8_t* bt = b_ring + static_cast<size_t>(j) * kBTile;
-                const uint4 v = *reinterpret_cast<const uint4*>(bt + t * (kMxChunkCols * 2) + (run * 32 + part * 8) * 2);
-                if (bar_sync_any(3, 128, !ok || *reinterpret_cast<volatile int*>(&abort_flag) != 0)) {
-                    ok = false;
-                    atomicExch(&abort_flag, 1);
-                    break;
-                }
-                x_split_run(v, bt, t, run, part);
-                fence_proxy_async_smem();   // the tensor core reads them through the async proxy
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full_x[j]);
-                // refill: the block kBsXSlots - kBsXLead ahead, into the slot
-                // of block i - kBsXLead once the MMAs have read that split
-                if (issuer && issued < n) {
-                    const int prev = issued - kBsXSlots;   // the slot's previous block
-                    if (prev < 0 || mbar_wait_bounded(&cvt_empty[issued % kBsXSlots],
-                                                      static_cast<uint32_t>(prev / kBsXSlots) & 1u))
-                        issue_x();
-                    else
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
+                    ok = mbar_wait_bounded(&x_full[s], ph);
+                    uint8_t* bt = b_ring + static_cast<size_t>(s) * kBTile;
+                    const uint4 v = *reinterpret_cast<const uint4*>(bt + t * (kMxChunkCols * 2) + (run * 32 + part * 8) * 2);
+                    if (bar_sync_any(3, 128, !ok || *reinterpret_cast<volatile int*>(&abort_flag) != 0)) {
+                        ok = false;
                         atomicExch(&abort_flag, 1);
+                        break;
+                    }
+                    x_split_run(v, bt, t, run, part);
+                    fence_proxy_async_smem();   // the tensor core reads them through the async proxy
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full_x[s]);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
-            // blocks still landing (after an abort): wait for them (bounded)
-            if (issuer)
-                for (int k = i; k < issued; ++k)
-                    if (!mbar_wait_bounded(&x_full[k % kBsXSlots], static_cast<uint32_t>(k / kBsXSlots) & 1u)) break;
         }
     };
 
@@ -931,7 +876,16 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                                      static_cast<uint32_t>((k_hi - k_lo) * 2));
             }
             pdl_wait();  // activations may be produced by the previous kernel
-            if (!BS) {   // (the block-scaled form's splitting warps load their own)
+            if (BS) {   // the bf16 blocks the splitting warps take (own barrier)
+                Cursor c0{0, 0, 0, 0, 0, 0, 0};
+                enter_unit(c0);
+                for (int i = 0; i < pre; ++i) {
+                    mbar_arrive_expect_tx(&x_full[i], kBsXTile);
+                    tma_load_3d(b_ring + static_cast<size_t>(i) * kBTile, &tmap_x, &x_full[i], c0.kb * KB, c0.r,
+                                c0.mt * BN);
+                    advance(c0);
+                }
+            } else {
                 // the same first positions again, for their activation blocks
                 Cursor c0{0, 0, 0, 0, 0, 0, 0};
                 enter_unit(c0);
@@ -953,7 +907,11 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
                 mbar_arrive_expect_tx(&full[s], tx);
                 load_w(s, cur.kb, cur.ht, cur.r);
-                if (!BS) {
+                if (BS) {
+                    mbar_arrive_expect_tx(&x_full[s], kBsXTile);
+                    tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, &x_full[s], cur.kb * KB, cur.r,
+                                cur.mt * BN);
+                } else {
                     if (MX) mbar_arrive_expect_tx(&full_x[s], kBTile);
                     tma_load_3d(b_ring + static_cast<size_t>(s) * kBTile, &tmap_x, MX ? &full_x[s] : &full[s],
                                 cur.kb * kTcKBlock, cur.r, cur.mt * BN);
@@ -971,7 +929,8 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             const int first = issued > S ? issued - S : 0;
             for (int i = first; i < issued; ++i)
                 if (!mbar_wait_bounded(&full[i % S], static_cast<uint32_t>(i / S) & 1u) ||
-                    (MX && !mbar_wait_bounded(&full_x[i % S], static_cast<uint32_t>(i / S) & 1u)))
+                    (MX && !mbar_wait_bounded(&full_x[i % S], static_cast<uint32_t>(i / S) & 1u)) ||
+                    (BS && !mbar_wait_bounded(&x_full[i % S], static_cast<uint32_t>(i / S) & 1u)))
                     break;
         }
     } else if (warp == 1) {
@@ -994,15 +953,15 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                 bool ok = true;
                 for (int kb = kb_lo; kb < kb_hi; ++kb, ++i) {
                     // MX: the converters consumed the codes; the MMA needs the activations
-                    // BS: the codes and scales, then split slot j
+                    // BS: the codes and scales, then the split activations
                     if (!mbar_wait_bounded(MX ? &full_x[s] : &full[s], ph) ||
                         (MX && !mbar_wait_bounded(&cvt_full[j], jph)) ||
-                        (BS && !mbar_wait_bounded(&full_x[j], jph))) {
+                        (BS && !mbar_wait_bounded(&full_x[s], ph))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    uint64_t bd = smem_desc_k128(b_ring + static_cast<size_t>(BS ? j : s) * kBTile);
+                    uint64_t bd = smem_desc_k128(b_ring + static_cast<size_t>(s) * kBTile);
                     if (x_atom) bd &= ~(0x3FFFull << 32);   // stride between 8-row groups: 0
                     if constexpr (MX) {
                         // A: the converted tile in tensor memory, 8 columns per 16 of K
@@ -1016,7 +975,7 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                         const uint32_t sfa = tmem_base + kSfaCol + 8u * static_cast<uint32_t>(s);
                         const uint32_t sfb = tmem_base + kSfbCol + 8u * static_cast<uint32_t>(s);
                         tmem_cp_32x128b_x4(sfa, smem_desc_rows16(s_ring + static_cast<size_t>(s) * kSTile));
-                        tmem_cp_32x128b_x4(sfb, smem_desc_rows16(b_ring + static_cast<size_t>(j) * kBTile + kBsSfbOff));
+                        tmem_cp_32x128b_x4(sfb, smem_desc_rows16(b_ring + static_cast<size_t>(s) * kBTile + kBsSfbOff));
                         const uint64_t ad = smem_desc_k128(a_ring + static_cast<size_t>(s) * kWTile);
                         // K = 32 a step (32 bytes of each row); step kk reads scale
                         // byte kk and goes to accumulator kk % kBsAccs
@@ -1033,12 +992,12 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
                             umma_bf16(d, ad + 2ull * kk, bd + 2ull * kk, kIdesc, (kb != kb_lo) || (kk != 0));
                     }
                     umma_commit(&empty[s]);  // frees the stage when these MMAs finish
-                    if (MX || BS) umma_commit(&cvt_empty[j]);   // and the converted (split) slot
+                    if (MX) umma_commit(&cvt_empty[j]);   // and the converted slot
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
                     }
-                    if (++j == (BS ? kBsXSlots : kSlots)) {
+                    if (++j == kSlots) {
                         j = 0;
                         jph ^= 1u;
                     }
@@ -1068,19 +1027,6 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         for (int lu = 0; lu < my_units; ++lu) {
             const int b = lu & 1;
             const uint32_t aph = static_cast<uint32_t>(lu >> 1) & 1u;
-            int r, ht, mt, sp;
-            unit_of(lu, r, ht, mt, sp);
-            // Counter fold: this CTA's place among the parts of its tile, taken
-            // before the accumulator is ready (the tags, not the tickets, say
-            // which parts have landed: the ticket only elects the CTA that
-            // folds), so the round trip overlaps the MMAs.
-            unsigned int ticket = 0, tag = 0;
-            if (MODE == kTcCounterFold) {
-                if (threadIdx.x == 64) ticket = atomicAdd(p.counters + ht * p.m_tiles + mt, 1u);
-                // this call's tag: the tile's folds so far + 1 (the previous
-                // call's fold is complete: the epilogue waited for the dependency)
-                tag = __ldcg(p.counters + p.h_tiles * p.m_tiles + ht * p.m_tiles + mt) + 1u;
-            }
             bool ok = mbar_wait_bounded(&acc_full[b], aph);
             // cluster fold: the peers have read the previous unit's partial tile
             if (kCluster && lu > 0)
@@ -1091,9 +1037,20 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             // The four epilogue warps leave together: one answer for all of them.
             if (bar_sync_any(2, 128, bad)) break;
             tc_fence_after_sync();
+            int r, ht, mt, sp;
+            unit_of(lu, r, ht, mt, sp);
             const int h = ht * kTcRows + q * 32 + lane;
             const int m0 = mt * BN;
             const size_t plane = static_cast<size_t>(p.tokens) * p.hidden;
+            // Counter fold: this CTA's place among the parts of its tile, taken
+            // now so the round trip overlaps the stores below.
+            unsigned int ticket = 0, tag = 0;
+            if (MODE == kTcCounterFold) {
+                if (threadIdx.x == 64) ticket = atomicAdd(p.counters + ht * p.m_tiles + mt, 1u);
+                // this call's tag: the tile's folds so far + 1 (the previous
+                // call's fold is complete: the epilogue waited for the dependency)
+                tag = __ldcg(p.counters + p.h_tiles * p.m_tiles + ht * p.m_tiles + mt) + 1u;
+            }
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];

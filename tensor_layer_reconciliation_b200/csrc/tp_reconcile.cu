@@ -286,17 +286,14 @@ TcConfig tc_config(const tp_plan* p, int64_t tokens, bool allow_split, int fmt =
     // converted bf16 tiles live in tensor memory).
     // At most 8 tokens: one 8-row atom of x a block instead of the BN-row tile
     c.x_rows = tokens <= 8 && c.m_tiles == 1 ? 8 : c.bn;
-    // (the block-scaled form's split activations have a ring of their own)
-    const bool split_ring = fmt == tpr::kFmtMxfp8Bs;
-    const size_t stage = tpr::fmt_code_tile(fmt) + tpr::fmt_scale_tile(fmt) +
-                         (split_ring ? 0 : tpr::fmt_b_tile(fmt, c.x_rows));
+    const size_t stage = tpr::fmt_code_tile(fmt) + tpr::fmt_scale_tile(fmt) + tpr::fmt_b_tile(fmt, c.x_rows);
     // the cluster fold's tile in shared memory: the tile's tokens x 128 rows,
     // bf16 partials or fp32 part sums
     const size_t part_tile = c.cluster_fold ? static_cast<size_t>(std::min<int64_t>(c.bn, tokens)) *
                                                   tpr::kTcRows * (c.splits > 1 ? 4 : 2)
                                             : 0;
     const size_t fixed = (4 * tpr::kTcMaxStages + 7 + 2 * tpr::kCvtSlotsMax) * sizeof(uint64_t) + 16 + 128 +
-                         1024 + part_tile + (split_ring ? tpr::kBsXSlots * tpr::kBsBTile : 0);
+                         1024 + part_tile;
     const size_t budget = std::min<size_t>(two_per_sm ? 110 * 1024 : 200 * 1024,
                                            static_cast<size_t>(p->smem_optin));
     c.stages = budget > fixed
