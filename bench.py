@@ -64,18 +64,18 @@ def _peaks():
 # sources means the kernels changed since, and the traffic is reported null.
 PROFILED_TRAFFIC = {
     # (workload, path): (bytes per call, kernel-source digest, the ncu capture)
-    ("decode_n2", "tensor"): (117927680, "0a546cf619614267",
+    ("decode_n2", "tensor"): (116805184, "fa9855c33663e1b4",
         "ncu dram__bytes of tc_partial_kernel<32> (counter fold) on decode_n2, one call per point kind"),
     ("decode_n4_m32", "tensor"): (119870080, "0a546cf619614267",
         "ncu dram__bytes of tc_partial_kernel<32> + ring_reduce_kernel on decode_n4_m32, one call per point kind"),
-    ("decode_n8_m64", "tensor"): (83639680, "0a546cf619614267",
+    ("decode_n8_m64", "tensor"): (81906688, "fa9855c33663e1b4",
         "ncu dram__bytes of tc_partial_kernel<64> + ring_reduce_kernel on decode_n8_m64, one call per point kind"),
-    ("prefill_n4", "tensor"): (888459776, "0a546cf619614267",
+    ("prefill_n4", "tensor"): (891593728, "fa9855c33663e1b4",
         "ncu dram__bytes of tc2_partial_kernel (fold in the epilogue) on prefill_n4, one call per point kind"),
     ("decode_n2", "exact-fused"): (117532032, "0a546cf619614267",
         "ncu dram__bytes of exact_partial_kernel<1> on decode_n2, one call per point kind"),
-    ("decode_n2", "mxfp8"): (62187008, "0a546cf619614267",
-        "ncu dram__bytes of tc_partial_kernel<32> MXFP8 form on decode_n2, one call per point kind"),
+    ("decode_n2", "mxfp8"): (59951552, "fa9855c33663e1b4",
+        "ncu dram__bytes of tc_partial_kernel<32> block-scaled MXFP8 form on decode_n2, one call per point kind"),
     ("decode_n2", "nvfp4"): (32578176, "0a546cf619614267",
         "ncu dram__bytes of tc_partial_kernel<32> NVFP4 form on decode_n2, one call per point kind"),
     ("decode_n2", "tensor-cluster"): (118056320, "0a546cf619614267",
@@ -657,8 +657,10 @@ def run_config(name, args, device, world, rank, local, peaks):
                   if wl.workspace is None else
                   "k-split parts, ring fold by the CTA completing a tile")
     kern_name = {
-        "mxfp8": (f"reconciliation call: tc_partial_kernel, MXFP8 form (codes widened to bf16 "
-                  f"tiles on chip; {fold_where})" if one_kernel else
+        "mxfp8": (f"reconciliation call: tc_partial_kernel, MXFP8 form ("
+                  + ("codes and scales to the block-scaled MMA, activations split into two E4M3 terms on chip"
+                     if cfg.tokens <= 8 else "codes widened to bf16 tiles on chip")
+                  + f"; {fold_where})" if one_kernel else
                   "reconciliation call: tc_partial_kernel, MXFP8 form, then a ring fold kernel"),
         "nvfp4": (f"reconciliation call: tc_partial_kernel, NVFP4 form (codes widened to bf16 "
                   f"tiles on chip; {fold_where})" if one_kernel else
