@@ -401,8 +401,13 @@ __device__ __forceinline__ void nv_convert_row(const uint8_t* code_row, const ui
 // a tile reads them without waiting for a count: a part whose tag is not yet
 // this call's is read again (bounded). Word-sized stores and loads are
 // single-copy atomic, so a part is never seen half-written.
+// A tagged part as it is now at gpu scope: a volatile relaxed load, so that
+// a polling loop reads memory again on every pass (a plain load of an address
+// the loop never writes may be hoisted out of it).
 __device__ __forceinline__ uint64_t ld_cg_u64(const uint64_t* p) {
-    return __ldcg(reinterpret_cast<const unsigned long long*>(p));
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
 }
 // The low half of a tagged part once its tag is `tag` (read again until then).
 __device__ __forceinline__ bool tagged_part(const uint64_t* p, uint32_t tag, uint32_t& v) {
@@ -1027,6 +1032,19 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
         for (int lu = 0; lu < my_units; ++lu) {
             const int b = lu & 1;
             const uint32_t aph = static_cast<uint32_t>(lu >> 1) & 1u;
+            int r, ht, mt, sp;
+            unit_of(lu, r, ht, mt, sp);
+            // Counter fold: this CTA's place among the parts of its tile, taken
+            // before the accumulator is ready (the tags, not the tickets, say
+            // which parts have landed: the ticket only elects the CTA that
+            // folds), so the round trip overlaps the MMAs.
+            unsigned int ticket = 0, tag = 0;
+            if (MODE == kTcCounterFold) {
+                if (threadIdx.x == 64) ticket = atomicAdd(p.counters + ht * p.m_tiles + mt, 1u);
+                // this call's tag: the tile's folds so far + 1 (the previous
+                // call's fold is complete: the epilogue waited for the dependency)
+                tag = __ldcg(p.counters + p.h_tiles * p.m_tiles + ht * p.m_tiles + mt) + 1u;
+            }
             bool ok = mbar_wait_bounded(&acc_full[b], aph);
             // cluster fold: the peers have read the previous unit's partial tile
             if (kCluster && lu > 0)
@@ -1037,20 +1055,9 @@ __global__ void __launch_bounds__(FMT != kFmtBf16 ? kTcMxThreads : kTcThreads, B
             // The four epilogue warps leave together: one answer for all of them.
             if (bar_sync_any(2, 128, bad)) break;
             tc_fence_after_sync();
-            int r, ht, mt, sp;
-            unit_of(lu, r, ht, mt, sp);
             const int h = ht * kTcRows + q * 32 + lane;
             const int m0 = mt * BN;
             const size_t plane = static_cast<size_t>(p.tokens) * p.hidden;
-            // Counter fold: this CTA's place among the parts of its tile, taken
-            // now so the round trip overlaps the stores below.
-            unsigned int ticket = 0, tag = 0;
-            if (MODE == kTcCounterFold) {
-                if (threadIdx.x == 64) ticket = atomicAdd(p.counters + ht * p.m_tiles + mt, 1u);
-                // this call's tag: the tile's folds so far + 1 (the previous
-                // call's fold is complete: the epilogue waited for the dependency)
-                tag = __ldcg(p.counters + p.h_tiles * p.m_tiles + ht * p.m_tiles + mt) + 1u;
-            }
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
