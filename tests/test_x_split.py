@@ -84,3 +84,26 @@ def test_split_exact_for_gaussian_runs():
     assert np.array_equal(got[~small], runs[~small])
     bound = np.broadcast_to(np.ldexp(1.0, e1 - 14), runs.shape)
     assert np.all(np.abs(runs - got)[small] <= bound[small] + 2.0 ** -137)
+
+
+def test_margin_bounds_the_split_partials():
+    """helpers.x_split_error_bound against the exact effect of the split on
+    each partial (sum over k of (x - split(x)) * w, one rank slice), on inputs
+    that put small values into runs with large maxima."""
+    from helpers import x_split_error_bound
+    rng = np.random.default_rng(11)
+    n, m, k, h = 2, 3, 256, 8
+    x = rng.standard_normal((m, k)).astype(np.float32)
+    x[:, ::7] *= 1e-5                                    # values far below their run's maximum
+    w = (0.02 * rng.standard_normal((h, k))).astype(np.float32)
+    xb, wb = oracle.bf16_rne(x), oracle.bf16_rne(w)
+    xv = oracle.f32(xb).astype(np.float64)
+    wv = oracle.f32(wb).astype(np.float64)
+    got, _, _ = split(xv.reshape(-1, 32))
+    err = (xv - got.reshape(m, k))
+    ks = k // n
+    exact = np.stack([np.abs(err[:, r * ks:(r + 1) * ks] @ wv[:, r * ks:(r + 1) * ks].T) for r in range(n)])
+    bound = x_split_error_bound(n, xb, wb)
+    assert exact.shape == bound.shape
+    assert np.all(exact <= bound)
+    assert exact.max() > 0                               # the case exercises inexact splits
