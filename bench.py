@@ -64,17 +64,17 @@ def _peaks():
 # sources means the kernels changed since, and the traffic is reported null.
 PROFILED_TRAFFIC = {
     # (workload, path): (bytes per call, kernel-source digest, the ncu capture)
-    ("decode_n2", "tensor"): (116298944, "fb8ed4f6a5e794b3",
+    ("decode_n2", "tensor"): (116298944, "6deafc10c0aa3bd1",
         "ncu dram__bytes of tc_partial_kernel<32> (counter fold) on decode_n2, one call per point kind"),
     ("decode_n4_m32", "tensor"): (119870080, "0a546cf619614267",
         "ncu dram__bytes of tc_partial_kernel<32> + ring_reduce_kernel on decode_n4_m32, one call per point kind"),
-    ("decode_n8_m64", "tensor"): (81532160, "fb8ed4f6a5e794b3",
+    ("decode_n8_m64", "tensor"): (81532160, "6deafc10c0aa3bd1",
         "ncu dram__bytes of tc_partial_kernel<64> + ring_reduce_kernel on decode_n8_m64, one call per point kind"),
-    ("prefill_n4", "tensor"): (886932608, "fb8ed4f6a5e794b3",
+    ("prefill_n4", "tensor"): (886932608, "6deafc10c0aa3bd1",
         "ncu dram__bytes of tc2_partial_kernel (fold in the epilogue) on prefill_n4, one call per point kind"),
     ("decode_n2", "exact-fused"): (117532032, "0a546cf619614267",
         "ncu dram__bytes of exact_partial_kernel<1> on decode_n2, one call per point kind"),
-    ("decode_n2", "mxfp8"): (60123584, "fb8ed4f6a5e794b3",
+    ("decode_n2", "mxfp8"): (60123584, "6deafc10c0aa3bd1",
         "ncu dram__bytes of tc_partial_kernel<32> block-scaled MXFP8 form on decode_n2, one call per point kind"),
     ("decode_n2", "nvfp4"): (32578176, "0a546cf619614267",
         "ncu dram__bytes of tc_partial_kernel<32> NVFP4 form on decode_n2, one call per point kind"),

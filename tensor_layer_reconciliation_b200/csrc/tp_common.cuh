@@ -199,70 +199,6 @@ __device__ __forceinline__ uint16_t ring_fold_f32_parts(const float* parts, int 
     return s;
 }
 
-// ring_fold_f32_parts for callers short of registers (the tensor-core
-// kernel's in-kernel fold): ranks one after another, the parts of a rank
-// loaded together. Same sums in the same order, so the same result.
-template <bool kL2>
-__device__ __forceinline__ uint16_t ring_fold_f32_parts_by_rank(const float* parts, int splits,
-                                                                int n_ranks, size_t plane, size_t off,
-                                                                int c) {
-    uint16_t s = 0;
-#pragma unroll 1
-    for (int i = 0; i < n_ranks; ++i) {
-        int rr = c + i;
-        if (rr >= n_ranks) rr -= n_ranks;
-        const float* q = parts + static_cast<size_t>(rr) * plane + off;
-        const size_t step = static_cast<size_t>(n_ranks) * plane;
-        float a[kMaxSplits];
-#pragma unroll
-        for (int sp = 0; sp < kMaxSplits; ++sp)
-            if (sp < splits) a[sp] = kL2 ? __ldcg(q + sp * step) : q[sp * step];
-        float f = a[0];
-#pragma unroll
-        for (int sp = 1; sp < kMaxSplits; ++sp)
-            if (sp < splits) f = __fadd_rn(f, a[sp]);
-        const uint16_t pr = f32_to_bf16_rne(f);
-        s = i == 0 ? pr : bf16_add(s, pr);
-    }
-    return s;
-}
-
-// ring_fold_f32_parts when N * SPLITS <= 16: the parts of every rank are
-// loaded before the first add, in 16 registers (a caller short of registers
-// can afford these; the fully unrolled 8 x 8 form it cannot). Same sums in
-// the same order, so the same result.
-template <bool kL2>
-__device__ __forceinline__ uint16_t ring_fold_f32_parts16(const float* parts, int splits, int n_ranks,
-                                                          size_t plane, size_t off, int c) {
-    constexpr int kVals = 16;
-    float a[kVals];
-    const int nv = n_ranks * splits;
-#pragma unroll
-    for (int j = 0; j < kVals; ++j) {
-        if (j < nv) {
-            const int i = j / splits, sp = j - (j / splits) * splits;
-            int rr = c + i;
-            if (rr >= n_ranks) rr -= n_ranks;
-            const float* q = parts + (static_cast<size_t>(sp) * n_ranks + rr) * plane + off;
-            a[j] = kL2 ? __ldcg(q) : *q;
-        }
-    }
-    uint16_t s = 0;
-    float f = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kVals; ++j) {
-        if (j < nv) {
-            const int sp = j - (j / splits) * splits;
-            f = sp == 0 ? a[j] : __fadd_rn(f, a[j]);
-            if (sp == splits - 1) {
-                const uint16_t pr = f32_to_bf16_rne(f);
-                s = j < splits ? pr : bf16_add(s, pr);
-            }
-        }
-    }
-    return s;
-}
-
 // --------------------------------------------------------------------- TMA --
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
