@@ -84,6 +84,8 @@ SHAPES = [             # N, M, K, H
     (8, 3, 4096, 1024),     # three tokens: K split, fp32 parts, split ring kernel
     (1, 4, 512, 256),       # N = 1
     (2, 1, 17408, 5120),    # the down-projection of the decode example, full size
+    (2, 1, 1152, 384),      # K/N = 576: the last 128-column stage lies half past K/N (block-scaled)
+    (2, 5, 1152, 256),      # five tokens, the same half stage, K split and the split ring kernel
     (8, 64, 1024, 4096),    # 64 tokens, 256 units: bf16 partials and the ring kernel
     (2, 300, 1024, 512),    # 256-token tiles with a K split: parts and the split ring kernel
     (8, 300, 1024, 4224),   # 256-token tiles, no split: bf16 partials and the ring kernel
